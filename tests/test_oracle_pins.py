@@ -1,0 +1,368 @@
+"""Pins for the CPU oracle: checks against things other than the oracle itself.
+
+* hand-worked examples under tests/golden/ (closed forms derived from the
+  definitions, each file citing the page and section it follows);
+* brute force on tiny inputs in plain Python loops (an O(d^2) rank count for
+  top-K, triple loops for the projections), independent of the oracle's sort
+  and matmul;
+* special cases that reduce to textbook results (K = d is the dense layer,
+  K = 0 is zero) and invariants that hold at any size.
+"""
+import itertools
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+import workloads
+from conftest import load_golden
+
+# ---------------------------------------------------------------- brute force
+
+
+def bf_keep(row, k):
+    """Kept set by rank counting: i is kept iff fewer than k entries beat it,
+    where j beats i when |x_j| > |x_i|, or |x_j| == |x_i| and j < i."""
+    d = len(row)
+    mags = [abs(float(v)) for v in row]
+    kept = []
+    for i in range(d):
+        beaters = sum(1 for j in range(d)
+                      if mags[j] > mags[i] or (mags[j] == mags[i] and j < i))
+        if beaters < k:
+            kept.append(i)
+    return kept
+
+
+def bf_matvec(xs_row, wt):
+    """y_j = sum_i xs_i * wt[i][j] by plain loops."""
+    d_in = len(wt)
+    d_out = len(wt[0])
+    return [sum(float(xs_row[i]) * float(wt[i][j]) for i in range(d_in)) for j in range(d_out)]
+
+
+# ---------------------------------------------------------------- top-K pins
+
+
+def test_topk_golden_hand():
+    g = load_golden("topk_hand.json")
+    for row in g["rows"]:
+        x = np.array([row["x"]], dtype=np.float32)
+        for k, want in row["keep"].items():
+            got = oracle.topk_keep(x, int(k))[0].tolist()
+            assert got == want, (row["x"], k)
+    r0 = g["rows"][0]
+    keep, m, xs = oracle.topk_mask(np.array([r0["x"]], dtype=np.float32), 4)
+    assert m[0].tolist() == r0["mask_k4"]
+    assert xs[0].tolist() == r0["xs_k4"]
+
+
+@pytest.mark.parametrize("seed", range(40))
+def test_topk_bruteforce_rank_tiny(seed):
+    g = np.random.default_rng(seed)
+    d = int(g.integers(1, 13))
+    palette = np.array([0.0, -0.0, 0.5, -0.5, 1.0, -1.0, 2.0, -2.0, 3.0], dtype=np.float32)
+    if seed % 2:
+        row = palette[g.integers(0, palette.size, d)]          # many ties
+    else:
+        row = g.standard_normal(d).astype(np.float32)           # distinct
+    for k in range(d + 1):
+        got = oracle.topk_keep(row[None, :], k)[0].tolist()
+        assert got == bf_keep(row, k), (row.tolist(), k)
+
+
+def test_topk_all_equal_and_signed_zero():
+    for d in (1, 5, 33):
+        for val in (1.25, -1.25, 0.0):
+            row = np.full((1, d), val, dtype=np.float32)
+            if val == 0.0:
+                row[0, ::2] = -0.0
+            for k in (0, 1, d // 2, d):
+                assert oracle.topk_keep(row, k)[0].tolist() == list(range(k))
+
+
+def test_topk_rejects_bad_k():
+    x = np.zeros((1, 4), np.float32)
+    for k in (-1, 5):
+        with pytest.raises(ValueError):
+            oracle.topk_keep(x, k)
+
+
+@pytest.mark.parametrize("d,k", [(4096, 2867), (11008, 7705), (4096, 1)])
+def test_topk_invariants_config_sizes(d, k):
+    x = workloads.normal_f32(workloads.rng(d + k), (3, d))
+    keep, m, xs = oracle.topk_mask(x, k)
+    assert keep.shape == (3, k)
+    assert np.all(m.sum(axis=1) == k)                       # exactly K selected
+    for t in range(3):
+        kept = np.abs(x[t, keep[t]])
+        dropped = np.abs(x[t, m[t] == 0])
+        if dropped.size:
+            assert kept.min() >= dropped.max()              # every kept >= every dropped
+        assert np.all(np.diff(keep[t]) > 0)                 # ascending, distinct
+    assert np.array_equal(xs != 0, m.astype(bool))
+
+
+# ---------------------------------------------------------------- sparse linear
+
+
+def test_sparse_linear_golden_hand():
+    g = load_golden("sparse_linear_hand.json")
+    x = np.array([g["x"]], dtype=np.float32)
+    wt = np.array(g["wt"], dtype=np.float32)
+    for k, want in g["y"].items():
+        assert oracle.sparse_linear(x, wt, int(k))[0].tolist() == want
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_sparse_linear_bruteforce_nonsquare(seed):
+    g = np.random.default_rng(100 + seed)
+    T, d_in, d_out = int(g.integers(1, 4)), int(g.integers(1, 9)), int(g.integers(1, 7))
+    x = g.standard_normal((T, d_in)).astype(np.float32)
+    wt = g.standard_normal((d_in, d_out)).astype(np.float32)
+    for k in range(d_in + 1):
+        y = oracle.sparse_linear(x, wt, k)
+        for t in range(T):
+            kept = set(bf_keep(x[t], k))
+            xs = [x[t, i] if i in kept else 0.0 for i in range(d_in)]
+            ref = bf_matvec(xs, wt.tolist())
+            assert np.allclose(y[t], ref, rtol=1e-12, atol=1e-12)
+
+
+def test_sparse_linear_k_eq_d_is_dense_and_k0_is_zero():
+    g = np.random.default_rng(7)
+    x = g.standard_normal((2, 6)).astype(np.float32)
+    wt = g.standard_normal((6, 5)).astype(np.float32)
+    dense = [bf_matvec(x[t], wt.tolist()) for t in range(2)]
+    assert np.allclose(oracle.sparse_linear(x, wt, 6), dense, rtol=1e-12, atol=1e-12)
+    assert np.all(oracle.sparse_linear(x, wt, 0) == 0.0)
+
+
+def test_sparse_linear_unselected_rows_do_not_matter():
+    g = np.random.default_rng(11)
+    x = g.standard_normal((1, 64)).astype(np.float32)
+    wt = g.standard_normal((64, 16)).astype(np.float32)
+    k = 20
+    keep = oracle.topk_keep(x, k)[0]
+    y0 = oracle.sparse_linear(x, wt, k)
+    dropped = np.setdiff1d(np.arange(64), keep)
+    wt2 = wt.copy()
+    wt2[dropped] = 1e6                        # masked columns contribute nothing
+    assert np.array_equal(oracle.sparse_linear(x, wt2, k), y0)
+    wt3 = wt.copy()
+    wt3[keep[0]] += 1.0                       # a kept row does contribute
+    assert not np.array_equal(oracle.sparse_linear(x, wt3, k), y0)
+
+
+# ---------------------------------------------------------------- FFN
+
+
+def test_ffn_golden_hand_relu2():
+    g = load_golden("ffn_hand.json")
+    x = np.array([g["x"]], dtype=np.float32)
+    c = g["relu2_glu"]
+    for k_h, want in c["y"].items():
+        r = oracle.sparse_ffn(x, g["wt_up"], g["wt_gate"], g["wt_down"], "relu2_glu",
+                              c["k_in"], int(k_h))
+        assert r["u"][0].tolist() == c["u"]
+        assert r["g"][0].tolist() == c["g"]
+        assert r["h"][0].tolist() == c["h"]
+        assert r["keep_h"][0].tolist() == c["keep_h"][k_h]
+        assert r["y"][0].tolist() == want
+
+
+def test_ffn_golden_hand_drelu():
+    g = load_golden("ffn_hand.json")
+    x = np.array([g["x"]], dtype=np.float32)
+    c = g["drelu"]
+    b = np.full(4, c["bias"])
+    r = oracle.sparse_ffn(x, g["wt_up"], g["wt_gate"], g["wt_down"], "drelu", c["k_in"],
+                          c["k_h"], b_up=b, b_gate=b)
+    assert r["u"][0].tolist() == c["u"]
+    assert r["g"][0].tolist() == c["g"]
+    assert r["h"][0].tolist() == c["h"]
+    assert r["keep_h"][0].tolist() == c["keep_h"]
+    assert r["y"][0].tolist() == c["y"]
+
+
+@pytest.mark.parametrize("act", ["relu2_glu", "drelu"])
+@pytest.mark.parametrize("seed", range(6))
+def test_ffn_bruteforce_tiny(act, seed):
+    g = np.random.default_rng(200 + seed)
+    dm, dff = int(g.integers(2, 7)), int(g.integers(2, 9))
+    x = g.standard_normal((1, dm)).astype(np.float32)
+    up = g.standard_normal((dm, dff))
+    gate = g.standard_normal((dm, dff))
+    down = g.standard_normal((dff, dm))
+    bu = g.standard_normal(dff) * 0.3
+    bg = g.standard_normal(dff) * 0.3
+    k_in = int(g.integers(0, dm + 1))
+    k_h = int(g.integers(0, dff + 1))
+    r = oracle.sparse_ffn(x, up, gate, down, act, k_in, k_h, b_up=bu, b_gate=bg)
+    kept = set(bf_keep(x[0], k_in))
+    xs = [x[0, i] if i in kept else 0.0 for i in range(dm)]
+    u = bf_matvec(xs, up.tolist())
+    gg = bf_matvec(xs, gate.tolist())
+    if act == "relu2_glu":
+        h = [max(u[j], 0.0) * max(u[j], 0.0) * gg[j] for j in range(dff)]
+    else:
+        h = [max(gg[j] + bg[j], 0.0) * max(u[j] + bu[j], 0.0) for j in range(dff)]
+    assert np.allclose(r["h"][0], h, rtol=1e-10, atol=1e-12)
+    kh = set(bf_keep(r["h"][0], k_h))
+    hs = [r["h"][0, j] if j in kh else 0.0 for j in range(dff)]
+    assert np.allclose(r["y"][0], bf_matvec(hs, down.tolist()), rtol=1e-10, atol=1e-12)
+
+
+def test_ffn_relu2_invariants():
+    w = workloads.WORKLOADS["ffn_relu2_llama7b"]
+    g = np.random.default_rng(5)
+    dm, dff = 256, 512
+    x = g.standard_normal((2, dm)).astype(np.float32)
+    up = g.standard_normal((dm, dff)) / 16
+    gate = g.standard_normal((dm, dff)) / 16
+    down = g.standard_normal((dff, dm)) / 22
+    r = oracle.sparse_ffn(x, up, gate, down, "relu2_glu", 179, 358)
+    sq = np.maximum(r["u"], 0) ** 2
+    assert np.all(sq >= 0)
+    assert np.all(r["h"][r["u"] <= 0] == 0)                 # zeros preserved
+    assert np.all(np.sign(r["h"][r["u"] > 0]) == np.sign(r["g"][r["u"] > 0]))
+    assert w.k_h == 7705 and w.k == 2867                    # floor(0.7 d)
+
+
+def test_ffn_drelu_invariants():
+    g = np.random.default_rng(6)
+    dm, dff = 128, 512
+    x = g.standard_normal((2, dm)).astype(np.float32)
+    up = g.standard_normal((dm, dff)) / math.sqrt(dm)
+    gate = g.standard_normal((dm, dff)) / math.sqrt(dm)
+    down = g.standard_normal((dff, dm)) / math.sqrt(dff)
+    b = np.full(dff, -0.8)
+    r = oracle.sparse_ffn(x, up, gate, down, "drelu", dm, 51, b_up=b, b_gate=b)
+    assert np.all(r["h"] >= 0)
+    assert np.all(r["h"][(r["u"] - 0.8 <= 0) | (r["g"] - 0.8 <= 0)] == 0)
+
+
+def test_ffn_k_full_is_dense_glu():
+    g = np.random.default_rng(8)
+    x = g.standard_normal((1, 5)).astype(np.float32)
+    up, gate, down = g.standard_normal((5, 7)), g.standard_normal((5, 7)), g.standard_normal((7, 5))
+    r = oracle.sparse_ffn(x, up, gate, down, "relu2_glu", 5, 7)
+    u = x.astype(np.float64) @ up
+    gg = x.astype(np.float64) @ gate
+    h = [max(u[0, j], 0) ** 2 * gg[0, j] for j in range(7)]
+    assert np.allclose(r["y"][0], bf_matvec(h, down.tolist()), rtol=1e-10)
+
+
+# ---------------------------------------------------------------- quantizers
+
+
+def test_absmax_quantize_golden_hand():
+    g = load_golden("quant_hand.json")
+    for c in g["act_cases"]:
+        q, gamma = oracle.absmax_quantize(np.array([c["x"]], dtype=np.float32), g["eps"])
+        assert q[0].tolist() == c["q"], c
+        if "gamma" in c:
+            assert float(gamma[0]) == c["gamma"]
+
+
+@pytest.mark.parametrize("seed", range(10))
+def test_absmax_quantize_properties(seed):
+    g = np.random.default_rng(300 + seed)
+    x = (g.standard_normal((4, 37)) * 10 ** g.uniform(-3, 3)).astype(np.float32)
+    q, gamma = oracle.absmax_quantize(x)
+    assert np.all(np.abs(q) <= 127)
+    q_neg, _ = oracle.absmax_quantize(-x)
+    assert np.array_equal(q_neg, -q)                        # symmetric
+    # q is x * 127 / (amax + eps) rounded: within 1/2 (+ float32 slack) in fp64
+    ref = x.astype(np.float64) * 127.0 / (np.abs(x).max(axis=1, keepdims=True) + 1e-5)
+    assert np.all(np.abs(q - ref) <= 0.5 + 1e-3)
+    # the largest |x| of each row lands on |q| = 127 or just under
+    am = np.argmax(np.abs(x), axis=1)
+    assert np.all(np.abs(q[np.arange(4), am]) >= 126)
+
+
+def test_ternary_quantize_golden_hand():
+    g = load_golden("quant_hand.json")
+    for c in g["ternary_cases"]:
+        t, alpha = oracle.ternary_quantize(np.array(c["w"], dtype=np.float32), g["eps"])
+        assert float(alpha) == c["alpha"]
+        assert t.tolist() == c["t"]
+
+
+def test_ternary_values_and_alpha_is_mean_abs():
+    w = workloads.weight_out_major(64, 96, 99)
+    t, alpha = oracle.ternary_quantize(w)
+    assert set(np.unique(t).tolist()) <= {-1, 0, 1}
+    eff = alpha * t.astype(np.float32)                      # weights in {-a, 0, a}
+    assert set(np.unique(np.abs(eff)).tolist()) <= {0.0, float(alpha)}
+    mean_abs = sum(abs(float(v)) for v in w.reshape(-1)) / w.size
+    assert abs(float(alpha) - mean_abs) <= 1e-7 * mean_abs
+    # round-clip: |W| >= 1.5 (alpha+eps) -> +-1 ; |W| < 0.5 (alpha+eps) -> 0
+    a = float(alpha) + 1e-5
+    assert np.all(t[np.abs(w) >= 1.5 * a] == np.sign(w[np.abs(w) >= 1.5 * a]))
+    assert np.all(t[np.abs(w) < 0.49 * a] == 0)
+
+
+def test_ternary_pack_golden_and_roundtrip():
+    g = load_golden("quant_hand.json")
+    c = g["pack_case"]
+    t = np.zeros((16, 2), dtype=np.int8)
+    t[:, 0] = c["t_col0"]
+    t[:, 1] = c["t_col1_all"]
+    p = oracle.ternary_pack(t)
+    assert p.tolist() == c["packed"]
+    assert np.array_equal(oracle.ternary_unpack(p, 16), t)
+    # brute-force bit layout on a random matrix
+    gen = np.random.default_rng(3)
+    t = gen.integers(-1, 2, size=(48, 5)).astype(np.int8)
+    p = oracle.ternary_pack(t)
+    for i, j in itertools.product(range(5), range(48)):
+        code = (int(p[i, j // 16]) >> (2 * (j % 16))) & 3
+        assert code == {0: 0, 1: 1, -1: 2}[int(t[j, i])]
+    assert np.array_equal(oracle.ternary_unpack(p, 48), t)
+
+
+def test_quant_sparse_linear_golden_hand():
+    g = load_golden("quant_hand.json")
+    c = g["linear_case"]
+    r = oracle.quant_sparse_linear(np.array([c["x"]], np.float32), np.array(c["t"]),
+                                   np.float32(c["alpha"]), c["k"])
+    assert r["keep"][0].tolist() == c["keep"]
+    assert r["acc"][0].tolist() == c["acc"]
+    assert np.allclose(r["y"][0], c["y_approx"], rtol=2e-7)
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_quant_sparse_linear_bruteforce(seed):
+    g = np.random.default_rng(400 + seed)
+    T, d_in, d_out = 2, int(g.integers(1, 10)), int(g.integers(1, 6))
+    x = g.standard_normal((T, d_in)).astype(np.float32)
+    t = g.integers(-1, 2, size=(d_out, d_in))
+    k = int(g.integers(0, d_in + 1))
+    r = oracle.quant_sparse_linear(x, t, np.float32(0.37), k)
+    for tt in range(T):
+        kept = set(bf_keep(r["q"][tt], k))              # top-K on |q|, not on |x|
+        for j in range(d_out):
+            acc = sum(int(r["q"][tt, i]) * int(t[j, i]) for i in range(d_in) if i in kept)
+            assert int(r["acc"][tt, j]) == acc
+    approx = r["acc"] * (0.37 * r["gamma"].astype(np.float64)[:, None] / 127.0)
+    assert np.allclose(r["y"], approx, rtol=1e-6, atol=1e-12)
+
+
+def test_quant_topk_on_q_ties():
+    # many equal |q| near the threshold: lower index first among equals
+    x = np.array([[0.5, -0.5, 1.0, 0.5, -0.5, 0.25]], dtype=np.float32)
+    r = oracle.quant_sparse_linear(x, np.eye(6, dtype=np.int64), np.float32(1.0), 3)
+    assert r["keep"][0].tolist() == [0, 1, 2]
+
+
+# ---------------------------------------------------------------- error measure
+
+
+def test_max_rel_err_definition():
+    ref = np.array([[1.0, -4.0, 2.0], [0.0, 0.0, 0.0]])
+    y = np.array([[1.1, -4.0, 2.0], [0.0, 0.5, 0.0]])
+    # row 0: 0.1 / 4 ; row 1 (all-zero reference): 0.5 / 1
+    assert oracle.max_rel_err(y, ref) == pytest.approx(0.5)
+    assert oracle.max_rel_err(y[:1], ref[:1]) == pytest.approx(0.025)
