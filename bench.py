@@ -1,0 +1,524 @@
+"""Benchmark: decode tokens/s and achieved HBM GB/s per sparse FFN layer.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--batch T]
+                    [--workload NAME] [--impl ours|reference]
+
+Default workload: the Llama-7B-shaped Q-Sparse FFN decode layer, bf16,
+d_model 4096 -> d_ff 11008 -> 4096, top-K keeping floor(0.7 d) of |x| and of
+|h|, h = ReLU(u)^2 * g, batch 1 token.  One step = one call of the whole layer
+(top-K on x, up/gate gather-GEMV with the gating epilogue, top-K on |h|, down
+gather-GEMV) on inputs already resident in HBM.  Steps rotate over several
+independent layers whose weights together are far larger than the 126 MB L2,
+so no step reads weights another step left in L2.
+
+Several GPUs (launched with torch.distributed.run): every rank runs its own
+replica of the layer on its own tokens (weak scaling, no data-path
+collective); the timed region is bracketed by barriers and the slowest rank's
+device time is reported.
+
+--impl reference times the CPU oracle (oracle/, fp64) on this machine's host
+cores on the same workload; it is the only other place this file runs it.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import workloads  # noqa: E402
+
+METRIC = "decode tokens/s and achieved HBM GB/s (% of B200 peak) per sparse FFN layer"
+UNIT = "tokens/s"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30000)
+    ap.add_argument("--warmup", type=int, default=300)
+    ap.add_argument("--batch", type=int, default=1, help="tokens per step (per GPU)")
+    ap.add_argument("--workload", default="ffn_relu2_llama7b",
+                    choices=["ffn_relu2_llama7b", "ffn_drelu_mistral7b"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--layers", type=int, default=0,
+                    help="independent layers to rotate over (0: enough to exceed 4x L2)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--ref-seconds", type=float, default=120.0)
+    a = ap.parse_args(argv)
+    if a.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if a.steps < 1:
+        ap.error("--steps must be >= 1")
+    return a
+
+
+# ---------------------------------------------------------------- distributed
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    return rank, world, local
+
+
+def dist_init(world: int, backend: str):
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist if world > 1 else None
+
+
+def max_over_ranks(value: float, dist, device) -> float:
+    """Slowest rank's number (all ranks get it)."""
+    if dist is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(value: float, dist, device) -> float:
+    if dist is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines: list[str] = []
+        self._t = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.gpu)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+            return
+        self._t = threading.Thread(target=self._read, daemon=True)
+        self._t.start()
+        time.sleep(0.25)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self._t is not None:
+            self._t.join(timeout=2)
+        return summarize_clocks(self.lines)
+
+
+def summarize_clocks(lines: list[str]) -> dict:
+    names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+    sm, smax, reasons = [], [], set()
+    for ln in lines:
+        parts = [p.strip() for p in ln.split(",")]
+        if len(parts) < 9:
+            continue
+        try:
+            sm.append(float(parts[1]))
+            smax.append(float(parts[2]))
+        except ValueError:
+            continue
+        for n, v in zip(names, parts[5:9]):
+            if v.lower() == "active":
+                reasons.add(n)
+    if not sm:
+        return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+    return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+            "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- peaks / profiles
+
+def load_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "source": "measured",
+                "bf16_tflops": float(d.get("bf16_tflops", 0) or 0)}
+    return {"hbm_gbs": 6650.0, "source": "fallback", "bf16_tflops": 1590.0}
+
+
+def kernel_source_digest() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for name in ("gemv.cu", "qs_internal.cuh"):
+        with open(os.path.join(ROOT, "top_activation_sparse_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str, batch: int) -> float | None:
+    """DRAM bytes per launch of the up/gate kernel from the committed ncu
+    summary, if it was taken on the current kernel source; else None."""
+    p = os.path.join(ROOT, "profiles", f"gemv_upgate_{workload}_T{batch}.md")
+    if not os.path.exists(p):
+        return None
+    vals = {}
+    with open(p) as f:
+        for ln in f:
+            if ln.startswith("- ") and ":" in ln:
+                k, v = ln[2:].split(":", 1)
+                vals[k.strip()] = v.strip().strip("`")
+    if vals.get("source_digest") != kernel_source_digest():
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+# ---------------------------------------------------------------- our arm
+
+def run_ours(args, rank, world, local):
+    import torch
+    import top_activation_sparse_b200 as qs
+    from top_activation_sparse_b200 import build as qs_build
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the library has no CPU path)")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist = dist_init(world, "nccl")
+    if rank == 0 or dist is None:
+        qs_build.build()
+    if dist is not None:
+        dist.barrier()
+    L = qs.lib()
+
+    w = workloads.WORKLOADS[args.workload]
+    T = args.batch
+    d_model, d_ff, k_in, k_h = w.d_in, w.d_out, w.k, w.k_h
+    act = qs.QS_ACT_RELU2_GLU if w.act == "relu2_glu" else qs.QS_ACT_DRELU
+    layer_bytes = 3 * d_model * d_ff * 2
+    n_layers = args.layers or max(2, math.ceil(4 * L2_BYTES / layer_bytes))
+
+    layers = [workloads.ffn_weights_device(w, l, device) for l in range(n_layers)]
+    bias = None
+    if w.bias is not None:
+        bias = torch.full((d_ff,), float(w.bias), dtype=torch.float32, device=device)
+    x = workloads.activations_device(w, T, device, salt=rank)
+    y = torch.empty(T, d_model, dtype=torch.bfloat16, device=device)
+    ws = qs.new_workspace(qs.QS_OP_SPARSE_FFN, T, d_model, d_ff, k_h, device)
+    stream = torch.cuda.current_stream(device)
+    sp = stream.cuda_stream
+    bptr = bias.data_ptr() if bias is not None else None
+
+    def c_args(l, ev_arr, kx=k_in, kh=k_h):
+        up, gate, down = layers[l]
+        return (x.data_ptr(), qs.QS_BF16, T, d_model, d_ff, act, kx, kh, up.data_ptr(),
+                gate.data_ptr(), bptr, bptr, down.data_ptr(), y.data_ptr(), None, None, ev_arr,
+                ws.data_ptr(), ws.numel(), sp)
+
+    fn = L.qs_sparse_ffn
+
+    # rows streamed per layer (algorithmic weight traffic)
+    rows = []
+    for l in range(n_layers):
+        st = fn(*c_args(l, None))
+        assert st == 0, qs.qs_status_string(st)
+        rows.append(qs.qs_workspace_stats(ws, qs.QS_OP_SPARSE_FFN, T, d_model, d_ff, k_h))
+    assert qs.qs_device_status(ws) == qs.QS_OK
+
+    # phase events on a sample of the timed steps
+    n_phase = min(args.steps, 256)
+    phase_steps = set(np.linspace(0, args.steps - 1, n_phase).astype(int).tolist())
+    phase_events = {}
+    for i in phase_steps:
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(qs.QS_FFN_PHASE_EVENTS)]
+        for e in evs:
+            e.record(stream)          # torch creates the CUDA event on first record
+        phase_events[i] = (evs, (ctypes.c_void_p * qs.QS_FFN_PHASE_EVENTS)(*[e.cuda_event for e in evs]))
+    torch.cuda.synchronize()
+    plain = [c_args(l, None) for l in range(n_layers)]
+    timed = {i: c_args(i % n_layers, phase_events[i][1]) for i in phase_steps}
+
+    def run(a):
+        st = fn(*a)
+        if st != 0:
+            raise RuntimeError(f"qs_sparse_ffn: {qs.qs_status_string(st)}")
+
+    for i in range(args.warmup):
+        run(plain[i % n_layers])
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        run(timed[i] if i in timed else plain[i % n_layers])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    clk = clocks.stop()
+    ms = t_start.elapsed_time(t_end)
+    assert qs.qs_device_status(ws) == qs.QS_OK
+    ms_max = max_over_ranks(ms, dist, device)
+    tokens = sum_over_ranks(float(T * args.steps), dist, device)
+    value = tokens / (ms_max / 1e3)
+
+    # per-phase device time on the sampled steps
+    ph = np.array([[phase_events[i][0][p].elapsed_time(phase_events[i][0][p + 1])
+                    for p in range(4)] for i in sorted(phase_steps)])
+    ph_us = ph.mean(axis=0) * 1e3
+    upgate_us = float(ph_us[1])
+
+    # algorithmic bytes of the dominant kernel (up/gate gather-GEMV) per launch:
+    # kept rows of W_up^T and W_gate^T + the kept (index, T values) entries it
+    # stages + h written (f32).
+    rows_x = float(np.mean([r[0] for r in rows]))
+    rows_h = float(np.mean([r[1] for r in rows]))
+    upgate_bytes = rows_x * d_ff * 2 * 2 + rows_x * (4 + 4 * T) + T * d_ff * 4
+    down_bytes = rows_h * d_model * 2 + rows_h * (4 + 4 * T) + T * d_model * 2
+    topk_bytes = T * d_model * 2 + T * d_ff * 4
+    layer_alg_bytes = upgate_bytes + down_bytes + topk_bytes
+    peaks = load_peaks()
+    achieved = upgate_bytes / (upgate_us * 1e-6) / 1e9
+    layer_gbs = layer_alg_bytes * T * args.steps / T / (ms / 1e3) / 1e9
+
+    # dense run of the same kernels (K = d): context for the sparsity win
+    for i in range(args.warmup):
+        run(c_args(i % n_layers, None, d_model, d_ff))
+    n_dense = max(1, min(args.steps, 2000))
+    torch.cuda.synchronize()
+    d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dense_args = [c_args(l, None, d_model, d_ff) for l in range(n_layers)]
+    d0.record(stream)
+    for i in range(n_dense):
+        run(dense_args[i % n_layers])
+    d1.record(stream)
+    torch.cuda.synchronize()
+    dense_ms = d0.elapsed_time(d1) / n_dense
+
+    # end to end through the public Python API with host buffers
+    x_host = x.cpu().pin_memory()
+    y_host = torch.empty(T, d_model, dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty_like(x)
+    n_e2e = max(1, min(args.steps, 5000))
+    lw = [layers[l] for l in range(n_layers)]
+    for i in range(args.warmup):
+        x_dev.copy_(x_host, non_blocking=True)
+        up, gate, down = lw[i % n_layers]
+        qs.qs_sparse_ffn(x_dev, up, gate, down, w.act, k_in, k_h, b_up=bias, b_gate=bias, y=y, ws=ws)
+        y_host.copy_(y, non_blocking=True)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(n_e2e):
+        x_dev.copy_(x_host, non_blocking=True)
+        up, gate, down = lw[i % n_layers]
+        qs.qs_sparse_ffn(x_dev, up, gate, down, w.act, k_in, k_h, b_up=bias, b_gate=bias, y=y, ws=ws)
+        y_host.copy_(y, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e_ms = max_over_ranks(e0.elapsed_time(e1), dist, device)
+    e_tokens = sum_over_ranks(float(T * n_e2e), dist, device)
+    e2e_value = e_tokens / (e_ms / 1e3)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        up, gate, down = (t.float().cpu().numpy() for t in layers[0])
+        cpu = cpu_oracle_rate(w, x.float().cpu().numpy(), up, gate, down, args.cpu_seconds)
+
+    traffic = profiled_traffic(args.workload, T)
+    result = {
+        "metric": METRIC,
+        "value": round(value, 1),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_max / args.steps, 6),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic: x ~ N(0,1), W ~ N(0,1/fan_in) (seeded; random-init weights)",
+        "config": {
+            "workload": f"{args.workload}: Q-Sparse FFN decode layer, d_model={d_model}, "
+                        f"d_ff={d_ff}, act={w.act}, K_x={k_in}, K_h={k_h}, bf16",
+            "batch_per_gpu": T,
+            "global_batch": T * world,
+            "layers_rotated": n_layers,
+            "l2": f"inputs larger than L2: {n_layers} independent layers "
+                  f"({n_layers * layer_bytes / 1e9:.2f} GB of weights) rotated per step",
+            "parallelism": f"replicas x{world} (no data-path collective)",
+        },
+        "hbm": {
+            "layer_gbs": round(layer_gbs, 1),
+            "layer_alg_bytes": int(layer_alg_bytes),
+            "frac_of_peak": round(layer_gbs / peaks["hbm_gbs"], 4),
+            "rows_streamed": {"x": rows_x, "h": rows_h},
+        },
+        "phases_us": {"topk_x": round(float(ph_us[0]), 3), "upgate": round(float(ph_us[1]), 3),
+                      "topk_h": round(float(ph_us[2]), 3), "down": round(float(ph_us[3]), 3)},
+        "roofline": {
+            "kernel": "gemv_kernel (up/gate gather-GEMV + gating epilogue)",
+            "bound": "hbm",
+            "achieved": round(achieved, 1),
+            "peak": peaks["hbm_gbs"],
+            "peak_source": peaks["source"],
+            "unit": "GB/s",
+            "frac": round(achieved / peaks["hbm_gbs"], 4),
+            "traffic": traffic,
+            "alg_bytes_per_launch": int(upgate_bytes),
+        },
+        "dense_same_kernels": {"ms_per_step": round(dense_ms, 6),
+                               "value": round(T / (dense_ms / 1e3), 1), "k_x": d_model,
+                               "k_h": d_ff},
+        "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "steps": n_e2e,
+                "h2d_bytes_per_step": int(x.numel() * x.element_size()),
+                "d2h_bytes_per_step": int(y.numel() * y.element_size())},
+        "gpu_launches": 4 * ((T + qs.QS_PREFILL_MIN_T - 1) // qs.QS_PREFILL_MIN_T) * args.steps,
+        "clocks": clk,
+    }
+    if cpu is not None:
+        result["cpu_baseline"] = cpu
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return result if rank == 0 else None
+
+
+# ---------------------------------------------------------------- oracle arms
+
+def _threads_in_use() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return int(max(n)) if n else 1
+    except Exception:
+        return 1
+
+
+def cpu_oracle_rate(w, x, up, gate, down, seconds: float) -> dict:
+    """Time the oracle as it stands on a bounded sample: whole-layer calls
+    for about `seconds` of host time (at least two)."""
+    import oracle
+    T = x.shape[0]
+    b = None if w.bias is None else np.full(w.d_out, w.bias)
+    n = 0
+    t0 = time.perf_counter()
+    while n < 2 or time.perf_counter() - t0 < seconds:
+        oracle.sparse_ffn(x, up, gate, down, w.act, w.k, w.k_h, b_up=b, b_gate=b)
+        n += 1
+    dt = time.perf_counter() - t0
+    return {"value": round(n * T / dt, 3), "unit": UNIT, "cores": _threads_in_use(),
+            "kind": "oracle",
+            "sample": f"{n} whole-layer oracle calls of {T} token(s) each, {dt:.1f} s, fp64 numpy"}
+
+
+def run_reference(args, rank, world, local):
+    """The oracle as the reference arm: rank 0 only, host cores only."""
+    if rank != 0:
+        return None
+    w = workloads.WORKLOADS[args.workload]
+    T = args.batch
+    x = workloads.activations(w, T)
+    up, gate, down = workloads.ffn_weights(w)
+    import oracle
+    b = None if w.bias is None else np.full(w.d_out, w.bias)
+
+    def step():
+        oracle.sparse_ffn(x, up, gate, down, w.act, w.k, w.k_h, b_up=b, b_gate=b)
+
+    t0 = time.perf_counter()
+    step()
+    one = time.perf_counter() - t0
+    budget = args.ref_seconds
+    warm = max(0, min(args.warmup, int(0.2 * budget / max(one, 1e-9))))
+    for _ in range(warm):
+        step()
+    n_run = max(1, min(args.steps, int(budget / max(one, 1e-9))))
+    t0 = time.perf_counter()
+    for _ in range(n_run):
+        step()
+    dt = time.perf_counter() - t0
+    value = n_run * T / dt
+    sample = (f"{n_run} of {args.steps} steps run (each the whole layer for {T} token(s)); "
+              f"{warm} warm-up; fp64 numpy oracle")
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": round(value, 3),
+        "unit": UNIT,
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(dt / n_run * 1e3, 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic: x ~ N(0,1), W ~ N(0,1/fan_in) (seeded)",
+        "config": {"workload": f"{args.workload} (same layer as --impl ours), CPU oracle",
+                   "batch_per_gpu": T, "global_batch": T, "parallelism": "host cores"},
+        "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": _threads_in_use(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        out = run_reference(args, rank, world, local)
+    else:
+        out = run_ours(args, rank, world, local)
+    if out is not None:
+        print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

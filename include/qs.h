@@ -1,0 +1,234 @@
+/*
+ * qs.h -- C ABI of the B200 (sm_100a) Q-Sparse top-K sparse projection library.
+ *
+ * What the library computes (sources are the pages this project follows):
+ *
+ *   Q-Sparse news article (zxwl-tech.com), section "Top-K sparsification"
+ *   (用Top-K函數實現稀疏化): every linear projection Y = X.W^T takes a
+ *   sparsified input.  For each token row x, |x| is ranked, the K largest
+ *   entries are kept (K preset), a 0/1 mask M of x's shape marks them, and
+ *   X_sparse = X (.) M replaces X in the matmul.  Because most of X_sparse is
+ *   zero, only the weight rows of the kept inputs have to be read.
+ *
+ * Conventions shared by every entry point
+ *
+ *   Layout.   Activations are row-major [T, d] (T token rows).  Weights are
+ *             given INPUT-MAJOR: wt = W^T, row-major [d_in, d_out], so that the
+ *             weights of one input feature i are the contiguous row wt[i, :].
+ *   Pointers. Every tensor pointer is a CUDA DEVICE pointer owned by the
+ *             caller, 16-byte aligned.  The library never allocates or frees
+ *             memory and keeps no state between calls; all scratch lives in
+ *             the caller's workspace `ws`.
+ *   Streams.  `stream` is a cudaStream_t passed as void* (NULL = the legacy
+ *             default stream).  Every call only enqueues work on that stream
+ *             and returns; nothing synchronises the host except
+ *             qs_device_status() and qs_workspace_stats().
+ *   Workspace. `ws` must hold at least qs_workspace_size(op, ...) bytes, be
+ *             16-byte aligned and be ZERO-FILLED before its first use
+ *             (qs_workspace_init does this).  Each call leaves its internal
+ *             counters at zero again when its kernels finish, so a workspace is
+ *             reused without clearing.  Calls that share one workspace must be
+ *             ordered (same stream, or event-ordered): overlapping them races.
+ *   Errors.   Argument errors are detected on the host, before anything is
+ *             enqueued, and returned as a qs_status; a failed launch returns
+ *             QS_ERR_CUDA.  Conditions only the device can see (a bounded wait
+ *             that gave up, an internal check) are recorded in the workspace's
+ *             status word and reported by qs_device_status().  No kernel traps.
+ *   Ties.     "The K largest |x|" is a total order: larger |x| first, equal |x|
+ *             -> lower index first; -0.0 and +0.0 are the same magnitude.  The
+ *             mask always has exactly K ones per row, even when fewer than K
+ *             entries are nonzero.  Inputs must be finite (NaN ranks above inf).
+ *   Numerics. Products accumulate in fp32 (int32 for the int8 x ternary path);
+ *             a bf16 output is rounded once, to nearest-even, at the end.
+ */
+#ifndef QS_H
+#define QS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum qs_status {
+  QS_OK = 0,
+  QS_ERR_INVALID_ARG = 1,   /* bad size, k, enum value, or a required pointer is NULL */
+  QS_ERR_ALIGNMENT = 2,     /* pointer not 16-byte aligned, or d_out not a multiple of the
+                               16-byte vector width (4 for f32, 8 for bf16, 16 packed) */
+  QS_ERR_WORKSPACE = 3,     /* ws NULL or smaller than qs_workspace_size() */
+  QS_ERR_CUDA = 4,          /* a CUDA runtime call or kernel launch failed */
+  QS_ERR_TIMEOUT = 5,       /* device: a bounded wait ran out (see qs_device_status) */
+  QS_ERR_DEVICE_CHECK = 6,  /* device: an internal consistency check failed */
+  QS_ERR_UNSUPPORTED = 7    /* arguments valid but outside what this build handles
+                               (e.g. d above QS_MAX_ROW) */
+} qs_status;
+
+typedef enum qs_dtype { QS_F32 = 0, QS_BF16 = 1 } qs_dtype;
+
+typedef enum qs_act {
+  QS_ACT_RELU2_GLU = 0,   /* h = ReLU(u)^2 * g           (Q-Sparse squared-ReLU FFN) */
+  QS_ACT_DRELU = 1        /* h = ReLU(g + b_gate) * ReLU(u + b_up)   (Turbo Sparse dReLU) */
+} qs_act;
+
+typedef enum qs_op {
+  QS_OP_TOPK_MASK = 0,
+  QS_OP_SPARSE_LINEAR = 1,
+  QS_OP_SPARSE_FFN = 2,
+  QS_OP_QUANT_SPARSE_LINEAR = 3,
+  QS_OP_TERNARY_PACK = 4
+} qs_op;
+
+/* Largest row length (d, d_in, d_ff) a top-K row may have: one CTA holds a
+ * row's keys in shared memory. */
+#define QS_MAX_ROW 49152
+/* From this many tokens on, qs_sparse_linear on bf16 runs the masked-dense
+ * tensor-core GEMM instead of the gather-GEMV. */
+#define QS_PREFILL_MIN_T 64
+/* Number of cudaEvent_t handles qs_sparse_ffn records when given phase events. */
+#define QS_FFN_PHASE_EVENTS 5
+
+/*
+ * qs_topk_mask -- top-K on |x| per row, with the mask and the sparsified input.
+ *   Source: Q-Sparse news article, section "Top-K sparsification" (rank |X|,
+ *   keep the K largest, binary mask M, X_sparse = X (.) M).
+ *
+ *   x     [T, d] in `dtype` (QS_F32 or QS_BF16), device.
+ *   k     0 <= k <= d.  k = d keeps every entry, k = 0 none.
+ *   idx   [T, k] int32 out: kept indices of each row, ascending.  Required if k > 0.
+ *   val   [T, k] `dtype` out or NULL: x at idx (the compacted value list).
+ *   mask  [T, d] uint8 out or NULL: 1 at kept positions, 0 elsewhere.
+ *   xs    [T, d] `dtype` out or NULL: X_sparse = x * mask (+0.0 where dropped).
+ *   ws    workspace of qs_workspace_size(QS_OP_TOPK_MASK, T, d, 0, k) bytes.
+ *   Errors: INVALID_ARG (T < 1, d < 1, k outside [0, d], NULL x/idx, bad dtype),
+ *   ALIGNMENT, WORKSPACE, UNSUPPORTED (d > QS_MAX_ROW), CUDA.
+ */
+qs_status qs_topk_mask(const void* x, int dtype, int T, int d, int k,
+                       int32_t* idx, void* val, uint8_t* mask, void* xs,
+                       void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * qs_sparse_linear -- Y = (X (.) M) . W^T with M the top-K mask of |X|.
+ *   Source: Q-Sparse news article, section "Top-K sparsification" (X_sparse
+ *   replaces X in the projection; zeros cut compute and memory traffic), and
+ *   the aibase.com summary, "Vantagens da ativacao esparsa" (I/O is the
+ *   bottleneck of inference, so only the kept inputs' weights are read).
+ *
+ *   x     [T, d_in] `dtype`.       wt  [d_in, d_out] `dtype` (= W^T).
+ *   y     [T, d_out] `dtype` out.  k   0 <= k <= d_in (k = d_in: dense layer).
+ *   Decode (T < QS_PREFILL_MIN_T, or f32): a gather-GEMV streams only the rows
+ *   wt[i, :] of inputs kept by some token.  Prefill (bf16, T >= QS_PREFILL_MIN_T):
+ *   X_sparse is materialised and multiplied on the tensor cores (tcgen05).
+ *   d_out must be a multiple of 8 (bf16) or 4 (f32).
+ *   Errors: INVALID_ARG, ALIGNMENT, WORKSPACE, UNSUPPORTED, CUDA.
+ */
+qs_status qs_sparse_linear(const void* x, int dtype, int T, int d_in, int d_out, int k,
+                           const void* wt, void* y, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * qs_sparse_ffn -- one sparse gated FFN layer.
+ *   x_s = topK(x, k_in);  u = x_s.W_up^T;  g = x_s.W_gate^T;
+ *   h   = act(u, g);      h_s = topK(h, k_h);   y = h_s.W_down^T.
+ *   Sources: Q-Sparse news article, Top-K section, feed-forward paragraph
+ *   (squared ReLU combined by a Hadamard product); aibase.com summary (top-K
+ *   on every linear projection); Turbo Sparse summary (blog.csdn.net), Eq. 2
+ *   (dReLU) and Eq. 3-4 (top k% of |h| by absolute value before W_down).
+ *
+ *   x         [T, d_model] `dtype` (bf16 or f32).
+ *   act       QS_ACT_RELU2_GLU or QS_ACT_DRELU.
+ *   k_in      0..d_model  (d_model = dense input).   k_h  0..d_ff.
+ *   wt_up, wt_gate  [d_model, d_ff] `dtype`.   wt_down [d_ff, d_model] `dtype`.
+ *   b_up, b_gate    [d_ff] f32 or NULL (= 0); added to u and g before the ReLUs
+ *                   of QS_ACT_DRELU; ignored by QS_ACT_RELU2_GLU.
+ *   y         [T, d_model] `dtype` out.
+ *   h_out     [T, d_ff] f32 out or NULL: h before its top-K.
+ *   idx_h_out [T, k_h] int32 out or NULL: indices kept by the top-K on |h|.
+ *   phase_events  NULL, or QS_FFN_PHASE_EVENTS cudaEvent_t handles (as void*)
+ *             recorded on `stream` before the first kernel and after the input
+ *             top-K, the up/gate projection, the top-K on |h| and the down
+ *             projection (for per-phase timing; recording them costs a little).
+ *   ws        qs_workspace_size(QS_OP_SPARSE_FFN, T, d_model, d_ff, k_h) bytes.
+ *   d_model and d_ff must be multiples of 8 (bf16) or 4 (f32).
+ *   Errors: INVALID_ARG, ALIGNMENT, WORKSPACE, UNSUPPORTED, CUDA.
+ */
+qs_status qs_sparse_ffn(const void* x, int dtype, int T, int d_model, int d_ff, int act,
+                        int k_in, int k_h, const void* wt_up, const void* wt_gate,
+                        const float* b_up, const float* b_gate, const void* wt_down,
+                        void* y, float* h_out, int32_t* idx_h_out,
+                        void* const* phase_events,
+                        void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * qs_quant_sparse_linear -- BitNet b1.58 + Q-Sparse projection.
+ *   Source: Q-Sparse news article, Top-K section, quantized-model paragraphs
+ *   (inputs are quantized before top-K, with an epsilon guarding a division;
+ *   1-bit weights scaled by alpha = mean|W|).  The lost formulas are read as:
+ *     gamma_t = max_j |x_tj| + eps;  s_t = 127 / gamma_t;
+ *     q_tj    = clamp(rint(x_tj * s_t), -127, 127)          (float32 steps)
+ *     keep    = topK(|q_t|, k)  (ties -> lower index)
+ *     acc_tj  = sum_{i in keep} q_ti * t_ij                  (exact int32)
+ *     y_tj    = float(acc_tj) * ((alpha * gamma_t) / 127)    (float32 steps)
+ *
+ *   x          [T, d_in] `dtype` (bf16 or f32).
+ *   wt_packed  [d_in, d_out/16] uint32: ternary W^T from qs_ternary_pack.
+ *   alpha      the weight scale qs_ternary_pack returned.   eps  e.g. 1e-5.
+ *   y          [T, d_out] f32 out.
+ *   acc        [T, d_out] int32 out or NULL.   q  [T, d_in] int8 out or NULL.
+ *   idx        [T, k] int32 out or NULL: kept indices, ascending.
+ *   d_out must be a multiple of 16; 127 * d_in < 2^24 keeps float(acc) exact.
+ *   Errors: INVALID_ARG, ALIGNMENT, WORKSPACE, UNSUPPORTED, CUDA.
+ */
+qs_status qs_quant_sparse_linear(const void* x, int dtype, int T, int d_in, int d_out, int k,
+                                 const uint32_t* wt_packed, float alpha, float eps,
+                                 float* y, int32_t* acc, int8_t* q, int32_t* idx,
+                                 void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * qs_ternary_pack -- ternary weight quantizer and 2-bit packing (offline step).
+ *   Source: Q-Sparse news article, quantized-model paragraph (alpha is the
+ *   mean absolute value of W).  Read as:
+ *     alpha = float(sum |W| in fp64 / (d_out * d_in));
+ *     t     = clamp(rint(W / (alpha + eps)), -1, 1)   (float32 division)
+ *   Packing: word [i, j/16] of the output holds t[j, i] at bits 2*(j%16),
+ *   code 00 = 0, 01 = +1, 10 = -1.
+ *
+ *   w          [d_out, d_in] f32 (output-major, as nn.Linear stores it).
+ *   wt_packed  [d_in, d_out/16] uint32 out.    alpha_out  1 f32 out (device).
+ *   d_out must be a multiple of 16.
+ *   Errors: INVALID_ARG, ALIGNMENT, WORKSPACE, CUDA.
+ */
+qs_status qs_ternary_pack(const float* w, int d_out, int d_in, float eps,
+                          uint32_t* wt_packed, float* alpha_out,
+                          void* ws, size_t ws_bytes, void* stream);
+
+/* Bytes of workspace `op` needs for these sizes (0 if the sizes are invalid).
+ * Arguments: QS_OP_TOPK_MASK (T, d, 0, k); QS_OP_SPARSE_LINEAR (T, d_in, d_out,
+ * k); QS_OP_SPARSE_FFN (T, d_model, d_ff, k_h); QS_OP_QUANT_SPARSE_LINEAR
+ * (T, d_in, d_out, k); QS_OP_TERNARY_PACK (0, d_in, d_out, 0).  The dtype does
+ * not change the size. */
+size_t qs_workspace_size(int op, int T, int d_in, int d_out, int k);
+
+/* Zero-fill `ws_bytes` of workspace on `stream` (enqueued, not synchronous). */
+qs_status qs_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronise `stream`, read and clear the workspace's device status word.
+ * Returns QS_OK, QS_ERR_TIMEOUT or QS_ERR_DEVICE_CHECK (or QS_ERR_CUDA). */
+qs_status qs_device_status(void* ws, void* stream);
+
+/* Synchronise `stream` and report, for the last call of `op` made with this
+ * workspace and these sizes, how many weight rows its projections streamed:
+ * rows[0] = distinct inputs with a kept nonzero value across the T tokens (the
+ * rows of wt / wt_up / wt_gate read), rows[1] = the same for h (rows of
+ * wt_down read; QS_OP_SPARSE_FFN only, else 0).  These counts are the
+ * algorithmic weight traffic: rows * d_out * sizeof(weight). */
+qs_status qs_workspace_stats(const void* ws, int op, int T, int d_in, int d_out, int k,
+                             int32_t* rows, void* stream);
+
+/* Human-readable name of a status code (static string). */
+const char* qs_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QS_H */

@@ -223,7 +223,7 @@ def ternary_pack(t) -> np.ndarray:
     code[t == -1] = 2
     ct = code.T.reshape(d_in, d_out // 16, 16)
     shifts = (2 * np.arange(16)).astype(np.uint32)
-    return np.bitwise_or.reduce(ct << shifts, axis=2).astype(np.uint32)
+    return np.ascontiguousarray(np.bitwise_or.reduce(ct << shifts, axis=2), dtype=np.uint32)
 
 
 def ternary_unpack(packed, d_out: int) -> np.ndarray:

@@ -1,0 +1,106 @@
+"""qs_sparse_ffn on the GPU against the fp64 oracle.
+
+h is computed on the GPU in f32 and on the oracle in fp64, so the top-K on
+|h| may pick a different element where two magnitudes sit within rounding of
+the threshold.  The checks therefore are: (1) h within the f32 tolerance;
+(2) the GPU's kept set is a valid top-K of the oracle's h up to
+eps_sel = 4 * TOL_F32 * max|h_t|; (3) y against the oracle re-run on the
+GPU's own selection of h (the input top-K, of given data, is bit-exact and
+checked through the row count)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import top_activation_sparse_b200 as qs
+import workloads
+from gpu_common import TOL_BF16, TOL_F32, check_status, need_gpu, to_dev, to_np
+
+pytestmark = pytest.mark.gpu
+
+_weights = {}
+
+
+def _ffn_weights(name):
+    if name not in _weights:
+        w = workloads.WORKLOADS[name]
+        _weights[name] = workloads.ffn_weights(w)
+    return _weights[name]
+
+
+def _check_ffn(x, up, gate, down, act, k_in, k_h, dtype, bias=None):
+    T, d_model = x.shape
+    d_ff = up.shape[1]
+    xt = to_dev(x, dtype)
+    upt, gatet, downt = to_dev(up, dtype), to_dev(gate, dtype), to_dev(down, dtype)
+    b = None if bias is None else torch.full((d_ff,), bias, dtype=torch.float32, device="cuda")
+    ws = qs.new_workspace(qs.QS_OP_SPARSE_FFN, T, d_model, d_ff, k_h, xt.device)
+    r = qs.qs_sparse_ffn(xt, upt, gatet, downt, act, k_in, k_h, b_up=b, b_gate=b,
+                         h_out=True, idx_h_out=True, ws=ws)
+    check_status(ws)
+    bnp = None if bias is None else np.full(d_ff, bias)
+    ref = oracle.sparse_ffn(x, up, gate, down, act, k_in, k_h, b_up=bnp, b_gate=bnp)
+    h_gpu = r.h.cpu().numpy()
+    assert oracle.max_rel_err(h_gpu, ref["h"]) <= TOL_F32
+    idx_h = r.idx_h.cpu().numpy().astype(np.int64)
+    swaps = 0
+    for t in range(T):
+        assert np.all(np.diff(idx_h[t]) > 0)
+        kept = np.zeros(d_ff, bool)
+        kept[idx_h[t]] = True
+        mag = np.abs(ref["h"][t])
+        eps_sel = 4 * TOL_F32 * mag.max()
+        if 0 < k_h < d_ff:
+            assert mag[kept].min() >= mag[~kept].max() - eps_sel
+        swaps += k_h - np.intersect1d(idx_h[t], ref["keep_h"][t]).size
+    ref_sel = oracle.sparse_ffn(x, up, gate, down, act, k_in, k_h, b_up=bnp, b_gate=bnp,
+                                keep_h=idx_h)
+    tol = TOL_F32 if dtype == "f32" else TOL_BF16
+    err = oracle.max_rel_err(to_np(r.y), ref_sel["y"])
+    assert err <= tol, err
+    # the row counts describe the last chunk of (at most 64) tokens
+    rows_x, rows_h = qs.qs_workspace_stats(ws, qs.QS_OP_SPARSE_FFN, T, d_model, d_ff, k_h)
+    t0 = ((T - 1) // qs.QS_PREFILL_MIN_T) * qs.QS_PREFILL_MIN_T
+    kx = ref["keep_x"][t0:]
+    assert rows_x == np.unique(kx[np.take_along_axis(x[t0:], kx, 1) != 0]).size
+    assert rows_h == np.unique(np.concatenate(
+        [idx_h[t][h_gpu[t, idx_h[t]] != 0] for t in range(t0, T)] + [np.zeros(0, np.int64)])).size
+    return swaps, ref
+
+
+@pytest.mark.parametrize("T", [1, 8])
+def test_ffn_relu2_llama7b(T):
+    """Llama-7B FFN decode, bf16: K = 0.7 d on x and on |h|, squared-ReLU gating."""
+    need_gpu()
+    w = workloads.WORKLOADS["ffn_relu2_llama7b"]
+    up, gate, down = _ffn_weights(w.name)
+    x = workloads.activations(w, T)
+    swaps, ref = _check_ffn(x, up, gate, down, "relu2_glu", w.k, w.k_h, "bf16")
+    assert swaps <= 2 * T
+
+
+@pytest.mark.parametrize("T", [1, 4])
+def test_ffn_drelu_mistral7b(T):
+    """Mistral-7B dReLU FFN decode, bf16: dense x, biases -0.8, keep top 10% of |h|."""
+    need_gpu()
+    w = workloads.WORKLOADS["ffn_drelu_mistral7b"]
+    up, gate, down = _ffn_weights(w.name)
+    x = workloads.activations(w, T)
+    swaps, ref = _check_ffn(x, up, gate, down, "drelu", w.k, w.k_h, "bf16", bias=w.bias)
+    assert swaps <= 2 * T
+    assert np.all(ref["h"] >= 0)
+
+
+@pytest.mark.parametrize("act", ["relu2_glu", "drelu"])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("T,dm,dff", [(1, 64, 96), (3, 200, 328), (9, 128, 256), (66, 64, 64)])
+def test_ffn_small_and_ragged(act, dtype, T, dm, dff):
+    need_gpu()
+    g = workloads.rng(T * 1000 + dm + dff)
+    x = workloads.round_to_dtype(workloads.normal_f32(g, (T, dm)), dtype)
+    up = workloads.round_to_dtype(workloads.normal_f32(g, (dm, dff), dm ** -0.5), dtype)
+    gate = workloads.round_to_dtype(workloads.normal_f32(g, (dm, dff), dm ** -0.5), dtype)
+    down = workloads.round_to_dtype(workloads.normal_f32(g, (dff, dm), dff ** -0.5), dtype)
+    bias = -0.3 if act == "drelu" else None
+    for k_in, k_h in ((dm, dff), ((7 * dm) // 10, (7 * dff) // 10), (1, 1), (dm, 0)):
+        _check_ffn(x, up, gate, down, act, k_in, k_h, dtype, bias=bias)

@@ -1,0 +1,490 @@
+// extern "C" entry points of include/qs.h: argument checks, the workspace
+// layout, and the order in which the kernels are enqueued.  Every step of the
+// computation runs in this library's CUDA kernels; there is no host fallback.
+#include <cstring>
+
+#include "qs_internal.cuh"
+
+namespace qs {
+namespace {
+
+// Token rows are processed in chunks of at most this many (decode kernels
+// keep one accumulator per token in registers; see plan_gemv).
+constexpr int kChunkT = QS_PREFILL_MIN_T;
+constexpr size_t kTicketBytes = 64 * 1024;       // fixed ticket region
+constexpr int kTicketCap = (int)(kTicketBytes / sizeof(int32_t));
+// fixed ticket slots
+constexpr int kTkTopkX = 0, kTkTopkH = 1, kTkAlpha = 2, kTkGemv = 8;
+
+size_t align_up(size_t v) { return (v + kWsAlign - 1) / kWsAlign * kWsAlign; }
+
+bool aligned16(const void* p) { return p == nullptr || ((uintptr_t)p & 15u) == 0; }
+
+int elem_bytes(int dtype) { return dtype == QS_F32 ? 4 : 2; }
+
+long rows_bound(int T, int d, int k) {
+  const long tk = (long)T * (long)k;
+  return tk < d ? tk : d;
+}
+
+}  // namespace
+
+// Same layout for every dtype: each buffer is sized for the larger of the
+// f32 and bf16 plans.  The status word and the ticket counters sit at fixed
+// offsets, so a zeroed workspace stays valid across ops and sizes.
+bool ws_layout(int op, int T, int d_in, int d_out, int k, WsLayout* L) {
+  *L = WsLayout{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + (bytes ? bytes : 1));
+    return o;
+  };
+  L->status = take(sizeof(DevStatus));
+  L->tickets = take(kTicketBytes);
+  L->n_tickets = kTicketCap;
+  L->cnt = take(4 * sizeof(int32_t));
+  L->ticket_topk_x = kTkTopkX;
+  L->ticket_topk_h = kTkTopkH;
+  L->ticket_alpha = kTkAlpha;
+  const int Tc = T < kChunkT ? T : kChunkT;
+  // Partial-sum buffers are sized for the largest plan any chunk (1..Tc
+  // tokens) of either dtype can pick: a short last chunk may split more.
+  auto max_parts = [&](int d_out_, int d_rows, int kk, int mats) {
+    size_t m = 0;
+    for (int t = 1; t <= Tc; ++t) {
+      const int rb = (int)rows_bound(t, d_rows, kk);
+      for (int eb = 2; eb <= 4; eb += 2) {
+        const GemvPlan p = plan_gemv(t, d_out_, rb, mats, eb);
+        if (p.parts_elems > m) m = p.parts_elems;
+      }
+    }
+    return m;
+  };
+  auto max_qparts = [&](int d_out_, int d_rows, int kk) {
+    size_t m = 0;
+    for (int t = 1; t <= Tc; ++t) {
+      const GemvPlan p = plan_qgemv(t, d_out_, (int)rows_bound(t, d_rows, kk));
+      if (p.parts_elems > m) m = p.parts_elems;
+    }
+    return m;
+  };
+  switch (op) {
+    case QS_OP_TOPK_MASK:
+      if (T < 1 || d_in < 1 || d_in > QS_MAX_ROW || k < 0 || k > d_in) return false;
+      break;
+    case QS_OP_SPARSE_LINEAR: {
+      if (T < 1 || d_in < 1 || d_out < 1 || d_in > QS_MAX_ROW || d_out > QS_MAX_ROW || k < 0 ||
+          k > d_in)
+        return false;
+      L->xsf_x = take((size_t)Tc * d_in * sizeof(float));
+      L->list_x = take((size_t)d_in * sizeof(int32_t));
+      L->lval_x = take((size_t)d_in * Tc * sizeof(float));
+      L->parts1_elems = max_parts(d_out, d_in, k, 1);
+      L->parts1 = take(L->parts1_elems * sizeof(float));
+      if (T >= kChunkT) L->xs_bf16 = take((size_t)T * d_in * sizeof(uint16_t));
+      break;
+    }
+    case QS_OP_SPARSE_FFN: {
+      if (T < 1 || d_in < 1 || d_out < 1 || d_in > QS_MAX_ROW || d_out > QS_MAX_ROW || k < 0 ||
+          k > d_out)
+        return false;
+      L->xsf_x = take((size_t)Tc * d_in * sizeof(float));
+      L->list_x = take((size_t)d_in * sizeof(int32_t));
+      L->lval_x = take((size_t)d_in * Tc * sizeof(float));
+      L->parts1_elems = max_parts(d_out, d_in, d_in, 2);
+      L->parts1 = take(L->parts1_elems * sizeof(float));
+      L->h = take((size_t)Tc * d_out * sizeof(float));
+      L->xsf_h = take((size_t)Tc * d_out * sizeof(float));
+      L->list_h = take((size_t)d_out * sizeof(int32_t));
+      L->lval_h = take((size_t)d_out * Tc * sizeof(float));
+      L->parts2_elems = max_parts(d_in, d_out, k, 1);
+      L->parts2 = take(L->parts2_elems * sizeof(float));
+      break;
+    }
+    case QS_OP_QUANT_SPARSE_LINEAR: {
+      if (T < 1 || d_in < 1 || d_out < 16 || d_in > QS_MAX_ROW || d_out > QS_MAX_ROW || k < 0 ||
+          k > d_in || (d_out % 16) != 0)
+        return false;
+      L->xq = take((size_t)Tc * d_in);
+      L->gamma = take((size_t)Tc * sizeof(float));
+      L->list_x = take((size_t)d_in * sizeof(int32_t));
+      L->lval_x = take((size_t)d_in * Tc);
+      L->parts1_elems = max_qparts(d_out, d_in, k);
+      L->parts1 = take(L->parts1_elems * sizeof(int32_t));
+      break;
+    }
+    case QS_OP_TERNARY_PACK:
+      if (d_in < 1 || d_out < 16 || (d_out % 16) != 0) return false;
+      L->alpha_parts = take(kPackSumBlocks * sizeof(double));
+      L->alpha = take(sizeof(float));
+      break;
+    default:
+      return false;
+  }
+  L->total = off;
+  return true;
+}
+
+}  // namespace qs
+
+using namespace qs;
+
+namespace {
+
+struct WsView {
+  unsigned char* base;
+  DevStatus* status() const { return reinterpret_cast<DevStatus*>(base); }
+  int32_t* ticket(const WsLayout& L, int slot) const {
+    return reinterpret_cast<int32_t*>(base + L.tickets) + slot;
+  }
+  template <typename T> T* at(size_t off) const { return reinterpret_cast<T*>(base + off); }
+};
+
+qs_status from_cuda(cudaError_t e) { return e == cudaSuccess ? QS_OK : QS_ERR_CUDA; }
+
+#define QS_TRY_CUDA(expr)                         \
+  do {                                            \
+    cudaError_t _e = (expr);                      \
+    if (_e != cudaSuccess) return QS_ERR_CUDA;    \
+  } while (0)
+
+qs_status check_ws(int op, int T, int d_in, int d_out, int k, void* ws, size_t ws_bytes,
+                   WsLayout* L) {
+  if (!ws_layout(op, T, d_in, d_out, k, L)) return QS_ERR_INVALID_ARG;
+  if (ws == nullptr || ws_bytes < L->total) return QS_ERR_WORKSPACE;
+  if (!aligned16(ws)) return QS_ERR_ALIGNMENT;
+  return QS_OK;
+}
+
+bool valid_dtype(int dt) { return dt == QS_F32 || dt == QS_BF16; }
+
+// A launch plan must fit the buffers the layout reserved for it.
+bool plan_fits(const WsLayout& L, const GemvPlan& p, size_t parts_cap, int ticket_offset) {
+  return p.parts_elems <= parts_cap && kTkGemv + ticket_offset + p.tickets <= L.n_tickets;
+}
+
+// Split the gemv ticket slots of one layout: first projection, then second.
+int32_t* gemv_tickets(const WsView& w, const WsLayout& L, int which, const GemvPlan& first) {
+  return w.ticket(L, kTkGemv + (which == 0 ? 0 : first.tickets));
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* qs_status_string(int status) {
+  switch (status) {
+    case QS_OK: return "QS_OK";
+    case QS_ERR_INVALID_ARG: return "QS_ERR_INVALID_ARG: invalid size, k, enum or NULL pointer";
+    case QS_ERR_ALIGNMENT: return "QS_ERR_ALIGNMENT: pointer or row length not 16-byte aligned";
+    case QS_ERR_WORKSPACE: return "QS_ERR_WORKSPACE: workspace missing or too small";
+    case QS_ERR_CUDA: return "QS_ERR_CUDA: a CUDA call or kernel launch failed";
+    case QS_ERR_TIMEOUT: return "QS_ERR_TIMEOUT: a bounded device wait ran out";
+    case QS_ERR_DEVICE_CHECK: return "QS_ERR_DEVICE_CHECK: a device-side consistency check failed";
+    case QS_ERR_UNSUPPORTED: return "QS_ERR_UNSUPPORTED: sizes outside what this build handles";
+    default: return "unknown qs_status";
+  }
+}
+
+size_t qs_workspace_size(int op, int T, int d_in, int d_out, int k) {
+  WsLayout L;
+  if (!ws_layout(op, T, d_in, d_out, k, &L)) return 0;
+  return L.total;
+}
+
+qs_status qs_workspace_init(void* ws, size_t ws_bytes, void* stream) {
+  if (ws == nullptr) return QS_ERR_INVALID_ARG;
+  return from_cuda(cudaMemsetAsync(ws, 0, ws_bytes, (cudaStream_t)stream));
+}
+
+qs_status qs_device_status(void* ws, void* stream) {
+  if (ws == nullptr) return QS_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  DevStatus st;
+  QS_TRY_CUDA(cudaStreamSynchronize(s));
+  QS_TRY_CUDA(cudaMemcpyAsync(&st, ws, sizeof(st), cudaMemcpyDeviceToHost, s));
+  QS_TRY_CUDA(cudaStreamSynchronize(s));
+  if (st.code == DEV_OK) return QS_OK;
+  QS_TRY_CUDA(cudaMemsetAsync(ws, 0, sizeof(st), s));
+  QS_TRY_CUDA(cudaStreamSynchronize(s));
+  return st.code == DEV_TIMEOUT ? QS_ERR_TIMEOUT : QS_ERR_DEVICE_CHECK;
+}
+
+qs_status qs_workspace_stats(const void* ws, int op, int T, int d_in, int d_out, int k,
+                             int32_t* rows, void* stream) {
+  if (ws == nullptr || rows == nullptr) return QS_ERR_INVALID_ARG;
+  WsLayout L;
+  if (!ws_layout(op, T, d_in, d_out, k, &L)) return QS_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  int32_t c[4] = {0, 0, 0, 0};
+  QS_TRY_CUDA(cudaMemcpyAsync(c, (const unsigned char*)ws + L.cnt, sizeof(c),
+                              cudaMemcpyDeviceToHost, s));
+  QS_TRY_CUDA(cudaStreamSynchronize(s));
+  rows[0] = c[0];
+  rows[1] = (op == QS_OP_SPARSE_FFN) ? c[1] : 0;
+  return QS_OK;
+}
+
+qs_status qs_topk_mask(const void* x, int dtype, int T, int d, int k, int32_t* idx, void* val,
+                       uint8_t* mask, void* xs, void* ws, size_t ws_bytes, void* stream) {
+  if (!valid_dtype(dtype) || x == nullptr || T < 1 || d < 1 || k < 0 || k > d)
+    return QS_ERR_INVALID_ARG;
+  if (k > 0 && idx == nullptr) return QS_ERR_INVALID_ARG;
+  if (d > QS_MAX_ROW) return QS_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(idx) || !aligned16(val) || !aligned16(mask) || !aligned16(xs))
+    return QS_ERR_ALIGNMENT;
+  WsLayout L;
+  qs_status st = check_ws(QS_OP_TOPK_MASK, T, d, 0, k, ws, ws_bytes, &L);
+  if (st != QS_OK) return st;
+  WsView w{(unsigned char*)ws};
+  TopkArgs a;
+  a.x = x; a.T = T; a.d = d; a.k = k;
+  a.kind = dtype == QS_F32 ? TK_F32 : TK_BF16;
+  a.idx = k > 0 ? idx : nullptr;
+  a.val = k > 0 ? val : nullptr;
+  a.mask = mask; a.xs = xs;
+  a.status = w.status();
+  return from_cuda(launch_topk(a, (cudaStream_t)stream));
+}
+
+qs_status qs_sparse_linear(const void* x, int dtype, int T, int d_in, int d_out, int k,
+                           const void* wt, void* y, void* ws, size_t ws_bytes, void* stream) {
+  if (!valid_dtype(dtype) || x == nullptr || wt == nullptr || y == nullptr || T < 1 || d_in < 1 ||
+      d_out < 1 || k < 0 || k > d_in)
+    return QS_ERR_INVALID_ARG;
+  if (d_in > QS_MAX_ROW || d_out > QS_MAX_ROW) return QS_ERR_UNSUPPORTED;
+  const int V = 16 / elem_bytes(dtype);
+  if ((d_out % V) != 0 || !aligned16(x) || !aligned16(wt) || !aligned16(y)) return QS_ERR_ALIGNMENT;
+  WsLayout L;
+  qs_status st = check_ws(QS_OP_SPARSE_LINEAR, T, d_in, d_out, k, ws, ws_bytes, &L);
+  if (st != QS_OK) return st;
+  WsView w{(unsigned char*)ws};
+  cudaStream_t s = (cudaStream_t)stream;
+  const int eb = elem_bytes(dtype);
+
+  // Prefill: many tokens make this a dense contraction over X_sparse.
+  if (dtype == QS_BF16 && T >= QS_PREFILL_MIN_T && prefill_supported(T, d_out, d_in)) {
+    TopkArgs a;
+    a.x = x; a.T = T; a.d = d_in; a.k = k; a.kind = TK_BF16;
+    a.xs = w.at<void>(L.xs_bf16);
+    a.status = w.status();
+    QS_TRY_CUDA(launch_topk(a, s));
+    PrefillArgs p;
+    p.xs = w.at<__nv_bfloat16>(L.xs_bf16);
+    p.wt = reinterpret_cast<const __nv_bfloat16*>(wt);
+    p.y = reinterpret_cast<__nv_bfloat16*>(y);
+    p.M = T; p.N = d_out; p.K = d_in;
+    p.status = w.status();
+    return from_cuda(launch_prefill_gemm(p, s));
+  }
+
+  for (int t0 = 0; t0 < T; t0 += kChunkT) {
+    const int Tc = (T - t0) < kChunkT ? (T - t0) : kChunkT;
+    TopkArgs a;
+    a.x = (const unsigned char*)x + (size_t)t0 * d_in * eb;
+    a.T = Tc; a.d = d_in; a.k = k;
+    a.kind = dtype == QS_F32 ? TK_F32 : TK_BF16;
+    a.xsf = Tc > 1 ? w.at<float>(L.xsf_x) : nullptr;   // only the union pass reads it
+    a.list = w.at<int32_t>(L.list_x);
+    a.list_val = w.at<float>(L.lval_x);
+    a.list_count = w.at<int32_t>(L.cnt) + 0;
+    a.ticket = w.ticket(L, kTkTopkX);
+    a.status = w.status();
+    const GemvPlan gp = plan_gemv(Tc, d_out, (int)rows_bound(Tc, d_in, k), 1, eb);
+    if (!plan_fits(L, gp, L.parts1_elems, 0)) return QS_ERR_UNSUPPORTED;
+    a.zero = w.at<float>(L.parts1);
+    a.zero_n = gp.parts_elems;
+    QS_TRY_CUDA(launch_topk(a, s));
+
+    GemvArgs g;
+    g.w[0] = wt;
+    g.d_in = d_in; g.d_out = d_out; g.T = Tc;
+    g.bf16 = dtype == QS_BF16;
+    g.mode = 0;
+    g.list = a.list; g.list_val = a.list_val; g.list_count = a.list_count;
+    g.parts = w.at<float>(L.parts1);
+    g.plan = gp;
+    g.tickets = gemv_tickets(w, L, 0, g.plan);
+    if (!plan_fits(L, g.plan, L.parts1_elems, 0)) return QS_ERR_UNSUPPORTED;
+    g.y = (unsigned char*)y + (size_t)t0 * d_out * eb;
+    g.status = w.status();
+    QS_TRY_CUDA(launch_gemv(g, s));
+  }
+  return QS_OK;
+}
+
+qs_status qs_sparse_ffn(const void* x, int dtype, int T, int d_model, int d_ff, int act,
+                        int k_in, int k_h, const void* wt_up, const void* wt_gate,
+                        const float* b_up, const float* b_gate, const void* wt_down, void* y,
+                        float* h_out, int32_t* idx_h_out, void* const* phase_events, void* ws,
+                        size_t ws_bytes, void* stream) {
+  if (!valid_dtype(dtype) || x == nullptr || wt_up == nullptr || wt_gate == nullptr ||
+      wt_down == nullptr || y == nullptr || T < 1 || d_model < 1 || d_ff < 1 || k_in < 0 ||
+      k_in > d_model || k_h < 0 || k_h > d_ff ||
+      (act != QS_ACT_RELU2_GLU && act != QS_ACT_DRELU))
+    return QS_ERR_INVALID_ARG;
+  if (d_model > QS_MAX_ROW || d_ff > QS_MAX_ROW) return QS_ERR_UNSUPPORTED;
+  const int eb = elem_bytes(dtype);
+  const int V = 16 / eb;
+  if ((d_model % V) != 0 || (d_ff % V) != 0) return QS_ERR_ALIGNMENT;
+  if (!aligned16(x) || !aligned16(wt_up) || !aligned16(wt_gate) || !aligned16(wt_down) ||
+      !aligned16(y) || !aligned16(h_out) || !aligned16(idx_h_out) || !aligned16(b_up) ||
+      !aligned16(b_gate))
+    return QS_ERR_ALIGNMENT;
+  WsLayout L;
+  qs_status st = check_ws(QS_OP_SPARSE_FFN, T, d_model, d_ff, k_h, ws, ws_bytes, &L);
+  if (st != QS_OK) return st;
+  WsView w{(unsigned char*)ws};
+  cudaStream_t s = (cudaStream_t)stream;
+  auto mark = [&](int i) -> cudaError_t {
+    if (phase_events == nullptr) return cudaSuccess;
+    return cudaEventRecord((cudaEvent_t)phase_events[i], s);
+  };
+
+  for (int t0 = 0; t0 < T; t0 += kChunkT) {
+    const int Tc = (T - t0) < kChunkT ? (T - t0) : kChunkT;
+    const bool timed = (t0 == 0);
+    if (timed) QS_TRY_CUDA(mark(0));
+
+    // 1. top-K on |x|
+    TopkArgs a;
+    a.x = (const unsigned char*)x + (size_t)t0 * d_model * eb;
+    a.T = Tc; a.d = d_model; a.k = k_in;
+    a.kind = dtype == QS_F32 ? TK_F32 : TK_BF16;
+    a.xsf = Tc > 1 ? w.at<float>(L.xsf_x) : nullptr;
+    a.list = w.at<int32_t>(L.list_x);
+    a.list_val = w.at<float>(L.lval_x);
+    a.list_count = w.at<int32_t>(L.cnt) + 0;
+    a.ticket = w.ticket(L, kTkTopkX);
+    a.status = w.status();
+    const GemvPlan p_ug = plan_gemv(Tc, d_ff, (int)rows_bound(Tc, d_model, d_model), 2, eb);
+    const GemvPlan p_dn = plan_gemv(Tc, d_model, (int)rows_bound(Tc, d_ff, k_h), 1, eb);
+    if (!plan_fits(L, p_ug, L.parts1_elems, 0) || !plan_fits(L, p_dn, L.parts2_elems, p_ug.tickets))
+      return QS_ERR_UNSUPPORTED;
+    a.zero = w.at<float>(L.parts1);
+    a.zero_n = p_ug.parts_elems;
+    QS_TRY_CUDA(launch_topk(a, s));
+    if (timed) QS_TRY_CUDA(mark(1));
+
+    // 2. up and gate projections over the kept rows, gating epilogue -> h
+    float* h = h_out ? h_out + (size_t)t0 * d_ff : w.at<float>(L.h);
+    GemvArgs g;
+    g.w[0] = wt_up; g.w[1] = wt_gate;
+    g.d_in = d_model; g.d_out = d_ff; g.T = Tc;
+    g.bf16 = dtype == QS_BF16;
+    g.mode = act == QS_ACT_RELU2_GLU ? 1 : 2;
+    g.list = a.list; g.list_val = a.list_val; g.list_count = a.list_count;
+    g.parts = w.at<float>(L.parts1);
+    g.plan = p_ug;
+    g.tickets = gemv_tickets(w, L, 0, g.plan);
+    g.h = h; g.b_up = b_up; g.b_gate = b_gate;
+    g.zero = w.at<float>(L.parts2);
+    g.zero_n = p_dn.parts_elems;
+    g.status = w.status();
+    QS_TRY_CUDA(launch_gemv(g, s));
+    if (timed) QS_TRY_CUDA(mark(2));
+
+    // 3. top-K on |h|
+    TopkArgs b;
+    b.x = h; b.T = Tc; b.d = d_ff; b.k = k_h; b.kind = TK_F32;
+    b.idx = (idx_h_out && k_h > 0) ? idx_h_out + (size_t)t0 * k_h : nullptr;
+    b.xsf = Tc > 1 ? w.at<float>(L.xsf_h) : nullptr;
+    b.list = w.at<int32_t>(L.list_h);
+    b.list_val = w.at<float>(L.lval_h);
+    b.list_count = w.at<int32_t>(L.cnt) + 1;
+    b.ticket = w.ticket(L, kTkTopkH);
+    b.status = w.status();
+    QS_TRY_CUDA(launch_topk(b, s));
+    if (timed) QS_TRY_CUDA(mark(3));
+
+    // 4. down projection over the kept nonzero h
+    GemvArgs dn;
+    dn.w[0] = wt_down;
+    dn.d_in = d_ff; dn.d_out = d_model; dn.T = Tc;
+    dn.bf16 = dtype == QS_BF16;
+    dn.mode = 0;
+    dn.list = b.list; dn.list_val = b.list_val; dn.list_count = b.list_count;
+    dn.parts = w.at<float>(L.parts2);
+    dn.plan = p_dn;
+    dn.tickets = gemv_tickets(w, L, 1, g.plan);
+    dn.y = (unsigned char*)y + (size_t)t0 * d_model * eb;
+    dn.status = w.status();
+    QS_TRY_CUDA(launch_gemv(dn, s));
+    if (timed) QS_TRY_CUDA(mark(4));
+  }
+  return QS_OK;
+}
+
+qs_status qs_quant_sparse_linear(const void* x, int dtype, int T, int d_in, int d_out, int k,
+                                 const uint32_t* wt_packed, float alpha, float eps, float* y,
+                                 int32_t* acc, int8_t* q, int32_t* idx, void* ws, size_t ws_bytes,
+                                 void* stream) {
+  if (!valid_dtype(dtype) || x == nullptr || wt_packed == nullptr || y == nullptr || T < 1 ||
+      d_in < 1 || d_out < 1 || k < 0 || k > d_in || !(eps >= 0.0f) || !(alpha == alpha))
+    return QS_ERR_INVALID_ARG;
+  if (d_in > QS_MAX_ROW || d_out > QS_MAX_ROW) return QS_ERR_UNSUPPORTED;
+  if ((d_out % 16) != 0 || !aligned16(x) || !aligned16(wt_packed) || !aligned16(y) ||
+      !aligned16(acc) || !aligned16(q) || !aligned16(idx))
+    return QS_ERR_ALIGNMENT;
+  WsLayout L;
+  qs_status st = check_ws(QS_OP_QUANT_SPARSE_LINEAR, T, d_in, d_out, k, ws, ws_bytes, &L);
+  if (st != QS_OK) return st;
+  WsView w{(unsigned char*)ws};
+  cudaStream_t s = (cudaStream_t)stream;
+  const int eb = elem_bytes(dtype);
+  for (int t0 = 0; t0 < T; t0 += kChunkT) {
+    const int Tc = (T - t0) < kChunkT ? (T - t0) : kChunkT;
+    TopkArgs a;
+    a.x = (const unsigned char*)x + (size_t)t0 * d_in * eb;
+    a.T = Tc; a.d = d_in; a.k = k;
+    a.kind = dtype == QS_F32 ? TK_QUANT_F32 : TK_QUANT_BF16;
+    a.eps = eps;
+    a.idx = (idx && k > 0) ? idx + (size_t)t0 * k : nullptr;
+    a.q_full = q ? q + (size_t)t0 * d_in : nullptr;
+    a.xq = Tc > 1 ? w.at<int8_t>(L.xq) : nullptr;     // only the union pass reads it
+    a.gamma = w.at<float>(L.gamma);
+    a.list = w.at<int32_t>(L.list_x);
+    a.list_q = w.at<int8_t>(L.lval_x);
+    a.list_count = w.at<int32_t>(L.cnt) + 0;
+    a.ticket = w.ticket(L, kTkTopkX);
+    a.status = w.status();
+    QS_TRY_CUDA(launch_topk(a, s));
+
+    QGemvArgs g;
+    g.wp = wt_packed; g.d_in = d_in; g.d_out = d_out; g.T = Tc;
+    g.gamma = a.gamma; g.alpha = alpha;
+    g.list = a.list; g.list_q = a.list_q; g.list_count = a.list_count;
+    g.parts = w.at<int32_t>(L.parts1);
+    g.plan = plan_qgemv(Tc, d_out, (int)rows_bound(Tc, d_in, k));
+    g.tickets = w.ticket(L, kTkGemv);
+    if (!plan_fits(L, g.plan, L.parts1_elems, 0)) return QS_ERR_UNSUPPORTED;
+    g.y = y + (size_t)t0 * d_out;
+    g.acc = acc ? acc + (size_t)t0 * d_out : nullptr;
+    g.status = w.status();
+    QS_TRY_CUDA(launch_qgemv(g, s));
+  }
+  return QS_OK;
+}
+
+qs_status qs_ternary_pack(const float* wmat, int d_out, int d_in, float eps, uint32_t* wt_packed,
+                          float* alpha_out, void* ws, size_t ws_bytes, void* stream) {
+  if (wmat == nullptr || wt_packed == nullptr || d_out < 16 || d_in < 1 || !(eps >= 0.0f))
+    return QS_ERR_INVALID_ARG;
+  if ((d_out % 16) != 0 || !aligned16(wmat) || !aligned16(wt_packed) || !aligned16(alpha_out))
+    return QS_ERR_ALIGNMENT;
+  WsLayout L;
+  qs_status st = check_ws(QS_OP_TERNARY_PACK, 0, d_in, d_out, 0, ws, ws_bytes, &L);
+  if (st != QS_OK) return st;
+  WsView w{(unsigned char*)ws};
+  PackArgs a;
+  a.w = wmat; a.d_out = d_out; a.d_in = d_in; a.eps = eps;
+  a.packed = wt_packed; a.alpha_out = alpha_out;
+  a.alpha_parts = w.at<double>(L.alpha_parts);
+  a.alpha_ws = w.at<float>(L.alpha);
+  a.ticket = w.ticket(L, kTkAlpha);
+  a.status = w.status();
+  return from_cuda(launch_ternary_pack(a, (cudaStream_t)stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,372 @@
+// Decode-regime gather-GEMV:  y[t, :] = sum_{i in rows} xs[t, i] * W^T[i, :]
+//
+// Source: Q-Sparse news article (zxwl-tech.com), section "Top-K
+// sparsification" (X_sparse replaces X in Y = X.W^T, so the zeroed inputs
+// need neither arithmetic nor their weights), and the aibase.com summary,
+// "Vantagens da ativacao esparsa" (memory traffic, not arithmetic, bounds
+// inference).  With W stored input-major (W^T, [d_in, d_out]) the weights of
+// one kept input are one contiguous row, so the kernel streams exactly the
+// rows listed by the top-K kernel (the union over the batch's tokens) and
+// nothing else.
+//
+// Mapping (B200: 148 SMs, HBM3e).  Measured on this pattern (2867 kept rows
+// of 22 KB): 512-byte segments per request stream at ~3.4 TB/s whatever the
+// load depth, while 1-D bulk copies (TMA) of multi-KB row segments reach
+// ~4.4-4.8 TB/s, close to a contiguous read.  So:
+//   * a row is cut into n_ct equal column tiles of a few KB (e.g. 4 x 5.5 KB
+//     for 11008 bf16 columns); a CTA owns one tile, one weight matrix and a
+//     contiguous slice of the row list (split-K);
+//   * one producer thread issues a cp.async.bulk per kept row into a ring of
+//     shared-memory stages guarded by mbarriers (transaction-count
+//     completion); each wait is bounded and reports DEV_TIMEOUT if it runs out;
+//   * each consumer thread owns one 16-byte column vector of the tile for the
+//     whole stream (f32 accumulators in registers, one per token), so no
+//     cross-warp reduction is needed;
+//   * the slice's row indices and per-token values are staged in shared
+//     memory first (one round trip: the top-K kernel stores each listed row's
+//     values next to the list);
+//   * split partials are added with f32 vector reductions (red.add.v4.f32)
+//     into an accumulator that the previous kernel of the call zeroed; the
+//     last CTA of a column tile to arrive (an atomic ticket, nobody waits)
+//     reads the sums once and runs the epilogue.  The epilogue
+//     is the output cast, or the FFN gating h = ReLU(u)^2 * g (Q-Sparse
+//     squared ReLU) or h = ReLU(g + b_g) * ReLU(u + b_u) (Turbo Sparse dReLU,
+//     Eq. 2).  The order of the split additions is not fixed, so the last
+//     bits of a split sum may differ between runs.
+#include "qs_internal.cuh"
+
+namespace qs {
+namespace {
+
+constexpr int kMaxConsumers = 384;
+constexpr int kMaxStages = 32;
+
+template <typename WT> struct VecTraits;
+template <> struct VecTraits<float> { static constexpr int V = 4; };
+template <> struct VecTraits<__nv_bfloat16> { static constexpr int V = 8; };
+
+template <typename WT>
+__device__ __forceinline__ void unpack(const uint4& q, float (&w)[VecTraits<WT>::V]) {
+  if constexpr (VecTraits<WT>::V == 8) {
+    w[0] = bf16lo(q.x); w[1] = bf16hi(q.x);
+    w[2] = bf16lo(q.y); w[3] = bf16hi(q.y);
+    w[4] = bf16lo(q.z); w[5] = bf16hi(q.z);
+    w[6] = bf16lo(q.w); w[7] = bf16hi(q.w);
+  } else {
+    w[0] = __uint_as_float(q.x); w[1] = __uint_as_float(q.y);
+    w[2] = __uint_as_float(q.z); w[3] = __uint_as_float(q.w);
+  }
+}
+
+__device__ __forceinline__ void red_add_v4(float* dst, float a0, float a1, float a2, float a3) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(a0), "f"(a1), "f"(a2),
+               "f"(a3)
+               : "memory");
+}
+
+template <int V>
+__device__ __forceinline__ void store_f32(float* dst, const float (&v)[V]) {
+#pragma unroll
+  for (int q = 0; q < V / 4; ++q)
+    reinterpret_cast<float4*>(dst)[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+}
+
+template <typename WT>
+__device__ __forceinline__ void store_y(void* y, size_t o, const float (&v)[VecTraits<WT>::V]) {
+  if constexpr (VecTraits<WT>::V == 8) {
+    uint4 q;
+    q.x = (uint32_t)f32_to_bf16_bits(v[0]) | ((uint32_t)f32_to_bf16_bits(v[1]) << 16);
+    q.y = (uint32_t)f32_to_bf16_bits(v[2]) | ((uint32_t)f32_to_bf16_bits(v[3]) << 16);
+    q.z = (uint32_t)f32_to_bf16_bits(v[4]) | ((uint32_t)f32_to_bf16_bits(v[5]) << 16);
+    q.w = (uint32_t)f32_to_bf16_bits(v[6]) | ((uint32_t)f32_to_bf16_bits(v[7]) << 16);
+    *reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(y) + o) = q;
+  } else {
+    store_f32<4>(reinterpret_cast<float*>(y) + o, v);
+  }
+}
+
+// Output of one column vector: y (MODE 0) or the gated hidden h (MODE 1/2).
+template <typename WT, int MODE>
+__device__ __forceinline__ void epilogue(const GemvArgs& a, int tok, int col,
+                                         const float (&u)[VecTraits<WT>::V],
+                                         const float (&g)[VecTraits<WT>::V]) {
+  constexpr int V = VecTraits<WT>::V;
+  const size_t o = (size_t)tok * a.d_out + col;
+  if constexpr (MODE == 0) {
+    store_y<WT>(a.y, o, u);
+  } else {
+    float hv[V];
+#pragma unroll
+    for (int e = 0; e < V; ++e) {
+      if constexpr (MODE == 1) {
+        const float r = fmaxf(u[e], 0.0f);           // u (up), g (gate)
+        hv[e] = (r * r) * g[e];
+      } else {
+        const float bu = a.b_up ? a.b_up[col + e] : 0.0f;
+        const float bg = a.b_gate ? a.b_gate[col + e] : 0.0f;
+        hv[e] = fmaxf(g[e] + bg, 0.0f) * fmaxf(u[e] + bu, 0.0f);
+      }
+    }
+    store_f32<V>(a.h + o, hv);
+  }
+}
+
+template <typename WT, int TT, int MODE>
+__global__ void __launch_bounds__(kMaxConsumers + 32, (TT <= 4) ? 2 : 1) gemv_kernel(GemvArgs a) {
+  constexpr int V = VecTraits<WT>::V;
+  extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ __align__(8) uint64_t s_full[kMaxStages];
+  __shared__ __align__(8) uint64_t s_empty[kMaxStages];
+  __shared__ int s_flag;
+  __shared__ int s_err;
+
+  const GemvPlan& P = a.plan;
+  const int NC = P.threads - 32;                 // consumer threads; the last warp produces
+  const int tid = threadIdx.x, lane = tid & 31;
+  const bool producer = tid >= NC;
+  const int tile_bytes = P.vec_tile * 16;
+  unsigned char* s_stage = smem;
+  int* s_rows = reinterpret_cast<int*>(smem + (size_t)P.nst * P.rps * tile_bytes);
+  float* s_vals = reinterpret_cast<float*>(s_rows + P.rcap);
+
+  const int S = P.S;
+  const int ct = blockIdx.x;
+  const int mat = blockIdx.y / S;
+  const int s = blockIdx.y - mat * S;
+  const int grp = blockIdx.z;
+  const int tok0 = grp * TT;
+  const int ntok = min(TT, a.T - tok0);
+  const int d_in = a.d_in, d_out = a.d_out;
+  const size_t row_bytes = (size_t)d_out * sizeof(WT);
+  const size_t cbyte = (size_t)ct * tile_bytes;
+  const int tbytes = (int)min((size_t)tile_bytes, row_bytes - cbyte);   // ragged last tile
+  const int tvec = tbytes / 16;
+  const unsigned char* Wb = reinterpret_cast<const unsigned char*>(a.w[mat]) + cbyte;
+  const int col = (ct * P.vec_tile + tid) * V;                            // this thread's columns
+
+  grid_zero(a.zero, a.zero_n);
+  const int n = min(max(*a.list_count, 0), d_in);
+  const int r0 = (int)(((long long)n * s) / S);
+  const int r1 = (int)(((long long)n * (s + 1)) / S);
+
+  if (tid == 0) {
+    for (int i = 0; i < P.nst; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_empty[i], NC / 32);
+    }
+    mbar_fence_init();
+    s_err = 0;
+  }
+  __syncthreads();
+
+  float acc[TT][V];
+#pragma unroll
+  for (int t = 0; t < TT; ++t)
+#pragma unroll
+    for (int e = 0; e < V; ++e) acc[t][e] = 0.0f;
+
+  int gst = 0;                                   // stages issued so far (slot/phase)
+  for (int pb = r0; pb < r1; pb += P.rcap) {
+    const int np = min(P.rcap, r1 - pb);
+    for (int j = tid; j < np; j += P.threads) {
+      int r = a.list[pb + j];
+      const bool ok = (unsigned)r < (unsigned)d_in;
+      if (!ok) {                                 // a corrupted list is reported, never followed
+        dev_fail(a.status, DEV_CHECK, 3, (uint32_t)r);
+        r = 0;
+      }
+      s_rows[j] = r;
+      const float* lv = a.list_val + (size_t)(pb + j) * a.T + tok0;
+#pragma unroll
+      for (int t = 0; t < TT; ++t) s_vals[t * P.rcap + j] = (ok && t < ntok) ? lv[t] : 0.0f;
+    }
+    __syncthreads();
+    const int nstage = (np + P.rps - 1) / P.rps;
+    if (producer) {
+      if (lane == 0) {
+        for (int st = 0; st < nstage; ++st) {
+          const int g = gst + st;
+          const int slot = g % P.nst;
+          if (g >= P.nst && !mbar_wait(&s_empty[slot], (uint32_t)((g / P.nst) - 1) & 1u)) {
+            dev_fail(a.status, DEV_TIMEOUT, 10, (uint32_t)g);
+            atomicExch(&s_err, 1);
+            break;
+          }
+          const int j0 = st * P.rps;
+          const int cnt = min(P.rps, np - j0);
+          mbar_arrive_expect_tx(&s_full[slot], (uint32_t)(cnt * tbytes));
+          for (int r = 0; r < cnt; ++r)
+            bulk_g2s(s_stage + ((size_t)slot * P.rps + r) * tile_bytes,
+                     Wb + (size_t)s_rows[j0 + r] * row_bytes, (uint32_t)tbytes, &s_full[slot]);
+        }
+      }
+    } else {
+      for (int st = 0; st < nstage; ++st) {
+        const int g = gst + st;
+        const int slot = g % P.nst;
+        bool ready = mbar_wait_backoff(&s_full[slot], (uint32_t)(g / P.nst) & 1u);
+        if (!ready) {
+          if (lane == 0) dev_fail(a.status, DEV_TIMEOUT, 11, (uint32_t)g);
+          atomicExch(&s_err, 1);
+        }
+        const int j0 = st * P.rps;
+        const int cnt = min(P.rps, np - j0);
+        if (ready && tid < tvec) {
+          for (int r = 0; r < cnt; ++r) {
+            const uint4 q = *reinterpret_cast<const uint4*>(
+                s_stage + ((size_t)slot * P.rps + r) * tile_bytes + (size_t)tid * 16);
+            float w[V];
+            unpack<WT>(q, w);
+#pragma unroll
+            for (int t = 0; t < TT; ++t) {
+              const float v = s_vals[t * P.rcap + j0 + r];
+#pragma unroll
+              for (int e = 0; e < V; ++e) acc[t][e] = fmaf(v, w[e], acc[t][e]);
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_empty[slot]);
+      }
+    }
+    gst += nstage;
+    __syncthreads();                             // piece consumed before restaging
+  }
+  if (s_err && tid == 0) {
+    // a wait gave up: let the copies already issued land before the CTA exits
+    for (int i = 0; i < P.nst && i < gst; ++i) {
+      const int g_last = gst - 1 - i;            // the newest stage of each slot
+      mbar_wait(&s_full[g_last % P.nst], (uint32_t)(g_last / P.nst) & 1u);
+    }
+  }
+
+  // ---- add this split's partial sums --------------------------------------
+  const bool mine = !producer && tid < tvec;
+  const bool direct = (MODE == 0) && (S == 1);
+  const size_t per_mat = (size_t)a.T * d_out;
+  if (mine) {
+    for (int t = 0; t < ntok; ++t) {
+      const int tok = tok0 + t;
+      if (direct) {
+        store_y<WT>(a.y, (size_t)tok * d_out + col, acc[t]);
+      } else {
+        float* dst = a.parts + (size_t)mat * per_mat + (size_t)tok * d_out + col;
+#pragma unroll
+        for (int q = 0; q < V / 4; ++q)
+          red_add_v4(dst + 4 * q, acc[t][4 * q], acc[t][4 * q + 1], acc[t][4 * q + 2], acc[t][4 * q + 3]);
+      }
+    }
+  }
+  if (direct) return;
+
+  // ---- the last CTA of this column tile: epilogue, then zero the sums -------
+  int32_t* ticket = a.tickets + (size_t)grp * P.n_ct + ct;
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_flag = (atomicAdd(ticket, 1) == P.mats * S - 1);
+  __syncthreads();
+  if (!s_flag) return;
+  __threadfence();
+  if (tid == 0) *ticket = 0;                     // leave the counter clean
+  if (mine) {
+    for (int t = 0; t < ntok; ++t) {
+      const int tok = tok0 + t;
+      float* pu = a.parts + (size_t)tok * d_out + col;
+      float* pg = pu + per_mat;
+      float u[V], g[V];
+#pragma unroll
+      for (int q = 0; q < V / 4; ++q) {
+        const float4 r = __ldcg(reinterpret_cast<const float4*>(pu) + q);
+        u[4 * q] = r.x; u[4 * q + 1] = r.y; u[4 * q + 2] = r.z; u[4 * q + 3] = r.w;
+      }
+      if (P.mats == 2) {
+#pragma unroll
+        for (int q = 0; q < V / 4; ++q) {
+          const float4 r = __ldcg(reinterpret_cast<const float4*>(pg) + q);
+          g[4 * q] = r.x; g[4 * q + 1] = r.y; g[4 * q + 2] = r.z; g[4 * q + 3] = r.w;
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < V; ++e) g[e] = 0.0f;
+      }
+      epilogue<WT, MODE>(a, tok, col, u, g);
+    }
+  }
+}
+
+template <typename WT, int TT, int MODE>
+cudaError_t launch3(const GemvArgs& a, cudaStream_t s) {
+  static unsigned configured = 0;
+  cudaError_t e = ensure_smem_attr(gemv_kernel<WT, TT, MODE>, 200 * 1024, &configured);
+  if (e != cudaSuccess) return e;
+  dim3 grid(a.plan.n_ct, a.plan.mats * a.plan.S, a.plan.groups);
+  gemv_kernel<WT, TT, MODE><<<grid, a.plan.threads, a.plan.smem, s>>>(a);
+  return cudaGetLastError();
+}
+
+template <typename WT, int TT>
+cudaError_t launch2(const GemvArgs& a, cudaStream_t s) {
+  switch (a.mode) {
+    case 0: return launch3<WT, TT, 0>(a, s);
+    case 1: return launch3<WT, TT, 1>(a, s);
+    case 2: return launch3<WT, TT, 2>(a, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+template <typename WT>
+cudaError_t launch1(const GemvArgs& a, cudaStream_t s) {
+  switch (a.plan.TT) {
+    case 1: return launch2<WT, 1>(a, s);
+    case 2: return launch2<WT, 2>(a, s);
+    case 4: return launch2<WT, 4>(a, s);
+    case 8: return launch2<WT, 8>(a, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace
+
+GemvPlan plan_gemv(int T, int d_out, int rows_bound, int mats, int elem_bytes) {
+  GemvPlan p{};
+  p.TT = (T <= 1) ? 1 : (T == 2 ? 2 : (T <= 4 ? 4 : 8));
+  p.groups = (T + p.TT - 1) / p.TT;
+  p.mats = mats;
+  const int vec_row = (int)(((long)d_out * elem_bytes) / 16);
+  int nct = (vec_row + kMaxConsumers - 1) / kMaxConsumers;
+  for (int c = nct; c <= nct + 8 && c <= vec_row; ++c)    // prefer equal tiles
+    if (vec_row % c == 0) { nct = c; break; }
+  p.n_ct = nct;
+  p.vec_tile = (vec_row + nct - 1) / nct;
+  p.threads = ((p.vec_tile + 31) / 32) * 32 + 32;
+  const int tile_bytes = p.vec_tile * 16;
+  p.rps = tile_bytes >= 8192 ? 1 : 8192 / tile_bytes;
+  if (p.rps > 8) p.rps = 8;
+  const int per_sm = (p.TT <= 4) ? 2 : 1;
+  const long stage_budget = per_sm == 2 ? 80 * 1024 : 160 * 1024;
+  long nst = stage_budget / ((long)p.rps * tile_bytes);
+  if (nst < 2) nst = 2;
+  if (nst > kMaxStages) nst = kMaxStages;
+  p.nst = (int)nst;
+  p.rcap = (p.TT == 1) ? 2048 : (p.TT == 8 ? 512 : 1024);
+  p.smem = (size_t)p.nst * p.rps * tile_bytes + (size_t)p.rcap * 4 * (1 + p.TT);
+  const long slots = (long)kNumSMs * per_sm;
+  const long units = (long)nct * mats * p.groups;
+  long S = slots / (units > 0 ? units : 1);
+  if (S < 1) S = 1;
+  const long max_by_rows = rows_bound / 16;      // keep >= ~16 rows per split
+  if (S > max_by_rows) S = max_by_rows > 0 ? max_by_rows : 1;
+  if (S > 256) S = 256;
+  p.S = (int)S;
+  p.ng = 1;
+  p.parts_elems = (size_t)mats * T * d_out;     // f32 accumulators, zeroed by the previous kernel
+  p.tickets = p.groups * nct;
+  return p;
+}
+
+cudaError_t launch_gemv(const GemvArgs& a, cudaStream_t s) {
+  if (a.T <= 0 || a.d_out <= 0) return cudaSuccess;
+  return a.bf16 ? launch1<__nv_bfloat16>(a, s) : launch1<float>(a, s);
+}
+
+}  // namespace qs

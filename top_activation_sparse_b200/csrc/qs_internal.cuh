@@ -1,0 +1,302 @@
+// Internal declarations shared by the library's translation units.
+// Nothing here is part of the C ABI (see include/qs.h).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "qs.h"
+
+namespace qs {
+
+// ---------------------------------------------------------------------------
+// device status word (first bytes of every workspace)
+// ---------------------------------------------------------------------------
+enum DevCode : uint32_t {
+  DEV_OK = 0,
+  DEV_TIMEOUT = 1,      // a bounded wait ran out
+  DEV_CHECK = 2,        // an internal consistency check failed
+};
+
+struct DevStatus {
+  uint32_t code;        // first error wins (atomicCAS from 0)
+  uint32_t where;       // which check / wait
+  uint32_t detail;      // free-form (an index, an iteration count)
+  uint32_t pad;
+};
+
+__device__ __forceinline__ void dev_fail(DevStatus* st, uint32_t code, uint32_t where,
+                                         uint32_t detail) {
+  if (st == nullptr) return;
+  if (atomicCAS(&st->code, 0u, code) == 0u) {
+    st->where = where;
+    st->detail = detail;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// small device helpers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
+  // weights are read exactly once per call: do not keep them in L1
+  uint4 r;
+  asm("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+      : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+      : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t ld_stream_u32(const void* p) {
+  uint32_t r;
+  asm("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(r) : "l"(p));
+  return r;
+}
+
+// ---- mbarrier / bulk-copy (TMA) helpers ------------------------------------
+// Every wait is bounded: after kWaitLimit polls it gives up and returns false,
+// and the caller records DEV_TIMEOUT instead of hanging the GPU.
+constexpr uint32_t kWaitLimit = 1u << 22;
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ void mbar_init(uint64_t* b, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(b)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_fence_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* b, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(done)
+      : "r"(smem_u32(b)), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity) {
+  for (uint32_t it = 0; it < kWaitLimit; ++it)
+    if (mbar_try_wait(b, parity)) return true;
+  return false;
+}
+// Consumer-side wait: poll with a short sleep so that waiting warps leave the
+// issue slots to the producer and to the warps that have data.
+__device__ __forceinline__ bool mbar_wait_backoff(uint64_t* b, uint32_t parity) {
+  for (uint32_t it = 0; it < kWaitLimit; ++it) {
+    if (mbar_try_wait(b, parity)) return true;
+    __nanosleep(64);
+  }
+  return false;
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* b) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b)) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* b, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)), "r"(bytes)
+               : "memory");
+}
+// 1-D bulk copy global -> this CTA's shared memory (no multicast); completion
+// is signalled on `bar` as transaction bytes.  16-byte aligned, size % 16 == 0.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ float bf16lo(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
+
+__device__ __forceinline__ uint16_t f32_to_bf16_bits(float f) {
+  return __bfloat16_as_ushort(__float2bfloat16_rn(f));
+}
+
+__device__ __forceinline__ unsigned lanemask_lt() {
+  unsigned m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+// Raise a kernel's dynamic shared-memory limit once per device.
+template <typename F>
+cudaError_t ensure_smem_attr(F* kernel, int bytes, unsigned* done_mask) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned bit = 1u << (dev & 31);
+  if (*done_mask & bit) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) *done_mask |= bit;
+  return e;
+}
+
+// ---------------------------------------------------------------------------
+// workspace layout (host side; one function sizes and places every buffer)
+// ---------------------------------------------------------------------------
+constexpr int kNumSMs = 148;          // B200; split counts are a pure function of sizes
+constexpr size_t kWsAlign = 256;
+
+struct GemvPlan {
+  int TT;          // tokens per pass (1, 2, 4, 8)
+  int groups;      // ceil(T / TT)
+  int n_ct;        // column tiles
+  int S;           // splits of the row list
+  int mats;        // weight matrices sharing the row list (2 for up/gate)
+  size_t parts_elems;  // partial-sum buffer, f32 elements (splits + split groups)
+  int tickets;     // ticket counters the launch uses
+  // gather-GEMV pipeline (bulk-copy ring), unused by the int8 path
+  int vec_tile;    // 16-byte vectors of one row segment (= consumer threads used)
+  int threads;     // consumer threads (multiple of 32) + one producer warp
+  int rps;         // rows per pipeline stage
+  int nst;         // pipeline stages
+  int ng;          // groups of up to 8 splits (two-level reduction)
+  int rcap;        // rows staged in shared memory per piece
+  size_t smem;     // dynamic shared memory bytes
+};
+
+GemvPlan plan_gemv(int T, int d_out, int rows_bound, int mats, int elem_bytes);
+GemvPlan plan_qgemv(int T, int d_out, int rows_bound);
+
+struct WsLayout {
+  size_t status = 0;          // DevStatus
+  size_t tickets = 0;         // int32 counters, zero between calls
+  int n_tickets = 0;
+  // stage 1: top-K on the projection input
+  size_t xsf_x = 0;           // [T, d_in] f32 dense masked values
+  size_t xq = 0;              // [T, d_in] int8 dense masked q (quant path)
+  size_t gamma = 0;           // [T] f32 (quant path)
+  size_t list_x = 0;          // [d_in] int32
+  size_t lval_x = 0;          // [d_in][T] f32 (or int8 for the quant path)
+  size_t cnt = 0;             // int32[4]: rows of list_x, rows of list_h, ...
+  // stage 2: projection(s)
+  size_t parts1 = 0;          // gemv partial sums
+  size_t h = 0;               // [T, d_ff] f32 (ffn)
+  size_t xsf_h = 0;           // [T, d_ff] f32 (ffn)
+  size_t list_h = 0;          // [d_ff] int32 (ffn)
+  size_t lval_h = 0;          // [d_ff][T] f32 (ffn)
+  size_t parts2 = 0;          // down-projection partials (ffn)
+  size_t xs_bf16 = 0;         // [T, d_in] bf16 (prefill)
+  size_t alpha_parts = 0;     // f64 partial sums (ternary pack)
+  size_t alpha = 0;           // f32 (ternary pack)
+  size_t total = 0;
+  size_t parts1_elems = 0, parts2_elems = 0;
+  int ticket_topk_x = 0, ticket_topk_h = 0, ticket_g1 = 0, ticket_g2 = 0, ticket_alpha = 0;
+};
+
+// Returns false if the sizes are invalid for `op`.
+bool ws_layout(int op, int T, int d_in, int d_out, int k, WsLayout* L);
+
+// ---------------------------------------------------------------------------
+// kernel launchers (host functions, defined next to their kernels)
+// ---------------------------------------------------------------------------
+enum TopkKind { TK_F32 = 0, TK_BF16 = 1, TK_QUANT_F32 = 2, TK_QUANT_BF16 = 3 };
+
+struct TopkArgs {
+  const void* x = nullptr;   // [T, d] input (f32 / bf16)
+  int T = 0, d = 0, k = 0;
+  int kind = TK_F32;
+  // optional outputs
+  int32_t* idx = nullptr;    // [T, k]
+  void* val = nullptr;       // [T, k] in the input dtype
+  uint8_t* mask = nullptr;   // [T, d]
+  void* xs = nullptr;        // [T, d] input dtype, masked
+  float* xsf = nullptr;      // [T, d] f32, masked (gemv input)
+  int8_t* xq = nullptr;      // [T, d] int8, masked q (quant gemv input)
+  int8_t* q_full = nullptr;  // [T, d] int8, all q (quant path debug output)
+  float* gamma = nullptr;    // [T] (quant path)
+  float eps = 0.f;           // (quant path)
+  int32_t* list = nullptr;   // [d] union of rows with a kept nonzero
+  float* list_val = nullptr; // [d][T] f32 values of the listed rows (projection input)
+  int8_t* list_q = nullptr;  // [d][T] int8 codes of the listed rows (quant path)
+  int32_t* list_count = nullptr;
+  int32_t* ticket = nullptr;
+  float* zero = nullptr;     // accumulators of the next kernel: set to 0 here
+  size_t zero_n = 0;         // floats, multiple of 4
+  DevStatus* status = nullptr;
+};
+
+cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s);
+
+// Zero `n` floats (n % 4 == 0) cooperatively across the whole grid.
+__device__ __forceinline__ void grid_zero(float* p, size_t n) {
+  if (p == nullptr) return;
+  const size_t nthr = (size_t)gridDim.x * gridDim.y * gridDim.z * blockDim.x;
+  const size_t cta = ((size_t)blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x;
+  const float4 z = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+  for (size_t i = cta * blockDim.x + threadIdx.x; i < n / 4; i += nthr)
+    reinterpret_cast<float4*>(p)[i] = z;
+}
+
+struct GemvArgs {
+  const void* w[2] = {nullptr, nullptr};  // W^T [d_in, d_out]
+  int d_in = 0, d_out = 0, T = 0;
+  int bf16 = 1;               // weight / output element type
+  int mode = 0;               // 0 plain, 1 relu2-glu, 2 drelu
+  const int32_t* list = nullptr;      // rows to stream
+  const float* list_val = nullptr;    // [n][T] their per-token values
+  const int32_t* list_count = nullptr;
+  float* parts = nullptr;
+  int32_t* tickets = nullptr;
+  void* y = nullptr;          // mode 0: [T, d_out] in the weight dtype
+  float* h = nullptr;         // mode 1/2: [T, d_out] f32
+  const float* b_up = nullptr;
+  const float* b_gate = nullptr;
+  float* zero = nullptr;       // accumulators of the next kernel: set to 0 here
+  size_t zero_n = 0;
+  DevStatus* status = nullptr;
+  GemvPlan plan{};
+};
+
+cudaError_t launch_gemv(const GemvArgs& a, cudaStream_t s);
+
+struct QGemvArgs {
+  const uint32_t* wp = nullptr;  // [d_in, d_out/16]
+  int d_in = 0, d_out = 0, T = 0;
+  const float* gamma = nullptr;  // [T]
+  float alpha = 0.f;
+  const int32_t* list = nullptr;
+  const int8_t* list_q = nullptr;  // [n][T] int8 codes of the listed rows
+  const int32_t* list_count = nullptr;
+  int32_t* parts = nullptr;
+  int32_t* tickets = nullptr;
+  float* y = nullptr;
+  int32_t* acc = nullptr;
+  DevStatus* status = nullptr;
+  GemvPlan plan{};
+};
+
+cudaError_t launch_qgemv(const QGemvArgs& a, cudaStream_t s);
+
+struct PackArgs {
+  const float* w = nullptr;  // [d_out, d_in]
+  int d_out = 0, d_in = 0;
+  float eps = 0.f;
+  uint32_t* packed = nullptr;
+  float* alpha_out = nullptr;
+  double* alpha_parts = nullptr;
+  float* alpha_ws = nullptr;
+  int32_t* ticket = nullptr;
+  DevStatus* status = nullptr;
+};
+
+constexpr int kPackSumBlocks = 592;   // fixed: the fp64 sum order does not depend on the GPU
+
+cudaError_t launch_ternary_pack(const PackArgs& a, cudaStream_t s);
+
+struct PrefillArgs {
+  const __nv_bfloat16* xs = nullptr;  // [M, K] masked activations (row-major)
+  const __nv_bfloat16* wt = nullptr;  // [K, N] W^T (row-major)
+  __nv_bfloat16* y = nullptr;         // [M, N]
+  int M = 0, N = 0, K = 0;
+  DevStatus* status = nullptr;
+};
+
+cudaError_t launch_prefill_gemm(const PrefillArgs& a, cudaStream_t s);
+bool prefill_supported(int M, int N, int K);
+
+}  // namespace qs

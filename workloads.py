@@ -183,3 +183,30 @@ def adversarial_rows(seed: int, T: int, d: int) -> np.ndarray:
         x[2, :] = np.float32(0.0)             # all zeros (with -0.0 mixed in)
         x[2, ::3] = np.float32(-0.0)
     return x
+
+
+def ffn_weights_device(w: Workload, layer: int, device, dtype=None):
+    """(W_up^T, W_gate^T, W_down^T) drawn on the device with torch's seeded
+    Philox generator: same distribution as :func:`ffn_weights` (N(0, 1/fan_in),
+    rounded once to the workload dtype), much faster at 7B sizes.  Used by the
+    benchmark, whose inputs do not need to match the numpy draws bit for bit."""
+    import torch
+    if dtype is None:
+        dtype = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    g = torch.Generator(device=device)
+    out = []
+    for j, (d_in, d_out) in enumerate(((w.d_in, w.d_out), (w.d_in, w.d_out), (w.d_out, w.d_in))):
+        g.manual_seed(w.seed(0, 1 + 3 * layer) + 0x1000000 * (j + 1))
+        t = torch.randn(d_in, d_out, generator=g, device=device, dtype=torch.float32)
+        t.mul_(1.0 / math.sqrt(d_in))
+        out.append(t.to(dtype))
+    return tuple(out)
+
+
+def activations_device(w: Workload, T: int, device, salt: int = 0):
+    """x [T, d_in] on the device from the numpy draw of :func:`activations`."""
+    import torch
+    x = torch.from_numpy(activations(w, T, salt))
+    if w.dtype == "bf16":
+        x = x.to(torch.bfloat16)
+    return x.to(device)
