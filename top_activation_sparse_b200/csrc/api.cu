@@ -15,6 +15,10 @@ constexpr size_t kTicketBytes = 64 * 1024;       // fixed ticket region
 constexpr int kTicketCap = (int)(kTicketBytes / sizeof(int32_t));
 // fixed ticket slots
 constexpr int kTkTopkX = 0, kTkTopkH = 1, kTkAlpha = 2, kTkGemv = 8;
+// union bitmasks of the several-token path (zero between calls)
+constexpr int kTkGemvEnd = 4096;
+constexpr int kUnionX = 4096, kUnionH = 4096 + QS_MAX_ROW / 32;
+static_assert(kUnionH + QS_MAX_ROW / 32 <= (int)(64 * 1024 / 4), "ticket region too small");
 
 size_t align_up(size_t v) { return (v + kWsAlign - 1) / kWsAlign * kWsAlign; }
 
@@ -161,7 +165,7 @@ bool valid_dtype(int dt) { return dt == QS_F32 || dt == QS_BF16; }
 
 // A launch plan must fit the buffers the layout reserved for it.
 bool plan_fits(const WsLayout& L, const GemvPlan& p, size_t parts_cap, int ticket_offset) {
-  return p.parts_elems <= parts_cap && kTkGemv + ticket_offset + p.tickets <= L.n_tickets;
+  return p.parts_elems <= parts_cap && kTkGemv + ticket_offset + p.tickets <= kTkGemvEnd;
 }
 
 // Split the gemv ticket slots of one layout: first projection, then second.
@@ -287,9 +291,10 @@ qs_status qs_sparse_linear(const void* x, int dtype, int T, int d_in, int d_out,
     a.kind = dtype == QS_F32 ? TK_F32 : TK_BF16;
     a.xsf = Tc > 1 ? w.at<float>(L.xsf_x) : nullptr;   // only the union pass reads it
     a.list = w.at<int32_t>(L.list_x);
-    a.list_val = w.at<float>(L.lval_x);
+    a.list_val = Tc == 1 ? w.at<float>(L.lval_x) : nullptr;
     a.list_count = w.at<int32_t>(L.cnt) + 0;
     a.ticket = w.ticket(L, kTkTopkX);
+    a.union_bits = reinterpret_cast<uint32_t*>(w.ticket(L, kUnionX));
     a.status = w.status();
     const GemvPlan gp = plan_gemv(Tc, d_out, (int)rows_bound(Tc, d_in, k), 1, eb);
     if (!plan_fits(L, gp, L.parts1_elems, 0)) return QS_ERR_UNSUPPORTED;
@@ -302,7 +307,7 @@ qs_status qs_sparse_linear(const void* x, int dtype, int T, int d_in, int d_out,
     g.d_in = d_in; g.d_out = d_out; g.T = Tc;
     g.bf16 = dtype == QS_BF16;
     g.mode = 0;
-    g.list = a.list; g.list_val = a.list_val; g.list_count = a.list_count;
+    g.list = a.list; g.list_val = a.list_val; g.xsf = a.xsf; g.list_count = a.list_count;
     g.parts = w.at<float>(L.parts1);
     g.plan = gp;
     g.tickets = gemv_tickets(w, L, 0, g.plan);
@@ -354,9 +359,10 @@ qs_status qs_sparse_ffn(const void* x, int dtype, int T, int d_model, int d_ff, 
     a.kind = dtype == QS_F32 ? TK_F32 : TK_BF16;
     a.xsf = Tc > 1 ? w.at<float>(L.xsf_x) : nullptr;
     a.list = w.at<int32_t>(L.list_x);
-    a.list_val = w.at<float>(L.lval_x);
+    a.list_val = Tc == 1 ? w.at<float>(L.lval_x) : nullptr;
     a.list_count = w.at<int32_t>(L.cnt) + 0;
     a.ticket = w.ticket(L, kTkTopkX);
+    a.union_bits = reinterpret_cast<uint32_t*>(w.ticket(L, kUnionX));
     a.status = w.status();
     const GemvPlan p_ug = plan_gemv(Tc, d_ff, (int)rows_bound(Tc, d_model, d_model), 2, eb);
     const GemvPlan p_dn = plan_gemv(Tc, d_model, (int)rows_bound(Tc, d_ff, k_h), 1, eb);
@@ -374,7 +380,7 @@ qs_status qs_sparse_ffn(const void* x, int dtype, int T, int d_model, int d_ff, 
     g.d_in = d_model; g.d_out = d_ff; g.T = Tc;
     g.bf16 = dtype == QS_BF16;
     g.mode = act == QS_ACT_RELU2_GLU ? 1 : 2;
-    g.list = a.list; g.list_val = a.list_val; g.list_count = a.list_count;
+    g.list = a.list; g.list_val = a.list_val; g.xsf = a.xsf; g.list_count = a.list_count;
     g.parts = w.at<float>(L.parts1);
     g.plan = p_ug;
     g.tickets = gemv_tickets(w, L, 0, g.plan);
@@ -391,9 +397,10 @@ qs_status qs_sparse_ffn(const void* x, int dtype, int T, int d_model, int d_ff, 
     b.idx = (idx_h_out && k_h > 0) ? idx_h_out + (size_t)t0 * k_h : nullptr;
     b.xsf = Tc > 1 ? w.at<float>(L.xsf_h) : nullptr;
     b.list = w.at<int32_t>(L.list_h);
-    b.list_val = w.at<float>(L.lval_h);
+    b.list_val = Tc == 1 ? w.at<float>(L.lval_h) : nullptr;
     b.list_count = w.at<int32_t>(L.cnt) + 1;
     b.ticket = w.ticket(L, kTkTopkH);
+    b.union_bits = reinterpret_cast<uint32_t*>(w.ticket(L, kUnionH));
     b.status = w.status();
     QS_TRY_CUDA(launch_topk(b, s));
     if (timed) QS_TRY_CUDA(mark(3));
@@ -404,7 +411,7 @@ qs_status qs_sparse_ffn(const void* x, int dtype, int T, int d_model, int d_ff, 
     dn.d_in = d_ff; dn.d_out = d_model; dn.T = Tc;
     dn.bf16 = dtype == QS_BF16;
     dn.mode = 0;
-    dn.list = b.list; dn.list_val = b.list_val; dn.list_count = b.list_count;
+    dn.list = b.list; dn.list_val = b.list_val; dn.xsf = b.xsf; dn.list_count = b.list_count;
     dn.parts = w.at<float>(L.parts2);
     dn.plan = p_dn;
     dn.tickets = gemv_tickets(w, L, 1, g.plan);
@@ -445,16 +452,17 @@ qs_status qs_quant_sparse_linear(const void* x, int dtype, int T, int d_in, int 
     a.xq = Tc > 1 ? w.at<int8_t>(L.xq) : nullptr;     // only the union pass reads it
     a.gamma = w.at<float>(L.gamma);
     a.list = w.at<int32_t>(L.list_x);
-    a.list_q = w.at<int8_t>(L.lval_x);
+    a.list_q = Tc == 1 ? w.at<int8_t>(L.lval_x) : nullptr;
     a.list_count = w.at<int32_t>(L.cnt) + 0;
     a.ticket = w.ticket(L, kTkTopkX);
+    a.union_bits = reinterpret_cast<uint32_t*>(w.ticket(L, kUnionX));
     a.status = w.status();
     QS_TRY_CUDA(launch_topk(a, s));
 
     QGemvArgs g;
     g.wp = wt_packed; g.d_in = d_in; g.d_out = d_out; g.T = Tc;
     g.gamma = a.gamma; g.alpha = alpha;
-    g.list = a.list; g.list_q = a.list_q; g.list_count = a.list_count;
+    g.list = a.list; g.list_q = a.list_q; g.xq = a.xq; g.list_count = a.list_count;
     g.parts = w.at<int32_t>(L.parts1);
     g.plan = plan_qgemv(Tc, d_out, (int)rows_bound(Tc, d_in, k));
     g.tickets = w.ticket(L, kTkGemv);

@@ -215,6 +215,7 @@ struct TopkArgs {
   int8_t* list_q = nullptr;  // [d][T] int8 codes of the listed rows (quant path)
   int32_t* list_count = nullptr;
   int32_t* ticket = nullptr;
+  uint32_t* union_bits = nullptr;  // [ceil(d/32)] zero between calls (several tokens)
   float* zero = nullptr;     // accumulators of the next kernel: set to 0 here
   size_t zero_n = 0;         // floats, multiple of 4
   DevStatus* status = nullptr;
@@ -238,7 +239,8 @@ struct GemvArgs {
   int bf16 = 1;               // weight / output element type
   int mode = 0;               // 0 plain, 1 relu2-glu, 2 drelu
   const int32_t* list = nullptr;      // rows to stream
-  const float* list_val = nullptr;    // [n][T] their per-token values
+  const float* list_val = nullptr;    // [n][T] their per-token values (one token), or
+  const float* xsf = nullptr;         // [T][d_in] dense masked values (several tokens)
   const int32_t* list_count = nullptr;
   float* parts = nullptr;
   int32_t* tickets = nullptr;
@@ -260,7 +262,8 @@ struct QGemvArgs {
   const float* gamma = nullptr;  // [T]
   float alpha = 0.f;
   const int32_t* list = nullptr;
-  const int8_t* list_q = nullptr;  // [n][T] int8 codes of the listed rows
+  const int8_t* list_q = nullptr;  // [n][T] int8 codes of the listed rows (one token), or
+  const int8_t* xq = nullptr;      // [T][d_in] dense masked codes (several tokens)
   const int32_t* list_count = nullptr;
   int32_t* parts = nullptr;
   int32_t* tickets = nullptr;

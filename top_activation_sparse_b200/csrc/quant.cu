@@ -70,9 +70,15 @@ __global__ void __launch_bounds__(kNT) qgemv_kernel(QGemvArgs a) {
         r = 0;
       }
       s_rows[j] = r;
-      const int8_t* lq = a.list_q + (size_t)(pb + j) * a.T + tok0;
+      if (a.list_q) {
+        const int8_t* lq = a.list_q + (size_t)(pb + j) * a.T + tok0;
 #pragma unroll
-      for (int t = 0; t < TT; ++t) s_q[t][j] = (ok && t < ntok) ? (int)lq[t] : 0;
+        for (int t = 0; t < TT; ++t) s_q[t][j] = (ok && t < ntok) ? (int)lq[t] : 0;
+      } else {
+#pragma unroll
+        for (int t = 0; t < TT; ++t)
+          s_q[t][j] = (ok && t < ntok) ? (int)a.xq[(size_t)(tok0 + t) * d_in + r] : 0;
+      }
     }
     __syncthreads();
     for (int j0 = warp * U; j0 < np; j0 += kNW * U) {

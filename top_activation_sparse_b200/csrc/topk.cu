@@ -321,16 +321,27 @@ __global__ void __launch_bounds__(NT) topk_kernel(TopkArgs a) {
     *a.list_count = tot_gt + (P != 0u ? min(tot_eq, remaining) : (int)t_eqnz);
   }
   __syncthreads();
-  for (int i = tid; i < d; i += NT) {            // coalesced dense outputs
-    const uint32_t ent = s_ent[i];
-    if constexpr (QUANT) {
-      if (a.xq) a.xq[rbase + i] = (int8_t)(ent >> 8);
-    } else {
-      if (a.xsf) a.xsf[rbase + i] = raw_to_f32<KIND>(ent);
-      if (a.xs) {
-        if constexpr (KIND == TK_F32) reinterpret_cast<uint32_t*>(a.xs)[rbase + i] = ent;
-        else reinterpret_cast<uint16_t*>(a.xs)[rbase + i] = (uint16_t)ent;
+  // coalesced dense outputs; with several tokens also OR this row's kept
+  // nonzeros into the union bitmask (one atomic per 32 inputs)
+  const bool want_union = (a.list != nullptr) && (a.T > 1);
+  for (int base = 0; base < d; base += NT) {
+    const int i = base + tid;
+    const bool valid = i < d;
+    const uint32_t ent = valid ? s_ent[i] : 0u;
+    if (valid) {
+      if constexpr (QUANT) {
+        if (a.xq) a.xq[rbase + i] = (int8_t)(ent >> 8);
+      } else {
+        if (a.xsf) a.xsf[rbase + i] = raw_to_f32<KIND>(ent);
+        if (a.xs) {
+          if constexpr (KIND == TK_F32) reinterpret_cast<uint32_t*>(a.xs)[rbase + i] = ent;
+          else reinterpret_cast<uint16_t*>(a.xs)[rbase + i] = (uint16_t)ent;
+        }
       }
+    }
+    if (want_union) {
+      const unsigned b = __ballot_sync(kFull, valid && (ent & MASK) != 0u);
+      if (lane == 0 && b != 0u) atomicOr(a.union_bits + (base + warp * 32) / 32, b);
     }
   }
 
@@ -342,39 +353,24 @@ __global__ void __launch_bounds__(NT) topk_kernel(TopkArgs a) {
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-    // (a) coalesced: mark inputs kept with a nonzero value by any token
-    //     (s_ent is free after the dense outputs above)
-    for (int i = tid; i < d; i += NT) {
-      bool nz = false;
-#pragma unroll 8
-      for (int t = 0; t < a.T; ++t) {
-        const size_t o = (size_t)t * (size_t)d + (size_t)i;
-        if constexpr (QUANT) nz |= (__ldcg(a.xq + o) != 0);
-        else nz |= (__ldcg(a.xsf + o) != 0.0f);
-      }
-      s_ent[i] = nz ? 1u : 0u;
-    }
-    __syncthreads();
-    // (b) chunked: list positions in index order, with the rows' values
+    // list the set bits in index order: a contiguous run of words per thread
+    const int nwords = (d + 31) / 32;
+    const int wpt = (nwords + NT - 1) / NT;
+    const int w0 = min(tid * wpt, nwords);
+    const int w1 = min(w0 + wpt, nwords);
     uint32_t n_any = 0;
-    for (int i = i0; i < i1; ++i) n_any += s_ent[i];
+    for (int w = w0; w < w1; ++w) n_any += __popc(__ldcg(a.union_bits + w));
     uint32_t e_any, e_unused, t_any, t_unused;
     block_scan2<NT>(n_any, 0u, s_scan[sbuf], e_any, e_unused, t_any, t_unused);
     int pos = (int)e_any;
-    for (int i = i0; i < i1; ++i) {
-      if (!s_ent[i]) continue;
-      a.list[pos] = i;
-#pragma unroll 8
-      for (int t = 0; t < a.T; ++t) {
-        const size_t o = (size_t)t * (size_t)d + (size_t)i;
-        const size_t lo = (size_t)pos * a.T + t;
-        if constexpr (QUANT) {
-          if (a.list_q) a.list_q[lo] = __ldcg(a.xq + o);
-        } else {
-          if (a.list_val) a.list_val[lo] = __ldcg(a.xsf + o);
-        }
+    for (int w = w0; w < w1; ++w) {
+      uint32_t bits = __ldcg(a.union_bits + w);
+      a.union_bits[w] = 0u;                      // leave the bitmask clean for the next call
+      while (bits) {
+        const int bpos = __ffs(bits) - 1;
+        a.list[pos++] = w * 32 + bpos;
+        bits &= bits - 1u;
       }
-      ++pos;
     }
     if (tid == 0) {
       *a.list_count = (int)t_any;
