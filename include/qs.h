@@ -227,6 +227,36 @@ qs_status qs_workspace_stats(const void* ws, int op, int T, int d_in, int d_out,
 /* Human-readable name of a status code (static string). */
 const char* qs_status_string(int status);
 
+/* Size of the fixed device scratch array behind qs_sparse_linear_noalloc. */
+#define QS_NOALLOC_SCRATCH_BYTES (4u << 20)
+
+/*
+ * qs_sparse_linear_noalloc -- qs_sparse_linear without a caller workspace.
+ *   The pages have no counterpart to this: it exists for callers that may not
+ *   allocate device memory (an op slot inside a framework that owns every
+ *   allocation, a service that freezes its memory after start-up, a plugin
+ *   without access to the host process's allocator).  Arguments and results
+ *   are those of qs_sparse_linear; the scratch space comes from one
+ *   QS_NOALLOC_SCRATCH_BYTES array built into the library, which every GPU
+ *   that loads the library holds until the process exits.
+ *
+ *   - Nothing is allocated or freed, by this call or by anything it calls.
+ *   - The first call on a device looks the array's address up for that device
+ *     (cudaGetSymbolAddress), so make that first call before any stream
+ *     capture.
+ *   - Each call first clears the array's status word and counters on `stream`
+ *     (cudaMemsetAsync); the rest of the array is rewritten before it is read.
+ *   - All calls share the array: calls whose kernels can overlap on the GPU
+ *     (different streams without ordering) race and give wrong results.
+ *   - Errors: as qs_sparse_linear, plus QS_ERR_UNSUPPORTED when these sizes
+ *     need more than QS_NOALLOC_SCRATCH_BYTES of scratch (that is,
+ *     qs_workspace_size(QS_OP_SPARSE_LINEAR, T, d_in, d_out, k) is larger),
+ *     returned before anything is enqueued.  qs_device_status is not
+ *     available for this entry point's scratch.
+ */
+qs_status qs_sparse_linear_noalloc(const void* x, int dtype, int T, int d_in, int d_out, int k,
+                                   const void* wt, void* y, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

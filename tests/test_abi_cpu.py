@@ -108,3 +108,12 @@ def test_python_binding_refuses_cpu_tensors(L):
     x = torch.zeros(1, 8)
     with pytest.raises(ValueError):
         qs.qs_topk_mask(x, 2)
+
+
+def test_noalloc_entry_point_checks_sizes_on_the_host(L):
+    # rejected before any CUDA call: works without a device
+    big = (64, 16384, 16384, 8192)
+    assert qs.qs_workspace_size(qs.QS_OP_SPARSE_LINEAR, *big) > qs.QS_NOALLOC_SCRATCH_BYTES
+    assert L.qs_sparse_linear_noalloc(_p(FAKE), 0, *big, _p(FAKE), _p(FAKE), None) == qs.QS_ERR_UNSUPPORTED
+    assert L.qs_sparse_linear_noalloc(None, 0, 1, 8, 8, 4, _p(FAKE), _p(FAKE), None) == qs.QS_ERR_INVALID_ARG
+    assert L.qs_sparse_linear_noalloc(_p(FAKE), 0, 1, 8, 8, 9, _p(FAKE), _p(FAKE), None) == qs.QS_ERR_INVALID_ARG

@@ -42,6 +42,7 @@ QS_OP_QUANT_SPARSE_LINEAR = 3
 QS_OP_TERNARY_PACK = 4
 
 QS_MAX_ROW = 49152
+QS_NOALLOC_SCRATCH_BYTES = 4 << 20
 QS_PREFILL_MIN_T = 64
 QS_FFN_PHASE_EVENTS = 5
 
@@ -72,6 +73,7 @@ _SIGNATURES = {
     "qs_device_status": (_i, [_vp, _vp]),
     "qs_workspace_stats": (_i, [_vp, _i, _i, _i, _i, _i, _vp, _vp]),
     "qs_status_string": (ctypes.c_char_p, [_i]),
+    "qs_sparse_linear_noalloc": (_i, [_vp, _i, _i, _i, _i, _i, _vp, _vp, _vp]),
 }
 
 _lib = None
@@ -241,6 +243,25 @@ def qs_sparse_linear(x: torch.Tensor, wt: torch.Tensor, k: int, y=None, ws=None,
     _check("qs_sparse_linear", lib().qs_sparse_linear(
         x.data_ptr(), _dtype_code(x), T, d_in, d_out, k, wt.data_ptr(), y.data_ptr(),
         ws.data_ptr(), ws.numel(), _stream_ptr(stream)))
+    return y
+
+
+def qs_sparse_linear_noalloc(x: torch.Tensor, wt: torch.Tensor, k: int, y=None,
+                             stream=None) -> torch.Tensor:
+    """qs_sparse_linear for callers that cannot allocate device memory: the
+    scratch comes from a fixed array inside the library (all calls share it;
+    calls that overlap on the GPU race).  y must be passed in by such callers;
+    if it is omitted it is allocated here, for convenience only."""
+    dev = _need_cuda(x, wt)
+    T, d_in = x.shape
+    d_out = wt.shape[1]
+    if wt.shape[0] != d_in or wt.dtype != x.dtype:
+        raise ValueError("wt must be [d_in, d_out] with x's dtype")
+    y = _out(y if y is not None else True, (T, d_out), x.dtype, dev)
+    _need_cuda(y)
+    _check("qs_sparse_linear_noalloc", lib().qs_sparse_linear_noalloc(
+        x.data_ptr(), _dtype_code(x), T, d_in, d_out, k, wt.data_ptr(), y.data_ptr(),
+        _stream_ptr(stream)))
     return y
 
 
