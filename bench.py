@@ -51,9 +51,11 @@ def parse_args(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=30000)
     ap.add_argument("--warmup", type=int, default=300)
-    ap.add_argument("--batch", type=int, default=1, help="tokens per step (per GPU)")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="tokens per step per GPU (default: 1 for decode workloads, the "
+                         "workload's own token count otherwise)")
     ap.add_argument("--workload", default="ffn_relu2_llama7b",
-                    choices=["ffn_relu2_llama7b", "ffn_drelu_mistral7b"])
+                    choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--layers", type=int, default=0,
                     help="independent layers to rotate over (0: enough to exceed 4x L2)")
@@ -61,6 +63,9 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-seconds", type=float, default=120.0)
     a = ap.parse_args(argv)
+    if a.batch <= 0:
+        w = workloads.WORKLOADS[a.workload]
+        a.batch = 1 if w.kind in ("ffn", "quant") else w.batches[0]
     if a.warmup < 3:
         ap.error("--warmup must be >= 3")
     if a.steps < 1:
@@ -182,19 +187,25 @@ def load_peaks() -> dict:
     return {"hbm_gbs": 6650.0, "source": "fallback", "bf16_tflops": 1590.0}
 
 
-def kernel_source_digest() -> str:
+KERNEL_SOURCES = {"gemv": "gemv.cu", "prefill": "prefill_gemm.cu", "qgemv": "quant.cu"}
+
+
+def kernel_source_digest(profile: str) -> str:
+    """Digest of the dominant kernel's source (its .cu and the shared header)."""
     import hashlib
     h = hashlib.sha256()
-    for name in ("gemv.cu", "qs_internal.cuh"):
+    main = KERNEL_SOURCES[profile.split("_")[0]]
+    for name in (main, "qs_internal.cuh"):
         with open(os.path.join(ROOT, "top_activation_sparse_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload: str, batch: int) -> float | None:
-    """DRAM bytes per launch of the up/gate kernel from the committed ncu
-    summary, if it was taken on the current kernel source; else None."""
-    p = os.path.join(ROOT, "profiles", f"gemv_upgate_{workload}_T{batch}.md")
+def profiled_traffic(profile: str) -> float | None:
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    summary profiles/<profile>.md, if it was taken on the current kernel
+    source; else None."""
+    p = os.path.join(ROOT, "profiles", f"{profile}.md")
     if not os.path.exists(p):
         return None
     vals = {}
@@ -203,7 +214,7 @@ def profiled_traffic(workload: str, batch: int) -> float | None:
             if ln.startswith("- ") and ":" in ln:
                 k, v = ln[2:].split(":", 1)
                 vals[k.strip()] = v.strip().strip("`")
-    if vals.get("source_digest") != kernel_source_digest():
+    if vals.get("source_digest") != kernel_source_digest(profile):
         return None
     try:
         return float(vals["dram_bytes_per_launch"])
@@ -212,6 +223,214 @@ def profiled_traffic(workload: str, batch: int) -> float | None:
 
 
 # ---------------------------------------------------------------- our arm
+
+def _mk_events(torch, stream, n):
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+    for e in evs:
+        e.record(stream)              # torch creates the CUDA event on its first record
+    return evs, (ctypes.c_void_p * n)(*[e.cuda_event for e in evs])
+
+
+def setup_ffn(args, qs, torch, device, stream, rank):
+    """One sparse FFN layer per step, rotating over independent layers."""
+    w = workloads.WORKLOADS[args.workload]
+    T = args.batch
+    d_model, d_ff, k_in, k_h = w.d_in, w.d_out, w.k, w.k_h
+    act = qs.QS_ACT_RELU2_GLU if w.act == "relu2_glu" else qs.QS_ACT_DRELU
+    layer_bytes = 3 * d_model * d_ff * 2
+    n_layers = args.layers or max(2, math.ceil(4 * L2_BYTES / layer_bytes))
+    layers = [workloads.ffn_weights_device(w, l, device) for l in range(n_layers)]
+    bias = None
+    if w.bias is not None:
+        bias = torch.full((d_ff,), float(w.bias), dtype=torch.float32, device=device)
+    x = workloads.activations_device(w, T, device, salt=rank)
+    y = torch.empty(T, d_model, dtype=torch.bfloat16, device=device)
+    ws = qs.new_workspace(qs.QS_OP_SPARSE_FFN, T, d_model, d_ff, k_h, device)
+    sp = stream.cuda_stream
+    bptr = bias.data_ptr() if bias is not None else None
+    fn = qs.lib().qs_sparse_ffn
+
+    def c_args(l, ev, kx=k_in, kh=k_h):
+        up, gate, down = layers[l]
+        return (x.data_ptr(), qs.QS_BF16, T, d_model, d_ff, act, kx, kh, up.data_ptr(),
+                gate.data_ptr(), bptr, bptr, down.data_ptr(), y.data_ptr(), None, None, ev,
+                ws.data_ptr(), ws.numel(), sp)
+
+    rows = []
+    for l in range(n_layers):
+        st = fn(*c_args(l, None))
+        assert st == 0, qs.qs_status_string(st)
+        rows.append(qs.qs_workspace_stats(ws, qs.QS_OP_SPARSE_FFN, T, d_model, d_ff, k_h))
+    assert qs.qs_device_status(ws) == qs.QS_OK
+    rows_x = float(np.mean([r[0] for r in rows]))
+    rows_h = float(np.mean([r[1] for r in rows]))
+    # algorithmic bytes of the up/gate kernel per launch: the kept rows of
+    # W_up^T and W_gate^T, the staged (index, T values) entries, h written (f32)
+    upgate_bytes = rows_x * d_ff * 2 * 2 + rows_x * (4 + 4 * T) + T * d_ff * 4
+    down_bytes = rows_h * d_model * 2 + rows_h * (4 + 4 * T) + T * d_model * 2
+    topk_bytes = T * d_model * 2 + T * d_ff * 4
+    lw = layers
+
+    def e2e_call(i, x_dev, y_dev):
+        up, gate, down = lw[i % n_layers]
+        qs.qs_sparse_ffn(x_dev, up, gate, down, w.act, k_in, k_h, b_up=bias, b_gate=bias, y=y_dev,
+                         ws=ws)
+
+    def cpu_rate():
+        up, gate, down = (t.float().cpu().numpy() for t in layers[0])
+        return cpu_oracle_ffn(w, x.float().cpu().numpy(), up, gate, down, args.cpu_seconds)
+
+    phases = ["topk_x", "upgate", "topk_h", "down"]
+    return {
+        "fn": fn, "T": T, "n_layers": n_layers, "ws": ws, "x": x, "y": y,
+        "args": lambda l, ev: c_args(l, ev), "n_events": qs.QS_FFN_PHASE_EVENTS,
+        "dense_args": (lambda l: c_args(l, None, d_model, d_ff)),
+        "phases": phases, "dominant": "upgate",
+        "kernel": "gemv_kernel (up/gate gather-GEMV with the gating epilogue)",
+        "bound": "hbm", "dom_work": upgate_bytes, "layer_work": upgate_bytes + down_bytes + topk_bytes,
+        "extra": {"rows_streamed": {"x": rows_x, "h": rows_h}},
+        "desc": (f"{args.workload}: sparse FFN decode layer, d_model={d_model}, d_ff={d_ff}, "
+                 f"act={w.act}, K_x={k_in}, K_h={k_h}, bf16"),
+        "l2": (f"inputs larger than L2: {n_layers} independent layers "
+               f"({n_layers * layer_bytes / 1e9:.2f} GB of weights) rotated per step"),
+        "e2e_call": e2e_call, "cpu_rate": cpu_rate, "launches": 4, "dtype": "bf16",
+        "profile": f"gemv_upgate_{args.workload}_T{T}",
+    }
+
+
+def setup_linear(args, qs, torch, device, stream, rank):
+    """One sparse projection per step (prefill GEMM for >= 64 bf16 tokens)."""
+    w = workloads.WORKLOADS[args.workload]
+    T = args.batch
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    eb = 2 if w.dtype == "bf16" else 4
+    wbytes = w.d_in * w.d_out * eb
+    n_layers = args.layers or max(2, math.ceil(2 * L2_BYTES / wbytes))
+    g = torch.Generator(device=device)
+    wts = []
+    for l in range(n_layers):
+        g.manual_seed(w.seed(0, 1 + l))
+        t = torch.randn(w.d_in, w.d_out, generator=g, device=device) * (w.d_in ** -0.5)
+        wts.append(t.to(tdt))
+    x = workloads.activations_device(w, T, device, salt=rank)
+    y = torch.empty(T, w.d_out, dtype=tdt, device=device)
+    ws = qs.new_workspace(qs.QS_OP_SPARSE_LINEAR, T, w.d_in, w.d_out, w.k, device)
+    sp = stream.cuda_stream
+    fn = qs.lib().qs_sparse_linear
+    dt = qs.QS_BF16 if w.dtype == "bf16" else qs.QS_F32
+
+    def c_args(l, ev, k=w.k):
+        return (x.data_ptr(), dt, T, w.d_in, w.d_out, k, wts[l].data_ptr(), y.data_ptr(), ev,
+                ws.data_ptr(), ws.numel(), sp)
+
+    assert fn(*c_args(0, None)) == 0
+    prefill = (w.dtype == "bf16" and T >= qs.QS_PREFILL_MIN_T)
+    if prefill:
+        # tensor-core bound: algorithmic FLOPs (kept inputs only) per launch
+        work = 2.0 * T * w.k * w.d_out
+        extra = {"executed_flops": 2.0 * T * w.d_in * w.d_out}
+        bound, kernel = "tensor", "prefill_gemm_kernel (tcgen05 masked-dense GEMM)"
+    else:
+        rows, _ = qs.qs_workspace_stats(ws, qs.QS_OP_SPARSE_LINEAR, T, w.d_in, w.d_out, w.k)
+        work = rows * w.d_out * eb + rows * (4 + 4 * T) + T * w.d_out * eb
+        extra = {"rows_streamed": rows}
+        bound, kernel = "hbm", "gemv_kernel (gather-GEMV)"
+
+    def e2e_call(i, x_dev, y_dev):
+        qs.qs_sparse_linear(x_dev, wts[i % n_layers], w.k, y=y_dev, ws=ws)
+
+    def cpu_rate():
+        import oracle
+        xs = x.float().cpu().numpy()
+        wt0 = wts[0].float().cpu().numpy()
+        rows_n = min(T, 8)
+        t0 = time.perf_counter()
+        n = 0
+        while n < 2 or time.perf_counter() - t0 < args.cpu_seconds:
+            oracle.sparse_linear(xs[:rows_n], wt0, w.k)
+            n += 1
+        dt_ = time.perf_counter() - t0
+        return {"value": round(n * rows_n / dt_, 3), "unit": UNIT, "cores": _threads_in_use(),
+                "kind": "oracle", "sample": f"{n} oracle calls of {rows_n} token(s), {dt_:.1f} s"}
+
+    return {
+        "fn": fn, "T": T, "n_layers": n_layers, "ws": ws, "x": x, "y": y,
+        "args": c_args, "n_events": qs.QS_LINEAR_PHASE_EVENTS,
+        "dense_args": (lambda l: c_args(l, None, w.d_in)),
+        "phases": ["topk", "projection"], "dominant": "projection", "kernel": kernel,
+        "bound": bound, "dom_work": work, "layer_work": work, "extra": extra,
+        "desc": (f"{args.workload}: sparse linear, T={T}, {w.d_in}->{w.d_out}, K={w.k}, "
+                 f"{w.dtype}"),
+        "l2": f"inputs larger than L2: {n_layers} weight copies ({n_layers * wbytes / 1e9:.2f} GB) rotated",
+        "e2e_call": e2e_call, "cpu_rate": cpu_rate, "launches": 2, "dtype": w.dtype,
+        "profile": f"{'prefill_gemm' if prefill else 'gemv'}_{args.workload}_T{T}",
+    }
+
+
+def setup_quant(args, qs, torch, device, stream, rank):
+    """BitNet b1.58 + Q-Sparse projection per step (int8 x packed ternary)."""
+    w = workloads.WORKLOADS[args.workload]
+    T = args.batch
+    n_words = w.d_out // 16
+    wbytes = w.d_in * n_words * 4
+    n_layers = args.layers or max(2, math.ceil(2 * L2_BYTES / wbytes))
+    g = torch.Generator(device=device)
+    packs, alphas = [], []
+    wsp = qs.new_workspace(qs.QS_OP_TERNARY_PACK, 0, w.d_in, w.d_out, 0, device)
+    for l in range(n_layers):
+        g.manual_seed(w.seed(0, 1 + l))
+        wf = torch.randn(w.d_out, w.d_in, generator=g, device=device) * (w.d_in ** -0.5)
+        p, a = qs.qs_ternary_pack(wf, 1e-5, ws=wsp)
+        packs.append(p)
+        alphas.append(float(a.item()))
+        del wf
+    x = workloads.activations_device(w, T, device, salt=rank)
+    y = torch.empty(T, w.d_out, dtype=torch.float32, device=device)
+    ws = qs.new_workspace(qs.QS_OP_QUANT_SPARSE_LINEAR, T, w.d_in, w.d_out, w.k, device)
+    sp = stream.cuda_stream
+    fn = qs.lib().qs_quant_sparse_linear
+
+    def c_args(l, ev, k=w.k):
+        return (x.data_ptr(), qs.QS_BF16, T, w.d_in, w.d_out, k, packs[l].data_ptr(),
+                ctypes.c_float(alphas[l]), ctypes.c_float(1e-5), y.data_ptr(), None, None, None, ev,
+                ws.data_ptr(), ws.numel(), sp)
+
+    assert fn(*c_args(0, None)) == 0
+    rows, _ = qs.qs_workspace_stats(ws, qs.QS_OP_QUANT_SPARSE_LINEAR, T, w.d_in, w.d_out, w.k)
+    work = rows * n_words * 4 + rows * (4 + T) + T * w.d_out * 4
+
+    def e2e_call(i, x_dev, y_dev):
+        qs.qs_quant_sparse_linear(x_dev, packs[i % n_layers], alphas[i % n_layers], w.k, y=y_dev,
+                                  ws=ws)
+
+    def cpu_rate():
+        import oracle
+        xs = x.float().cpu().numpy()
+        t = oracle.ternary_unpack(packs[0].cpu().numpy().view(np.uint32), w.d_out)
+        rows_n = min(T, 8)
+        t0 = time.perf_counter()
+        n = 0
+        while n < 2 or time.perf_counter() - t0 < args.cpu_seconds:
+            oracle.quant_sparse_linear(xs[:rows_n], t, alphas[0], w.k)
+            n += 1
+        dt_ = time.perf_counter() - t0
+        return {"value": round(n * rows_n / dt_, 3), "unit": UNIT, "cores": _threads_in_use(),
+                "kind": "oracle", "sample": f"{n} oracle calls of {rows_n} token(s), {dt_:.1f} s"}
+
+    return {
+        "fn": fn, "T": T, "n_layers": n_layers, "ws": ws, "x": x, "y": y,
+        "args": c_args, "n_events": qs.QS_LINEAR_PHASE_EVENTS,
+        "dense_args": (lambda l: c_args(l, None, w.d_in)),
+        "phases": ["quant_topk", "projection"], "dominant": "projection",
+        "kernel": "qgemv_kernel (int8 x ternary gather)", "bound": "hbm", "dom_work": work,
+        "layer_work": work, "extra": {"rows_streamed": rows},
+        "desc": (f"{args.workload}: int8 x ternary sparse projection, T={T}, {w.d_in}->{w.d_out}, "
+                 f"K={w.k}, packed 2-bit weights"),
+        "l2": f"inputs larger than L2: {n_layers} packed weight copies ({n_layers * wbytes / 1e9:.2f} GB) rotated",
+        "e2e_call": e2e_call, "cpu_rate": cpu_rate, "launches": 2, "dtype": "int8",
+        "profile": f"qgemv_{args.workload}_T{T}",
+    }
+
 
 def run_ours(args, rank, world, local):
     import torch
@@ -227,59 +446,26 @@ def run_ours(args, rank, world, local):
         qs_build.build()
     if dist is not None:
         dist.barrier()
-    L = qs.lib()
-
-    w = workloads.WORKLOADS[args.workload]
-    T = args.batch
-    d_model, d_ff, k_in, k_h = w.d_in, w.d_out, w.k, w.k_h
-    act = qs.QS_ACT_RELU2_GLU if w.act == "relu2_glu" else qs.QS_ACT_DRELU
-    layer_bytes = 3 * d_model * d_ff * 2
-    n_layers = args.layers or max(2, math.ceil(4 * L2_BYTES / layer_bytes))
-
-    layers = [workloads.ffn_weights_device(w, l, device) for l in range(n_layers)]
-    bias = None
-    if w.bias is not None:
-        bias = torch.full((d_ff,), float(w.bias), dtype=torch.float32, device=device)
-    x = workloads.activations_device(w, T, device, salt=rank)
-    y = torch.empty(T, d_model, dtype=torch.bfloat16, device=device)
-    ws = qs.new_workspace(qs.QS_OP_SPARSE_FFN, T, d_model, d_ff, k_h, device)
+    qs.lib()
     stream = torch.cuda.current_stream(device)
-    sp = stream.cuda_stream
-    bptr = bias.data_ptr() if bias is not None else None
-
-    def c_args(l, ev_arr, kx=k_in, kh=k_h):
-        up, gate, down = layers[l]
-        return (x.data_ptr(), qs.QS_BF16, T, d_model, d_ff, act, kx, kh, up.data_ptr(),
-                gate.data_ptr(), bptr, bptr, down.data_ptr(), y.data_ptr(), None, None, ev_arr,
-                ws.data_ptr(), ws.numel(), sp)
-
-    fn = L.qs_sparse_ffn
-
-    # rows streamed per layer (algorithmic weight traffic)
-    rows = []
-    for l in range(n_layers):
-        st = fn(*c_args(l, None))
-        assert st == 0, qs.qs_status_string(st)
-        rows.append(qs.qs_workspace_stats(ws, qs.QS_OP_SPARSE_FFN, T, d_model, d_ff, k_h))
-    assert qs.qs_device_status(ws) == qs.QS_OK
-
-    # phase events on a sample of the timed steps
-    n_phase = min(args.steps, 256)
-    phase_steps = set(np.linspace(0, args.steps - 1, n_phase).astype(int).tolist())
-    phase_events = {}
-    for i in phase_steps:
-        evs = [torch.cuda.Event(enable_timing=True) for _ in range(qs.QS_FFN_PHASE_EVENTS)]
-        for e in evs:
-            e.record(stream)          # torch creates the CUDA event on first record
-        phase_events[i] = (evs, (ctypes.c_void_p * qs.QS_FFN_PHASE_EVENTS)(*[e.cuda_event for e in evs]))
-    torch.cuda.synchronize()
-    plain = [c_args(l, None) for l in range(n_layers)]
-    timed = {i: c_args(i % n_layers, phase_events[i][1]) for i in phase_steps}
+    kind = workloads.WORKLOADS[args.workload].kind
+    setup = {"ffn": setup_ffn, "linear": setup_linear, "prefill": setup_linear,
+             "quant": setup_quant}[kind]
+    c = setup(args, qs, torch, device, stream, rank)
+    fn, T, n_layers = c["fn"], c["T"], c["n_layers"]
 
     def run(a):
         st = fn(*a)
         if st != 0:
-            raise RuntimeError(f"qs_sparse_ffn: {qs.qs_status_string(st)}")
+            raise RuntimeError(f"{fn.__name__}: {qs.qs_status_string(st)}")
+
+    # phase events on a sample of the timed steps
+    n_phase = min(args.steps, 256)
+    phase_steps = set(np.linspace(0, args.steps - 1, n_phase).astype(int).tolist())
+    ev = {i: _mk_events(torch, stream, c["n_events"]) for i in phase_steps}
+    torch.cuda.synchronize()
+    plain = [c["args"](l, None) for l in range(n_layers)]
+    timed = {i: c["args"](i % n_layers, ev[i][1]) for i in phase_steps}
 
     for i in range(args.warmup):
         run(plain[i % n_layers])
@@ -299,54 +485,51 @@ def run_ours(args, rank, world, local):
         dist.barrier()
     clk = clocks.stop()
     ms = t_start.elapsed_time(t_end)
-    assert qs.qs_device_status(ws) == qs.QS_OK
+    assert qs.qs_device_status(c["ws"]) == qs.QS_OK
     ms_max = max_over_ranks(ms, dist, device)
     tokens = sum_over_ranks(float(T * args.steps), dist, device)
     value = tokens / (ms_max / 1e3)
 
-    # per-phase device time on the sampled steps
-    ph = np.array([[phase_events[i][0][p].elapsed_time(phase_events[i][0][p + 1])
-                    for p in range(4)] for i in sorted(phase_steps)])
-    ph_us = ph.mean(axis=0) * 1e3
-    upgate_us = float(ph_us[1])
-
-    # algorithmic bytes of the dominant kernel (up/gate gather-GEMV) per launch:
-    # kept rows of W_up^T and W_gate^T + the kept (index, T values) entries it
-    # stages + h written (f32).
-    rows_x = float(np.mean([r[0] for r in rows]))
-    rows_h = float(np.mean([r[1] for r in rows]))
-    upgate_bytes = rows_x * d_ff * 2 * 2 + rows_x * (4 + 4 * T) + T * d_ff * 4
-    down_bytes = rows_h * d_model * 2 + rows_h * (4 + 4 * T) + T * d_model * 2
-    topk_bytes = T * d_model * 2 + T * d_ff * 4
-    layer_alg_bytes = upgate_bytes + down_bytes + topk_bytes
+    names = c["phases"]
+    ph = np.array([[ev[i][0][p].elapsed_time(ev[i][0][p + 1]) for p in range(len(names))]
+                   for i in sorted(phase_steps)])
+    ph_us = {n: round(float(v), 3) for n, v in zip(names, ph.mean(axis=0) * 1e3)}
+    dom_us = ph_us[c["dominant"]]
     peaks = load_peaks()
-    achieved = upgate_bytes / (upgate_us * 1e-6) / 1e9
-    layer_gbs = layer_alg_bytes * T * args.steps / T / (ms / 1e3) / 1e9
+    if c["bound"] == "hbm":
+        achieved = c["dom_work"] / (dom_us * 1e-6) / 1e9
+        peak, unit = peaks["hbm_gbs"], "GB/s"
+    else:
+        achieved = c["dom_work"] / (dom_us * 1e-6) / 1e12
+        peak, unit = peaks["bf16_tflops"], "TFLOP/s"
+    step_s = ms / 1e3 / args.steps
 
     # dense run of the same kernels (K = d): context for the sparsity win
-    for i in range(args.warmup):
-        run(c_args(i % n_layers, None, d_model, d_ff))
-    n_dense = max(1, min(args.steps, 2000))
-    torch.cuda.synchronize()
-    d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    dense_args = [c_args(l, None, d_model, d_ff) for l in range(n_layers)]
-    d0.record(stream)
-    for i in range(n_dense):
-        run(dense_args[i % n_layers])
-    d1.record(stream)
-    torch.cuda.synchronize()
-    dense_ms = d0.elapsed_time(d1) / n_dense
+    dense = None
+    if c.get("dense_args") is not None:
+        dargs = [c["dense_args"](l) for l in range(n_layers)]
+        for i in range(args.warmup):
+            run(dargs[i % n_layers])
+        n_dense = max(1, min(args.steps, 2000))
+        torch.cuda.synchronize()
+        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        d0.record(stream)
+        for i in range(n_dense):
+            run(dargs[i % n_layers])
+        d1.record(stream)
+        torch.cuda.synchronize()
+        dense_ms = d0.elapsed_time(d1) / n_dense
+        dense = {"ms_per_step": round(dense_ms, 6), "value": round(T / (dense_ms / 1e3), 1)}
 
-    # end to end through the public Python API with host buffers
+    # end to end through the public Python API, host buffers in and out
+    x, y = c["x"], c["y"]
     x_host = x.cpu().pin_memory()
-    y_host = torch.empty(T, d_model, dtype=torch.bfloat16).pin_memory()
+    y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
     x_dev = torch.empty_like(x)
     n_e2e = max(1, min(args.steps, 5000))
-    lw = [layers[l] for l in range(n_layers)]
     for i in range(args.warmup):
         x_dev.copy_(x_host, non_blocking=True)
-        up, gate, down = lw[i % n_layers]
-        qs.qs_sparse_ffn(x_dev, up, gate, down, w.act, k_in, k_h, b_up=bias, b_gate=bias, y=y, ws=ws)
+        c["e2e_call"](i, x_dev, y)
         y_host.copy_(y, non_blocking=True)
     torch.cuda.synchronize()
     if dist is not None:
@@ -355,8 +538,7 @@ def run_ours(args, rank, world, local):
     e0.record(stream)
     for i in range(n_e2e):
         x_dev.copy_(x_host, non_blocking=True)
-        up, gate, down = lw[i % n_layers]
-        qs.qs_sparse_ffn(x_dev, up, gate, down, w.act, k_in, k_h, b_up=bias, b_gate=bias, y=y, ws=ws)
+        c["e2e_call"](i, x_dev, y)
         y_host.copy_(y, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
@@ -366,10 +548,11 @@ def run_ours(args, rank, world, local):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        up, gate, down = (t.float().cpu().numpy() for t in layers[0])
-        cpu = cpu_oracle_rate(w, x.float().cpu().numpy(), up, gate, down, args.cpu_seconds)
+        cpu = c["cpu_rate"]()
 
-    traffic = profiled_traffic(args.workload, T)
+    chunks = (T + qs.QS_PREFILL_MIN_T - 1) // qs.QS_PREFILL_MIN_T
+    if c["launches"] == 2 and T >= qs.QS_PREFILL_MIN_T:
+        chunks = 1
     result = {
         "metric": METRIC,
         "value": round(value, 1),
@@ -381,44 +564,39 @@ def run_ours(args, rank, world, local):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16",
+        "dtype": c["dtype"],
         "data": "synthetic: x ~ N(0,1), W ~ N(0,1/fan_in) (seeded; random-init weights)",
         "config": {
-            "workload": f"{args.workload}: Q-Sparse FFN decode layer, d_model={d_model}, "
-                        f"d_ff={d_ff}, act={w.act}, K_x={k_in}, K_h={k_h}, bf16",
+            "workload": c["desc"],
             "batch_per_gpu": T,
             "global_batch": T * world,
             "layers_rotated": n_layers,
-            "l2": f"inputs larger than L2: {n_layers} independent layers "
-                  f"({n_layers * layer_bytes / 1e9:.2f} GB of weights) rotated per step",
+            "l2": c["l2"],
             "parallelism": f"replicas x{world} (no data-path collective)",
         },
         "hbm": {
-            "layer_gbs": round(layer_gbs, 1),
-            "layer_alg_bytes": int(layer_alg_bytes),
-            "frac_of_peak": round(layer_gbs / peaks["hbm_gbs"], 4),
-            "rows_streamed": {"x": rows_x, "h": rows_h},
+            "step_alg_gbs": round(c["layer_work"] / step_s / 1e9, 1) if c["bound"] == "hbm" else None,
+            "frac_of_peak": (round(c["layer_work"] / step_s / 1e9 / peaks["hbm_gbs"], 4)
+                             if c["bound"] == "hbm" else None),
+            **c["extra"],
         },
-        "phases_us": {"topk_x": round(float(ph_us[0]), 3), "upgate": round(float(ph_us[1]), 3),
-                      "topk_h": round(float(ph_us[2]), 3), "down": round(float(ph_us[3]), 3)},
+        "phases_us": ph_us,
         "roofline": {
-            "kernel": "gemv_kernel (up/gate gather-GEMV + gating epilogue)",
-            "bound": "hbm",
+            "kernel": c["kernel"],
+            "bound": c["bound"],
             "achieved": round(achieved, 1),
-            "peak": peaks["hbm_gbs"],
+            "peak": peak,
             "peak_source": peaks["source"],
-            "unit": "GB/s",
-            "frac": round(achieved / peaks["hbm_gbs"], 4),
-            "traffic": traffic,
-            "alg_bytes_per_launch": int(upgate_bytes),
+            "unit": unit,
+            "frac": round(achieved / peak, 4),
+            "traffic": profiled_traffic(c["profile"]),
+            "alg_work_per_launch": int(c["dom_work"]),
         },
-        "dense_same_kernels": {"ms_per_step": round(dense_ms, 6),
-                               "value": round(T / (dense_ms / 1e3), 1), "k_x": d_model,
-                               "k_h": d_ff},
+        "dense_same_kernels": dense,
         "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "steps": n_e2e,
                 "h2d_bytes_per_step": int(x.numel() * x.element_size()),
                 "d2h_bytes_per_step": int(y.numel() * y.element_size())},
-        "gpu_launches": 4 * ((T + qs.QS_PREFILL_MIN_T - 1) // qs.QS_PREFILL_MIN_T) * args.steps,
+        "gpu_launches": c["launches"] * chunks * args.steps,
         "clocks": clk,
     }
     if cpu is not None:
@@ -440,7 +618,7 @@ def _threads_in_use() -> int:
         return 1
 
 
-def cpu_oracle_rate(w, x, up, gate, down, seconds: float) -> dict:
+def cpu_oracle_ffn(w, x, up, gate, down, seconds: float) -> dict:
     """Time the oracle as it stands on a bounded sample: whole-layer calls
     for about `seconds` of host time (at least two)."""
     import oracle
@@ -461,15 +639,26 @@ def run_reference(args, rank, world, local):
     """The oracle as the reference arm: rank 0 only, host cores only."""
     if rank != 0:
         return None
+    import oracle
     w = workloads.WORKLOADS[args.workload]
     T = args.batch
     x = workloads.activations(w, T)
-    up, gate, down = workloads.ffn_weights(w)
-    import oracle
-    b = None if w.bias is None else np.full(w.d_out, w.bias)
+    if w.kind == "ffn":
+        up, gate, down = workloads.ffn_weights(w)
+        b = None if w.bias is None else np.full(w.d_out, w.bias)
 
-    def step():
-        oracle.sparse_ffn(x, up, gate, down, w.act, w.k, w.k_h, b_up=b, b_gate=b)
+        def step():
+            oracle.sparse_ffn(x, up, gate, down, w.act, w.k, w.k_h, b_up=b, b_gate=b)
+    elif w.kind == "quant":
+        t, alpha = oracle.ternary_quantize(workloads.weight_out_major(w.d_out, w.d_in, w.seed(0, 1)))
+
+        def step():
+            oracle.quant_sparse_linear(x, t, alpha, w.k)
+    else:
+        wt = workloads.weight_t(w.d_in, w.d_out, w.seed(0, 1), w.dtype)
+
+        def step():
+            oracle.sparse_linear(x, wt, w.k)
 
     t0 = time.perf_counter()
     step()
@@ -484,7 +673,7 @@ def run_reference(args, rank, world, local):
         step()
     dt = time.perf_counter() - t0
     value = n_run * T / dt
-    sample = (f"{n_run} of {args.steps} steps run (each the whole layer for {T} token(s)); "
+    sample = (f"{n_run} of {args.steps} steps run (each the whole workload for {T} token(s)); "
               f"{warm} warm-up; fp64 numpy oracle")
     return {
         "impl": "reference",
@@ -500,7 +689,7 @@ def run_reference(args, rank, world, local):
         "vs_baseline": None,
         "dtype": "f64",
         "data": "synthetic: x ~ N(0,1), W ~ N(0,1/fan_in) (seeded)",
-        "config": {"workload": f"{args.workload} (same layer as --impl ours), CPU oracle",
+        "config": {"workload": f"{args.workload} (same workload as --impl ours), CPU oracle",
                    "batch_per_gpu": T, "global_batch": T, "parallelism": "host cores"},
         "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": _threads_in_use(),
                          "kind": "oracle", "sample": sample},

@@ -87,6 +87,9 @@ typedef enum qs_op {
 #define QS_PREFILL_MIN_T 64
 /* Number of cudaEvent_t handles qs_sparse_ffn records when given phase events. */
 #define QS_FFN_PHASE_EVENTS 5
+/* ... and qs_sparse_linear / qs_quant_sparse_linear (before the top-K, after
+ * the top-K, after the projection; first chunk of QS_PREFILL_MIN_T tokens). */
+#define QS_LINEAR_PHASE_EVENTS 3
 
 /*
  * qs_topk_mask -- top-K on |x| per row, with the mask and the sparsified input.
@@ -120,10 +123,14 @@ qs_status qs_topk_mask(const void* x, int dtype, int T, int d, int k,
  *   wt[i, :] of inputs kept by some token.  Prefill (bf16, T >= QS_PREFILL_MIN_T):
  *   X_sparse is materialised and multiplied on the tensor cores (tcgen05).
  *   d_out must be a multiple of 8 (bf16) or 4 (f32).
+ *   phase_events  NULL, or QS_LINEAR_PHASE_EVENTS cudaEvent_t handles (as void*)
+ *             recorded on `stream` before the top-K, after it, and after the
+ *             projection (timing hook; recording them costs a little).
  *   Errors: INVALID_ARG, ALIGNMENT, WORKSPACE, UNSUPPORTED, CUDA.
  */
 qs_status qs_sparse_linear(const void* x, int dtype, int T, int d_in, int d_out, int k,
-                           const void* wt, void* y, void* ws, size_t ws_bytes, void* stream);
+                           const void* wt, void* y, void* const* phase_events,
+                           void* ws, size_t ws_bytes, void* stream);
 
 /*
  * qs_sparse_ffn -- one sparse gated FFN layer.
@@ -175,12 +182,14 @@ qs_status qs_sparse_ffn(const void* x, int dtype, int T, int d_model, int d_ff, 
  *   y          [T, d_out] f32 out.
  *   acc        [T, d_out] int32 out or NULL.   q  [T, d_in] int8 out or NULL.
  *   idx        [T, k] int32 out or NULL: kept indices, ascending.
+ *   phase_events  NULL or QS_LINEAR_PHASE_EVENTS events (as qs_sparse_linear).
  *   d_out must be a multiple of 16; 127 * d_in < 2^24 keeps float(acc) exact.
  *   Errors: INVALID_ARG, ALIGNMENT, WORKSPACE, UNSUPPORTED, CUDA.
  */
 qs_status qs_quant_sparse_linear(const void* x, int dtype, int T, int d_in, int d_out, int k,
                                  const uint32_t* wt_packed, float alpha, float eps,
                                  float* y, int32_t* acc, int8_t* q, int32_t* idx,
+                                 void* const* phase_events,
                                  void* ws, size_t ws_bytes, void* stream);
 
 /*

@@ -79,10 +79,10 @@ def test_invalid_arguments_are_rejected_on_the_host(L):
     assert L.qs_topk_mask(_p(FAKE), 0, 1, 8, 2, _p(FAKE), None, None, None, ws, 16, s) == qs.QS_ERR_WORKSPACE
     assert L.qs_topk_mask(_p(FAKE), 0, 1, 8, 2, _p(FAKE), None, None, None, None, wsb, s) == qs.QS_ERR_WORKSPACE
     # qs_sparse_linear: d_out not a multiple of the vector width (bf16 needs 8)
-    assert L.qs_sparse_linear(_p(FAKE), 1, 1, 64, 12, 8, _p(FAKE), _p(FAKE), ws, wsb, s) == qs.QS_ERR_ALIGNMENT
-    assert L.qs_sparse_linear(_p(FAKE), 1, 1, 64, 16, 65, _p(FAKE), _p(FAKE), ws, wsb, s) == qs.QS_ERR_INVALID_ARG
-    assert L.qs_sparse_linear(_p(FAKE), 1, 1, 64, 16, -1, _p(FAKE), _p(FAKE), ws, wsb, s) == qs.QS_ERR_INVALID_ARG
-    assert L.qs_sparse_linear(_p(FAKE), 1, 1, 64, 16, 8, None, _p(FAKE), ws, wsb, s) == qs.QS_ERR_INVALID_ARG
+    assert L.qs_sparse_linear(_p(FAKE), 1, 1, 64, 12, 8, _p(FAKE), _p(FAKE), None, ws, wsb, s) == qs.QS_ERR_ALIGNMENT
+    assert L.qs_sparse_linear(_p(FAKE), 1, 1, 64, 16, 65, _p(FAKE), _p(FAKE), None, ws, wsb, s) == qs.QS_ERR_INVALID_ARG
+    assert L.qs_sparse_linear(_p(FAKE), 1, 1, 64, 16, -1, _p(FAKE), _p(FAKE), None, ws, wsb, s) == qs.QS_ERR_INVALID_ARG
+    assert L.qs_sparse_linear(_p(FAKE), 1, 1, 64, 16, 8, None, _p(FAKE), None, ws, wsb, s) == qs.QS_ERR_INVALID_ARG
     # qs_sparse_ffn: bad activation, k_h > d_ff
     args = [_p(FAKE), 1, 1, 64, 128, 0, 32, 64, _p(FAKE), _p(FAKE), None, None, _p(FAKE), _p(FAKE),
             None, None, None, ws, wsb, s]
@@ -94,9 +94,9 @@ def test_invalid_arguments_are_rejected_on_the_host(L):
     assert L.qs_sparse_ffn(*bad) == qs.QS_ERR_ALIGNMENT
     # qs_quant_sparse_linear: d_out % 16, negative eps
     assert L.qs_quant_sparse_linear(_p(FAKE), 1, 1, 64, 40, 8, _p(FAKE), ctypes.c_float(1.0),
-                                    ctypes.c_float(1e-5), _p(FAKE), None, None, None, ws, wsb, s) == qs.QS_ERR_ALIGNMENT
+                                    ctypes.c_float(1e-5), _p(FAKE), None, None, None, None, ws, wsb, s) == qs.QS_ERR_ALIGNMENT
     assert L.qs_quant_sparse_linear(_p(FAKE), 1, 1, 64, 32, 8, _p(FAKE), ctypes.c_float(1.0),
-                                    ctypes.c_float(-1.0), _p(FAKE), None, None, None, ws, wsb, s) == qs.QS_ERR_INVALID_ARG
+                                    ctypes.c_float(-1.0), _p(FAKE), None, None, None, None, ws, wsb, s) == qs.QS_ERR_INVALID_ARG
     # qs_ternary_pack: d_out % 16
     assert L.qs_ternary_pack(_p(FAKE), 24, 8, ctypes.c_float(1e-5), _p(FAKE), None, ws, wsb, s) == qs.QS_ERR_ALIGNMENT
     assert L.qs_workspace_init(None, 16, s) == qs.QS_ERR_INVALID_ARG

@@ -96,3 +96,37 @@ def test_linear_never_reads_unselected_rows(dtype):
     # split sums are added in no fixed order, so compare to rounding only
     tol = 1e-5 if dtype == "f32" else 2 ** -7
     assert oracle.max_rel_err(to_np(y_poison), to_np(y_clean)) <= tol
+
+
+# ---- prefill: bf16 with >= 64 tokens runs the tcgen05 masked-dense GEMM ----
+
+def test_prefill_2048_tokens_outliers():
+    """2048 tokens x 4096 -> 11008, 1% outlier channels x20, K = 2048: rows
+    sampled across all 16 M-blocks checked against the fp64 oracle."""
+    need_gpu()
+    w = workloads.WORKLOADS["prefill_bf16_2048"]
+    x = workloads.activations(w, 2048)
+    wt = workloads.weight_t(w.d_in, w.d_out, w.seed(0, 1), "bf16")
+    y, _ = _run(x, wt, w.k, "bf16")
+    rows = np.arange(0, 2048, 16)
+    ref = oracle.sparse_linear(x[rows], wt, w.k)
+    assert oracle.max_rel_err(to_np(y)[rows], ref) <= TOL_BF16
+
+
+@pytest.mark.parametrize("T,d_in,d_out,k", [
+    (64, 64, 256, 32),        # one k-block, one N tile, M tail (64 < 128)
+    (200, 136, 264, 70),      # K tail (136 = 2 x 64 + 8), N tail (264 = 256 + 8), M tail
+    (130, 4096, 512, 4096),   # dense (K = d_in), M tail of 2 rows
+    (256, 1000, 1024, 1),     # one kept input per token
+    (128, 512, 520, 0),       # K = 0: all zero
+])
+def test_prefill_ragged_tiles(T, d_in, d_out, k):
+    need_gpu()
+    g = workloads.rng(T + d_in + d_out + k)
+    x = workloads.round_to_dtype(workloads.normal_f32(g, (T, d_in)), "bf16")
+    wt = workloads.round_to_dtype(workloads.normal_f32(g, (d_in, d_out), d_in ** -0.5), "bf16")
+    y, _ = _run(x, wt, k, "bf16")
+    if k == 0:
+        assert torch.count_nonzero(y).item() == 0
+        return
+    assert oracle.max_rel_err(to_np(y), oracle.sparse_linear(x, wt, k)) <= TOL_BF16

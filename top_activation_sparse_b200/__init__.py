@@ -45,6 +45,7 @@ QS_MAX_ROW = 49152
 QS_NOALLOC_SCRATCH_BYTES = 4 << 20
 QS_PREFILL_MIN_T = 64
 QS_FFN_PHASE_EVENTS = 5
+QS_LINEAR_PHASE_EVENTS = 3
 
 _ACTS = {"relu2_glu": QS_ACT_RELU2_GLU, "drelu": QS_ACT_DRELU}
 
@@ -62,11 +63,11 @@ _f = ctypes.c_float
 
 _SIGNATURES = {
     "qs_topk_mask": (_i, [_vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
-    "qs_sparse_linear": (_i, [_vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _sz, _vp]),
+    "qs_sparse_linear": (_i, [_vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _sz, _vp]),
     "qs_sparse_ffn": (_i, [_vp, _i, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                            _vp, _vp, _vp, _sz, _vp]),
     "qs_quant_sparse_linear": (_i, [_vp, _i, _i, _i, _i, _i, _vp, _f, _f, _vp, _vp, _vp, _vp,
-                                    _vp, _sz, _vp]),
+                                    _vp, _vp, _sz, _vp]),
     "qs_ternary_pack": (_i, [_vp, _i, _i, _f, _vp, _vp, _vp, _sz, _vp]),
     "qs_workspace_size": (_sz, [_i, _i, _i, _i, _i]),
     "qs_workspace_init": (_i, [_vp, _sz, _vp]),
@@ -229,8 +230,16 @@ def qs_topk_mask(x: torch.Tensor, k: int, idx=True, val=None, mask=None, xs=None
     return TopkResult(idx, val, mask, xs)
 
 
-def qs_sparse_linear(x: torch.Tensor, wt: torch.Tensor, k: int, y=None, ws=None,
-                     stream=None) -> torch.Tensor:
+def _events(phase_events, n):
+    if phase_events is None:
+        return None
+    if len(phase_events) != n:
+        raise ValueError(f"phase_events must hold {n} events")
+    return (ctypes.c_void_p * n)(*[e.cuda_event for e in phase_events])
+
+
+def qs_sparse_linear(x: torch.Tensor, wt: torch.Tensor, k: int, y=None, phase_events=None,
+                     ws=None, stream=None) -> torch.Tensor:
     """Y = (X (.) topK-mask(|X|)) . W^T with wt = W^T [d_in, d_out]."""
     dev = _need_cuda(x, wt)
     T, d_in = x.shape
@@ -242,7 +251,8 @@ def qs_sparse_linear(x: torch.Tensor, wt: torch.Tensor, k: int, y=None, ws=None,
     ws = _workspace(ws, QS_OP_SPARSE_LINEAR, T, d_in, d_out, k, dev)
     _check("qs_sparse_linear", lib().qs_sparse_linear(
         x.data_ptr(), _dtype_code(x), T, d_in, d_out, k, wt.data_ptr(), y.data_ptr(),
-        ws.data_ptr(), ws.numel(), _stream_ptr(stream)))
+        _events(phase_events, QS_LINEAR_PHASE_EVENTS), ws.data_ptr(), ws.numel(),
+        _stream_ptr(stream)))
     return y
 
 
@@ -289,11 +299,7 @@ def qs_sparse_ffn(x, wt_up, wt_gate, wt_down, act, k_in: int, k_h: int, b_up=Non
     h_out = _out(h_out, (T, d_ff), torch.float32, dev)
     idx_h_out = _out(idx_h_out, (T, k_h), torch.int32, dev)
     _need_cuda(y, h_out, idx_h_out)
-    ev = None
-    if phase_events is not None:
-        if len(phase_events) != QS_FFN_PHASE_EVENTS:
-            raise ValueError(f"phase_events must hold {QS_FFN_PHASE_EVENTS} events")
-        ev = (ctypes.c_void_p * QS_FFN_PHASE_EVENTS)(*[e.cuda_event for e in phase_events])
+    ev = _events(phase_events, QS_FFN_PHASE_EVENTS)
     ws = _workspace(ws, QS_OP_SPARSE_FFN, T, d_model, d_ff, k_h, dev)
     _check("qs_sparse_ffn", lib().qs_sparse_ffn(
         x.data_ptr(), _dtype_code(x), T, d_model, d_ff, act_code, k_in, k_h,
@@ -311,7 +317,8 @@ class QuantResult(NamedTuple):
 
 
 def qs_quant_sparse_linear(x, wt_packed, alpha: float, k: int, eps: float = 1e-5, y=None,
-                           acc=None, q=None, idx=None, ws=None, stream=None) -> QuantResult:
+                           acc=None, q=None, idx=None, phase_events=None, ws=None,
+                           stream=None) -> QuantResult:
     """int8 (per-token absmax) x ternary (packed 2-bit) projection of the top-K of |q|."""
     dev = _need_cuda(x, wt_packed)
     T, d_in = x.shape
@@ -326,7 +333,8 @@ def qs_quant_sparse_linear(x, wt_packed, alpha: float, k: int, eps: float = 1e-5
     ws = _workspace(ws, QS_OP_QUANT_SPARSE_LINEAR, T, d_in, d_out, k, dev)
     _check("qs_quant_sparse_linear", lib().qs_quant_sparse_linear(
         x.data_ptr(), _dtype_code(x), T, d_in, d_out, k, wt_packed.data_ptr(), float(alpha),
-        float(eps), y.data_ptr(), _ptr(acc), _ptr(q), _ptr(idx), ws.data_ptr(), ws.numel(),
+        float(eps), y.data_ptr(), _ptr(acc), _ptr(q), _ptr(idx),
+        _events(phase_events, QS_LINEAR_PHASE_EVENTS), ws.data_ptr(), ws.numel(),
         _stream_ptr(stream)))
     return QuantResult(y, acc, q, idx)
 

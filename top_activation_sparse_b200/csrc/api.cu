@@ -253,7 +253,8 @@ qs_status qs_topk_mask(const void* x, int dtype, int T, int d, int k, int32_t* i
 }
 
 qs_status qs_sparse_linear(const void* x, int dtype, int T, int d_in, int d_out, int k,
-                           const void* wt, void* y, void* ws, size_t ws_bytes, void* stream) {
+                           const void* wt, void* y, void* const* phase_events, void* ws,
+                           size_t ws_bytes, void* stream) {
   if (!valid_dtype(dtype) || x == nullptr || wt == nullptr || y == nullptr || T < 1 || d_in < 1 ||
       d_out < 1 || k < 0 || k > d_in)
     return QS_ERR_INVALID_ARG;
@@ -266,24 +267,34 @@ qs_status qs_sparse_linear(const void* x, int dtype, int T, int d_in, int d_out,
   WsView w{(unsigned char*)ws};
   cudaStream_t s = (cudaStream_t)stream;
   const int eb = elem_bytes(dtype);
+  auto mark = [&](int i) -> cudaError_t {
+    if (phase_events == nullptr) return cudaSuccess;
+    return cudaEventRecord((cudaEvent_t)phase_events[i], s);
+  };
 
   // Prefill: many tokens make this a dense contraction over X_sparse.
   if (dtype == QS_BF16 && T >= QS_PREFILL_MIN_T && prefill_supported(T, d_out, d_in)) {
+    QS_TRY_CUDA(mark(0));
     TopkArgs a;
     a.x = x; a.T = T; a.d = d_in; a.k = k; a.kind = TK_BF16;
     a.xs = w.at<void>(L.xs_bf16);
     a.status = w.status();
     QS_TRY_CUDA(launch_topk(a, s));
+    QS_TRY_CUDA(mark(1));
     PrefillArgs p;
     p.xs = w.at<__nv_bfloat16>(L.xs_bf16);
     p.wt = reinterpret_cast<const __nv_bfloat16*>(wt);
     p.y = reinterpret_cast<__nv_bfloat16*>(y);
     p.M = T; p.N = d_out; p.K = d_in;
     p.status = w.status();
-    return from_cuda(launch_prefill_gemm(p, s));
+    QS_TRY_CUDA(launch_prefill_gemm(p, s));
+    QS_TRY_CUDA(mark(2));
+    return QS_OK;
   }
 
   for (int t0 = 0; t0 < T; t0 += kChunkT) {
+    const bool timed = (t0 == 0);
+    if (timed) QS_TRY_CUDA(mark(0));
     const int Tc = (T - t0) < kChunkT ? (T - t0) : kChunkT;
     TopkArgs a;
     a.x = (const unsigned char*)x + (size_t)t0 * d_in * eb;
@@ -301,6 +312,7 @@ qs_status qs_sparse_linear(const void* x, int dtype, int T, int d_in, int d_out,
     a.zero = w.at<float>(L.parts1);
     a.zero_n = gp.parts_elems;
     QS_TRY_CUDA(launch_topk(a, s));
+    if (timed) QS_TRY_CUDA(mark(1));
 
     GemvArgs g;
     g.w[0] = wt;
@@ -315,6 +327,7 @@ qs_status qs_sparse_linear(const void* x, int dtype, int T, int d_in, int d_out,
     g.y = (unsigned char*)y + (size_t)t0 * d_out * eb;
     g.status = w.status();
     QS_TRY_CUDA(launch_gemv(g, s));
+    if (timed) QS_TRY_CUDA(mark(2));
   }
   return QS_OK;
 }
@@ -425,7 +438,8 @@ qs_status qs_sparse_ffn(const void* x, int dtype, int T, int d_model, int d_ff, 
 
 qs_status qs_quant_sparse_linear(const void* x, int dtype, int T, int d_in, int d_out, int k,
                                  const uint32_t* wt_packed, float alpha, float eps, float* y,
-                                 int32_t* acc, int8_t* q, int32_t* idx, void* ws, size_t ws_bytes,
+                                 int32_t* acc, int8_t* q, int32_t* idx,
+                                 void* const* phase_events, void* ws, size_t ws_bytes,
                                  void* stream) {
   if (!valid_dtype(dtype) || x == nullptr || wt_packed == nullptr || y == nullptr || T < 1 ||
       d_in < 1 || d_out < 1 || k < 0 || k > d_in || !(eps >= 0.0f) || !(alpha == alpha))
@@ -440,8 +454,14 @@ qs_status qs_quant_sparse_linear(const void* x, int dtype, int T, int d_in, int 
   WsView w{(unsigned char*)ws};
   cudaStream_t s = (cudaStream_t)stream;
   const int eb = elem_bytes(dtype);
+  auto mark = [&](int i) -> cudaError_t {
+    if (phase_events == nullptr) return cudaSuccess;
+    return cudaEventRecord((cudaEvent_t)phase_events[i], s);
+  };
   for (int t0 = 0; t0 < T; t0 += kChunkT) {
     const int Tc = (T - t0) < kChunkT ? (T - t0) : kChunkT;
+    const bool timed = (t0 == 0);
+    if (timed) QS_TRY_CUDA(mark(0));
     TopkArgs a;
     a.x = (const unsigned char*)x + (size_t)t0 * d_in * eb;
     a.T = Tc; a.d = d_in; a.k = k;
@@ -458,6 +478,7 @@ qs_status qs_quant_sparse_linear(const void* x, int dtype, int T, int d_in, int 
     a.union_bits = reinterpret_cast<uint32_t*>(w.ticket(L, kUnionX));
     a.status = w.status();
     QS_TRY_CUDA(launch_topk(a, s));
+    if (timed) QS_TRY_CUDA(mark(1));
 
     QGemvArgs g;
     g.wp = wt_packed; g.d_in = d_in; g.d_out = d_out; g.T = Tc;
@@ -471,6 +492,7 @@ qs_status qs_quant_sparse_linear(const void* x, int dtype, int T, int d_in, int 
     g.acc = acc ? acc + (size_t)t0 * d_out : nullptr;
     g.status = w.status();
     QS_TRY_CUDA(launch_qgemv(g, s));
+    if (timed) QS_TRY_CUDA(mark(2));
   }
   return QS_OK;
 }

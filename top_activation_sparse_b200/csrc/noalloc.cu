@@ -59,5 +59,5 @@ extern "C" qs_status qs_sparse_linear_noalloc(const void* x, int dtype, int T, i
   qs::WsLayout L;
   if (!qs::ws_layout(QS_OP_SPARSE_LINEAR, T, d_in, d_out, k, &L)) return QS_ERR_INVALID_ARG;
   if (cudaMemsetAsync(ws, 0, L.cnt, (cudaStream_t)stream) != cudaSuccess) return QS_ERR_CUDA;
-  return qs_sparse_linear(x, dtype, T, d_in, d_out, k, wt, y, ws, kScratchBytes, stream);
+  return qs_sparse_linear(x, dtype, T, d_in, d_out, k, wt, y, nullptr, ws, kScratchBytes, stream);
 }

@@ -1,12 +1,298 @@
-// Prefill masked-dense GEMM: Y = X_sparse . W^T on the tensor cores.
-// (Placeholder until the tcgen05 kernel lands: reports "unsupported" so that
-// qs_sparse_linear keeps prefill sizes on the gather-GEMV path.)
+// Prefill masked-dense GEMM on the 5th-generation tensor cores:
+//   Y[M, N] = X_sparse[M, K] . W^T[K, N]      (bf16 in, f32 accumulate, bf16 out)
+//
+// Source: Q-Sparse paper summary (shd-paper.top), abstract and method
+// sections (Block Q-Sparse makes the sparsity usable for batched training and
+// inference); with thousands of tokens each keeping its own top-K, almost
+// every weight row is needed by some token, so the projection is a dense
+// contraction over the masked activations and belongs on the tensor cores.
+//
+// sm_100a design (one output tile of 128 x 256 per CTA, one CTA per SM):
+//   * TMA (cp.async.bulk.tensor, 128-byte swizzle, no multicast) loads an A
+//     tile of X_sparse (128 rows x 64 K, K-major) and a B tile of W^T (64 K x
+//     256 N, N-major, as four 64-column boxes) per stage into a 4-stage ring;
+//   * one thread issues tcgen05.mma.kind::f16 (bf16 x bf16 -> f32) with the
+//     accumulator in tensor memory (TMEM, 256 columns x 128 lanes) and frees
+//     each stage with tcgen05.commit on that stage's "empty" mbarrier;
+//   * four epilogue warps read the accumulator with tcgen05.ld (each warp its
+//     32 TMEM lanes = 32 rows), round to bf16 and store Y;
+//   * CTAs are ordered M-block fastest, so the CTAs resident at one time share
+//     W^T tiles through the L2;
+//   * every mbarrier wait is bounded: on a timeout the CTA records
+//     DEV_TIMEOUT, waits (bounded) for its own copies and MMAs in flight,
+//     frees its TMEM and returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
 #include "qs_internal.cuh"
 
 namespace qs {
+namespace {
 
-bool prefill_supported(int, int, int) { return false; }
+constexpr int BM = 128, BN = 256, BK = 64;
+constexpr int kStages = 4;
+constexpr int kABytes = BM * BK * 2;                 // 16 KB
+constexpr int kBBox = 64 * BK * 2;                   // one 64-column box of B: 8 KB
+constexpr int kBBytes = (BN / 64) * kBBox;           // 32 KB
+constexpr int kStageBytes = kABytes + kBBytes;       // 48 KB
+constexpr int kSmemBytes = kStages * kStageBytes + 1024;
+constexpr int kThreads = 192;                        // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
+constexpr uint32_t kTmemCols = 256;
 
-cudaError_t launch_prefill_gemm(const PrefillArgs&, cudaStream_t) { return cudaErrorNotSupported; }
+// tcgen05 instruction descriptor, kind::f16: D f32, A bf16 (K-major),
+// B bf16 (MN-major), N = 256, M = 128.
+constexpr uint32_t kIdesc = (1u << 4)            // accumulator format: f32
+                          | (1u << 7)            // A format: bf16
+                          | (1u << 10)           // B format: bf16
+                          | (0u << 15)           // A major-ness: K
+                          | (1u << 16)           // B major-ness: MN
+                          | ((uint32_t)(BN >> 3) << 17)
+                          | ((uint32_t)(BM >> 4) << 24);
+
+// Shared-memory matrix descriptor (sm_100 version bits), 128-byte swizzle.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.u32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// 32 consecutive f32 accumulator columns of this warp's 32 TMEM lanes.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
+      "%30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(uint32_t lo_f32, uint32_t hi_f32) {
+  return (uint32_t)f32_to_bf16_bits(__uint_as_float(lo_f32)) |
+         ((uint32_t)f32_to_bf16_bits(__uint_as_float(hi_f32)) << 16);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    prefill_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
+                        const __grid_constant__ CUtensorMap map_b, __nv_bfloat16* __restrict__ y,
+                        int M, int N, int K, DevStatus* status) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  __shared__ __align__(8) uint64_t s_full[kStages];
+  __shared__ __align__(8) uint64_t s_empty[kStages];
+  __shared__ __align__(8) uint64_t s_accum;
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_abort;
+
+  // 1024-byte aligned ring (128-byte swizzle atoms repeat every 1 KB)
+  const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.x * BM;          // M-block fastest
+  const int n0 = blockIdx.y * BN;
+  const int nk = (K + BK - 1) / BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&s_full[s], 1);
+      mbar_init(&s_empty[s], 1);
+    }
+    mbar_init(&s_accum, 1);
+    mbar_fence_init();
+    s_abort = 0;
+  }
+  if (warp == 0) {   // whole warp: allocate the accumulator columns
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&s_tmem)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+
+  if (warp == 0 && lane == 0) {
+    // ---- TMA producer ----
+    int issued = 0;
+    for (int kb = 0; kb < nk; ++kb) {
+      const int s = kb % kStages;
+      if (kb >= kStages && !mbar_wait(&s_empty[s], (uint32_t)((kb / kStages) - 1) & 1u)) {
+        dev_fail(status, DEV_TIMEOUT, 20, (uint32_t)kb);
+        atomicExch(&s_abort, 1);
+        break;
+      }
+      if (*(volatile int*)&s_abort) break;
+      const uint32_t sa = base + (uint32_t)(s * kStageBytes);
+      const uint32_t sb = sa + kABytes;
+      mbar_arrive_expect_tx(&s_full[s], (uint32_t)kStageBytes);
+      tma_load_2d(sa, &map_a, kb * BK, m0, &s_full[s]);
+#pragma unroll
+      for (int j = 0; j < BN / 64; ++j) tma_load_2d(sb + j * kBBox, &map_b, n0 + 64 * j, kb * BK, &s_full[s]);
+      ++issued;
+    }
+    // on an abort, let the copies already issued land before the CTA exits
+    if (*(volatile int*)&s_abort) {
+      for (int i = 0; i < kStages && i < issued; ++i) {
+        const int kb = issued - 1 - i;
+        mbar_wait(&s_full[kb % kStages], (uint32_t)(kb / kStages) & 1u);
+      }
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ---- MMA issuer ----
+    int done = 0;
+    for (int kb = 0; kb < nk; ++kb) {
+      const int s = kb % kStages;
+      if (!mbar_wait(&s_full[s], (uint32_t)(kb / kStages) & 1u)) {
+        dev_fail(status, DEV_TIMEOUT, 21, (uint32_t)kb);
+        atomicExch(&s_abort, 1);
+        break;
+      }
+      if (*(volatile int*)&s_abort) break;
+      tc_fence_after();
+      const uint32_t sa = base + (uint32_t)(s * kStageBytes);
+      const uint32_t sb = sa + kABytes;
+#pragma unroll
+      for (int kk = 0; kk < BK / 16; ++kk) {
+        // A: K-major, 128-byte rows, 8-row groups 1 KB apart; K step = 32 bytes
+        const uint64_t ad = smem_desc(sa + kk * 32, 16, 1024);
+        // B: N-major, 128-byte K rows, 8-row groups 1 KB apart (SBO),
+        //    64-column boxes 8 KB apart (LBO); K step = 16 rows = 2 KB
+        const uint64_t bd = smem_desc(sb + kk * 2048, kBBox, 1024);
+        umma_bf16(tmem, ad, bd, (kb > 0 || kk > 0) ? 1u : 0u);
+      }
+      umma_commit(&s_empty[s]);          // frees the stage once these MMAs have read it
+      ++done;
+    }
+    umma_commit(&s_accum);               // accumulator complete (or abandoned)
+  } else if (warp >= 2) {
+    // ---- epilogue: TMEM -> registers -> bf16 -> global ----
+    const bool ok = mbar_wait_backoff(&s_accum, 0u);
+    if (!ok) {
+      if (lane == 0) dev_fail(status, DEV_TIMEOUT, 22, 0u);
+      atomicExch(&s_abort, 1);
+    }
+    tc_fence_after();
+    const int q = warp & 3;                      // this warp's TMEM lane quarter
+    const int row = m0 + q * 32 + lane;
+    const bool abort = *(volatile int*)&s_abort;
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 32) {
+      uint32_t r[32];
+      tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c, r);
+      if (abort || row >= M) continue;
+      __nv_bfloat16* dst = y + (size_t)row * N + n0 + c;
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        if (n0 + c + 8 * v + 8 > N) break;       // N is a multiple of 8
+        uint4 o;
+        o.x = pack_bf16x2(r[8 * v + 0], r[8 * v + 1]);
+        o.y = pack_bf16x2(r[8 * v + 2], r[8 * v + 3]);
+        o.z = pack_bf16x2(r[8 * v + 4], r[8 * v + 5]);
+        o.w = pack_bf16x2(r[8 * v + 6], r[8 * v + 7]);
+        *reinterpret_cast<uint4*>(dst + 8 * v) = o;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static std::once_flag once;
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 tensor map: dims {inner, outer}, row pitch in bytes, box {bx, by}.
+bool make_map(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint64_t pitch,
+              uint32_t bx, uint32_t by) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {pitch};
+  cuuint32_t box[2] = {bx, by};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool prefill_supported(int M, int N, int K) {
+  // TMA needs 16-byte row pitches; the epilogue stores 8 columns at a time
+  return M >= 1 && N >= 8 && K >= 8 && (N % 8) == 0 && (K % 8) == 0 && encode_fn() != nullptr;
+}
+
+cudaError_t launch_prefill_gemm(const PrefillArgs& a, cudaStream_t s) {
+  CUtensorMap ma, mb;
+  // A = X_sparse [M, K] row-major: inner K, box 64 x 128
+  if (!make_map(&ma, a.xs, (uint64_t)a.K, (uint64_t)a.M, (uint64_t)a.K * 2, BK, BM))
+    return cudaErrorInvalidValue;
+  // B = W^T [K, N] row-major: inner N, box 64 (N) x 64 (K)
+  if (!make_map(&mb, a.wt, (uint64_t)a.N, (uint64_t)a.K, (uint64_t)a.N * 2, 64, BK))
+    return cudaErrorInvalidValue;
+  static unsigned configured = 0;
+  cudaError_t e = ensure_smem_attr(prefill_gemm_kernel, kSmemBytes, &configured);
+  if (e != cudaSuccess) return e;
+  dim3 grid((a.M + BM - 1) / BM, (a.N + BN - 1) / BN);
+  prefill_gemm_kernel<<<grid, kThreads, kSmemBytes, s>>>(ma, mb, a.y, a.M, a.N, a.K, a.status);
+  return cudaGetLastError();
+}
 
 }  // namespace qs
