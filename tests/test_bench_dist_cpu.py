@@ -1,0 +1,80 @@
+"""Host logic of the benchmark's multi-rank path, on CPU with gloo (2 ranks).
+
+Every rank runs its own replica (weak scaling, no data-path collective); the
+only collectives are the barrier and the max / sum of the per-rank timings,
+which these tests check.  Also: argument parsing and the clock summary."""
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import bench
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    r, w, local = bench.dist_env()
+    d = bench.dist_init(w, "gloo")
+    try:
+        dev = torch.device("cpu")
+        ms = 10.0 + 5.0 * r                      # the slower rank decides
+        mx = bench.max_over_ranks(ms, d, dev)
+        tok = bench.sum_over_ranks(100.0 * (r + 1), d, dev)
+        out[r] = (r, w, local, mx, tok)
+    finally:
+        d.barrier()
+        d.destroy_process_group()
+
+
+def test_two_rank_timing_reduction():
+    port = _free_port()
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.spawn(_worker, args=(2, port, out), nprocs=2, join=True)
+        res = dict(out)
+    assert sorted(res) == [0, 1]
+    for r, (rank, world, local, mx, tok) in res.items():
+        assert (rank, world, local) == (r, 2, r)
+        assert mx == 15.0                        # max over ranks
+        assert tok == 300.0                      # whole-job units
+
+
+def test_single_rank_needs_no_process_group(monkeypatch):
+    for k in ("WORLD_SIZE", "RANK", "LOCAL_RANK"):
+        monkeypatch.delenv(k, raising=False)
+    rank, world, local = bench.dist_env()
+    assert (rank, world, local) == (0, 1, 0)
+    assert bench.dist_init(world, "gloo") is None
+    assert bench.max_over_ranks(3.5, None, None) == 3.5
+
+
+def test_parse_args_defaults_and_guards():
+    a = bench.parse_args([])
+    assert a.gpus == 1 and a.warmup >= 3 and a.steps >= 1
+    assert a.workload == "ffn_relu2_llama7b" and a.batch == 1
+    assert bench.parse_args(["--workload", "prefill_bf16_2048"]).batch == 2048
+    with pytest.raises(SystemExit):
+        bench.parse_args(["--warmup", "2"])
+
+
+def test_clock_summary():
+    lines = [
+        "0, 1965, 1965, 700.1, 0x0, Not Active, Not Active, Not Active, Not Active",
+        "0, 1950, 1965, 990.0, 0x4, Not Active, Not Active, Not Active, Active",
+        "0, 1965, 1965, 800.0, 0x0, Not Active, Not Active, Not Active, Not Active",
+        "garbage",
+    ]
+    s = bench.summarize_clocks(lines)
+    assert s["sm_mhz"] == 1965.0 and s["sm_max_mhz"] == 1965.0 and s["samples"] == 3
+    assert s["reasons"] == ["sw_power_cap"]
+    assert bench.summarize_clocks([])["samples"] == 0
