@@ -144,6 +144,7 @@ __global__ void __launch_bounds__(kMaxConsumers + 32, (TT <= 4) ? 2 : 1) gemv_ke
   const unsigned char* Wb = reinterpret_cast<const unsigned char*>(a.w[mat]) + cbyte;
   const int col = (ct * P.vec_tile + tid) * V;                            // this thread's columns
 
+  pdl_begin();
   grid_zero(a.zero, a.zero_n);
   const int n = min(max(*a.list_count, 0), d_in);
   const int r0 = (int)(((long long)n * s) / S);
@@ -306,7 +307,8 @@ cudaError_t launch3(const GemvArgs& a, cudaStream_t s) {
   cudaError_t e = ensure_smem_attr(gemv_kernel<WT, TT, MODE>, 200 * 1024, &configured);
   if (e != cudaSuccess) return e;
   dim3 grid(a.plan.n_ct, a.plan.mats * a.plan.S, a.plan.groups);
-  gemv_kernel<WT, TT, MODE><<<grid, a.plan.threads, a.plan.smem, s>>>(a);
+  e = launch_pdl(gemv_kernel<WT, TT, MODE>, grid, dim3(a.plan.threads), a.plan.smem, s, a);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -119,6 +119,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const __grid_constant__ CUtensorMap map_b, __nv_bfloat16* __restrict__ y,
                         int M, int N, int K, DevStatus* status) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
+  pdl_begin();
   __shared__ __align__(8) uint64_t s_full[kStages];
   __shared__ __align__(8) uint64_t s_empty[kStages];
   __shared__ __align__(8) uint64_t s_accum;
@@ -291,7 +292,9 @@ cudaError_t launch_prefill_gemm(const PrefillArgs& a, cudaStream_t s) {
   cudaError_t e = ensure_smem_attr(prefill_gemm_kernel, kSmemBytes, &configured);
   if (e != cudaSuccess) return e;
   dim3 grid((a.M + BM - 1) / BM, (a.N + BN - 1) / BN);
-  prefill_gemm_kernel<<<grid, kThreads, kSmemBytes, s>>>(ma, mb, a.y, a.M, a.N, a.K, a.status);
+  e = launch_pdl(prefill_gemm_kernel, grid, dim3(kThreads), (size_t)kSmemBytes, s, ma, mb, a.y, a.M,
+                 a.N, a.K, a.status);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

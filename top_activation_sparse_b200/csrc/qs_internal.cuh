@@ -122,6 +122,36 @@ __device__ __forceinline__ unsigned lanemask_lt() {
   return m;
 }
 
+// ---- programmatic dependent launch ----------------------------------------
+// Kernels of one call are launched with programmatic stream serialization:
+// the next kernel's CTAs may be scheduled while this one runs, which hides the
+// launch latency.  Every kernel first waits for the previous grid to finish
+// (griddepcontrol.wait, a no-op when not launched that way) and only then
+// touches memory, so the stream order of the results is unchanged.  The next
+// grid is released only once every CTA of this one has executed
+// launch_dependents (or exited), so it never takes resources this grid's
+// later waves need.
+__device__ __forceinline__ void pdl_begin() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // Raise a kernel's dynamic shared-memory limit once per device.
 template <typename F>
 cudaError_t ensure_smem_attr(F* kernel, int bytes, unsigned* done_mask) {

@@ -47,6 +47,7 @@ __global__ void __launch_bounds__(kNT) qgemv_kernel(QGemvArgs a) {
   const int wcol = ct * kTileWords + lane;
   const bool colok = wcol < n_words;
 
+  pdl_begin();
   for (int q = tid; q < TT * TILE; q += kNT) (&s_acc[0][0])[q] = 0;
 
   const int n = min(max(*a.list_count, 0), d_in);
@@ -157,7 +158,8 @@ __global__ void __launch_bounds__(kNT) qgemv_kernel(QGemvArgs a) {
 template <int TT>
 cudaError_t qlaunch(const QGemvArgs& a, cudaStream_t s) {
   dim3 grid(a.plan.n_ct, a.plan.S, a.plan.groups);
-  qgemv_kernel<TT><<<grid, kNT, 0, s>>>(a);
+  cudaError_t e = launch_pdl(qgemv_kernel<TT>, grid, dim3(kNT), 0, s, a);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

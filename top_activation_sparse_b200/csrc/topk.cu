@@ -142,6 +142,7 @@ __global__ void __launch_bounds__(NT) topk_kernel(TopkArgs a) {
   const size_t rbase = (size_t)row * (size_t)d;
   int sbuf = 0;
 
+  pdl_begin();
   grid_zero(a.zero, a.zero_n);
   uint32_t my_nnz = 0;
 
@@ -386,7 +387,8 @@ cudaError_t launch_kind(const TopkArgs& a, cudaStream_t s) {
   cudaError_t e = ensure_smem_attr(topk_kernel<KIND, NT>, (int)(QS_MAX_ROW * sizeof(uint32_t)),
                                    &configured);
   if (e != cudaSuccess) return e;
-  topk_kernel<KIND, NT><<<a.T, NT, smem, s>>>(a);
+  e = launch_pdl(topk_kernel<KIND, NT>, dim3(a.T), dim3(NT), smem, s, a);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
