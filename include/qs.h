@@ -55,7 +55,8 @@ typedef enum qs_status {
   QS_OK = 0,
   QS_ERR_INVALID_ARG = 1,   /* bad size, k, enum value, or a required pointer is NULL */
   QS_ERR_ALIGNMENT = 2,     /* pointer not 16-byte aligned, or d_out not a multiple of the
-                               16-byte vector width (4 for f32, 8 for bf16, 16 packed) */
+                               16-byte vector width (4 for f32, 8 for bf16; 64 for the
+                               packed int8 x ternary projection) */
   QS_ERR_WORKSPACE = 3,     /* ws NULL or smaller than qs_workspace_size() */
   QS_ERR_CUDA = 4,          /* a CUDA runtime call or kernel launch failed */
   QS_ERR_TIMEOUT = 5,       /* device: a bounded wait ran out (see qs_device_status) */
@@ -183,7 +184,8 @@ qs_status qs_sparse_ffn(const void* x, int dtype, int T, int d_model, int d_ff, 
  *   acc        [T, d_out] int32 out or NULL.   q  [T, d_in] int8 out or NULL.
  *   idx        [T, k] int32 out or NULL: kept indices, ascending.
  *   phase_events  NULL or QS_LINEAR_PHASE_EVENTS events (as qs_sparse_linear).
- *   d_out must be a multiple of 16; 127 * d_in < 2^24 keeps float(acc) exact.
+ *   d_out must be a multiple of 64 (whole packed rows move in 16-byte bulk
+ *   copies); 127 * d_in < 2^24 keeps float(acc) exact.
  *   Errors: INVALID_ARG, ALIGNMENT, WORKSPACE, UNSUPPORTED, CUDA.
  */
 qs_status qs_quant_sparse_linear(const void* x, int dtype, int T, int d_in, int d_out, int k,

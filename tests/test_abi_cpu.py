@@ -49,7 +49,8 @@ def test_workspace_size_is_host_only_and_sane(L):
     b = f(qs.QS_OP_SPARSE_FFN, 8, 4096, 11008, 7705)
     assert 0 < a < b
     assert f(qs.QS_OP_QUANT_SPARSE_LINEAR, 32, 4096, 11008, 1597) > 0
-    assert f(qs.QS_OP_QUANT_SPARSE_LINEAR, 1, 4096, 11000, 1597) == 0   # d_out % 16
+    assert f(qs.QS_OP_QUANT_SPARSE_LINEAR, 1, 4096, 11000, 1597) == 0   # d_out % 64
+    assert f(qs.QS_OP_QUANT_SPARSE_LINEAR, 1, 4096, 48, 1597) == 0
     assert f(qs.QS_OP_TERNARY_PACK, 0, 4096, 11008, 0) > 0
     assert f(99, 1, 1, 1, 1) == 0
     # more than the decode chunk of tokens does not grow the decode buffers

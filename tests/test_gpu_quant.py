@@ -70,7 +70,7 @@ def test_quant_sparse_linear_bitnet_shapes(name, T):
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_quant_edge_cases(dtype):
     need_gpu()
-    d_in, d_out = 300, 48
+    d_in, d_out = 300, 64
     W = workloads.weight_out_major(d_out, d_in, 9)
     t, alpha = oracle.ternary_quantize(W)
     packed = oracle.ternary_pack(t)
@@ -93,3 +93,13 @@ def test_quant_chunked_tokens():
     t, alpha = oracle.ternary_quantize(W)
     x = workloads.round_to_dtype(workloads.normal_f32(workloads.rng(13), (70, d_in)), "bf16")
     _check_quant(x, "bf16", t, alpha, oracle.ternary_pack(t), 100)
+
+
+def test_quant_rejects_unaligned_packed_rows():
+    """Packed rows move in 16-byte bulk copies: d_out must be a multiple of 64."""
+    need_gpu()
+    x = torch.zeros(1, 32, device="cuda")
+    p = torch.zeros(32, 3, dtype=torch.int32, device="cuda")      # d_out = 48
+    with pytest.raises(qs.QSError) as e:
+        qs.qs_quant_sparse_linear(x, p, 1.0, 8)
+    assert e.value.status == qs.QS_ERR_ALIGNMENT

@@ -107,15 +107,15 @@ bool ws_layout(int op, int T, int d_in, int d_out, int k, WsLayout* L) {
       break;
     }
     case QS_OP_QUANT_SPARSE_LINEAR: {
-      if (T < 1 || d_in < 1 || d_out < 16 || d_in > QS_MAX_ROW || d_out > QS_MAX_ROW || k < 0 ||
-          k > d_in || (d_out % 16) != 0)
+      if (T < 1 || d_in < 1 || d_out < 64 || d_in > QS_MAX_ROW || d_out > QS_MAX_ROW || k < 0 ||
+          k > d_in || (d_out % 64) != 0)
         return false;
       L->xq = take((size_t)Tc * d_in);
       L->gamma = take((size_t)Tc * sizeof(float));
       L->list_x = take((size_t)d_in * sizeof(int32_t));
       L->lval_x = take((size_t)d_in * Tc);
       L->parts1_elems = max_qparts(d_out, d_in, k);
-      L->parts1 = take(L->parts1_elems * sizeof(int32_t));
+      L->parts1 = take(L->parts1_elems * sizeof(float));
       break;
     }
     case QS_OP_TERNARY_PACK:
@@ -445,7 +445,7 @@ qs_status qs_quant_sparse_linear(const void* x, int dtype, int T, int d_in, int 
       d_in < 1 || d_out < 1 || k < 0 || k > d_in || !(eps >= 0.0f) || !(alpha == alpha))
     return QS_ERR_INVALID_ARG;
   if (d_in > QS_MAX_ROW || d_out > QS_MAX_ROW) return QS_ERR_UNSUPPORTED;
-  if ((d_out % 16) != 0 || !aligned16(x) || !aligned16(wt_packed) || !aligned16(y) ||
+  if (!qgemv_supported(d_out) || !aligned16(x) || !aligned16(wt_packed) || !aligned16(y) ||
       !aligned16(acc) || !aligned16(q) || !aligned16(idx))
     return QS_ERR_ALIGNMENT;
   WsLayout L;
@@ -477,6 +477,10 @@ qs_status qs_quant_sparse_linear(const void* x, int dtype, int T, int d_in, int 
     a.ticket = w.ticket(L, kTkTopkX);
     a.union_bits = reinterpret_cast<uint32_t*>(w.ticket(L, kUnionX));
     a.status = w.status();
+    const GemvPlan qp = plan_qgemv(Tc, d_out, (int)rows_bound(Tc, d_in, k));
+    if (!plan_fits(L, qp, L.parts1_elems, 0)) return QS_ERR_UNSUPPORTED;
+    a.zero = w.at<float>(L.parts1);
+    a.zero_n = qp.parts_elems;
     QS_TRY_CUDA(launch_topk(a, s));
     if (timed) QS_TRY_CUDA(mark(1));
 
@@ -484,10 +488,9 @@ qs_status qs_quant_sparse_linear(const void* x, int dtype, int T, int d_in, int 
     g.wp = wt_packed; g.d_in = d_in; g.d_out = d_out; g.T = Tc;
     g.gamma = a.gamma; g.alpha = alpha;
     g.list = a.list; g.list_q = a.list_q; g.xq = a.xq; g.list_count = a.list_count;
-    g.parts = w.at<int32_t>(L.parts1);
-    g.plan = plan_qgemv(Tc, d_out, (int)rows_bound(Tc, d_in, k));
+    g.parts = w.at<float>(L.parts1);
+    g.plan = qp;
     g.tickets = w.ticket(L, kTkGemv);
-    if (!plan_fits(L, g.plan, L.parts1_elems, 0)) return QS_ERR_UNSUPPORTED;
     g.y = y + (size_t)t0 * d_out;
     g.acc = acc ? acc + (size_t)t0 * d_out : nullptr;
     g.status = w.status();

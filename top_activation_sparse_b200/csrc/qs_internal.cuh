@@ -191,6 +191,7 @@ struct GemvPlan {
 
 GemvPlan plan_gemv(int T, int d_out, int rows_bound, int mats, int elem_bytes);
 GemvPlan plan_qgemv(int T, int d_out, int rows_bound);
+bool qgemv_supported(int d_out);
 
 struct WsLayout {
   size_t status = 0;          // DevStatus
@@ -295,7 +296,7 @@ struct QGemvArgs {
   const int8_t* list_q = nullptr;  // [n][T] int8 codes of the listed rows (one token), or
   const int8_t* xq = nullptr;      // [T][d_in] dense masked codes (several tokens)
   const int32_t* list_count = nullptr;
-  int32_t* parts = nullptr;
+  float* parts = nullptr;          // [T][d_out] f32 accumulators (exact integers), zeroed before
   int32_t* tickets = nullptr;
   float* y = nullptr;
   int32_t* acc = nullptr;

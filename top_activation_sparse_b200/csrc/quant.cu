@@ -21,49 +21,128 @@
 namespace qs {
 namespace {
 
-constexpr int kNT = 256;
-constexpr int kNW = kNT / 32;
-constexpr int kPiece = 256;
-constexpr int kTileWords = 32;          // one 32-bit word (16 columns) per lane
+// ---- int8 x ternary gather-GEMV ----------------------------------------------
+// Packed rows are streamed like the bf16 gather-GEMV: one producer thread
+// issues a cp.async.bulk per kept row (whole rows, or a few column tiles) into a
+// ring of ~16 KB shared-memory stages.
+//
+// Decoding.  Each code c (00 = 0, 01 = +1, 10 = -1) is first mapped to
+// u = t + 1 in {0, 1, 2} with four logic operations per word.  Codes j and j+8
+// of a word then sit 16 bits apart, so one (shift, and) pulls out the pair as
+// two 16-bit lanes and one integer multiply-add accumulates q * u for both:
+// two outputs per IMAD.  A lane holds sum q*u with |q| <= 127 and u <= 2, so it
+// stays inside int16 for up to 128 rows; every <= 128 rows the lanes are
+// unpacked into int32 accumulators and the sum of q over those rows is taken
+// off (sum q*t = sum q*u - sum q).  Everything is integer: the result is exact
+// and independent of the order of the additions.
+//
+// Split partials are added with f32 vector reductions: every partial is an
+// integer with |value| <= 127 * d_in < 2^24, so the f32 additions are exact and
+// the result does not depend on their order.
+
+template <int TT> struct QTune {
+  static constexpr int LPT = (TT == 1) ? 32 : (TT == 2 ? 16 : (TT == 4 ? 8 : 4));  // lane pairs per thread
+  static constexpr int WPT = LPT >= 8 ? LPT / 8 : 1;   // packed words a thread reads per row
+  static constexpr int KPW = LPT >= 8 ? 8 : LPT;       // lane pairs a thread takes from each word
+  static constexpr int kMaxConsumers = 192;            // two CTAs per SM
+};
+constexpr int kLaneRows = 128;                           // rows between lane flushes
+
+__device__ __forceinline__ void red_add_v4_f32(float* dst, float a0, float a1, float a2, float a3) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(a0), "f"(a1),
+               "f"(a2), "f"(a3)
+               : "memory");
+}
+
+// codes (00 = 0, 01 = +1, 10 = -1) -> u = t + 1 (00, 01, 10 for -1, 0, +1)
+__device__ __forceinline__ uint32_t ternary_to_u(uint32_t w) {
+  const uint32_t hi = (w << 1) & 0xAAAAAAAAu;              // +1 -> bit 1 of the field
+  const uint32_t zero = ~(w | (w >> 1)) & 0x55555555u;     // 0 -> bit 0 of the field
+  return hi | zero;
+}
 
 template <int TT>
-__global__ void __launch_bounds__(kNT) qgemv_kernel(QGemvArgs a) {
-  constexpr int U = (TT <= 2) ? 8 : 4;
-  constexpr int TILE = kTileWords * 16;  // 512 columns
-  __shared__ int s_rows[kPiece];
-  __shared__ int s_q[TT][kPiece];
-  __shared__ int s_acc[TT][TILE];
-  __shared__ int s_last;
+__global__ void __launch_bounds__(QTune<TT>::kMaxConsumers + 32, 2) qgemv_kernel(QGemvArgs a) {
+  using Q = QTune<TT>;
+  constexpr int WPT = Q::WPT, KPW = Q::KPW, LPT = Q::LPT;
+  extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ __align__(8) uint64_t s_full[32];
+  __shared__ __align__(8) uint64_t s_empty[32];
+  __shared__ int s_flag;
+  __shared__ int s_err;
 
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int S = a.plan.S;
+  const GemvPlan& P = a.plan;
+  const int NC = P.threads - 32;
+  const int tid = threadIdx.x, lane = tid & 31;
+  const bool producer = tid >= NC;
+  const int tile_bytes = P.vec_tile * 4;               // vec_tile = packed words per tile
+  unsigned char* s_stage = smem;
+  int* s_rows = reinterpret_cast<int*>(smem + (size_t)P.nst * P.rps * tile_bytes);
+  int8_t* s_q = reinterpret_cast<int8_t*>(s_rows + P.rcap);   // [rcap][TT]
+
+  const int S = P.S;
   const int ct = blockIdx.x;
   const int s = blockIdx.y;
   const int grp = blockIdx.z;
   const int tok0 = grp * TT;
   const int ntok = min(TT, a.T - tok0);
   const int d_in = a.d_in, d_out = a.d_out;
-  const int n_words = d_out / 16;
-  const int wcol = ct * kTileWords + lane;
-  const bool colok = wcol < n_words;
+  const int row_words = d_out / 16;
+  const int cword = ct * P.vec_tile;
+  const int twords = min(P.vec_tile, row_words - cword);
+  const int tbytes = twords * 4;
+  const unsigned char* Wb = reinterpret_cast<const unsigned char*>(a.wp) + (size_t)cword * 4;
+  const int lp0 = tid * LPT;                             // this thread's first lane pair of the tile
+  const int w0 = lp0 >> 3;                               // its first word
+  const int k0 = lp0 & 7;                                // its first pair inside that word
 
   pdl_begin();
-  for (int q = tid; q < TT * TILE; q += kNT) (&s_acc[0][0])[q] = 0;
-
   const int n = min(max(*a.list_count, 0), d_in);
   const int r0 = (int)(((long long)n * s) / S);
   const int r1 = (int)(((long long)n * (s + 1)) / S);
 
-  int acc[TT][16];
-#pragma unroll
-  for (int t = 0; t < TT; ++t)
-#pragma unroll
-    for (int c = 0; c < 16; ++c) acc[t][c] = 0;
+  if (tid == 0) {
+    for (int i = 0; i < P.nst; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_empty[i], NC / 32);
+    }
+    mbar_fence_init();
+    s_err = 0;
+  }
+  __syncthreads();
 
-  for (int pb = r0; pb < r1; pb += kPiece) {
-    const int np = min(kPiece, r1 - pb);
-    __syncthreads();
-    for (int j = tid; j < np; j += kNT) {
+  uint32_t pk[TT][WPT * KPW];      // two 16-bit lanes: outputs (k, k + 8) of a word
+  int acc[TT][WPT * KPW * 2];      // int32: [i][kk][lo, hi]
+  int qwin[TT];                    // sum of q over the rows since the last flush
+#pragma unroll
+  for (int t = 0; t < TT; ++t) {
+    qwin[t] = 0;
+#pragma unroll
+    for (int c = 0; c < WPT * KPW; ++c) pk[t][c] = 0u;
+#pragma unroll
+    for (int c = 0; c < WPT * KPW * 2; ++c) acc[t][c] = 0;
+  }
+  auto flush = [&]() {
+#pragma unroll
+    for (int t = 0; t < TT; ++t) {
+#pragma unroll
+      for (int c = 0; c < WPT * KPW; ++c) {
+        const uint32_t v = pk[t][c];
+        const int lo = (int)(int16_t)(uint16_t)(v & 0xFFFFu);   // signed low lane
+        const int hi = (int)(v - (uint32_t)lo) >> 16;           // signed high lane
+        acc[t][2 * c] += lo - qwin[t];
+        acc[t][2 * c + 1] += hi - qwin[t];
+        pk[t][c] = 0u;
+      }
+      qwin[t] = 0;
+    }
+  };
+  int since = 0;                                         // rows in the lanes
+
+  int gst = 0;
+  for (int pb = r0; pb < r1; pb += P.rcap) {
+    const int np = min(P.rcap, r1 - pb);
+    for (int j = tid; j < np; j += P.threads) {
       int r = a.list[pb + j];
       const bool ok = (unsigned)r < (unsigned)d_in;
       if (!ok) {
@@ -71,94 +150,161 @@ __global__ void __launch_bounds__(kNT) qgemv_kernel(QGemvArgs a) {
         r = 0;
       }
       s_rows[j] = r;
-      if (a.list_q) {
-        const int8_t* lq = a.list_q + (size_t)(pb + j) * a.T + tok0;
 #pragma unroll
-        for (int t = 0; t < TT; ++t) s_q[t][j] = (ok && t < ntok) ? (int)lq[t] : 0;
-      } else {
-#pragma unroll
-        for (int t = 0; t < TT; ++t)
-          s_q[t][j] = (ok && t < ntok) ? (int)a.xq[(size_t)(tok0 + t) * d_in + r] : 0;
+      for (int t = 0; t < TT; ++t) {
+        int8_t qv = 0;
+        if (ok && t < ntok)
+          qv = a.list_q ? a.list_q[(size_t)(pb + j) * a.T + tok0 + t]
+                        : a.xq[(size_t)(tok0 + t) * d_in + r];
+        s_q[j * TT + t] = qv;
       }
     }
     __syncthreads();
-    for (int j0 = warp * U; j0 < np; j0 += kNW * U) {
-      uint32_t wv[U];
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int j = j0 + u;
-        wv[u] = (j < np && colok) ? ld_stream_u32(a.wp + (size_t)s_rows[j] * n_words + wcol) : 0u;
-      }
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int j = j0 + u;
-        int qv[TT];
-#pragma unroll
-        for (int t = 0; t < TT; ++t) qv[t] = (j < np) ? s_q[t][j] : 0;
-        const uint32_t w = wv[u];
-#pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const int code = (int)((w >> (2 * c)) & 3u);
-          const int tv = (code & 1) - (code >> 1);     // 01 -> +1, 10 -> -1, 00 -> 0
-#pragma unroll
-          for (int t = 0; t < TT; ++t) acc[t][c] += qv[t] * tv;
+    const int nstage = (np + P.rps - 1) / P.rps;
+    if (producer) {
+      if (lane == 0) {
+        for (int st = 0; st < nstage; ++st) {
+          const int g = gst + st;
+          const int slot = g % P.nst;
+          if (g >= P.nst && !mbar_wait(&s_empty[slot], (uint32_t)((g / P.nst) - 1) & 1u)) {
+            dev_fail(a.status, DEV_TIMEOUT, 12, (uint32_t)g);
+            atomicExch(&s_err, 1);
+            break;
+          }
+          const int j0 = st * P.rps;
+          const int cnt = min(P.rps, np - j0);
+          mbar_arrive_expect_tx(&s_full[slot], (uint32_t)(cnt * tbytes));
+          for (int r = 0; r < cnt; ++r)
+            bulk_g2s(s_stage + ((size_t)slot * P.rps + r) * tile_bytes,
+                     Wb + (size_t)s_rows[j0 + r] * row_words * 4, (uint32_t)tbytes, &s_full[slot]);
         }
       }
-    }
-  }
-
-  // ---- combine warps (integer adds: exact in any order) --------------------
-#pragma unroll
-  for (int t = 0; t < TT; ++t)
-#pragma unroll
-    for (int c = 0; c < 16; ++c)
-      if (acc[t][c] != 0) atomicAdd(&s_acc[t][lane * 16 + c], acc[t][c]);
-  __syncthreads();
-
-  const bool direct = (S == 1);
-  for (int q = tid; q < TT * TILE; q += kNT) {
-    const int t = q / TILE;
-    const int gc = ct * TILE + (q - t * TILE);
-    if (t >= ntok || gc >= d_out) continue;
-    const int tok = tok0 + t;
-    const int v = s_acc[t][q - t * TILE];
-    if (direct) {
-      const float r = __fdiv_rn(__fmul_rn(a.alpha, a.gamma[tok]), 127.0f);
-      a.y[(size_t)tok * d_out + gc] = __fmul_rn(__int2float_rn(v), r);
-      if (a.acc) a.acc[(size_t)tok * d_out + gc] = v;
     } else {
-      a.parts[((size_t)s * a.T + tok) * d_out + gc] = v;
+      for (int st = 0; st < nstage; ++st) {
+        const int g = gst + st;
+        const int slot = g % P.nst;
+        const bool ready = mbar_wait_backoff(&s_full[slot], (uint32_t)(g / P.nst) & 1u);
+        if (!ready) {
+          if (lane == 0) dev_fail(a.status, DEV_TIMEOUT, 13, (uint32_t)g);
+          atomicExch(&s_err, 1);
+        }
+        const int j0 = st * P.rps;
+        const int cnt = min(P.rps, np - j0);
+        if (ready && w0 < twords) {
+          for (int r = 0; r < cnt; ++r) {
+            const uint32_t* rw =
+                reinterpret_cast<const uint32_t*>(s_stage + ((size_t)slot * P.rps + r) * tile_bytes) + w0;
+            int qv[TT];
+#pragma unroll
+            for (int t = 0; t < TT; ++t) {
+              qv[t] = s_q[(j0 + r) * TT + t];
+              qwin[t] += qv[t];
+            }
+#pragma unroll
+            for (int i = 0; i < WPT; ++i) {
+              const uint32_t u = ternary_to_u((w0 + i < twords) ? rw[i] : 0u) >> (2 * k0);
+#pragma unroll
+              for (int kk = 0; kk < KPW; ++kk) {
+                const uint32_t pair = (u >> (2 * kk)) & 0x00030003u;
+#pragma unroll
+                for (int t = 0; t < TT; ++t) pk[t][i * KPW + kk] += (uint32_t)qv[t] * pair;
+              }
+            }
+          }
+          since += cnt;
+          if (since + P.rps > kLaneRows) {
+            flush();
+            since = 0;
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_empty[slot]);
+      }
+    }
+    gst += nstage;
+    __syncthreads();
+  }
+  if (s_err && tid == 0) {
+    for (int i = 0; i < P.nst && i < gst; ++i) {
+      const int g_last = gst - 1 - i;
+      mbar_wait(&s_full[g_last % P.nst], (uint32_t)(g_last / P.nst) & 1u);
     }
   }
-  if (direct) return;
 
-  __threadfence();
-  __syncthreads();
-  int32_t* ticket = a.tickets + grp * a.plan.n_ct + ct;
-  if (tid == 0) s_last = (atomicAdd(ticket, 1) == S - 1);
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  for (int q = tid; q < TT * TILE; q += kNT) {
-    const int t = q / TILE;
-    const int gc = ct * TILE + (q - t * TILE);
-    if (t >= ntok || gc >= d_out) continue;
-    const int tok = tok0 + t;
-    const int32_t* p = a.parts + (size_t)tok * d_out + gc;
-    const size_t step = (size_t)a.T * d_out;
-    int v = 0;
-    for (int s2 = 0; s2 < S; ++s2) v += __ldcg(p + (size_t)s2 * step);
-    const float r = __fdiv_rn(__fmul_rn(a.alpha, a.gamma[tok]), 127.0f);
-    a.y[(size_t)tok * d_out + gc] = __fmul_rn(__int2float_rn(v), r);
-    if (a.acc) a.acc[(size_t)tok * d_out + gc] = v;
+  // ---- add this split's (integer) partials, exactly, as f32 --------------------
+  // lane pair (i, kk) holds output columns 16 (w0 + i) + k0 + kk and that + 8
+  const bool mine = !producer && w0 < twords;
+  if (mine) {
+    flush();
+    for (int t = 0; t < ntok; ++t) {
+      float* dst = a.parts + (size_t)(tok0 + t) * d_out + (size_t)(cword + w0) * 16 + k0;
+#pragma unroll
+      for (int i = 0; i < WPT; ++i) {
+        if (w0 + i >= twords) break;
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int kk = 0; kk < KPW; kk += 4)
+            red_add_v4_f32(dst + i * 16 + h * 8 + kk, (float)acc[t][(i * KPW + kk) * 2 + h],
+                           (float)acc[t][(i * KPW + kk + 1) * 2 + h],
+                           (float)acc[t][(i * KPW + kk + 2) * 2 + h],
+                           (float)acc[t][(i * KPW + kk + 3) * 2 + h]);
+      }
+    }
   }
+
+  // ---- last CTA of this column tile: rescale ----------------------------------
+  int32_t* ticket = a.tickets + grp * P.n_ct + ct;
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_flag = (atomicAdd(ticket, 1) == S - 1);
+  __syncthreads();
+  if (!s_flag) return;
+  __threadfence();
   if (tid == 0) *ticket = 0;
+  if (mine) {
+    for (int t = 0; t < ntok; ++t) {
+      const int tok = tok0 + t;
+      const float r = __fdiv_rn(__fmul_rn(a.alpha, a.gamma[tok]), 127.0f);
+      const size_t o = (size_t)tok * d_out + (size_t)(cword + w0) * 16 + k0;
+      float4 v[WPT][2][KPW / 4];
+#pragma unroll
+      for (int i = 0; i < WPT; ++i)
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int kk = 0; kk < KPW; kk += 4)
+            v[i][h][kk / 4] = (w0 + i < twords)
+                                  ? __ldcg(reinterpret_cast<const float4*>(a.parts + o + i * 16 + h * 8 + kk))
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int i = 0; i < WPT; ++i) {
+        if (w0 + i >= twords) break;
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int kk = 0; kk < KPW; kk += 4) {
+            const float4 f = v[i][h][kk / 4];
+            const int4 iv = make_int4(__float2int_rn(f.x), __float2int_rn(f.y), __float2int_rn(f.z),
+                                      __float2int_rn(f.w));
+            const size_t e = o + i * 16 + h * 8 + kk;
+            reinterpret_cast<float4*>(a.y + e)[0] =
+                make_float4(__fmul_rn(__int2float_rn(iv.x), r), __fmul_rn(__int2float_rn(iv.y), r),
+                            __fmul_rn(__int2float_rn(iv.z), r), __fmul_rn(__int2float_rn(iv.w), r));
+            if (a.acc) reinterpret_cast<int4*>(a.acc + e)[0] = iv;
+          }
+      }
+    }
+  }
 }
 
 template <int TT>
 cudaError_t qlaunch(const QGemvArgs& a, cudaStream_t s) {
+  static unsigned configured = 0;
+  cudaError_t e = ensure_smem_attr(qgemv_kernel<TT>, 200 * 1024, &configured);
+  if (e != cudaSuccess) return e;
   dim3 grid(a.plan.n_ct, a.plan.S, a.plan.groups);
-  cudaError_t e = launch_pdl(qgemv_kernel<TT>, grid, dim3(kNT), 0, s, a);
+  e = launch_pdl(qgemv_kernel<TT>, grid, dim3(a.plan.threads), a.plan.smem, s, a);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -224,22 +370,45 @@ GemvPlan plan_qgemv(int T, int d_out, int rows_bound) {
   GemvPlan p{};
   p.TT = (T <= 1) ? 1 : (T == 2 ? 2 : (T <= 4 ? 4 : 8));
   p.groups = (T + p.TT - 1) / p.TT;
-  const int n_words = d_out / 16;
-  p.n_ct = (n_words + kTileWords - 1) / kTileWords;
   p.mats = 1;
-  const int per_sm = (p.TT <= 2) ? 6 : (p.TT == 4 ? 4 : 2);
-  const long slots = (long)kNumSMs * per_sm;
+  const int lpt = (p.TT == 1) ? 32 : (p.TT == 2 ? 16 : (p.TT == 4 ? 8 : 4));   // lane pairs / thread
+  const int max_cons = 192;
+  const int row_words = d_out / 16;
+  const int max_words = max_cons * lpt / 8;                 // a multiple of 4
+  // near-equal column tiles of a multiple of 4 words (16-byte bulk copies)
+  int nct = (row_words + max_words - 1) / max_words;
+  if (nct < 1) nct = 1;
+  int tile = ((row_words + nct - 1) / nct + 3) / 4 * 4;
+  if (tile > max_words) tile = max_words;
+  p.n_ct = (row_words + tile - 1) / tile;
+  p.vec_tile = tile;                                          // packed words per tile
+  const int cons = (tile * 8 + lpt - 1) / lpt;
+  p.threads = ((cons + 31) / 32) * 32 + 32;
+  const int tile_bytes = tile * 4;
+  p.rps = (16384 + tile_bytes / 2) / tile_bytes;
+  if (p.rps < 1) p.rps = 1;
+  if (p.rps > 16) p.rps = 16;
+  const long ring = 90 * 1024;                               // two CTAs per SM
+  long nst = ring / ((long)p.rps * tile_bytes);
+  if (nst < 3) nst = 3;
+  if (nst > 32) nst = 32;
+  p.nst = (int)nst;
+  p.rcap = 1024;
+  p.smem = (size_t)p.nst * p.rps * tile_bytes + (size_t)p.rcap * (4 + p.TT);
+  const long slots = (long)kNumSMs * 2;
   const long units = (long)p.n_ct * p.groups;
   long S = slots / (units > 0 ? units : 1);
   if (S < 1) S = 1;
-  const long max_by_rows = rows_bound / 16;
+  const long max_by_rows = rows_bound / 8;       // keep >= ~8 rows per split
   if (S > max_by_rows) S = max_by_rows > 0 ? max_by_rows : 1;
   if (S > 256) S = 256;
   p.S = (int)S;
-  p.parts_elems = (size_t)p.S * (size_t)T * d_out;
+  p.parts_elems = (size_t)T * d_out;             // f32 accumulators, zeroed by the top-K kernel
   p.tickets = p.groups * p.n_ct;
   return p;
 }
+
+bool qgemv_supported(int d_out) { return d_out % 64 == 0; }   // 16-byte aligned packed rows
 
 cudaError_t launch_qgemv(const QGemvArgs& a, cudaStream_t s) {
   if (a.T <= 0) return cudaSuccess;
