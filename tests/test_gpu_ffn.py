@@ -104,3 +104,67 @@ def test_ffn_small_and_ragged(act, dtype, T, dm, dff):
     bias = -0.3 if act == "drelu" else None
     for k_in, k_h in ((dm, dff), ((7 * dm) // 10, (7 * dff) // 10), (1, 1), (dm, 0)):
         _check_ffn(x, up, gate, down, act, k_in, k_h, dtype, bias=bias)
+
+
+def _check_ffn_list_path(x, up, gate, down, act, k_in, k_h, dtype, bias=None, ws=None):
+    """One token, no idx_h_out: the up/gate epilogue marks the nonzero h in a
+    bitmask and the top-K on h starts from it (all nonzeros when there are at
+    most K of them, else a full selection).  The kept set is checked through
+    the row count and y against the oracle re-run on the top-K of the GPU's
+    own h (ranking given f32 values is exact)."""
+    T, d_model = x.shape
+    d_ff = up.shape[1]
+    xt = to_dev(x, dtype)
+    upt, gatet, downt = to_dev(up, dtype), to_dev(gate, dtype), to_dev(down, dtype)
+    b = None if bias is None else torch.full((d_ff,), bias, dtype=torch.float32, device="cuda")
+    if ws is None:
+        ws = qs.new_workspace(qs.QS_OP_SPARSE_FFN, T, d_model, d_ff, k_h, xt.device)
+    r = qs.qs_sparse_ffn(xt, upt, gatet, downt, act, k_in, k_h, b_up=b, b_gate=b, h_out=True, ws=ws)
+    check_status(ws)
+    bnp = None if bias is None else np.full(d_ff, bias)
+    ref = oracle.sparse_ffn(x, up, gate, down, act, k_in, k_h, b_up=bnp, b_gate=bnp)
+    h_gpu = r.h.cpu().numpy()
+    assert oracle.max_rel_err(h_gpu, ref["h"]) <= TOL_F32
+    keep_h = oracle.topk_keep(h_gpu.astype(np.float64), k_h)
+    ref_sel = oracle.sparse_ffn(x, up, gate, down, act, k_in, k_h, b_up=bnp, b_gate=bnp,
+                                keep_h=keep_h)
+    tol = TOL_F32 if dtype == "f32" else TOL_BF16
+    assert oracle.max_rel_err(to_np(r.y), ref_sel["y"]) <= tol
+    _, rows_h = qs.qs_workspace_stats(ws, qs.QS_OP_SPARSE_FFN, T, d_model, d_ff, k_h)
+    assert rows_h == int(np.count_nonzero(h_gpu[0, keep_h[0]]))
+    return r, ws
+
+
+def test_ffn_one_token_list_path_llama7b():
+    """Llama-7B shape: about half of h is zero, fewer than K_h nonzeros, so the
+    kept rows are exactly the nonzero h.  Two tokens in a row on one workspace
+    (the bitmask must be left clear), then a several-token call."""
+    need_gpu()
+    w = workloads.WORKLOADS["ffn_relu2_llama7b"]
+    up, gate, down = _ffn_weights(w.name)
+    x2 = workloads.activations(w, 2)
+    # two different tokens in a row: a bitmask left over from the first call
+    # would add the first token's nonzero h to the second token's row count
+    _, ws = _check_ffn_list_path(x2[:1], up, gate, down, "relu2_glu", w.k, w.k_h, "bf16")
+    _check_ffn_list_path(x2[1:], up, gate, down, "relu2_glu", w.k, w.k_h, "bf16", ws=ws)
+    x8 = workloads.activations(w, 8)
+    _check_ffn(x8, up, gate, down, "relu2_glu", w.k, w.k_h, "bf16")
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("dm,dff", [(64, 96), (200, 328), (128, 1000), (96, 16384)])
+def test_ffn_one_token_list_path_small(dtype, dm, dff):
+    """Both branches of the bitmask start: K_h above and below the nonzero
+    count of h (and K_h = 0, K_h = d_ff), ragged d_ff, the largest d_ff it takes."""
+    need_gpu()
+    g = workloads.rng(dm * 7 + dff)
+    x = workloads.round_to_dtype(workloads.normal_f32(g, (1, dm)), dtype)
+    up = workloads.round_to_dtype(workloads.normal_f32(g, (dm, dff), dm ** -0.5), dtype)
+    gate = workloads.round_to_dtype(workloads.normal_f32(g, (dm, dff), dm ** -0.5), dtype)
+    down = workloads.round_to_dtype(workloads.normal_f32(g, (dff, dm), dff ** -0.5), dtype)
+    k_hs = (dff, (7 * dff) // 10, dff // 5, 1, 0)
+    need = max(qs.qs_workspace_size(qs.QS_OP_SPARSE_FFN, 1, dm, dff, k) for k in k_hs)
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")      # one workspace for every call
+    for act, bias in (("relu2_glu", None), ("drelu", -0.3)):
+        for k_h in k_hs:
+            _check_ffn_list_path(x, up, gate, down, act, (7 * dm) // 10, k_h, dtype, bias=bias, ws=ws)

@@ -401,6 +401,10 @@ qs_status qs_sparse_ffn(const void* x, int dtype, int T, int d_model, int d_ff, 
     g.zero = w.at<float>(L.parts2);
     g.zero_n = p_dn.parts_elems;
     g.status = w.status();
+    // one token, list outputs only: the epilogue marks the nonzero h, and the
+    // top-K on h starts from that bitmask (it clears it again)
+    const bool h_bits = Tc == 1 && idx_h_out == nullptr && topk_bitmask_supported(Tc, d_ff, TK_F32);
+    if (h_bits) g.hbits = reinterpret_cast<uint32_t*>(w.ticket(L, kUnionH));
     QS_TRY_CUDA(launch_gemv(g, s));
     if (timed) QS_TRY_CUDA(mark(2));
 
@@ -414,6 +418,7 @@ qs_status qs_sparse_ffn(const void* x, int dtype, int T, int d_model, int d_ff, 
     b.list_count = w.at<int32_t>(L.cnt) + 1;
     b.ticket = w.ticket(L, kTkTopkH);
     b.union_bits = reinterpret_cast<uint32_t*>(w.ticket(L, kUnionH));
+    if (h_bits) b.nz_bits = b.union_bits;
     b.status = w.status();
     QS_TRY_CUDA(launch_topk(b, s));
     if (timed) QS_TRY_CUDA(mark(3));

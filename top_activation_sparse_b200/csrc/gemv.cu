@@ -108,6 +108,12 @@ __device__ __forceinline__ void epilogue(const GemvArgs& a, int tok, int col,
       }
     }
     store_f32<V>(a.h + o, hv);
+    if (a.hbits != nullptr) {                      // one token: publish which h are nonzero
+      uint32_t m = 0;
+#pragma unroll
+      for (int e = 0; e < V; ++e) m |= (hv[e] != 0.0f ? 1u : 0u) << e;
+      if (m != 0u) atomicOr(a.hbits + col / 32, m << (col % 32));
+    }
   }
 }
 

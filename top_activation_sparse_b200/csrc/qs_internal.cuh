@@ -247,12 +247,21 @@ struct TopkArgs {
   int32_t* list_count = nullptr;
   int32_t* ticket = nullptr;
   uint32_t* union_bits = nullptr;  // [ceil(d/32)] zero between calls (several tokens)
+  uint32_t* nz_bits = nullptr;     // one token: bitmask of the row's nonzero entries, written by
+                                   // the kernel that produced the row; read, then zeroed, here
   float* zero = nullptr;     // accumulators of the next kernel: set to 0 here
   size_t zero_n = 0;         // floats, multiple of 4
   DevStatus* status = nullptr;
+  // set by launch_topk from the sizes
+  int stage = 0;             // the row's list (or idx) is staged in shared memory
+  int hist16 = 0;            // bf16: one 15-bit radix pass (packed 16-bit counters)
+  int zero_ctas = 0;         // CTAs after the T row CTAs that only zero `zero`
 };
 
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s);
+// True when launch_topk takes a one-token row of this size through the list
+// kernel, which can consume (and then clears) a producer's nonzero bitmask.
+bool topk_bitmask_supported(int T, int d, int kind);
 
 // Zero `n` floats (n % 4 == 0) cooperatively across the whole grid.
 __device__ __forceinline__ void grid_zero(float* p, size_t n) {
@@ -281,6 +290,7 @@ struct GemvArgs {
   const float* b_gate = nullptr;
   float* zero = nullptr;       // accumulators of the next kernel: set to 0 here
   size_t zero_n = 0;
+  uint32_t* hbits = nullptr;   // mode 1/2, one token: OR the bitmask of nonzero h in here
   DevStatus* status = nullptr;
   GemvPlan plan{};
 };

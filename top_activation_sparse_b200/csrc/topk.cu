@@ -28,6 +28,8 @@
 // values, or int8 codes) and a list of input rows that carry a kept nonzero
 // value; with several token rows the last CTA to finish (an atomic ticket, no
 // waiting) merges the rows into the union list.
+#include <algorithm>
+
 #include "qs_internal.cuh"
 
 namespace qs {
@@ -127,7 +129,7 @@ __global__ void __launch_bounds__(NT) topk_kernel(TopkArgs a) {
   constexpr uint32_t MASK = KT::kMask;
   constexpr bool QUANT = (KIND == TK_QUANT_F32 || KIND == TK_QUANT_BF16);
 
-  extern __shared__ uint32_t s_ent[];          // [d]
+  extern __shared__ uint32_t s_ent[];          // [d], then the staged list [k], then hist16
   __shared__ int s_hist[kMaxBins];
   __shared__ uint32_t s_scan[2][2 * (NW + 1)];
   __shared__ uint32_t s_sel[3];
@@ -143,7 +145,18 @@ __global__ void __launch_bounds__(NT) topk_kernel(TopkArgs a) {
   int sbuf = 0;
 
   pdl_begin();
-  grid_zero(a.zero, a.zero_n);
+  if (row >= a.T) {
+    // zeroing CTAs: clear the next kernel's accumulators, nothing else
+    if (a.zero != nullptr) {
+      const size_t nthr = (size_t)a.zero_ctas * NT;
+      const float4 z = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      for (size_t i = (size_t)(row - a.T) * NT + tid; i < a.zero_n / 4; i += nthr)
+        reinterpret_cast<float4*>(a.zero)[i] = z;
+    }
+    return;
+  }
+  // dynamic layout (word offsets rounded to 4 so that hist16 is 16-byte aligned)
+  uint32_t* s_stg = s_ent + ((d + 3) & ~3);      // [k] when a.stage
   uint32_t my_nnz = 0;
 
   // ---- 1. entries --------------------------------------------------------
@@ -204,6 +217,56 @@ __global__ void __launch_bounds__(NT) topk_kernel(TopkArgs a) {
     // At most K nonzero entries: every nonzero beats every zero, so all of
     // them are kept together with the lowest-index zeros (threshold key 0).
     P = 0u; shift = 0; remaining = k - nnz;
+  } else if (KIND == TK_BF16 && NT == 1024 && a.hist16) {
+    // One pass over the whole 15-bit |x| key: 32768 bins kept as packed
+    // 16-bit counters (a bin counts at most d < 65536 entries, so the low
+    // half never carries into the high half).
+    uint32_t* h16 = s_stg + (a.stage ? ((k + 3) & ~3) : 0);
+    for (int j = tid; j < 4096; j += NT) reinterpret_cast<uint4*>(h16)[j] = make_uint4(0u, 0u, 0u, 0u);
+    __syncthreads();
+    for (int i = tid; i < d; i += NT) {
+      const uint32_t key = s_ent[i] & 0x7fffu;
+      atomicAdd(&h16[key >> 1], 1u << ((key & 1u) * 16u));
+    }
+    __syncthreads();
+    if (tid == 0) s_sel[0] = 0xffffffffu;
+    // thread j sums bins [32768 - 32 (j+1), 32768 - 32 j): largest keys first
+    uint32_t local = 0;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint4 v = reinterpret_cast<const uint4*>(h16)[4095 - 4 * tid - q];
+      local += (v.x & 0xffffu) + (v.x >> 16) + (v.y & 0xffffu) + (v.y >> 16) + (v.z & 0xffffu) +
+               (v.z >> 16) + (v.w & 0xffffu) + (v.w >> 16);
+    }
+    uint32_t excl, unused_e, tot, unused_t;
+    block_scan2<NT>(local, 0u, s_scan[sbuf], excl, unused_e, tot, unused_t);
+    sbuf ^= 1;
+    remaining = k;
+    if ((int)excl < remaining && remaining <= (int)(excl + local)) {
+      int run = (int)excl;
+      const int top = 32767 - 32 * tid;
+      for (int b = 0; b < 32; ++b) {
+        const int bin = top - b;
+        const int c = (int)((h16[bin >> 1] >> ((bin & 1) * 16)) & 0xffffu);
+        if (run + c >= remaining) {
+          s_sel[0] = (uint32_t)bin;
+          s_sel[1] = (uint32_t)run;
+          s_sel[2] = (uint32_t)c;
+          break;
+        }
+        run += c;
+      }
+    }
+    __syncthreads();
+    const uint32_t digit = s_sel[0];
+    shift = 0;
+    if (digit == 0xffffffffu) {                     // counts inconsistent: report
+      if (tid == 0) dev_fail(a.status, DEV_CHECK, 1, (uint32_t)row);
+      P = 0xffffffffu;
+    } else {
+      remaining -= (int)s_sel[1];
+      P = digit;
+    }
   } else {
     uint32_t prefix = 0;
     remaining = k;
@@ -283,6 +346,8 @@ __global__ void __launch_bounds__(NT) topk_kernel(TopkArgs a) {
   // whole digit is kept (early stop), so its nonzero count is exact.
   int nzb = gtb + (P != 0u ? min(eqb, remaining) : (int)e_eqnz);
   const bool list_direct = (a.list != nullptr) && (a.T == 1);
+  const bool stage_list = list_direct && a.stage;            // list positions < list count <= k
+  const bool stage_idx = !list_direct && a.stage && a.idx;   // idx positions < k
   for (int i = i0; i < i1; ++i) {
     const uint32_t ent = s_ent[i];
     const uint32_t key = ent & MASK;
@@ -293,21 +358,29 @@ __global__ void __launch_bounds__(NT) topk_kernel(TopkArgs a) {
     if (sel) {
       const int pos = gtb + min(eqb, remaining);
       if (pos < k) {
-        const size_t o = (size_t)row * (size_t)k + (size_t)pos;
-        if (a.idx) a.idx[o] = i;
-        if (a.val) {
-          if constexpr (KIND == TK_F32) reinterpret_cast<uint32_t*>(a.val)[o] = ent;
-          else if constexpr (KIND == TK_BF16) reinterpret_cast<uint16_t*>(a.val)[o] = (uint16_t)ent;
+        if (stage_idx) {
+          s_stg[pos] = (uint32_t)i;
+        } else {
+          const size_t o = (size_t)row * (size_t)k + (size_t)pos;
+          if (a.idx) a.idx[o] = i;
+          if (a.val) {
+            if constexpr (KIND == TK_F32) reinterpret_cast<uint32_t*>(a.val)[o] = ent;
+            else if constexpr (KIND == TK_BF16) reinterpret_cast<uint16_t*>(a.val)[o] = (uint16_t)ent;
+          }
         }
       } else {
         dev_fail(a.status, DEV_CHECK, 2, (uint32_t)row);   // inconsistent select
       }
       if (list_direct && key != 0u) {
-        a.list[nzb] = i;
-        if constexpr (QUANT) {
-          if (a.list_q) a.list_q[nzb] = (int8_t)(ent >> 8);
+        if (stage_list) {
+          s_stg[nzb] = (uint32_t)i;
         } else {
-          if (a.list_val) a.list_val[nzb] = raw_to_f32<KIND>(ent);
+          a.list[nzb] = i;
+          if constexpr (QUANT) {
+            if (a.list_q) a.list_q[nzb] = (int8_t)(ent >> 8);
+          } else {
+            if (a.list_val) a.list_val[nzb] = raw_to_f32<KIND>(ent);
+          }
         }
         ++nzb;
       }
@@ -322,6 +395,35 @@ __global__ void __launch_bounds__(NT) topk_kernel(TopkArgs a) {
     *a.list_count = tot_gt + (P != 0u ? min(tot_eq, remaining) : (int)t_eqnz);
   }
   __syncthreads();
+  // staged list / idx: coalesced copy-out (kept entries keep their bits in s_ent)
+  if (stage_list) {
+    const int tot_gt = (int)(t_ge & 0xffffu), tot_eq = (int)(t_ge >> 16);
+    const int cnt = min(k, tot_gt + (P != 0u ? min(tot_eq, remaining) : (int)t_eqnz));
+    for (int j = tid; j < cnt; j += NT) {
+      const int i = (int)s_stg[j];
+      const uint32_t ent = s_ent[i];
+      a.list[j] = i;
+      if constexpr (QUANT) {
+        if (a.list_q) a.list_q[j] = (int8_t)(ent >> 8);
+      } else {
+        if (a.list_val) a.list_val[j] = raw_to_f32<KIND>(ent);
+      }
+    }
+  }
+  if (stage_idx) {
+    const int tot_gt = (int)(t_ge & 0xffffu), tot_eq = (int)(t_ge >> 16);
+    const int nsel = min(k, tot_gt + min(tot_eq, remaining));
+    for (int j = tid; j < nsel; j += NT) {
+      const int i = (int)s_stg[j];
+      const uint32_t ent = s_ent[i];
+      const size_t o = (size_t)row * (size_t)k + (size_t)j;
+      a.idx[o] = i;
+      if (a.val) {
+        if constexpr (KIND == TK_F32) reinterpret_cast<uint32_t*>(a.val)[o] = ent;
+        else if constexpr (KIND == TK_BF16) reinterpret_cast<uint16_t*>(a.val)[o] = (uint16_t)ent;
+      }
+    }
+  }
   // coalesced dense outputs; with several tokens also OR this row's kept
   // nonzeros into the union bitmask (one atomic per 32 inputs)
   const bool want_union = (a.list != nullptr) && (a.T > 1);
@@ -380,14 +482,584 @@ __global__ void __launch_bounds__(NT) topk_kernel(TopkArgs a) {
   }
 }
 
-template <int KIND, int NT>
-cudaError_t launch_kind(const TopkArgs& a, cudaStream_t s) {
-  const size_t smem = (size_t)a.d * sizeof(uint32_t);
-  static unsigned configured = 0;
-  cudaError_t e = ensure_smem_attr(topk_kernel<KIND, NT>, (int)(QS_MAX_ROW * sizeof(uint32_t)),
-                                   &configured);
+// ---- register-resident variant (rows of up to 16 K elements) -------------
+// Each thread keeps EPT elements of the row in registers, element j*NT + tid
+// in slot j, so loads and stores of a slot are coalesced and ballots over a
+// slot follow index order.  Radix digits are 8 bits (256 bins, scanned by one
+// warp).  Compaction: one ballot per slot gives each warp its counts of
+// entries above / at the threshold; one warp turns the (slot, warp) table into
+// exclusive prefixes, and every kept entry then knows its final position from
+// the prefix plus its rank in the ballot: no per-element shared-memory traffic
+// and three barriers for the whole compaction.
+template <int KIND> struct RegKeys;
+template <> struct RegKeys<TK_F32> {
+  static constexpr int kPasses = 4;
+  __device__ static constexpr int shift(int p) { return p == 0 ? 23 : (p == 1 ? 15 : (p == 2 ? 7 : 0)); }
+  __device__ static constexpr int width(int p) { return p == 3 ? 7 : 8; }
+};
+template <> struct RegKeys<TK_BF16> {
+  static constexpr int kPasses = 2;
+  __device__ static constexpr int shift(int p) { return p == 0 ? 7 : 0; }
+  __device__ static constexpr int width(int p) { return p == 0 ? 8 : 7; }
+};
+struct RegQuantKeys {
+  static constexpr int kPasses = 1;
+  __device__ static constexpr int shift(int) { return 0; }
+  __device__ static constexpr int width(int) { return 8; }
+};
+template <> struct RegKeys<TK_QUANT_F32> : RegQuantKeys {};
+template <> struct RegKeys<TK_QUANT_BF16> : RegQuantKeys {};
+
+// K-th largest key of the row held in registers: after this an entry is kept
+// iff (key >> shift) > P, or it equals P and fewer than `remaining` equal
+// entries precede it.  Each radix pass: a 256-bin shared-memory histogram,
+// one warp scans it (largest digits first) and publishes the digit.  `hist`
+// holds NP cleared histograms, `sel` three words.
+template <int KIND, int NT, int EPT>
+__device__ __forceinline__ void reg_select(const uint32_t (&ent)[EPT], int d, int k, int nnz,
+                                           int (*hist)[256], uint32_t* sel, DevStatus* status,
+                                           int row, uint32_t& P, int& shift, int& remaining) {
+  using RK = RegKeys<KIND>;
+  constexpr uint32_t MASK = KeyTraits<KIND>::kMask;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (k <= 0) {
+    P = 0xffffffffu; shift = 31; remaining = 0;        // nothing is kept
+    return;
+  }
+  if (k >= d) {
+    P = 0u; shift = 31; remaining = d;                 // every key >> 31 == 0: all kept
+    return;
+  }
+  if (nnz <= k) {
+    // at most K nonzero entries: all of them, plus the lowest-index zeros
+    P = 0u; shift = 0; remaining = k - nnz;
+    return;
+  }
+  uint32_t prefix = 0;
+  remaining = k;
+  shift = 0;
+#pragma unroll 1
+  for (int p = 0; p < RK::kPasses; ++p) {
+    const int sh = RK::shift(p);
+    const int nb = 1 << RK::width(p);
+    const int hi = sh + RK::width(p);
+    const uint32_t himask = hi >= 32 ? 0u : (0xffffffffu << hi);
+    int* h = hist[p];
+#pragma unroll
+    for (int j = 0; j < EPT; ++j) {
+      const uint32_t key = ent[j] & MASK;
+      if (j * NT + tid < d && ((key ^ prefix) & himask) == 0u)
+        atomicAdd(&h[(key >> sh) & (uint32_t)(nb - 1)], 1);
+    }
+    __syncthreads();
+    if (warp == 0) {
+      // lane l: bins [nb - (l+1) bpl, nb - l bpl), largest digits first
+      const int bpl = nb / 32;
+      const int top = nb - 1 - lane * bpl;
+      int cnt[8];
+      int local = 0;
+#pragma unroll
+      for (int b = 0; b < 8; ++b) {
+        cnt[b] = b < bpl ? h[top - b] : 0;
+        local += cnt[b];
+      }
+      int inc = local;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(kFull, inc, o);
+        if (lane >= o) inc += v;
+      }
+      const int excl = inc - local;
+      const bool mine = excl < remaining && remaining <= inc;
+      if (__ballot_sync(kFull, mine) == 0u && lane == 0) sel[0] = 0xffffffffu;
+      if (mine) {
+        int run = excl;
+        bool done = false;
+#pragma unroll
+        for (int b = 0; b < 8; ++b) {
+          if (!done && b < bpl) {
+            if (run + cnt[b] >= remaining) {
+              sel[0] = (uint32_t)(top - b);
+              sel[1] = (uint32_t)run;
+              sel[2] = (uint32_t)cnt[b];
+              done = true;
+            } else {
+              run += cnt[b];
+            }
+          }
+        }
+      }
+    }
+    __syncthreads();
+    const uint32_t digit = sel[0];
+    if (digit == 0xffffffffu) {                        // counts inconsistent: report, keep nothing
+      if (tid == 0) dev_fail(status, DEV_CHECK, 1, (uint32_t)row);
+      P = 0xffffffffu; shift = 0; remaining = 0;
+      return;
+    }
+    remaining -= (int)sel[1];
+    prefix |= digit << sh;
+    shift = sh;
+    if ((int)sel[2] == remaining) break;               // the whole digit is kept
+    // every thread has read sel before the next pass's first barrier
+  }
+  P = prefix >> shift;
+}
+
+// One token row, list outputs only (the projection path): the kept nonzero
+// entries in index order with their values, and their count.  An entry is in
+// the list iff it is kept and nonzero, which is
+//   key != 0                           when P == 0 (every nonzero is kept), else
+//   c > P, or c == P among the first `remaining` such entries (c = key >> shift).
+template <int KIND, int NT, int EPT>
+__global__ void __launch_bounds__(NT) topk_list_kernel(TopkArgs a) {
+  constexpr int NW = NT / 32;
+  constexpr int NP = RegKeys<KIND>::kPasses;
+  constexpr int E = EPT * NW;
+  constexpr uint32_t MASK = KeyTraits<KIND>::kMask;
+  constexpr bool QUANT = (KIND == TK_QUANT_F32 || KIND == TK_QUANT_BF16);
+
+  __shared__ int s_hist[NP][256];
+  __shared__ uint32_t s_cnt[E];                     // definite | ties << 16 per (slot, warp)
+  __shared__ uint32_t s_wred[NW];
+  __shared__ uint32_t s_wnnz[NW];
+  __shared__ uint32_t s_tot;
+  __shared__ uint32_t s_sel[3];
+
+  const int d = a.d;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t lt = (1u << lane) - 1u;
+
+  pdl_begin();
+  if constexpr (!QUANT) {
+    if (a.nz_bits != nullptr) {
+      // The producer left a bitmask of the row's nonzero entries (d <= 32 NT,
+      // one word per thread).  With at most K nonzeros the list is exactly the
+      // nonzeros in index order, and every CTA of the grid writes its NT
+      // entries at positions given by a prefix over the bitmask.  Otherwise
+      // CTA 0 goes on with the full selection below.
+      __shared__ uint32_t s_word[NT];
+      __shared__ uint32_t s_wpre[NT];
+      __shared__ uint32_t s_scan[2 * (NW + 1)];
+      __shared__ int s_last;
+      const int nwords = (d + 31) >> 5;
+      const uint32_t bits = tid < nwords ? __ldcg(a.nz_bits + tid) : 0u;
+      const int e = (int)blockIdx.x * NT + tid;
+      const uint32_t raw = e < d ? load_raw<KIND>(a.x, e) : 0u;
+      uint32_t excl, unused_e, tot, unused_t;
+      block_scan2<NT>((uint32_t)__popc(bits), 0u, s_scan, excl, unused_e, tot, unused_t);
+      s_word[tid] = bits;
+      s_wpre[tid] = excl;
+      __syncthreads();
+      if (tid == 0) s_last = (atomicAdd(a.ticket, 1) == (int)gridDim.x - 1);
+      __syncthreads();
+      if (s_last) {                                  // every CTA has read the bitmask
+        if (tid < nwords) a.nz_bits[tid] = 0u;
+        if (tid == 0) *a.ticket = 0;
+      }
+      if ((int)tot <= a.k) {
+        if (blockIdx.x == 0 && tid == 0) *a.list_count = (int)tot;
+        if (e < d) {
+          const uint32_t wb = s_word[e >> 5];
+          if ((wb >> lane) & 1u) {
+            const int pos = (int)s_wpre[e >> 5] + __popc(wb & lt);
+            a.list[pos] = e;
+            a.list_val[pos] = raw_to_f32<KIND>(raw);
+          }
+        }
+        return;
+      }
+      if (blockIdx.x != 0) return;
+      __syncthreads();                               // s_scan is reused below
+    }
+  }
+  if (blockIdx.x >= 1) {
+    if (a.zero != nullptr) {
+      const size_t nthr = (size_t)a.zero_ctas * NT;
+      const float4 z = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      for (size_t i = (size_t)(blockIdx.x - 1) * NT + tid; i < a.zero_n / 4; i += nthr)
+        reinterpret_cast<float4*>(a.zero)[i] = z;
+    }
+    return;
+  }
+  for (int j = tid; j < NP * 256; j += NT) (&s_hist[0][0])[j] = 0;
+
+  uint32_t ent[EPT];
+#pragma unroll
+  for (int j = 0; j < EPT; ++j) {
+    const int e = j * NT + tid;
+    ent[j] = e < d ? load_raw<KIND>(a.x, e) : 0u;
+  }
+  if constexpr (QUANT) {
+    uint32_t m = 0;
+#pragma unroll
+    for (int j = 0; j < EPT; ++j) m = max(m, raw_abs_f32bits<KIND>(ent[j]));   // padding is 0
+    m = __reduce_max_sync(kFull, m);
+    if (lane == 0) s_wred[warp] = m;
+    __syncthreads();
+    const uint32_t amax_bits = __reduce_max_sync(kFull, lane < NW ? s_wred[lane] : 0u);
+    const float gamma = __fadd_rn(__uint_as_float(amax_bits), a.eps);
+    const float scale = __fdiv_rn(127.0f, gamma);
+    if (tid == 0 && a.gamma) a.gamma[0] = gamma;
+#pragma unroll
+    for (int j = 0; j < EPT; ++j) {
+      int qi = __float2int_rn(__fmul_rn(raw_to_f32<KIND>(ent[j]), scale));
+      qi = min(127, max(-127, qi));
+      const uint32_t mag = (uint32_t)(qi < 0 ? -qi : qi);
+      ent[j] = j * NT + tid < d ? (mag | ((uint32_t)(uint8_t)(int8_t)qi << 8)) : 0u;
+    }
+  }
+  uint32_t my_nnz = 0;
+#pragma unroll
+  for (int j = 0; j < EPT; ++j) my_nnz += ((ent[j] & MASK) != 0u);   // padding is 0
+  my_nnz = __reduce_add_sync(kFull, my_nnz);
+  if (lane == 0) s_wnnz[warp] = my_nnz;
+  __syncthreads();
+  const int nnz = (int)__reduce_add_sync(kFull, lane < NW ? s_wnnz[lane] : 0u);
+
+  uint32_t P;
+  int shift, remaining;
+  reg_select<KIND, NT, EPT>(ent, d, a.k, nnz, s_hist, s_sel, a.status, 0, P, shift, remaining);
+  const bool ties = P != 0u;
+
+#pragma unroll
+  for (int j = 0; j < EPT; ++j) {
+    const uint32_t key = ent[j] & MASK;              // padding: key 0, never listed
+    const uint32_t c = key >> shift;
+    const uint32_t bd = __ballot_sync(kFull, ties ? c > P : key != 0u);
+    const uint32_t bt = __ballot_sync(kFull, ties && c == P);
+    if (lane == j) s_cnt[j * NW + warp] = (uint32_t)__popc(bd) | ((uint32_t)__popc(bt) << 16);
+  }
+  __syncthreads();
+  if (warp == 0) {
+    constexpr int CH = (E + 31) / 32;
+    const int b0 = min(lane * CH, E), b1 = min(b0 + CH, E);
+    uint32_t sg = 0;
+    for (int i = b0; i < b1; ++i) sg += s_cnt[i];
+    uint32_t ig = sg;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t v = __shfl_up_sync(kFull, ig, o);
+      if (lane >= o) ig += v;
+    }
+    uint32_t eg = ig - sg;
+    for (int i = b0; i < b1; ++i) {
+      const uint32_t c = s_cnt[i];
+      s_cnt[i] = eg;
+      eg += c;
+    }
+    if (lane == 31) s_tot = ig;
+  }
+  __syncthreads();
+  if (tid == 0) *a.list_count = (int)(s_tot & 0xffffu) + min((int)(s_tot >> 16), remaining);
+#pragma unroll
+  for (int j = 0; j < EPT; ++j) {
+    const uint32_t key = ent[j] & MASK;
+    const uint32_t c = key >> shift;
+    const bool def = ties ? c > P : key != 0u;
+    const bool tie = ties && c == P;
+    const uint32_t bd = __ballot_sync(kFull, def);
+    const uint32_t bt = __ballot_sync(kFull, tie);
+    const uint32_t pre = s_cnt[j * NW + warp];
+    const int def_b = (int)(pre & 0xffffu) + __popc(bd & lt);
+    const int tie_b = (int)(pre >> 16) + __popc(bt & lt);
+    if (def || (tie && tie_b < remaining)) {
+      const int pos = def_b + min(tie_b, remaining);
+      a.list[pos] = j * NT + tid;
+      if constexpr (QUANT) a.list_q[pos] = (int8_t)(ent[j] >> 8);
+      else a.list_val[pos] = raw_to_f32<KIND>(ent[j]);
+    }
+  }
+}
+
+template <int KIND, int NT, int EPT>
+__global__ void __launch_bounds__(NT) topk_reg_kernel(TopkArgs a) {
+  using RK = RegKeys<KIND>;
+  constexpr int NW = NT / 32;
+  constexpr int NP = RK::kPasses;
+  constexpr int E = EPT * NW;                       // (slot, warp) table size
+  constexpr uint32_t MASK = KeyTraits<KIND>::kMask;
+  constexpr bool QUANT = (KIND == TK_QUANT_F32 || KIND == TK_QUANT_BF16);
+
+  __shared__ int s_hist[NP][256];
+  __shared__ uint32_t s_cnt[E];                     // gt | eq << 16 per (slot, warp), then prefixes
+  __shared__ uint32_t s_cnz[E];                     // eq with a nonzero key, then prefixes
+  __shared__ uint32_t s_wred[NW];
+  __shared__ uint32_t s_wnnz[NW];
+  __shared__ uint32_t s_tot[2];
+  __shared__ uint32_t s_sel[3];
+  __shared__ uint32_t s_scan[2 * (NW + 1)];
+  __shared__ int s_last;
+
+  const int row = blockIdx.x;
+  const int d = a.d;
+  const int k = a.k;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const size_t rbase = (size_t)row * (size_t)d;
+  const uint32_t lt = (1u << lane) - 1u;
+
+  pdl_begin();
+  if (row >= a.T) {
+    if (a.zero != nullptr) {
+      const size_t nthr = (size_t)a.zero_ctas * NT;
+      const float4 z = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      for (size_t i = (size_t)(row - a.T) * NT + tid; i < a.zero_n / 4; i += nthr)
+        reinterpret_cast<float4*>(a.zero)[i] = z;
+    }
+    return;
+  }
+  for (int j = tid; j < NP * 256; j += NT) (&s_hist[0][0])[j] = 0;
+
+  // ---- 1. entries in registers ---------------------------------------------
+  uint32_t ent[EPT];
+#pragma unroll
+  for (int j = 0; j < EPT; ++j) {
+    const int e = j * NT + tid;
+    ent[j] = e < d ? load_raw<KIND>(a.x, rbase + e) : 0u;
+  }
+  if constexpr (QUANT) {
+    uint32_t m = 0;
+#pragma unroll
+    for (int j = 0; j < EPT; ++j)
+      if (j * NT + tid < d) m = max(m, raw_abs_f32bits<KIND>(ent[j]));
+    m = __reduce_max_sync(kFull, m);
+    if (lane == 0) s_wred[warp] = m;
+    __syncthreads();
+    const uint32_t amax_bits = __reduce_max_sync(kFull, lane < NW ? s_wred[lane] : 0u);
+    const float gamma = __fadd_rn(__uint_as_float(amax_bits), a.eps);
+    const float scale = __fdiv_rn(127.0f, gamma);
+    if (tid == 0 && a.gamma) a.gamma[row] = gamma;
+#pragma unroll
+    for (int j = 0; j < EPT; ++j) {
+      const int e = j * NT + tid;
+      if (e < d) {
+        int qi = __float2int_rn(__fmul_rn(raw_to_f32<KIND>(ent[j]), scale));
+        qi = min(127, max(-127, qi));
+        const uint32_t mag = (uint32_t)(qi < 0 ? -qi : qi);
+        ent[j] = mag | ((uint32_t)(uint8_t)(int8_t)qi << 8);
+        if (a.q_full) a.q_full[rbase + e] = (int8_t)qi;
+      }
+    }
+  }
+  uint32_t my_nnz = 0;
+#pragma unroll
+  for (int j = 0; j < EPT; ++j) my_nnz += (j * NT + tid < d && (ent[j] & MASK) != 0u);
+  my_nnz = __reduce_add_sync(kFull, my_nnz);
+  if (lane == 0) s_wnnz[warp] = my_nnz;
+  __syncthreads();                                  // also orders the histogram clear
+  const int nnz = (int)__reduce_add_sync(kFull, lane < NW ? s_wnnz[lane] : 0u);
+
+  // ---- 2. the K-th largest key ----------------------------------------------
+  uint32_t P;
+  int shift;
+  int remaining;
+  reg_select<KIND, NT, EPT>(ent, d, k, nnz, s_hist, s_sel, a.status, row, P, shift, remaining);
+
+  // ---- 3. compaction in index order ------------------------------------------
+#pragma unroll
+  for (int j = 0; j < EPT; ++j) {
+    const bool valid = j * NT + tid < d;
+    const uint32_t key = ent[j] & MASK;
+    const uint32_t c = key >> shift;
+    const bool eq = valid && c == P;
+    const uint32_t bg = __ballot_sync(kFull, valid && c > P);
+    const uint32_t be = __ballot_sync(kFull, eq);
+    const uint32_t bz = __ballot_sync(kFull, eq && key != 0u);
+    if (lane == j) {
+      s_cnt[j * NW + warp] = (uint32_t)__popc(bg) | ((uint32_t)__popc(be) << 16);
+      s_cnz[j * NW + warp] = (uint32_t)__popc(bz);
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    // exclusive prefixes over the (slot, warp) table, warps fastest: index order
+    constexpr int CH = (E + 31) / 32;
+    const int b0 = min(lane * CH, E), b1 = min(b0 + CH, E);
+    uint32_t sg = 0, sz = 0;
+    for (int i = b0; i < b1; ++i) { sg += s_cnt[i]; sz += s_cnz[i]; }
+    uint32_t ig = sg, iz = sz;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t vg = __shfl_up_sync(kFull, ig, o);
+      const uint32_t vz = __shfl_up_sync(kFull, iz, o);
+      if (lane >= o) { ig += vg; iz += vz; }
+    }
+    uint32_t eg = ig - sg, ez = iz - sz;
+    for (int i = b0; i < b1; ++i) {
+      const uint32_t cg = s_cnt[i], cz = s_cnz[i];
+      s_cnt[i] = eg; s_cnz[i] = ez;
+      eg += cg; ez += cz;
+    }
+    if (lane == 31) { s_tot[0] = ig; s_tot[1] = iz; }
+  }
+  __syncthreads();
+  const int tot_gt = (int)(s_tot[0] & 0xffffu), tot_eq = (int)(s_tot[0] >> 16);
+  const int tot_eqnz = (int)s_tot[1];
+  const bool list_direct = (a.list != nullptr) && (a.T == 1);
+  if (list_direct && tid == 0) *a.list_count = tot_gt + (P != 0u ? min(tot_eq, remaining) : tot_eqnz);
+  const bool want_union = (a.list != nullptr) && (a.T > 1);
+#pragma unroll
+  for (int j = 0; j < EPT; ++j) {
+    const int e = j * NT + tid;
+    const bool valid = e < d;
+    const uint32_t key = ent[j] & MASK;
+    const uint32_t c = key >> shift;
+    const bool gt = valid && c > P;
+    const bool eq = valid && c == P;
+    const uint32_t bg = __ballot_sync(kFull, gt);
+    const uint32_t be = __ballot_sync(kFull, eq);
+    const uint32_t bz = __ballot_sync(kFull, eq && key != 0u);
+    const uint32_t pre = s_cnt[j * NW + warp];
+    const int gt_b = (int)(pre & 0xffffu) + __popc(bg & lt);
+    const int eq_b = (int)(pre >> 16) + __popc(be & lt);
+    const int eqnz_b = (int)s_cnz[j * NW + warp] + __popc(bz & lt);
+    const bool sel = gt || (eq && eq_b < remaining);
+    if (sel) {
+      const int pos = gt_b + min(eq_b, remaining);
+      if (pos < k) {
+        const size_t o = (size_t)row * (size_t)k + (size_t)pos;
+        if (a.idx) a.idx[o] = e;
+        if (a.val) {
+          if constexpr (KIND == TK_F32) reinterpret_cast<uint32_t*>(a.val)[o] = ent[j];
+          else if constexpr (KIND == TK_BF16) reinterpret_cast<uint16_t*>(a.val)[o] = (uint16_t)ent[j];
+        }
+      } else {
+        dev_fail(a.status, DEV_CHECK, 2, (uint32_t)row);
+      }
+      if (list_direct && key != 0u) {
+        const int nzp = gt_b + (P != 0u ? min(eq_b, remaining) : eqnz_b);
+        a.list[nzp] = e;
+        if constexpr (QUANT) {
+          if (a.list_q) a.list_q[nzp] = (int8_t)(ent[j] >> 8);
+        } else {
+          if (a.list_val) a.list_val[nzp] = raw_to_f32<KIND>(ent[j]);
+        }
+      }
+    }
+    if (valid) {
+      const uint32_t v = sel ? ent[j] : 0u;
+      if (a.mask) a.mask[rbase + e] = sel ? 1 : 0;
+      if constexpr (QUANT) {
+        if (a.xq) a.xq[rbase + e] = (int8_t)(v >> 8);
+      } else {
+        if (a.xsf) a.xsf[rbase + e] = raw_to_f32<KIND>(v);
+        if (a.xs) {
+          if constexpr (KIND == TK_F32) reinterpret_cast<uint32_t*>(a.xs)[rbase + e] = v;
+          else reinterpret_cast<uint16_t*>(a.xs)[rbase + e] = (uint16_t)v;
+        }
+      }
+    }
+    if (want_union) {
+      const uint32_t b = __ballot_sync(kFull, sel && key != 0u);
+      if (lane == 0 && b != 0u) atomicOr(a.union_bits + (j * NT + warp * 32) / 32, b);
+    }
+  }
+
+  // ---- 4. union of the rows' kept nonzeros (several tokens) ------------------
+  if (want_union) {
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) s_last = (atomicAdd(a.ticket, 1) == a.T - 1);
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    const int nwords = (d + 31) / 32;
+    const int wpt = (nwords + NT - 1) / NT;
+    const int w0 = min(tid * wpt, nwords);
+    const int w1 = min(w0 + wpt, nwords);
+    uint32_t n_any = 0;
+    for (int w = w0; w < w1; ++w) n_any += __popc(__ldcg(a.union_bits + w));
+    uint32_t e_any, e_unused, t_any, t_unused;
+    block_scan2<NT>(n_any, 0u, s_scan, e_any, e_unused, t_any, t_unused);
+    int pos = (int)e_any;
+    for (int w = w0; w < w1; ++w) {
+      uint32_t bits = __ldcg(a.union_bits + w);
+      a.union_bits[w] = 0u;
+      while (bits) {
+        const int bpos = __ffs(bits) - 1;
+        a.list[pos++] = w * 32 + bpos;
+        bits &= bits - 1u;
+      }
+    }
+    if (tid == 0) {
+      *a.list_count = (int)t_any;
+      *a.ticket = 0;
+    }
+  }
+}
+
+// The list-only kernel serves one token row whose only outputs are the list,
+// its values and count (and gamma): the projection path's decode step.
+bool list_only(const TopkArgs& a) {
+  const bool quant = a.kind == TK_QUANT_F32 || a.kind == TK_QUANT_BF16;
+  return a.T == 1 && a.list != nullptr && a.list_count != nullptr && a.idx == nullptr &&
+         a.val == nullptr && a.mask == nullptr && a.xs == nullptr && a.xsf == nullptr &&
+         a.xq == nullptr && a.q_full == nullptr &&
+         (quant ? a.list_q != nullptr : a.list_val != nullptr);
+}
+
+template <int KIND, int NT, int EPT>
+cudaError_t launch_reg(const TopkArgs& a_in, cudaStream_t s) {
+  TopkArgs a = a_in;
+  a.stage = 0;
+  a.hist16 = 0;
+  a.zero_ctas = 0;
+  if (a.zero != nullptr && a.zero_n >= 4)
+    a.zero_ctas = (int)std::min<size_t>((a.zero_n / 4 + NT - 1) / NT, 32);
+  cudaError_t e;
+  if (list_only(a) && a.nz_bits != nullptr) {
+    if (a.zero != nullptr || NT != 1024 || a.kind == TK_QUANT_F32 || a.kind == TK_QUANT_BF16)
+      return cudaErrorInvalidValue;                 // not a configuration the API builds
+    a.zero_ctas = 0;
+    e = launch_pdl(topk_list_kernel<KIND, NT, EPT>, dim3((a.d + NT - 1) / NT), dim3(NT), (size_t)0, s, a);
+  } else if (list_only(a))
+    e = launch_pdl(topk_list_kernel<KIND, NT, EPT>, dim3(1 + a.zero_ctas), dim3(NT), (size_t)0, s, a);
+  else
+    e = launch_pdl(topk_reg_kernel<KIND, NT, EPT>, dim3(a.T + a.zero_ctas), dim3(NT), (size_t)0, s, a);
   if (e != cudaSuccess) return e;
-  e = launch_pdl(topk_kernel<KIND, NT>, dim3(a.T), dim3(NT), smem, s, a);
+  return cudaGetLastError();
+}
+
+// Register-resident launch when the row fits (EPT <= 16); false otherwise.
+template <int KIND>
+bool try_launch_reg(const TopkArgs& a, cudaStream_t s, cudaError_t* err) {
+  if (a.T >= 2 * kNumSMs) {                      // many rows: 256-thread CTAs
+    if (a.d <= 256 * 4) { *err = launch_reg<KIND, 256, 4>(a, s); return true; }
+    if (a.d <= 256 * 8) { *err = launch_reg<KIND, 256, 8>(a, s); return true; }
+    if (a.d <= 256 * 16) { *err = launch_reg<KIND, 256, 16>(a, s); return true; }
+    return false;
+  }
+  if (a.d <= 1024 * 1) { *err = launch_reg<KIND, 1024, 1>(a, s); return true; }
+  if (a.d <= 1024 * 2) { *err = launch_reg<KIND, 1024, 2>(a, s); return true; }
+  if (a.d <= 1024 * 4) { *err = launch_reg<KIND, 1024, 4>(a, s); return true; }
+  if (a.d <= 1024 * 8) { *err = launch_reg<KIND, 1024, 8>(a, s); return true; }
+  if (a.d <= 1024 * 12) { *err = launch_reg<KIND, 1024, 12>(a, s); return true; }
+  if (a.d <= 1024 * 16) { *err = launch_reg<KIND, 1024, 16>(a, s); return true; }
+  return false;
+}
+
+constexpr size_t kTopkSmemMax = 216 * 1024;   // dynamic; the static arrays take ~9 KB
+static_assert((size_t)QS_MAX_ROW * 4 <= kTopkSmemMax, "a full row must fit");
+
+template <int KIND, int NT>
+cudaError_t launch_kind(const TopkArgs& a_in, cudaStream_t s) {
+  TopkArgs a = a_in;
+  const bool list_direct = a.list != nullptr && a.T == 1;
+  const bool want_stage = list_direct || a.idx != nullptr;
+  const size_t d4 = ((size_t)a.d + 3) / 4 * 4, k4 = ((size_t)a.k + 3) / 4 * 4;
+  a.stage = (want_stage && (d4 + k4) * 4 <= kTopkSmemMax) ? 1 : 0;
+  const size_t words = d4 + (a.stage ? k4 : 0);
+  a.hist16 = (KIND == TK_BF16 && NT == 1024 && (words + 16384) * 4 <= kTopkSmemMax) ? 1 : 0;
+  const size_t smem = (words + (a.hist16 ? 16384 : 0)) * sizeof(uint32_t);
+  a.zero_ctas = 0;
+  if (a.zero != nullptr && a.zero_n >= 4) {
+    const size_t v = a.zero_n / 4;
+    a.zero_ctas = (int)std::min<size_t>((v + NT - 1) / NT, 32);
+  }
+  static unsigned configured = 0;
+  cudaError_t e = ensure_smem_attr(topk_kernel<KIND, NT>, (int)kTopkSmemMax, &configured);
+  if (e != cudaSuccess) return e;
+  e = launch_pdl(topk_kernel<KIND, NT>, dim3(a.T + a.zero_ctas), dim3(NT), smem, s, a);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -405,8 +1077,23 @@ cudaError_t launch_nt(const TopkArgs& a, cudaStream_t s) {
 
 }  // namespace
 
+bool topk_bitmask_supported(int T, int d, int kind) {
+  return T == 1 && d >= 1 && d <= 1024 * 16 && (kind == TK_F32 || kind == TK_BF16);
+}
+
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s) {
   if (a.T <= 0 || a.d <= 0) return cudaSuccess;
+  cudaError_t err = cudaSuccess;
+  bool done = false;
+  switch (a.kind) {
+    case TK_F32: done = try_launch_reg<TK_F32>(a, s, &err); break;
+    case TK_BF16: done = try_launch_reg<TK_BF16>(a, s, &err); break;
+    case TK_QUANT_F32: done = try_launch_reg<TK_QUANT_F32>(a, s, &err); break;
+    case TK_QUANT_BF16: done = try_launch_reg<TK_QUANT_BF16>(a, s, &err); break;
+    default: return cudaErrorInvalidValue;
+  }
+  if (done) return err;
+  // longer rows: the shared-memory kernel
   // Few rows: a full 1024-thread CTA per row keeps the latency down.  Many
   // rows (prefill): 256-thread CTAs so that several rows share an SM.
   if (a.T >= 2 * kNumSMs) return launch_nt<256>(a, s);
