@@ -177,14 +177,14 @@ struct GemvPlan {
   int n_ct;        // column tiles
   int S;           // splits of the row list
   int mats;        // weight matrices sharing the row list (2 for up/gate)
-  size_t parts_elems;  // partial-sum buffer, f32 elements (splits + split groups)
+  size_t parts_elems;  // partial-sum buffer, f32 elements (all copies)
   int tickets;     // ticket counters the launch uses
   // gather-GEMV pipeline (bulk-copy ring), unused by the int8 path
   int vec_tile;    // 16-byte vectors of one row segment (= consumer threads used)
   int threads;     // consumer threads (multiple of 32) + one producer warp
   int rps;         // rows per pipeline stage
   int nst;         // pipeline stages
-  int ng;          // groups of up to 8 splits (two-level reduction)
+  int copies;      // accumulator copies: split s adds into copy s % copies (fewer adds per address)
   int rcap;        // rows staged in shared memory per piece
   size_t smem;     // dynamic shared memory bytes
 };

@@ -237,7 +237,8 @@ __global__ void __launch_bounds__(QTune<TT>::kMaxConsumers + 32, 2) qgemv_kernel
   if (mine) {
     flush();
     for (int t = 0; t < ntok; ++t) {
-      float* dst = a.parts + (size_t)(tok0 + t) * d_out + (size_t)(cword + w0) * 16 + k0;
+      float* dst = a.parts + (size_t)(s % P.copies) * a.T * d_out + (size_t)(tok0 + t) * d_out +
+                   (size_t)(cword + w0) * 16 + k0;
 #pragma unroll
       for (int i = 0; i < WPT; ++i) {
         if (w0 + i >= twords) break;
@@ -273,10 +274,22 @@ __global__ void __launch_bounds__(QTune<TT>::kMaxConsumers + 32, 2) qgemv_kernel
 #pragma unroll
         for (int h = 0; h < 2; ++h)
 #pragma unroll
-          for (int kk = 0; kk < KPW; kk += 4)
-            v[i][h][kk / 4] = (w0 + i < twords)
-                                  ? __ldcg(reinterpret_cast<const float4*>(a.parts + o + i * 16 + h * 8 + kk))
-                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int kk = 0; kk < KPW; kk += 4) v[i][h][kk / 4] = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int c = 0; c < P.copies; ++c) {
+        const float* pc = a.parts + (size_t)c * a.T * d_out + o;
+#pragma unroll
+        for (int i = 0; i < WPT; ++i) {
+          if (w0 + i >= twords) break;
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int kk = 0; kk < KPW; kk += 4) {
+              const float4 f = __ldcg(reinterpret_cast<const float4*>(pc + i * 16 + h * 8 + kk));
+              float4& acc4 = v[i][h][kk / 4];
+              acc4.x += f.x; acc4.y += f.y; acc4.z += f.z; acc4.w += f.w;
+            }
+        }
+      }
 #pragma unroll
       for (int i = 0; i < WPT; ++i) {
         if (w0 + i >= twords) break;
@@ -374,7 +387,10 @@ GemvPlan plan_qgemv(int T, int d_out, int rows_bound) {
   const int lpt = (p.TT == 1) ? 32 : (p.TT == 2 ? 16 : (p.TT == 4 ? 8 : 4));   // lane pairs / thread
   const int max_cons = 192;
   const int row_words = d_out / 16;
-  const int max_words = max_cons * lpt / 8;                 // a multiple of 4
+  // one token: tiles of <= 192 words (3 KB of packed row), so that the
+  // epilogue is spread over several CTAs and fewer splits share an address
+  // (measured on 4096 -> 11008: 4 tiles 16.4 us, 1 tile 21.6 us)
+  const int max_words = (p.TT == 1) ? 192 : max_cons * lpt / 8;   // a multiple of 4
   // near-equal column tiles of a multiple of 4 words (16-byte bulk copies)
   int nct = (row_words + max_words - 1) / max_words;
   if (nct < 1) nct = 1;
@@ -403,7 +419,10 @@ GemvPlan plan_qgemv(int T, int d_out, int rows_bound) {
   if (S > max_by_rows) S = max_by_rows > 0 ? max_by_rows : 1;
   if (S > 256) S = 256;
   p.S = (int)S;
-  p.parts_elems = (size_t)T * d_out;             // f32 accumulators, zeroed by the top-K kernel
+  // one accumulator copy: summing copies in the epilogue cost more than the
+  // contention it removed on these sizes (measured)
+  p.copies = 1;
+  p.parts_elems = (size_t)p.copies * T * d_out;  // zeroed by the top-K kernel
   p.tickets = p.groups * p.n_ct;
   return p;
 }
