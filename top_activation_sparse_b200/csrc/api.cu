@@ -54,22 +54,29 @@ bool ws_layout(int op, int T, int d_in, int d_out, int k, WsLayout* L) {
   const int Tc = T < kChunkT ? T : kChunkT;
   // Partial-sum buffers are sized for the largest plan any chunk (1..Tc
   // tokens) of either dtype can pick: a short last chunk may split more.
-  auto max_parts = [&](int d_out_, int d_rows, int kk, int mats) {
+  // The number of accumulator copies grows with the splits, i.e. with K, so
+  // the buffers are sized for every K up to the row length: a workspace stays
+  // valid for calls of the same sizes with any K.
+  (void)k;
+  auto max_parts = [&](int d_out_, int d_rows, int /*kk*/, int mats) {
     size_t m = 0;
     for (int t = 1; t <= Tc; ++t) {
-      const int rb = (int)rows_bound(t, d_rows, kk);
-      for (int eb = 2; eb <= 4; eb += 2) {
-        const GemvPlan p = plan_gemv(t, d_out_, rb, mats, eb);
-        if (p.parts_elems > m) m = p.parts_elems;
+      for (int rb : {(int)rows_bound(t, d_rows, 1), (int)rows_bound(t, d_rows, d_rows)}) {
+        for (int eb = 2; eb <= 4; eb += 2) {
+          const GemvPlan p = plan_gemv(t, d_out_, rb, mats, eb);
+          if (p.parts_elems > m) m = p.parts_elems;
+        }
       }
     }
     return m;
   };
-  auto max_qparts = [&](int d_out_, int d_rows, int kk) {
+  auto max_qparts = [&](int d_out_, int d_rows, int /*kk*/) {
     size_t m = 0;
     for (int t = 1; t <= Tc; ++t) {
-      const GemvPlan p = plan_qgemv(t, d_out_, (int)rows_bound(t, d_rows, kk));
-      if (p.parts_elems > m) m = p.parts_elems;
+      for (int rb : {(int)rows_bound(t, d_rows, 1), (int)rows_bound(t, d_rows, d_rows)}) {
+        const GemvPlan p = plan_qgemv(t, d_out_, rb);
+        if (p.parts_elems > m) m = p.parts_elems;
+      }
     }
     return m;
   };
