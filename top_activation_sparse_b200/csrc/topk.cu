@@ -515,19 +515,27 @@ template <> struct RegKeys<TK_QUANT_BF16> : RegQuantKeys {};
 // entries precede it.  Each radix pass: a 256-bin shared-memory histogram,
 // one warp scans it (largest digits first) and publishes the digit.  `hist`
 // holds NP cleared histograms, `sel` three words.
-template <int KIND, int NT, int EPT>
+// Element j of a thread is row entry j*NT + tid (CONTIG false) or tid*EPT + j
+// (CONTIG true).  `tied` returns how many entries equal the threshold key
+// when that is known to be at most `remaining` (all of them kept), else a
+// larger value.
+template <int KIND, int NT, int EPT, bool CONTIG = false>
 __device__ __forceinline__ void reg_select(const uint32_t (&ent)[EPT], int d, int k, int nnz,
                                            int (*hist)[256], uint32_t* sel, DevStatus* status,
-                                           int row, uint32_t& P, int& shift, int& remaining) {
+                                           int row, uint32_t& P, int& shift, int& remaining,
+                                           int* tied = nullptr) {
   using RK = RegKeys<KIND>;
   constexpr uint32_t MASK = KeyTraits<KIND>::kMask;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tied) *tied = 0x7fffffff;
   if (k <= 0) {
     P = 0xffffffffu; shift = 31; remaining = 0;        // nothing is kept
+    if (tied) *tied = 0;
     return;
   }
   if (k >= d) {
     P = 0u; shift = 31; remaining = d;                 // every key >> 31 == 0: all kept
+    if (tied) *tied = d;
     return;
   }
   if (nnz <= k) {
@@ -548,7 +556,8 @@ __device__ __forceinline__ void reg_select(const uint32_t (&ent)[EPT], int d, in
 #pragma unroll
     for (int j = 0; j < EPT; ++j) {
       const uint32_t key = ent[j] & MASK;
-      if (j * NT + tid < d && ((key ^ prefix) & himask) == 0u)
+      const int e = CONTIG ? tid * EPT + j : j * NT + tid;
+      if (e < d && ((key ^ prefix) & himask) == 0u)
         atomicAdd(&h[(key >> sh) & (uint32_t)(nb - 1)], 1);
     }
     __syncthreads();
@@ -600,7 +609,11 @@ __device__ __forceinline__ void reg_select(const uint32_t (&ent)[EPT], int d, in
     remaining -= (int)sel[1];
     prefix |= digit << sh;
     shift = sh;
-    if ((int)sel[2] == remaining) break;               // the whole digit is kept
+    if ((int)sel[2] == remaining) {                    // the whole digit is kept
+      if (tied) *tied = remaining;
+      break;
+    }
+    if (p == RK::kPasses - 1 && tied) *tied = (int)sel[2];   // entries equal to the full key
     // every thread has read sel before the next pass's first barrier
   }
   P = prefix >> shift;
@@ -988,6 +1001,93 @@ __global__ void __launch_bounds__(NT) topk_reg_kernel(TopkArgs a) {
   }
 }
 
+// Many bf16 rows whose only output is X_sparse (the prefill path): each thread
+// owns 16 contiguous entries, loaded and stored as two 16-byte vectors.  Zero
+// entries are 0 in X_sparse whether kept or not, so ties need ranking only at
+// a nonzero threshold that splits them (a block scan of per-thread counts).
+template <int NT>
+__global__ void __launch_bounds__(NT) topk_dense_bf16_kernel(TopkArgs a) {
+  constexpr int EPT = 16;
+  constexpr int NW = NT / 32;
+  constexpr int NP = RegKeys<TK_BF16>::kPasses;
+  constexpr uint32_t MASK = KeyTraits<TK_BF16>::kMask;
+  __shared__ int s_hist[NP][256];
+  __shared__ uint32_t s_sel[3];
+  __shared__ uint32_t s_wnnz[NW];
+  __shared__ uint32_t s_scan[2 * (NW + 1)];
+
+  const int row = blockIdx.x;
+  const int d = a.d;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int e0 = tid * EPT;
+  const uint16_t* xr = reinterpret_cast<const uint16_t*>(a.x) + (size_t)row * d;
+  uint16_t* xsr = reinterpret_cast<uint16_t*>(a.xs) + (size_t)row * d;
+
+  pdl_begin();
+  for (int j = tid; j < NP * 256; j += NT) (&s_hist[0][0])[j] = 0;
+  uint32_t ent[EPT];
+  if (e0 + EPT <= d) {                               // d % 8 == 0: rows are 16-byte aligned
+    const uint4 v0 = ld_stream_v4(xr + e0);
+    const uint4 v1 = ld_stream_v4(xr + e0 + 8);
+    const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+    for (int q = 0; q < 8; ++q) { ent[2 * q] = w[q] & 0xffffu; ent[2 * q + 1] = w[q] >> 16; }
+  } else {
+#pragma unroll
+    for (int j = 0; j < EPT; ++j) ent[j] = e0 + j < d ? (uint32_t)xr[e0 + j] : 0u;
+  }
+  uint32_t my_nnz = 0;
+#pragma unroll
+  for (int j = 0; j < EPT; ++j) my_nnz += ((ent[j] & MASK) != 0u);
+  my_nnz = __reduce_add_sync(kFull, my_nnz);
+  if (lane == 0) s_wnnz[warp] = my_nnz;
+  __syncthreads();
+  const int nnz = (int)__reduce_add_sync(kFull, lane < NW ? s_wnnz[lane] : 0u);
+
+  uint32_t P;
+  int shift, remaining, tied;
+  reg_select<TK_BF16, NT, EPT, true>(ent, d, a.k, nnz, s_hist, s_sel, a.status, row, P, shift,
+                                     remaining, &tied);
+  // ties at a nonzero threshold that are not all kept: rank them by index
+  int eq_b = 0;
+  if (P != 0u && remaining < tied) {
+    uint32_t my_eq = 0;
+#pragma unroll
+    for (int j = 0; j < EPT; ++j) my_eq += (e0 + j < d && ((ent[j] & MASK) >> shift) == P);
+    uint32_t excl, unused_e, tot, unused_t;
+    block_scan2<NT>(my_eq, 0u, s_scan, excl, unused_e, tot, unused_t);
+    eq_b = (int)excl;
+  } else {
+    eq_b = -0x40000000;                              // every tie is below `remaining`
+  }
+  uint32_t out[8];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) out[q] = 0u;
+#pragma unroll
+  for (int j = 0; j < EPT; ++j) {
+    const uint32_t c = (ent[j] & MASK) >> shift;
+    const bool eq = c == P;
+    const bool keep = c > P || (eq && eq_b < remaining);
+    eq_b += eq;
+    if (keep) out[j >> 1] |= ent[j] << (16 * (j & 1));
+  }
+  if (e0 + EPT <= d) {
+    reinterpret_cast<uint4*>(xsr + e0)[0] = make_uint4(out[0], out[1], out[2], out[3]);
+    reinterpret_cast<uint4*>(xsr + e0)[1] = make_uint4(out[4], out[5], out[6], out[7]);
+  } else {
+#pragma unroll
+    for (int j = 0; j < EPT; ++j)
+      if (e0 + j < d) xsr[e0 + j] = (uint16_t)(out[j >> 1] >> (16 * (j & 1)));
+  }
+}
+
+bool dense_only_bf16(const TopkArgs& a) {
+  return a.kind == TK_BF16 && a.xs != nullptr && a.idx == nullptr && a.val == nullptr &&
+         a.mask == nullptr && a.xsf == nullptr && a.xq == nullptr && a.list == nullptr &&
+         a.zero == nullptr && a.d <= 256 * 16 && (a.d % 8) == 0 &&
+         ((uintptr_t)a.x & 15u) == 0 && ((uintptr_t)a.xs & 15u) == 0;
+}
+
 // The list-only kernel serves one token row whose only outputs are the list,
 // its values and count (and gamma): the projection path's decode step.
 bool list_only(const TopkArgs& a) {
@@ -1024,6 +1124,11 @@ cudaError_t launch_reg(const TopkArgs& a_in, cudaStream_t s) {
 template <int KIND>
 bool try_launch_reg(const TopkArgs& a, cudaStream_t s, cudaError_t* err) {
   if (a.T >= 2 * kNumSMs) {                      // many rows: 256-thread CTAs
+    if (KIND == TK_BF16 && dense_only_bf16(a)) {
+      *err = launch_pdl(topk_dense_bf16_kernel<256>, dim3(a.T), dim3(256), (size_t)0, s, a);
+      if (*err == cudaSuccess) *err = cudaGetLastError();
+      return true;
+    }
     if (a.d <= 256 * 4) { *err = launch_reg<KIND, 256, 4>(a, s); return true; }
     if (a.d <= 256 * 8) { *err = launch_reg<KIND, 256, 8>(a, s); return true; }
     if (a.d <= 256 * 16) { *err = launch_reg<KIND, 256, 16>(a, s); return true; }
