@@ -309,6 +309,282 @@ __global__ void __launch_bounds__(kMaxConsumers + 32, (TT <= 4) ? 2 : 1) gemv_ke
   }
 }
 
+// ---- batched decode on the tensor cores ------------------------------------
+// With 4 or 8 tokens the FMA path spends 32-64 FMAs per 16-byte weight vector
+// and stops being HBM-bound.  Here the staged rows feed warp-level
+// mma.sync m16n8k16 (bf16 x bf16 -> f32): A = the weight tile read as
+// [16 columns x 16 rows] with ldmatrix.trans (rows sit in shared memory with
+// their columns contiguous), B = the 16 rows' values for 8 token slots
+// (rounded to bf16), C = 16 columns x 8 tokens in registers.  Rows are staged
+// 16 per ring stage at a padded pitch (tile bytes + 16), which keeps the
+// ldmatrix row addresses in distinct bank groups.  Split sums, tickets and
+// the epilogue are those of gemv_kernel.
+constexpr int kMmaWarps = 8;                       // consumer warps
+constexpr int kMmaBPW = 12;                        // 16-column blocks per warp (max)
+constexpr int kMmaRows = 16;                       // rows per stage (the MMA's K)
+
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1,
+                                              uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                               uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+template <int TT, int MODE>
+__global__ void __launch_bounds__(kMmaWarps * 32 + 32, 2) gemv_mma_kernel(GemvArgs a) {
+  constexpr int V = 8;
+  constexpr int NC = kMmaWarps * 32;
+  extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ __align__(8) uint64_t s_full[kMaxStages];
+  __shared__ __align__(8) uint64_t s_empty[kMaxStages];
+  __shared__ int s_flag;
+  __shared__ int s_err;
+
+  const GemvPlan& P = a.plan;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const bool producer = warp == kMmaWarps;
+  const int pitch = P.vec_tile * 16 + 16;
+  const int stage_bytes = kMmaRows * pitch;
+  unsigned char* s_stage = smem;
+  int* s_rows = reinterpret_cast<int*>(smem + (size_t)P.nst * stage_bytes);
+  float* s_vals = reinterpret_cast<float*>(s_rows + P.rcap);
+
+  const int S = P.S;
+  const int ct = blockIdx.x;
+  const int mat = blockIdx.y / S;
+  const int s = blockIdx.y - mat * S;
+  const int grp = blockIdx.z;
+  const int tok0 = grp * TT;
+  const int ntok = min(TT, a.T - tok0);
+  const int d_in = a.d_in, d_out = a.d_out;
+  const size_t row_bytes = (size_t)d_out * 2;
+  const size_t cbyte = (size_t)ct * P.vec_tile * 16;
+  const int tbytes = (int)min((size_t)P.vec_tile * 16, row_bytes - cbyte);
+  const int tvec = tbytes / 16;
+  const int nblk = tbytes / 32;                    // 16-column blocks (d_out % 16 == 0)
+  const unsigned char* Wb = reinterpret_cast<const unsigned char*>(a.w[mat]) + cbyte;
+
+  pdl_begin();
+  grid_zero(a.zero, a.zero_n);
+  const int n = min(max(*a.list_count, 0), d_in);
+  const int r0 = (int)(((long long)n * s) / S);
+  const int r1 = (int)(((long long)n * (s + 1)) / S);
+
+  if (tid == 0) {
+    for (int i = 0; i < P.nst; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_empty[i], kMmaWarps);
+    }
+    mbar_fence_init();
+    s_err = 0;
+  }
+  __syncthreads();
+
+  float acc[kMmaBPW][4];
+#pragma unroll
+  for (int b = 0; b < kMmaBPW; ++b)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[b][e] = 0.0f;
+
+  // ldmatrix row address of this lane inside a 16 x 16 block: matrices
+  // (k 0-7, m 0-7), (k 0-7, m 8-15), (k 8-15, m 0-7), (k 8-15, m 8-15)
+  const int q = lane >> 3;
+  const uint32_t lane_off = (uint32_t)(((q >> 1) * 8 + (lane & 7)) * pitch + (q & 1) * 16);
+  const uint32_t ring_addr = (uint32_t)__cvta_generic_to_shared(s_stage);
+  const int bn = lane >> 2;                         // token slot of this lane's B values
+  const int bk = (lane & 3) * 2;                    // first row of this lane's B values
+
+  int gst = 0;
+  for (int pb = r0; pb < r1; pb += P.rcap) {
+    const int np = min(P.rcap, r1 - pb);
+    for (int j = tid; j < np; j += blockDim.x) {
+      int r = a.list[pb + j];
+      const bool ok = (unsigned)r < (unsigned)d_in;
+      if (!ok) {
+        dev_fail(a.status, DEV_CHECK, 3, (uint32_t)r);
+        r = 0;
+      }
+      s_rows[j] = r;
+#pragma unroll
+      for (int t = 0; t < TT; ++t)
+        s_vals[t * P.rcap + j] = (ok && t < ntok)
+                                     ? (a.list_val ? a.list_val[(size_t)(pb + j) * a.T + tok0 + t]
+                                                   : a.xsf[(size_t)(tok0 + t) * d_in + r])
+                                     : 0.0f;
+    }
+    __syncthreads();
+    const int nstage = (np + kMmaRows - 1) / kMmaRows;
+    if (producer) {
+      if (lane == 0) {
+        for (int st = 0; st < nstage; ++st) {
+          const int g = gst + st;
+          const int slot = g % P.nst;
+          if (g >= P.nst && !mbar_wait(&s_empty[slot], (uint32_t)((g / P.nst) - 1) & 1u)) {
+            dev_fail(a.status, DEV_TIMEOUT, 14, (uint32_t)g);
+            atomicExch(&s_err, 1);
+            break;
+          }
+          const int j0 = st * kMmaRows;
+          const int cnt = min(kMmaRows, np - j0);
+          mbar_arrive_expect_tx(&s_full[slot], (uint32_t)(cnt * tbytes));
+          for (int r = 0; r < cnt; ++r)
+            bulk_g2s(s_stage + (size_t)slot * stage_bytes + (size_t)r * pitch,
+                     Wb + (size_t)s_rows[j0 + r] * row_bytes, (uint32_t)tbytes, &s_full[slot]);
+        }
+      }
+    } else {
+      for (int st = 0; st < nstage; ++st) {
+        const int g = gst + st;
+        const int slot = g % P.nst;
+        const bool ready = mbar_wait_backoff(&s_full[slot], (uint32_t)(g / P.nst) & 1u);
+        if (!ready) {
+          if (lane == 0) dev_fail(a.status, DEV_TIMEOUT, 15, (uint32_t)g);
+          atomicExch(&s_err, 1);
+        }
+        const int j0 = st * kMmaRows;
+        const int cnt = min(kMmaRows, np - j0);
+        unsigned char* sb = s_stage + (size_t)slot * stage_bytes;
+        if (cnt < kMmaRows) {
+          // rows past the list's end: zero them (a stale NaN times a zero value
+          // would still poison the sum); consumer warps sync on a named barrier
+          for (int i = tid; i < (kMmaRows - cnt) * tvec; i += NC) {
+            const int rr = cnt + i / tvec, vv = i % tvec;
+            *reinterpret_cast<uint4*>(sb + (size_t)rr * pitch + (size_t)vv * 16) = make_uint4(0u, 0u, 0u, 0u);
+          }
+          asm volatile("bar.sync 1, %0;" ::"r"(NC) : "memory");
+        }
+        if (ready) {
+          // B: rows bk, bk+1 and bk+8, bk+9 of the stage for token slot bn
+          float x0 = 0.f, x1 = 0.f, x8 = 0.f, x9 = 0.f;
+          if (bn < TT) {
+            const float* vp = s_vals + bn * P.rcap + j0;
+            if (bk < cnt) x0 = vp[bk];
+            if (bk + 1 < cnt) x1 = vp[bk + 1];
+            if (bk + 8 < cnt) x8 = vp[bk + 8];
+            if (bk + 9 < cnt) x9 = vp[bk + 9];
+          }
+          const uint32_t b0 = pack_bf16x2(x0, x1), b1 = pack_bf16x2(x8, x9);
+          const uint32_t base = ring_addr + (uint32_t)((size_t)slot * stage_bytes) + lane_off;
+#pragma unroll
+          for (int b = 0; b < kMmaBPW; ++b) {
+            const int blk = warp + b * kMmaWarps;
+            if (blk < nblk) {
+              uint32_t a0, a1, a2, a3;
+              ldsm_x4_trans(base + (uint32_t)(blk * 32), a0, a1, a2, a3);
+              mma_bf16_16816(acc[b], a0, a1, a2, a3, b0, b1);
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_empty[slot]);
+      }
+    }
+    gst += nstage;
+    __syncthreads();
+  }
+  if (s_err && tid == 0) {
+    for (int i = 0; i < P.nst && i < gst; ++i) {
+      const int g_last = gst - 1 - i;
+      mbar_wait(&s_full[g_last % P.nst], (uint32_t)(g_last / P.nst) & 1u);
+    }
+  }
+
+  // ---- split sums: C[m][n] with m = lane/4 (+8), n = 2 (lane%4) (+1) ----------
+  const size_t per_mat = (size_t)a.T * d_out;
+  if (!producer) {
+    float* base = a.parts + (size_t)(s % P.copies) * P.mats * per_mat + (size_t)mat * per_mat;
+    const int cb = (int)(cbyte / 2);
+#pragma unroll
+    for (int b = 0; b < kMmaBPW; ++b) {
+      const int blk = warp + b * kMmaWarps;
+      if (blk < nblk) {
+        const int m = cb + blk * 16 + (lane >> 2);
+        const int t0 = (lane & 3) * 2;
+        if (t0 < ntok) {
+          atomicAdd(base + (size_t)(tok0 + t0) * d_out + m, acc[b][0]);
+          atomicAdd(base + (size_t)(tok0 + t0) * d_out + m + 8, acc[b][2]);
+        }
+        if (t0 + 1 < ntok) {
+          atomicAdd(base + (size_t)(tok0 + t0 + 1) * d_out + m, acc[b][1]);
+          atomicAdd(base + (size_t)(tok0 + t0 + 1) * d_out + m + 8, acc[b][3]);
+        }
+      }
+    }
+  }
+
+  // ---- the last CTA of this column tile: epilogue -----------------------------
+  int32_t* ticket = a.tickets + (size_t)grp * P.n_ct + ct;
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_flag = (atomicAdd(ticket, 1) == P.mats * S - 1);
+  __syncthreads();
+  if (!s_flag) return;
+  __threadfence();
+  if (tid == 0) *ticket = 0;
+  const size_t copy_stride = (size_t)P.mats * per_mat;
+  for (int v = tid; v < tvec; v += blockDim.x) {
+    const int col = (ct * P.vec_tile + v) * V;
+    for (int t = 0; t < ntok; ++t) {
+      const int tok = tok0 + t;
+      const float* pu = a.parts + (size_t)tok * d_out + col;
+      float u[V], gv[V];
+#pragma unroll
+      for (int e = 0; e < V; ++e) { u[e] = 0.0f; gv[e] = 0.0f; }
+      for (int c = 0; c < P.copies; ++c) {
+#pragma unroll
+        for (int qq = 0; qq < 2; ++qq) {
+          const float4 r = __ldcg(reinterpret_cast<const float4*>(pu + c * copy_stride) + qq);
+          u[4 * qq] += r.x; u[4 * qq + 1] += r.y; u[4 * qq + 2] += r.z; u[4 * qq + 3] += r.w;
+        }
+        if (P.mats == 2) {
+#pragma unroll
+          for (int qq = 0; qq < 2; ++qq) {
+            const float4 r = __ldcg(reinterpret_cast<const float4*>(pu + c * copy_stride + per_mat) + qq);
+            gv[4 * qq] += r.x; gv[4 * qq + 1] += r.y; gv[4 * qq + 2] += r.z; gv[4 * qq + 3] += r.w;
+          }
+        }
+      }
+      epilogue<__nv_bfloat16, MODE>(a, tok, col, u, gv);
+    }
+  }
+}
+
+template <int TT, int MODE>
+cudaError_t launch_mma(const GemvArgs& a, cudaStream_t s) {
+  static unsigned configured = 0;
+  cudaError_t e = ensure_smem_attr(gemv_mma_kernel<TT, MODE>, 200 * 1024, &configured);
+  if (e != cudaSuccess) return e;
+  dim3 grid(a.plan.n_ct, a.plan.mats * a.plan.S, a.plan.groups);
+  e = launch_pdl(gemv_mma_kernel<TT, MODE>, grid, dim3(kMmaWarps * 32 + 32), a.plan.smem, s, a);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+template <int TT>
+cudaError_t launch_mma_mode(const GemvArgs& a, cudaStream_t s) {
+  switch (a.mode) {
+    case 0: return launch_mma<TT, 0>(a, s);
+    case 1: return launch_mma<TT, 1>(a, s);
+    case 2: return launch_mma<TT, 2>(a, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
 template <typename WT, int TT, int MODE>
 cudaError_t launch3(const GemvArgs& a, cudaStream_t s) {
   static unsigned configured = 0;
@@ -343,7 +619,49 @@ cudaError_t launch1(const GemvArgs& a, cudaStream_t s) {
 
 }  // namespace
 
+// Plan of the tensor-core kernel (bf16, 4 or 8 tokens, d_out % 16 == 0).
+GemvPlan plan_gemv_mma(int T, int d_out, int rows_bound, int mats) {
+  GemvPlan p{};
+  p.mma = 1;
+  p.TT = T <= 4 ? 4 : 8;
+  p.groups = (T + p.TT - 1) / p.TT;
+  p.mats = mats;
+  const int blocks = d_out / 16;
+  const int max_blk = kMmaWarps * kMmaBPW;
+  int nct = (blocks + max_blk - 1) / max_blk;
+  for (int c = nct; c <= nct + 8 && c <= blocks; ++c)   // prefer equal tiles
+    if (blocks % c == 0) { nct = c; break; }
+  const int blk_tile = (blocks + nct - 1) / nct;
+  p.n_ct = (blocks + blk_tile - 1) / blk_tile;
+  p.vec_tile = blk_tile * 2;
+  p.threads = kMmaWarps * 32 + 32;
+  p.rps = kMmaRows;
+  const long stage = (long)kMmaRows * (p.vec_tile * 16 + 16);
+  long nst = (90L * 1024) / stage;
+  if (nst < 2) nst = 2;
+  if (nst > 4) nst = 4;
+  p.nst = (int)nst;
+  p.rcap = 512;
+  p.smem = (size_t)p.nst * stage + (size_t)p.rcap * 4 * (1 + p.TT);
+  const long slots = (long)kNumSMs * 2;
+  const long units = (long)p.n_ct * mats * p.groups;
+  long S = slots / (units > 0 ? units : 1);
+  if (S < 1) S = 1;
+  const long max_by_rows = rows_bound / 32;      // >= two stages per split
+  if (S > max_by_rows) S = max_by_rows > 0 ? max_by_rows : 1;
+  if (S > 256) S = 256;
+  p.S = (int)S;
+  p.copies = (int)(S / 32);
+  if (p.copies < 1) p.copies = 1;
+  if (p.copies > 4) p.copies = 4;
+  p.parts_elems = (size_t)p.copies * mats * T * d_out;
+  p.tickets = p.groups * p.n_ct;
+  return p;
+}
+
 GemvPlan plan_gemv(int T, int d_out, int rows_bound, int mats, int elem_bytes) {
+  if (elem_bytes == 2 && T >= 3 && d_out % 16 == 0 && d_out >= 16)
+    return plan_gemv_mma(T, d_out, rows_bound, mats);
   GemvPlan p{};
   p.TT = (T <= 1) ? 1 : (T == 2 ? 2 : (T <= 4 ? 4 : 8));
   p.groups = (T + p.TT - 1) / p.TT;
@@ -392,6 +710,14 @@ GemvPlan plan_gemv(int T, int d_out, int rows_bound, int mats, int elem_bytes) {
 
 cudaError_t launch_gemv(const GemvArgs& a, cudaStream_t s) {
   if (a.T <= 0 || a.d_out <= 0) return cudaSuccess;
+  if (a.plan.mma) {
+    if (!a.bf16) return cudaErrorInvalidValue;
+    switch (a.plan.TT) {
+      case 4: return launch_mma_mode<4>(a, s);
+      case 8: return launch_mma_mode<8>(a, s);
+      default: return cudaErrorInvalidValue;
+    }
+  }
   return a.bf16 ? launch1<__nv_bfloat16>(a, s) : launch1<float>(a, s);
 }
 

@@ -185,6 +185,7 @@ struct GemvPlan {
   int rps;         // rows per pipeline stage
   int nst;         // pipeline stages
   int copies;      // accumulator copies: split s adds into copy s % copies (fewer adds per address)
+  int mma;         // bf16, 4-8 tokens: the tensor-core (mma.sync) kernel
   int rcap;        // rows staged in shared memory per piece
   size_t smem;     // dynamic shared memory bytes
 };
