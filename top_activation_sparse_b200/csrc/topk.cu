@@ -969,7 +969,12 @@ __global__ void __launch_bounds__(NT) topk_reg_kernel(TopkArgs a) {
   }
 
   // ---- 4. union of the rows' kept nonzeros (several tokens) ------------------
+  // The last row CTA lists the set bits: one word per thread for the prefix
+  // (d <= 32 NT here), then one word per warp per step with the ballot rank,
+  // so that the 32 entries of a word are stored together.
   if (want_union) {
+    __shared__ uint32_t s_uword[NT];
+    __shared__ uint32_t s_upre[NT];
     __threadfence();
     __syncthreads();
     if (tid == 0) s_last = (atomicAdd(a.ticket, 1) == a.T - 1);
@@ -977,22 +982,16 @@ __global__ void __launch_bounds__(NT) topk_reg_kernel(TopkArgs a) {
     if (!s_last) return;
     __threadfence();
     const int nwords = (d + 31) / 32;
-    const int wpt = (nwords + NT - 1) / NT;
-    const int w0 = min(tid * wpt, nwords);
-    const int w1 = min(w0 + wpt, nwords);
-    uint32_t n_any = 0;
-    for (int w = w0; w < w1; ++w) n_any += __popc(__ldcg(a.union_bits + w));
+    const uint32_t bits = tid < nwords ? __ldcg(a.union_bits + tid) : 0u;
     uint32_t e_any, e_unused, t_any, t_unused;
-    block_scan2<NT>(n_any, 0u, s_scan, e_any, e_unused, t_any, t_unused);
-    int pos = (int)e_any;
-    for (int w = w0; w < w1; ++w) {
-      uint32_t bits = __ldcg(a.union_bits + w);
-      a.union_bits[w] = 0u;
-      while (bits) {
-        const int bpos = __ffs(bits) - 1;
-        a.list[pos++] = w * 32 + bpos;
-        bits &= bits - 1u;
-      }
+    block_scan2<NT>((uint32_t)__popc(bits), 0u, s_scan, e_any, e_unused, t_any, t_unused);
+    s_uword[tid] = bits;
+    s_upre[tid] = e_any;
+    if (tid < nwords) a.union_bits[tid] = 0u;    // leave the bitmask clean for the next call
+    __syncthreads();
+    for (int w = warp; w < nwords; w += NW) {
+      const uint32_t wb = s_uword[w];
+      if ((wb >> lane) & 1u) a.list[s_upre[w] + __popc(wb & lt)] = w * 32 + lane;
     }
     if (tid == 0) {
       *a.list_count = (int)t_any;
