@@ -119,6 +119,8 @@ def test_prefill_2048_tokens_outliers():
     (130, 4096, 512, 4096),   # dense (K = d_in), M tail of 2 rows
     (256, 1000, 1024, 1),     # one kept input per token
     (128, 512, 520, 0),       # K = 0: all zero
+    (1024, 256, 8200, 100),   # 264 tiles: CTAs take a second tile (the other accumulator), N tail
+    (2048, 128, 8192, 64),    # 512 tiles: 3-4 tiles per CTA, each accumulator reused
 ])
 def test_prefill_ragged_tiles(T, d_in, d_out, k):
     need_gpu()

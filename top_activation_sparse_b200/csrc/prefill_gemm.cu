@@ -7,15 +7,17 @@
 // every weight row is needed by some token, so the projection is a dense
 // contraction over the masked activations and belongs on the tensor cores.
 //
-// sm_100a design (one output tile of 128 x 256 per CTA, one CTA per SM):
+// sm_100a design (persistent: one CTA per SM walks output tiles of 128 x 256):
 //   * TMA (cp.async.bulk.tensor, 128-byte swizzle, no multicast) loads an A
 //     tile of X_sparse (128 rows x 64 K, K-major) and a B tile of W^T (64 K x
 //     256 N, N-major, as four 64-column boxes) per stage into a 4-stage ring;
 //   * one thread issues tcgen05.mma.kind::f16 (bf16 x bf16 -> f32) with the
-//     accumulator in tensor memory (TMEM, 256 columns x 128 lanes) and frees
-//     each stage with tcgen05.commit on that stage's "empty" mbarrier;
-//   * four epilogue warps read the accumulator with tcgen05.ld (each warp its
-//     32 TMEM lanes = 32 rows), round to bf16 and store Y;
+//     accumulator in tensor memory (two accumulators of 256 columns x 128
+//     lanes, used by alternate tiles) and frees each stage with
+//     tcgen05.commit on that stage's "empty" mbarrier;
+//   * four epilogue warps read a finished accumulator with tcgen05.ld (each
+//     warp its 32 TMEM lanes = 32 rows), round to bf16 and store Y while the
+//     MMAs of the next tile fill the other accumulator;
 //   * CTAs are ordered M-block fastest, so the CTAs resident at one time share
 //     W^T tiles through the L2;
 //   * every mbarrier wait is bounded: on a timeout the CTA records
@@ -39,7 +41,8 @@ constexpr int kBBytes = (BN / 64) * kBBox;           // 32 KB
 constexpr int kStageBytes = kABytes + kBBytes;       // 48 KB
 constexpr int kSmemBytes = kStages * kStageBytes + 1024;
 constexpr int kThreads = 192;                        // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
-constexpr uint32_t kTmemCols = 256;
+constexpr int kEpiThreads = 128;
+constexpr uint32_t kTmemCols = 512;                  // two 256-column accumulators
 
 // tcgen05 instruction descriptor, kind::f16: D f32, A bf16 (K-major),
 // B bf16 (MN-major), N = 256, M = 128.
@@ -122,27 +125,36 @@ __global__ void __launch_bounds__(kThreads, 1)
   pdl_begin();
   __shared__ __align__(8) uint64_t s_full[kStages];
   __shared__ __align__(8) uint64_t s_empty[kStages];
-  __shared__ __align__(8) uint64_t s_accum;
+  __shared__ __align__(8) uint64_t s_tfull[2];      // accumulator b complete (MMA -> epilogue)
+  __shared__ __align__(8) uint64_t s_tempty[2];     // accumulator b drained (epilogue -> MMA)
+  __shared__ __align__(8) uint64_t s_done;          // every MMA issued has completed
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
 
   // 1024-byte aligned ring (128-byte swizzle atoms repeat every 1 KB)
   const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.x * BM;          // M-block fastest
-  const int n0 = blockIdx.y * BN;
+  const int mblocks = (M + BM - 1) / BM;
+  const int ntiles = mblocks * ((N + BN - 1) / BN);
   const int nk = (K + BK - 1) / BK;
+  // tiles of this CTA: blockIdx.x, + gridDim.x, ...  (M-block fastest, so the
+  // CTAs busy at one time share W^T tiles through the L2)
+  const int my_tiles = blockIdx.x < ntiles ? (ntiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&s_full[s], 1);
       mbar_init(&s_empty[s], 1);
     }
-    mbar_init(&s_accum, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&s_tfull[b], 1);
+      mbar_init(&s_tempty[b], kEpiThreads);
+    }
+    mbar_init(&s_done, 1);
     mbar_fence_init();
     s_abort = 0;
   }
-  if (warp == 0) {   // whole warp: allocate the accumulator columns
+  if (warp == 0) {   // whole warp: two accumulators of 256 columns
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_u32(&s_tmem)),
                  "r"(kTmemCols)
@@ -155,85 +167,114 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = s_tmem;
 
   if (warp == 0 && lane == 0) {
-    // ---- TMA producer ----
-    int issued = 0;
-    for (int kb = 0; kb < nk; ++kb) {
-      const int s = kb % kStages;
-      if (kb >= kStages && !mbar_wait(&s_empty[s], (uint32_t)((kb / kStages) - 1) & 1u)) {
-        dev_fail(status, DEV_TIMEOUT, 20, (uint32_t)kb);
-        atomicExch(&s_abort, 1);
-        break;
-      }
-      if (*(volatile int*)&s_abort) break;
-      const uint32_t sa = base + (uint32_t)(s * kStageBytes);
-      const uint32_t sb = sa + kABytes;
-      mbar_arrive_expect_tx(&s_full[s], (uint32_t)kStageBytes);
-      tma_load_2d(sa, &map_a, kb * BK, m0, &s_full[s]);
+    // ---- TMA producer: the ring runs on across this CTA's tiles ----
+    int it = 0;
+    for (int lt = 0; lt < my_tiles && !*(volatile int*)&s_abort; ++lt) {
+      const int t = (int)blockIdx.x + lt * (int)gridDim.x;
+      const int m0 = (t % mblocks) * BM, n0 = (t / mblocks) * BN;
+      for (int kb = 0; kb < nk; ++kb, ++it) {
+        const int s = it % kStages;
+        if (it >= kStages && !mbar_wait(&s_empty[s], (uint32_t)((it / kStages) - 1) & 1u)) {
+          dev_fail(status, DEV_TIMEOUT, 20, (uint32_t)it);
+          atomicExch(&s_abort, 1);
+          break;
+        }
+        if (*(volatile int*)&s_abort) break;
+        const uint32_t sa = base + (uint32_t)(s * kStageBytes);
+        const uint32_t sb = sa + kABytes;
+        mbar_arrive_expect_tx(&s_full[s], (uint32_t)kStageBytes);
+        tma_load_2d(sa, &map_a, kb * BK, m0, &s_full[s]);
 #pragma unroll
-      for (int j = 0; j < BN / 64; ++j) tma_load_2d(sb + j * kBBox, &map_b, n0 + 64 * j, kb * BK, &s_full[s]);
-      ++issued;
+        for (int j = 0; j < BN / 64; ++j)
+          tma_load_2d(sb + j * kBBox, &map_b, n0 + 64 * j, kb * BK, &s_full[s]);
+      }
     }
     // on an abort, let the copies already issued land before the CTA exits
     if (*(volatile int*)&s_abort) {
-      for (int i = 0; i < kStages && i < issued; ++i) {
-        const int kb = issued - 1 - i;
-        mbar_wait(&s_full[kb % kStages], (uint32_t)(kb / kStages) & 1u);
+      for (int i = 0; i < kStages && i < it; ++i) {
+        const int g = it - 1 - i;
+        mbar_wait(&s_full[g % kStages], (uint32_t)(g / kStages) & 1u);
       }
     }
   } else if (warp == 1 && lane == 0) {
-    // ---- MMA issuer ----
-    int done = 0;
-    for (int kb = 0; kb < nk; ++kb) {
-      const int s = kb % kStages;
-      if (!mbar_wait(&s_full[s], (uint32_t)(kb / kStages) & 1u)) {
-        dev_fail(status, DEV_TIMEOUT, 21, (uint32_t)kb);
+    // ---- MMA issuer: accumulator lt & 1, reused once the epilogue drained it ----
+    int it = 0;
+    bool issued = false;
+    for (int lt = 0; lt < my_tiles && !*(volatile int*)&s_abort; ++lt) {
+      const int b = lt & 1;
+      if (lt >= 2 && !mbar_wait(&s_tempty[b], (uint32_t)((lt >> 1) - 1) & 1u)) {
+        dev_fail(status, DEV_TIMEOUT, 23, (uint32_t)lt);
         atomicExch(&s_abort, 1);
         break;
       }
-      if (*(volatile int*)&s_abort) break;
       tc_fence_after();
-      const uint32_t sa = base + (uint32_t)(s * kStageBytes);
-      const uint32_t sb = sa + kABytes;
+      const uint32_t acc = tmem + (uint32_t)(b * BN);
+      for (int kb = 0; kb < nk; ++kb, ++it) {
+        const int s = it % kStages;
+        if (!mbar_wait(&s_full[s], (uint32_t)(it / kStages) & 1u)) {
+          dev_fail(status, DEV_TIMEOUT, 21, (uint32_t)it);
+          atomicExch(&s_abort, 1);
+          break;
+        }
+        if (*(volatile int*)&s_abort) break;
+        tc_fence_after();
+        const uint32_t sa = base + (uint32_t)(s * kStageBytes);
+        const uint32_t sb = sa + kABytes;
 #pragma unroll
-      for (int kk = 0; kk < BK / 16; ++kk) {
-        // A: K-major, 128-byte rows, 8-row groups 1 KB apart; K step = 32 bytes
-        const uint64_t ad = smem_desc(sa + kk * 32, 16, 1024);
-        // B: N-major, 128-byte K rows, 8-row groups 1 KB apart (SBO),
-        //    64-column boxes 8 KB apart (LBO); K step = 16 rows = 2 KB
-        const uint64_t bd = smem_desc(sb + kk * 2048, kBBox, 1024);
-        umma_bf16(tmem, ad, bd, (kb > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < BK / 16; ++kk) {
+          // A: K-major, 128-byte rows, 8-row groups 1 KB apart; K step = 32 bytes
+          const uint64_t ad = smem_desc(sa + kk * 32, 16, 1024);
+          // B: N-major, 128-byte K rows, 8-row groups 1 KB apart (SBO),
+          //    64-column boxes 8 KB apart (LBO); K step = 16 rows = 2 KB
+          const uint64_t bd = smem_desc(sb + kk * 2048, kBBox, 1024);
+          umma_bf16(acc, ad, bd, (kb > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(&s_empty[s]);          // frees the stage once these MMAs have read it
+        issued = true;
       }
-      umma_commit(&s_empty[s]);          // frees the stage once these MMAs have read it
-      ++done;
+      umma_commit(&s_tfull[b]);            // accumulator b complete (or abandoned)
     }
-    umma_commit(&s_accum);               // accumulator complete (or abandoned)
+    // every MMA issued has completed before TMEM is freed
+    if (issued) {
+      umma_commit(&s_done);
+      mbar_wait(&s_done, 0u);
+    }
   } else if (warp >= 2) {
-    // ---- epilogue: TMEM -> registers -> bf16 -> global ----
-    const bool ok = mbar_wait_backoff(&s_accum, 0u);
-    if (!ok) {
-      if (lane == 0) dev_fail(status, DEV_TIMEOUT, 22, 0u);
-      atomicExch(&s_abort, 1);
-    }
-    tc_fence_after();
+    // ---- epilogue: TMEM -> registers -> bf16 -> global, overlapping the next tile's MMAs ----
     const int q = warp & 3;                      // this warp's TMEM lane quarter
-    const int row = m0 + q * 32 + lane;
-    const bool abort = *(volatile int*)&s_abort;
-#pragma unroll 1
-    for (int c = 0; c < BN; c += 32) {
-      uint32_t r[32];
-      tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)c, r);
-      if (abort || row >= M) continue;
-      __nv_bfloat16* dst = y + (size_t)row * N + n0 + c;
-#pragma unroll
-      for (int v = 0; v < 4; ++v) {
-        if (n0 + c + 8 * v + 8 > N) break;       // N is a multiple of 8
-        uint4 o;
-        o.x = pack_bf16x2(r[8 * v + 0], r[8 * v + 1]);
-        o.y = pack_bf16x2(r[8 * v + 2], r[8 * v + 3]);
-        o.z = pack_bf16x2(r[8 * v + 4], r[8 * v + 5]);
-        o.w = pack_bf16x2(r[8 * v + 6], r[8 * v + 7]);
-        *reinterpret_cast<uint4*>(dst + 8 * v) = o;
+    for (int lt = 0; lt < my_tiles; ++lt) {
+      const int b = lt & 1;
+      const int t = (int)blockIdx.x + lt * (int)gridDim.x;
+      const int m0 = (t % mblocks) * BM, n0 = (t / mblocks) * BN;
+      if (!mbar_wait_backoff(&s_tfull[b], (uint32_t)(lt >> 1) & 1u)) {
+        if (lane == 0) dev_fail(status, DEV_TIMEOUT, 22, (uint32_t)lt);
+        atomicExch(&s_abort, 1);
+        break;
       }
+      tc_fence_after();
+      const bool abort = *(volatile int*)&s_abort;
+      const int row = m0 + q * 32 + lane;
+      const uint32_t acc = tmem + (uint32_t)(b * BN) + ((uint32_t)(q * 32) << 16);
+#pragma unroll 1
+      for (int c = 0; c < BN; c += 32) {
+        uint32_t r[32];
+        tmem_ld32(acc + (uint32_t)c, r);
+        if (abort || row >= M) continue;
+        __nv_bfloat16* dst = y + (size_t)row * N + n0 + c;
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          if (n0 + c + 8 * v + 8 > N) break;       // N is a multiple of 8
+          uint4 o;
+          o.x = pack_bf16x2(r[8 * v + 0], r[8 * v + 1]);
+          o.y = pack_bf16x2(r[8 * v + 2], r[8 * v + 3]);
+          o.z = pack_bf16x2(r[8 * v + 4], r[8 * v + 5]);
+          o.w = pack_bf16x2(r[8 * v + 6], r[8 * v + 7]);
+          *reinterpret_cast<uint4*>(dst + 8 * v) = o;
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&s_tempty[b]);                   // this thread's reads of accumulator b are done
+      if (abort) break;
     }
   }
   tc_fence_before();
@@ -291,7 +332,9 @@ cudaError_t launch_prefill_gemm(const PrefillArgs& a, cudaStream_t s) {
   static unsigned configured = 0;
   cudaError_t e = ensure_smem_attr(prefill_gemm_kernel, kSmemBytes, &configured);
   if (e != cudaSuccess) return e;
-  dim3 grid((a.M + BM - 1) / BM, (a.N + BN - 1) / BN);
+  // persistent: one CTA per SM, each walking tiles blockIdx.x + i * gridDim.x
+  const int tiles = ((a.M + BM - 1) / BM) * ((a.N + BN - 1) / BN);
+  dim3 grid(tiles < kNumSMs ? tiles : kNumSMs);
   e = launch_pdl(prefill_gemm_kernel, grid, dim3(kThreads), (size_t)kSmemBytes, s, ma, mb, a.y, a.M,
                  a.N, a.K, a.status);
   if (e != cudaSuccess) return e;
