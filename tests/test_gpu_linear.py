@@ -49,8 +49,12 @@ def test_linear_bf16_llama_up_shape(T):
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-@pytest.mark.parametrize("T,d_in,d_out", [(1, 1, 8), (5, 1000, 264), (2, 77, 136), (70, 300, 96)])
+@pytest.mark.parametrize("T,d_in,d_out", [(1, 1, 8), (5, 1000, 264), (2, 77, 136), (70, 300, 96),
+                                           (6, 333, 1552), (4, 20, 160)])
 def test_linear_ragged_sizes(dtype, T, d_in, d_out):
+    """Ragged sizes; bf16 with 3-64 tokens and d_out % 16 == 0 takes the
+    tensor-core path: (6, 333, 1552) has a short last column tile (97 blocks
+    of 16 in 2 tiles), (4, 20, 160) fewer kept rows than one 16-row stage."""
     need_gpu()
     g = workloads.rng(T + d_in + d_out)
     x = workloads.round_to_dtype(workloads.normal_f32(g, (T, d_in)), dtype)
