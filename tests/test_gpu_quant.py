@@ -103,3 +103,17 @@ def test_quant_rejects_unaligned_packed_rows():
     with pytest.raises(qs.QSError) as e:
         qs.qs_quant_sparse_linear(x, p, 1.0, 8)
     assert e.value.status == qs.QS_ERR_ALIGNMENT
+
+
+@pytest.mark.parametrize("T", [12, 20])
+@pytest.mark.parametrize("k", [1, 37, 300])
+def test_quant_tensor_core_token_groups(T, k):
+    """8 or more tokens take the tensor-core kernel (m16n8k32 s8): 12 and 20
+    tokens use 16- and 24-token groups with empty token slots; K = 1 and 37
+    leave a short last stage of 32 rows.  Everything bit-exact."""
+    need_gpu()
+    d_in, d_out = 300, 320
+    W = workloads.weight_out_major(d_out, d_in, 21)
+    t, alpha = oracle.ternary_quantize(W)
+    x = workloads.round_to_dtype(workloads.normal_f32(workloads.rng(22 + T), (T, d_in)), "bf16")
+    _check_quant(x, "bf16", t, alpha, oracle.ternary_pack(t), k)

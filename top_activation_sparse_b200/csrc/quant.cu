@@ -311,6 +311,261 @@ __global__ void __launch_bounds__(QTune<TT>::kMaxConsumers + 32, 2) qgemv_kernel
   }
 }
 
+// ---- 8 to 32 tokens: int8 x ternary on the tensor cores ------------------------
+// The lane-pair decode spends about one instruction per multiply-add, so with
+// many tokens the kernel is integer-issue bound.  Here warp-level
+// mma.sync m16n8k32 (s8 x s8 -> s32) does the multiply-adds: A = 16 output
+// columns x 32 kept rows of ternary weights, decoded by each lane straight
+// from the packed words into its fragment (a shift and mask per row, two byte
+// permutes, 0/1/2 -> 0/+1/-1 per byte); B = the 32 rows' int8 codes of 8
+// tokens, read as 32-bit groups from a token-major copy in shared memory.
+// Integer throughout: exact, and the split sums stay exact in f32.
+constexpr int kQmWarps = 8;
+constexpr int kQmRows = 32;                        // rows per stage (the MMA's K)
+
+__device__ __forceinline__ void mma_s8_16832(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                             uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// codes of 4 rows (packed words w0..w3, already shifted so that column m sits
+// in bits 0-1 and column m+8 in bits 16-17) -> int8 weights of column m (lo)
+// and of column m+8 (hi), row i in byte i
+__device__ __forceinline__ void decode4(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3,
+                                        uint32_t& lo, uint32_t& hi) {
+  const uint32_t p01 = (w0 & 0x00030003u) | ((w1 & 0x00030003u) << 8);
+  const uint32_t p23 = (w2 & 0x00030003u) | ((w3 & 0x00030003u) << 8);
+  const uint32_t clo = __byte_perm(p01, p23, 0x5410);
+  const uint32_t chi = __byte_perm(p01, p23, 0x7632);
+  // byte code 0 -> 0, 1 -> +1, 2 -> -1 (0xFF)
+  lo = clo | (((clo >> 1) & 0x01010101u) * 0xFFu);
+  hi = chi | (((chi >> 1) & 0x01010101u) * 0xFFu);
+}
+
+template <int NB>
+__global__ void __launch_bounds__(kQmWarps * 32 + 32, 2) qgemv_mma_kernel(QGemvArgs a) {
+  constexpr int TT = NB * 8;
+  constexpr int BPW = 12 / NB;                     // 16-column blocks (packed words) per warp
+  extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ __align__(8) uint64_t s_full[32];
+  __shared__ __align__(8) uint64_t s_empty[32];
+  __shared__ int s_flag;
+  __shared__ int s_err;
+
+  const GemvPlan& P = a.plan;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const bool producer = warp == kQmWarps;
+  const int pitch = P.vec_tile * 4 + 16;           // bytes per staged row (tile + pad)
+  const int stage_bytes = kQmRows * pitch;
+  unsigned char* s_stage = smem;
+  int* s_rows = reinterpret_cast<int*>(smem + (size_t)P.nst * stage_bytes);
+  int8_t* s_qT = reinterpret_cast<int8_t*>(s_rows + P.rcap);   // [TT][rcap], token-major
+
+  const int S = P.S;
+  const int ct = blockIdx.x;
+  const int s = blockIdx.y;
+  const int grp = blockIdx.z;
+  const int tok0 = grp * TT;
+  const int ntok = min(TT, a.T - tok0);
+  const int d_in = a.d_in, d_out = a.d_out;
+  const int row_words = d_out / 16;
+  const int cword = ct * P.vec_tile;
+  const int twords = min(P.vec_tile, row_words - cword);
+  const int tbytes = twords * 4;
+  const unsigned char* Wb = reinterpret_cast<const unsigned char*>(a.wp) + (size_t)cword * 4;
+
+  pdl_begin();
+  const int n = min(max(*a.list_count, 0), d_in);
+  const int r0 = (int)(((long long)n * s) / S);
+  const int r1 = (int)(((long long)n * (s + 1)) / S);
+
+  if (tid == 0) {
+    for (int i = 0; i < P.nst; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_empty[i], kQmWarps);
+    }
+    mbar_fence_init();
+    s_err = 0;
+  }
+  __syncthreads();
+
+  int acc[BPW][NB][4];
+#pragma unroll
+  for (int b = 0; b < BPW; ++b)
+#pragma unroll
+    for (int nb = 0; nb < NB; ++nb)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[b][nb][e] = 0;
+
+  const int g = lane >> 2;                          // A row (column m) / B column (token)
+  const int k0 = (lane & 3) * 4;                    // first of this lane's 4 rows
+  const int shift = 2 * g;                          // column g of a packed word
+
+  int gst = 0;
+  for (int pb = r0; pb < r1; pb += P.rcap) {
+    const int np = min(P.rcap, r1 - pb);
+    for (int j = tid; j < np; j += blockDim.x) {
+      int r = a.list[pb + j];
+      const bool ok = (unsigned)r < (unsigned)d_in;
+      if (!ok) {
+        dev_fail(a.status, DEV_CHECK, 4, (uint32_t)r);
+        r = 0;
+      }
+      s_rows[j] = r;
+#pragma unroll
+      for (int t = 0; t < TT; ++t)
+        s_qT[t * P.rcap + j] = (ok && t < ntok) ? a.xq[(size_t)(tok0 + t) * d_in + r] : (int8_t)0;
+    }
+    __syncthreads();
+    const int nstage = (np + kQmRows - 1) / kQmRows;
+    if (producer) {
+      if (lane == 0) {
+        for (int st = 0; st < nstage; ++st) {
+          const int gg = gst + st;
+          const int slot = gg % P.nst;
+          if (gg >= P.nst && !mbar_wait(&s_empty[slot], (uint32_t)((gg / P.nst) - 1) & 1u)) {
+            dev_fail(a.status, DEV_TIMEOUT, 16, (uint32_t)gg);
+            atomicExch(&s_err, 1);
+            break;
+          }
+          const int j0 = st * kQmRows;
+          const int cnt = min(kQmRows, np - j0);
+          mbar_arrive_expect_tx(&s_full[slot], (uint32_t)(cnt * tbytes));
+          for (int r = 0; r < cnt; ++r)
+            bulk_g2s(s_stage + (size_t)slot * stage_bytes + (size_t)r * pitch,
+                     Wb + (size_t)s_rows[j0 + r] * row_words * 4, (uint32_t)tbytes, &s_full[slot]);
+        }
+      }
+    } else {
+      for (int st = 0; st < nstage; ++st) {
+        const int gg = gst + st;
+        const int slot = gg % P.nst;
+        const bool ready = mbar_wait_backoff(&s_full[slot], (uint32_t)(gg / P.nst) & 1u);
+        if (!ready) {
+          if (lane == 0) dev_fail(a.status, DEV_TIMEOUT, 17, (uint32_t)gg);
+          atomicExch(&s_err, 1);
+        }
+        const int j0 = st * kQmRows;
+        const int cnt = min(kQmRows, np - j0);
+        if (ready) {
+          // B: rows k0..k0+3 and k0+16..k0+19 of token nb*8 + g; rows past the
+          // stage's end contribute 0 (their staged weights are stale)
+          const int v0 = min(max(cnt - k0, 0), 4), v1 = min(max(cnt - k0 - 16, 0), 4);
+          const uint32_t m0 = v0 >= 4 ? 0xffffffffu : ((1u << (8 * v0)) - 1u);
+          const uint32_t m1 = v1 >= 4 ? 0xffffffffu : ((1u << (8 * v1)) - 1u);
+          uint32_t b0[NB], b1[NB];
+#pragma unroll
+          for (int nb = 0; nb < NB; ++nb) {
+            const int8_t* qp = s_qT + (nb * 8 + g) * P.rcap + j0 + k0;
+            b0[nb] = *reinterpret_cast<const uint32_t*>(qp) & m0;
+            b1[nb] = *reinterpret_cast<const uint32_t*>(qp + 16) & m1;
+          }
+          const unsigned char* sb = s_stage + (size_t)slot * stage_bytes;
+#pragma unroll
+          for (int b = 0; b < BPW; ++b) {
+            const int blk = warp + b * kQmWarps;
+            if (blk < twords) {
+              const unsigned char* wp = sb + (size_t)k0 * pitch + (size_t)blk * 4;
+              const uint32_t w0 = *reinterpret_cast<const uint32_t*>(wp) >> shift;
+              const uint32_t w1 = *reinterpret_cast<const uint32_t*>(wp + pitch) >> shift;
+              const uint32_t w2 = *reinterpret_cast<const uint32_t*>(wp + 2 * pitch) >> shift;
+              const uint32_t w3 = *reinterpret_cast<const uint32_t*>(wp + 3 * pitch) >> shift;
+              const unsigned char* wq = wp + (size_t)16 * pitch;
+              const uint32_t x0 = *reinterpret_cast<const uint32_t*>(wq) >> shift;
+              const uint32_t x1 = *reinterpret_cast<const uint32_t*>(wq + pitch) >> shift;
+              const uint32_t x2 = *reinterpret_cast<const uint32_t*>(wq + 2 * pitch) >> shift;
+              const uint32_t x3 = *reinterpret_cast<const uint32_t*>(wq + 3 * pitch) >> shift;
+              uint32_t a0, a1, a2, a3;
+              decode4(w0, w1, w2, w3, a0, a1);
+              decode4(x0, x1, x2, x3, a2, a3);
+#pragma unroll
+              for (int nb = 0; nb < NB; ++nb) mma_s8_16832(acc[b][nb], a0, a1, a2, a3, b0[nb], b1[nb]);
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_empty[slot]);
+      }
+    }
+    gst += nstage;
+    __syncthreads();
+  }
+  if (s_err && tid == 0) {
+    for (int i = 0; i < P.nst && i < gst; ++i) {
+      const int g_last = gst - 1 - i;
+      mbar_wait(&s_full[g_last % P.nst], (uint32_t)(g_last / P.nst) & 1u);
+    }
+  }
+
+  // ---- split sums (exact integers in f32): D[m][n], m = g (+8), n = 2 (lane%4) (+1)
+  if (!producer) {
+    float* base = a.parts + (size_t)(s % P.copies) * a.T * d_out;
+    const int tn = (lane & 3) * 2;
+#pragma unroll
+    for (int b = 0; b < BPW; ++b) {
+      const int blk = warp + b * kQmWarps;
+      if (blk < twords) {
+        const int col = (cword + blk) * 16 + g;
+#pragma unroll
+        for (int nb = 0; nb < NB; ++nb) {
+          const int t = nb * 8 + tn;
+          if (t < ntok) {
+            atomicAdd(base + (size_t)(tok0 + t) * d_out + col, (float)acc[b][nb][0]);
+            atomicAdd(base + (size_t)(tok0 + t) * d_out + col + 8, (float)acc[b][nb][2]);
+          }
+          if (t + 1 < ntok) {
+            atomicAdd(base + (size_t)(tok0 + t + 1) * d_out + col, (float)acc[b][nb][1]);
+            atomicAdd(base + (size_t)(tok0 + t + 1) * d_out + col + 8, (float)acc[b][nb][3]);
+          }
+        }
+      }
+    }
+  }
+
+  // ---- last CTA of this column tile: rescale -----------------------------------
+  int32_t* ticket = a.tickets + grp * P.n_ct + ct;
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_flag = (atomicAdd(ticket, 1) == S - 1);
+  __syncthreads();
+  if (!s_flag) return;
+  __threadfence();
+  if (tid == 0) *ticket = 0;
+  const int q4 = twords * 4;                       // float4 groups of the tile, per token
+  for (int i = tid; i < ntok * q4; i += blockDim.x) {
+    const int t = i / q4;
+    const int tok = tok0 + t;
+    const size_t o = (size_t)tok * d_out + (size_t)cword * 16 + (size_t)(i - t * q4) * 4;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int c = 0; c < P.copies; ++c) {
+      const float4 f = __ldcg(reinterpret_cast<const float4*>(a.parts + (size_t)c * a.T * d_out + o));
+      v.x += f.x; v.y += f.y; v.z += f.z; v.w += f.w;
+    }
+    const float r = __fdiv_rn(__fmul_rn(a.alpha, a.gamma[tok]), 127.0f);
+    const int4 iv = make_int4(__float2int_rn(v.x), __float2int_rn(v.y), __float2int_rn(v.z),
+                              __float2int_rn(v.w));
+    reinterpret_cast<float4*>(a.y + o)[0] =
+        make_float4(__fmul_rn(__int2float_rn(iv.x), r), __fmul_rn(__int2float_rn(iv.y), r),
+                    __fmul_rn(__int2float_rn(iv.z), r), __fmul_rn(__int2float_rn(iv.w), r));
+    if (a.acc) reinterpret_cast<int4*>(a.acc + o)[0] = iv;
+  }
+}
+
+template <int NB>
+cudaError_t qlaunch_mma(const QGemvArgs& a, cudaStream_t s) {
+  static unsigned configured = 0;
+  cudaError_t e = ensure_smem_attr(qgemv_mma_kernel<NB>, 200 * 1024, &configured);
+  if (e != cudaSuccess) return e;
+  dim3 grid(a.plan.n_ct, a.plan.S, a.plan.groups);
+  e = launch_pdl(qgemv_mma_kernel<NB>, grid, dim3(kQmWarps * 32 + 32), a.plan.smem, s, a);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
 template <int TT>
 cudaError_t qlaunch(const QGemvArgs& a, cudaStream_t s) {
   static unsigned configured = 0;
@@ -379,7 +634,47 @@ __global__ void __launch_bounds__(kPackNT) pack_kernel(PackArgs a) {
 
 }  // namespace
 
+// Plan of the tensor-core kernel: 8-32 tokens per group (n-blocks of 8).
+GemvPlan plan_qgemv_mma(int T, int d_out, int rows_bound) {
+  GemvPlan p{};
+  p.mma = 1;
+  p.TT = T >= 32 ? 32 : ((T + 7) / 8) * 8;
+  p.groups = (T + p.TT - 1) / p.TT;
+  p.mats = 1;
+  const int nb = p.TT / 8;
+  const int row_words = d_out / 16;
+  const int max_words = kQmWarps * (12 / nb);      // 96, 48, 32, 24: multiples of 4
+  int nct = (row_words + max_words - 1) / max_words;
+  if (nct < 1) nct = 1;
+  int tile = ((row_words + nct - 1) / nct + 3) / 4 * 4;
+  if (tile > max_words) tile = max_words;
+  p.n_ct = (row_words + tile - 1) / tile;
+  p.vec_tile = tile;                               // packed words per tile
+  p.threads = kQmWarps * 32 + 32;
+  p.rps = kQmRows;
+  const long stage = (long)kQmRows * (tile * 4 + 16);
+  long nst = (90L * 1024) / stage;
+  if (nst < 2) nst = 2;
+  if (nst > 16) nst = 16;
+  p.nst = (int)nst;
+  p.rcap = 512;
+  p.smem = (size_t)p.nst * stage + (size_t)p.rcap * (4 + p.TT);
+  const long slots = (long)kNumSMs * 2;
+  const long units = (long)p.n_ct * p.groups;
+  long S = slots / (units > 0 ? units : 1);
+  if (S < 1) S = 1;
+  const long max_by_rows = rows_bound / kQmRows;
+  if (S > max_by_rows) S = max_by_rows > 0 ? max_by_rows : 1;
+  if (S > 256) S = 256;
+  p.S = (int)S;
+  p.copies = 1;
+  p.parts_elems = (size_t)T * d_out;
+  p.tickets = p.groups * p.n_ct;
+  return p;
+}
+
 GemvPlan plan_qgemv(int T, int d_out, int rows_bound) {
+  if (T >= 8) return plan_qgemv_mma(T, d_out, rows_bound);
   GemvPlan p{};
   p.TT = (T <= 1) ? 1 : (T == 2 ? 2 : (T <= 4 ? 4 : 8));
   p.groups = (T + p.TT - 1) / p.TT;
@@ -431,6 +726,16 @@ bool qgemv_supported(int d_out) { return d_out % 64 == 0; }   // 16-byte aligned
 
 cudaError_t launch_qgemv(const QGemvArgs& a, cudaStream_t s) {
   if (a.T <= 0) return cudaSuccess;
+  if (a.plan.mma) {
+    if (a.xq == nullptr) return cudaErrorInvalidValue;   // several tokens: dense codes
+    switch (a.plan.TT) {
+      case 8: return qlaunch_mma<1>(a, s);
+      case 16: return qlaunch_mma<2>(a, s);
+      case 24: return qlaunch_mma<3>(a, s);
+      case 32: return qlaunch_mma<4>(a, s);
+      default: return cudaErrorInvalidValue;
+    }
+  }
   switch (a.plan.TT) {
     case 1: return qlaunch<1>(a, s);
     case 2: return qlaunch<2>(a, s);
