@@ -504,24 +504,32 @@ __global__ void __launch_bounds__(kMmaWarps * 32 + 32, 2) gemv_mma_kernel(GemvAr
     }
   }
 
-  // ---- split sums: C[m][n] with m = lane/4 (+8), n = 2 (lane%4) (+1) ----------
-  const size_t per_mat = (size_t)a.T * d_out;
+  // ---- split sums --------------------------------------------------------------
+  // The accumulators of this kernel are column-major, [column][Tp] (tokens
+  // contiguous, Tp = T rounded up to 4), so that one lane adds 4 tokens of one
+  // column with one vector reduction: lanes 2i and 2i+1 (tokens n..n+1 and
+  // n+2..n+3 of columns m and m+8) swap halves, then the even lane adds
+  // column m, the odd lane column m+8.  (Scalar adds per element cost ~4x the
+  // reduction operations and were the bottleneck.)
+  const int Tp = (a.T + 3) & ~3;
+  const size_t per_mat = (size_t)d_out * Tp;
   if (!producer) {
     float* base = a.parts + (size_t)(s % P.copies) * P.mats * per_mat + (size_t)mat * per_mat;
     const int cb = (int)(cbyte / 2);
+    const int tig = lane & 3;
+    const bool even = (tig & 1) == 0;
+    const int t = (tig & 2) * 2;                    // first of this lane's 4 tokens
 #pragma unroll
     for (int b = 0; b < kMmaBPW; ++b) {
       const int blk = warp + b * kMmaWarps;
-      if (blk < nblk) {
-        const int m = cb + blk * 16 + (lane >> 2);
-        const int t0 = (lane & 3) * 2;
-        if (t0 < ntok) {
-          atomicAdd(base + (size_t)(tok0 + t0) * d_out + m, acc[b][0]);
-          atomicAdd(base + (size_t)(tok0 + t0) * d_out + m + 8, acc[b][2]);
-        }
-        if (t0 + 1 < ntok) {
-          atomicAdd(base + (size_t)(tok0 + t0 + 1) * d_out + m, acc[b][1]);
-          atomicAdd(base + (size_t)(tok0 + t0 + 1) * d_out + m + 8, acc[b][3]);
+      if (blk < nblk) {                            // warp-uniform
+        const float r0 = __shfl_xor_sync(0xffffffffu, even ? acc[b][2] : acc[b][0], 1);
+        const float r1 = __shfl_xor_sync(0xffffffffu, even ? acc[b][3] : acc[b][1], 1);
+        const int col = cb + blk * 16 + (lane >> 2) + (even ? 0 : 8);
+        if (t < ntok) {
+          float* dst = base + (size_t)col * Tp + tok0 + t;
+          if (even) red_add_v4(dst, acc[b][0], acc[b][1], r0, r1);
+          else red_add_v4(dst, r0, r1, acc[b][2], acc[b][3]);
         }
       }
     }
@@ -537,30 +545,25 @@ __global__ void __launch_bounds__(kMmaWarps * 32 + 32, 2) gemv_mma_kernel(GemvAr
   __threadfence();
   if (tid == 0) *ticket = 0;
   const size_t copy_stride = (size_t)P.mats * per_mat;
-  for (int v = tid; v < tvec; v += blockDim.x) {
+  // (column vector, token) pairs, tokens fastest: neighbouring threads read
+  // neighbouring accumulators
+  for (int i = tid; i < tvec * ntok; i += blockDim.x) {
+    const int v = i / ntok, tt = i - v * ntok;
     const int col = (ct * P.vec_tile + v) * V;
-    for (int t = 0; t < ntok; ++t) {
-      const int tok = tok0 + t;
-      const float* pu = a.parts + (size_t)tok * d_out + col;
-      float u[V], gv[V];
+    const int tok = tok0 + tt;
+    const float* pu = a.parts + (size_t)col * Tp + tok;
+    float u[V], gv[V];
 #pragma unroll
-      for (int e = 0; e < V; ++e) { u[e] = 0.0f; gv[e] = 0.0f; }
-      for (int c = 0; c < P.copies; ++c) {
+    for (int e = 0; e < V; ++e) { u[e] = 0.0f; gv[e] = 0.0f; }
+    for (int c = 0; c < P.copies; ++c) {
 #pragma unroll
-        for (int qq = 0; qq < 2; ++qq) {
-          const float4 r = __ldcg(reinterpret_cast<const float4*>(pu + c * copy_stride) + qq);
-          u[4 * qq] += r.x; u[4 * qq + 1] += r.y; u[4 * qq + 2] += r.z; u[4 * qq + 3] += r.w;
-        }
-        if (P.mats == 2) {
+      for (int e = 0; e < V; ++e) u[e] += __ldcg(pu + c * copy_stride + (size_t)e * Tp);
+      if (P.mats == 2) {
 #pragma unroll
-          for (int qq = 0; qq < 2; ++qq) {
-            const float4 r = __ldcg(reinterpret_cast<const float4*>(pu + c * copy_stride + per_mat) + qq);
-            gv[4 * qq] += r.x; gv[4 * qq + 1] += r.y; gv[4 * qq + 2] += r.z; gv[4 * qq + 3] += r.w;
-          }
-        }
+        for (int e = 0; e < V; ++e) gv[e] += __ldcg(pu + c * copy_stride + per_mat + (size_t)e * Tp);
       }
-      epilogue<__nv_bfloat16, MODE>(a, tok, col, u, gv);
     }
+    epilogue<__nv_bfloat16, MODE>(a, tok, col, u, gv);
   }
 }
 
@@ -654,7 +657,7 @@ GemvPlan plan_gemv_mma(int T, int d_out, int rows_bound, int mats) {
   p.copies = (int)(S / 32);
   if (p.copies < 1) p.copies = 1;
   if (p.copies > 4) p.copies = 4;
-  p.parts_elems = (size_t)p.copies * mats * T * d_out;
+  p.parts_elems = (size_t)p.copies * mats * d_out * (size_t)((T + 3) & ~3);   // [column][T up to 4]
   p.tickets = p.groups * p.n_ct;
   return p;
 }

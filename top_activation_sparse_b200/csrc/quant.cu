@@ -501,25 +501,32 @@ __global__ void __launch_bounds__(kQmWarps * 32 + 32, 2) qgemv_mma_kernel(QGemvA
     }
   }
 
-  // ---- split sums (exact integers in f32): D[m][n], m = g (+8), n = 2 (lane%4) (+1)
+  // ---- split sums (exact integers in f32) ----------------------------------------
+  // Column-major accumulators [column][Tp] (Tp = T rounded up to 4): lanes 2i
+  // and 2i+1 swap halves so that each adds 4 tokens of one column with one
+  // vector reduction (see the bf16 tensor-core gather-GEMV).
+  const int Tp = (a.T + 3) & ~3;
   if (!producer) {
-    float* base = a.parts + (size_t)(s % P.copies) * a.T * d_out;
-    const int tn = (lane & 3) * 2;
+    float* base = a.parts + (size_t)(s % P.copies) * d_out * Tp;
+    const int tig = lane & 3;
+    const bool even = (tig & 1) == 0;
+    const int tq = (tig & 2) * 2;
 #pragma unroll
     for (int b = 0; b < BPW; ++b) {
       const int blk = warp + b * kQmWarps;
-      if (blk < twords) {
-        const int col = (cword + blk) * 16 + g;
+      if (blk < twords) {                          // warp-uniform
+        const int col = (cword + blk) * 16 + g + (even ? 0 : 8);
 #pragma unroll
         for (int nb = 0; nb < NB; ++nb) {
-          const int t = nb * 8 + tn;
+          const float c0 = (float)acc[b][nb][0], c1 = (float)acc[b][nb][1];
+          const float c2 = (float)acc[b][nb][2], c3 = (float)acc[b][nb][3];
+          const float r0 = __shfl_xor_sync(0xffffffffu, even ? c2 : c0, 1);
+          const float r1 = __shfl_xor_sync(0xffffffffu, even ? c3 : c1, 1);
+          const int t = nb * 8 + tq;
           if (t < ntok) {
-            atomicAdd(base + (size_t)(tok0 + t) * d_out + col, (float)acc[b][nb][0]);
-            atomicAdd(base + (size_t)(tok0 + t) * d_out + col + 8, (float)acc[b][nb][2]);
-          }
-          if (t + 1 < ntok) {
-            atomicAdd(base + (size_t)(tok0 + t + 1) * d_out + col, (float)acc[b][nb][1]);
-            atomicAdd(base + (size_t)(tok0 + t + 1) * d_out + col + 8, (float)acc[b][nb][3]);
+            float* dst = base + (size_t)col * Tp + tok0 + t;
+            if (even) red_add_v4_f32(dst, c0, c1, r0, r1);
+            else red_add_v4_f32(dst, r0, r1, c2, c3);
           }
         }
       }
@@ -535,19 +542,21 @@ __global__ void __launch_bounds__(kQmWarps * 32 + 32, 2) qgemv_mma_kernel(QGemvA
   if (!s_flag) return;
   __threadfence();
   if (tid == 0) *ticket = 0;
-  const int q4 = twords * 4;                       // float4 groups of the tile, per token
+  const int q4 = twords * 4;                       // float4 groups of the tile
   for (int i = tid; i < ntok * q4; i += blockDim.x) {
-    const int t = i / q4;
+    const int qi = i / ntok, t = i - qi * ntok;    // tokens fastest
     const int tok = tok0 + t;
-    const size_t o = (size_t)tok * d_out + (size_t)cword * 16 + (size_t)(i - t * q4) * 4;
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    const int col = cword * 16 + qi * 4;
+    float v[4] = {0.f, 0.f, 0.f, 0.f};
     for (int c = 0; c < P.copies; ++c) {
-      const float4 f = __ldcg(reinterpret_cast<const float4*>(a.parts + (size_t)c * a.T * d_out + o));
-      v.x += f.x; v.y += f.y; v.z += f.z; v.w += f.w;
+      const float* pc = a.parts + (size_t)c * d_out * Tp + (size_t)col * Tp + tok;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) v[e] += __ldcg(pc + (size_t)e * Tp);
     }
     const float r = __fdiv_rn(__fmul_rn(a.alpha, a.gamma[tok]), 127.0f);
-    const int4 iv = make_int4(__float2int_rn(v.x), __float2int_rn(v.y), __float2int_rn(v.z),
-                              __float2int_rn(v.w));
+    const int4 iv = make_int4(__float2int_rn(v[0]), __float2int_rn(v[1]), __float2int_rn(v[2]),
+                              __float2int_rn(v[3]));
+    const size_t o = (size_t)tok * d_out + col;
     reinterpret_cast<float4*>(a.y + o)[0] =
         make_float4(__fmul_rn(__int2float_rn(iv.x), r), __fmul_rn(__int2float_rn(iv.y), r),
                     __fmul_rn(__int2float_rn(iv.z), r), __fmul_rn(__int2float_rn(iv.w), r));
@@ -668,7 +677,7 @@ GemvPlan plan_qgemv_mma(int T, int d_out, int rows_bound) {
   if (S > 256) S = 256;
   p.S = (int)S;
   p.copies = 1;
-  p.parts_elems = (size_t)T * d_out;
+  p.parts_elems = (size_t)d_out * (size_t)((T + 3) & ~3);   // [column][T up to 4]
   p.tickets = p.groups * p.n_ct;
   return p;
 }
