@@ -196,22 +196,24 @@ __global__ void __launch_bounds__(kMaxConsumers + 32, (TT <= 4) ? 2 : 1) gemv_ke
     __syncthreads();
     const int nstage = (np + P.rps - 1) / P.rps;
     if (producer) {
-      if (lane == 0) {
-        for (int st = 0; st < nstage; ++st) {
-          const int g = gst + st;
-          const int slot = g % P.nst;
-          if (g >= P.nst && !mbar_wait(&s_empty[slot], (uint32_t)((g / P.nst) - 1) & 1u)) {
-            dev_fail(a.status, DEV_TIMEOUT, 10, (uint32_t)g);
-            atomicExch(&s_err, 1);
-            break;
-          }
-          const int j0 = st * P.rps;
-          const int cnt = min(P.rps, np - j0);
-          mbar_arrive_expect_tx(&s_full[slot], (uint32_t)(cnt * tbytes));
-          for (int r = 0; r < cnt; ++r)
-            bulk_g2s(s_stage + ((size_t)slot * P.rps + r) * tile_bytes,
-                     Wb + (size_t)s_rows[j0 + r] * row_bytes, (uint32_t)tbytes, &s_full[slot]);
+      // the producer warp's lanes issue a stage's copies side by side
+      for (int st = 0; st < nstage; ++st) {
+        const int g = gst + st;
+        const int slot = g % P.nst;
+        int ok = 1;
+        if (lane == 0 && g >= P.nst && !mbar_wait(&s_empty[slot], (uint32_t)((g / P.nst) - 1) & 1u)) {
+          dev_fail(a.status, DEV_TIMEOUT, 10, (uint32_t)g);
+          atomicExch(&s_err, 1);
+          ok = 0;
         }
+        if (__shfl_sync(0xffffffffu, ok, 0) == 0) break;
+        const int j0 = st * P.rps;
+        const int cnt = min(P.rps, np - j0);
+        if (lane == 0) mbar_arrive_expect_tx(&s_full[slot], (uint32_t)(cnt * tbytes));
+        __syncwarp();
+        for (int rr = lane; rr < cnt; rr += 32)
+          bulk_g2s(s_stage + ((size_t)slot * P.rps + rr) * tile_bytes,
+                   Wb + (size_t)s_rows[j0 + rr] * row_bytes, (uint32_t)tbytes, &s_full[slot]);
       }
     } else {
       for (int st = 0; st < nstage; ++st) {
@@ -430,22 +432,24 @@ __global__ void __launch_bounds__(kMmaWarps * 32 + 32, 2) gemv_mma_kernel(GemvAr
     __syncthreads();
     const int nstage = (np + kMmaRows - 1) / kMmaRows;
     if (producer) {
-      if (lane == 0) {
-        for (int st = 0; st < nstage; ++st) {
-          const int g = gst + st;
-          const int slot = g % P.nst;
-          if (g >= P.nst && !mbar_wait(&s_empty[slot], (uint32_t)((g / P.nst) - 1) & 1u)) {
-            dev_fail(a.status, DEV_TIMEOUT, 14, (uint32_t)g);
-            atomicExch(&s_err, 1);
-            break;
-          }
-          const int j0 = st * kMmaRows;
-          const int cnt = min(kMmaRows, np - j0);
-          mbar_arrive_expect_tx(&s_full[slot], (uint32_t)(cnt * tbytes));
-          for (int r = 0; r < cnt; ++r)
-            bulk_g2s(s_stage + (size_t)slot * stage_bytes + (size_t)r * pitch,
-                     Wb + (size_t)s_rows[j0 + r] * row_bytes, (uint32_t)tbytes, &s_full[slot]);
+      // the producer warp's lanes issue a stage's copies side by side
+      for (int st = 0; st < nstage; ++st) {
+        const int g = gst + st;
+        const int slot = g % P.nst;
+        int ok = 1;
+        if (lane == 0 && g >= P.nst && !mbar_wait(&s_empty[slot], (uint32_t)((g / P.nst) - 1) & 1u)) {
+          dev_fail(a.status, DEV_TIMEOUT, 14, (uint32_t)g);
+          atomicExch(&s_err, 1);
+          ok = 0;
         }
+        if (__shfl_sync(0xffffffffu, ok, 0) == 0) break;
+        const int j0 = st * kMmaRows;
+        const int cnt = min(kMmaRows, np - j0);
+        if (lane == 0) mbar_arrive_expect_tx(&s_full[slot], (uint32_t)(cnt * tbytes));
+        __syncwarp();
+        for (int rr = lane; rr < cnt; rr += 32)
+          bulk_g2s(s_stage + (size_t)slot * stage_bytes + (size_t)rr * pitch,
+                   Wb + (size_t)s_rows[j0 + rr] * row_bytes, (uint32_t)tbytes, &s_full[slot]);
       }
     } else {
       for (int st = 0; st < nstage; ++st) {
