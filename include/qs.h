@@ -216,7 +216,8 @@ qs_status qs_ternary_pack(const float* w, int d_out, int d_in, float eps,
  * Arguments: QS_OP_TOPK_MASK (T, d, 0, k); QS_OP_SPARSE_LINEAR (T, d_in, d_out,
  * k); QS_OP_SPARSE_FFN (T, d_model, d_ff, k_h); QS_OP_QUANT_SPARSE_LINEAR
  * (T, d_in, d_out, k); QS_OP_TERNARY_PACK (0, d_in, d_out, 0).  The dtype does
- * not change the size. */
+ * not change the size, and a workspace of this size also serves calls with the
+ * same sizes and any other k. */
 size_t qs_workspace_size(int op, int T, int d_in, int d_out, int k);
 
 /* Zero-fill `ws_bytes` of workspace on `stream` (enqueued, not synchronous). */

@@ -12,13 +12,14 @@
 // Mapping (B200: 148 SMs, HBM3e).  Measured on this pattern (2867 kept rows
 // of 22 KB): 512-byte segments per request stream at ~3.4 TB/s whatever the
 // load depth, while 1-D bulk copies (TMA) of multi-KB row segments reach
-// ~4.4-4.8 TB/s, close to a contiguous read.  So:
+// 6.0 TB/s over 4 GiB (5.5 KB every 22 KB; plain reads peak at 7.1 TB/s).  So:
 //   * a row is cut into n_ct equal column tiles of a few KB (e.g. 4 x 5.5 KB
 //     for 11008 bf16 columns); a CTA owns one tile, one weight matrix and a
 //     contiguous slice of the row list (split-K);
-//   * one producer thread issues a cp.async.bulk per kept row into a ring of
-//     shared-memory stages guarded by mbarriers (transaction-count
-//     completion); each wait is bounded and reports DEV_TIMEOUT if it runs out;
+//   * the producer warp issues a cp.async.bulk per kept row (a stage's rows
+//     from its lanes side by side) into a ring of shared-memory stages guarded
+//     by mbarriers (transaction-count completion); each wait is bounded and
+//     reports DEV_TIMEOUT if it runs out;
 //   * each consumer thread owns one 16-byte column vector of the tile for the
 //     whole stream (f32 accumulators in registers, one per token), so no
 //     cross-warp reduction is needed;

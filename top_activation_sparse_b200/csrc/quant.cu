@@ -22,9 +22,9 @@ namespace qs {
 namespace {
 
 // ---- int8 x ternary gather-GEMV ----------------------------------------------
-// Packed rows are streamed like the bf16 gather-GEMV: one producer thread
-// issues a cp.async.bulk per kept row (whole rows, or a few column tiles) into a
-// ring of ~16 KB shared-memory stages.
+// Packed rows are streamed like the bf16 gather-GEMV: the producer warp
+// issues a cp.async.bulk per kept row (a column tile of it) into a ring of
+// ~16 KB shared-memory stages.
 //
 // Decoding.  Each code c (00 = 0, 01 = +1, 10 = -1) is first mapped to
 // u = t + 1 in {0, 1, 2} with four logic operations per word.  Codes j and j+8
