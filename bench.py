@@ -190,14 +190,41 @@ def load_peaks() -> dict:
 KERNEL_SOURCES = {"gemv": "gemv.cu", "prefill": "prefill_gemm.cu", "qgemv": "quant.cu"}
 
 
+def _code_only(text: str) -> str:
+    """C/C++ source without comments and blank-line noise: a comment edit does
+    not change the compiled kernel, so it must not void a profile."""
+    import re
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c == '"' or c == "'":                       # string / char literal
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    lines = (re.sub(r"[ \t]+", " ", line).strip() for line in "".join(out).splitlines())
+    return "\n".join(line for line in lines if line)
+
+
 def kernel_source_digest(profile: str) -> str:
-    """Digest of the dominant kernel's source (its .cu and the shared header)."""
+    """Digest of the dominant kernel's code (its .cu and the shared header,
+    comments stripped)."""
     import hashlib
     h = hashlib.sha256()
     main = KERNEL_SOURCES[profile.split("_")[0]]
     for name in (main, "qs_internal.cuh"):
-        with open(os.path.join(ROOT, "top_activation_sparse_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "top_activation_sparse_b200", "csrc", name), encoding="utf-8") as f:
+            h.update(_code_only(f.read()).encode("utf-8"))
     return h.hexdigest()[:16]
 
 

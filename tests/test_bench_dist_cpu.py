@@ -78,3 +78,21 @@ def test_clock_summary():
     assert s["sm_mhz"] == 1965.0 and s["sm_max_mhz"] == 1965.0 and s["samples"] == 3
     assert s["reasons"] == ["sw_power_cap"]
     assert bench.summarize_clocks([])["samples"] == 0
+
+
+def test_profile_digest_ignores_comments():
+    """A profile stays valid across comment edits, not across code edits."""
+    code = 'int f(int a) { // add one\n  return a + 1; /* done */ }\nconst char* s = "// not a comment";\n'
+    same = 'int f(int a) {\n  return a + 1; }\n\n\nconst char* s = "// not a comment";  // note\n'
+    other = 'int f(int a) {\n  return a + 2; }\nconst char* s = "// not a comment";\n'
+    assert bench._code_only(code) == bench._code_only(same)
+    assert bench._code_only(code) != bench._code_only(other)
+    assert '"// not a comment"' in bench._code_only(code)
+
+
+def test_committed_profiles_match_the_kernels():
+    """Every committed profile's digest matches the current kernel code, so
+    the bench line reports its DRAM traffic."""
+    for name in ("gemv_upgate_ffn_relu2_llama7b_T1", "prefill_gemm_prefill_bf16_2048_T2048",
+                 "qgemv_quant_up_4096x11008_T32"):
+        assert bench.profiled_traffic(name) is not None, name
