@@ -8,7 +8,7 @@
 // contraction over the masked activations and belongs on the tensor cores.
 //
 // sm_100a design (persistent: one CTA per SM walks output tiles of 128 x 256):
-//   * TMA (cp.async.bulk.tensor, 128-byte swizzle, no multicast) loads an A
+//   * TMA (cp.async.bulk.tensor, 128-byte swizzle, one CTA per copy) loads an A
 //     tile of X_sparse (128 rows x 64 K, K-major) and a B tile of W^T (64 K x
 //     256 N, N-major, as four 64-column boxes) per stage into a 4-stage ring;
 //   * one thread issues tcgen05.mma.kind::f16 (bf16 x bf16 -> f32) with the

@@ -99,7 +99,7 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* b, uint32_t byte
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)), "r"(bytes)
                : "memory");
 }
-// 1-D bulk copy global -> this CTA's shared memory (no multicast); completion
+// 1-D bulk copy global -> this CTA's shared memory (this CTA only); completion
 // is signalled on `bar` as transaction bytes.  16-byte aligned, size % 16 == 0.
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile(
