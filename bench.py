@@ -258,6 +258,18 @@ def _mk_events(torch, stream, n):
     return evs, (ctypes.c_void_p * n)(*[e.cuda_event for e in evs])
 
 
+def workload_desc(args, T: int) -> str:
+    """The workload's description, identical in both arms' `config`."""
+    w = workloads.WORKLOADS[args.workload]
+    if w.kind == "ffn":
+        return (f"{args.workload}: sparse FFN decode layer, d_model={w.d_in}, d_ff={w.d_out}, "
+                f"act={w.act}, K_x={w.k}, K_h={w.k_h}, bf16")
+    if w.kind == "quant":
+        return (f"{args.workload}: int8 x ternary sparse projection, T={T}, {w.d_in}->{w.d_out}, "
+                f"K={w.k}, packed 2-bit weights")
+    return f"{args.workload}: sparse linear, T={T}, {w.d_in}->{w.d_out}, K={w.k}, {w.dtype}"
+
+
 def setup_ffn(args, qs, torch, device, stream, rank):
     """One sparse FFN layer per step, rotating over independent layers."""
     w = workloads.WORKLOADS[args.workload]
@@ -316,8 +328,7 @@ def setup_ffn(args, qs, torch, device, stream, rank):
         "kernel": "gemv_kernel (up/gate gather-GEMV with the gating epilogue)",
         "bound": "hbm", "dom_work": upgate_bytes, "layer_work": upgate_bytes + down_bytes + topk_bytes,
         "extra": {"rows_streamed": {"x": rows_x, "h": rows_h}},
-        "desc": (f"{args.workload}: sparse FFN decode layer, d_model={d_model}, d_ff={d_ff}, "
-                 f"act={w.act}, K_x={k_in}, K_h={k_h}, bf16"),
+        "desc": workload_desc(args, T),
         "l2": (f"inputs larger than L2: {n_layers} independent layers "
                f"({n_layers * layer_bytes / 1e9:.2f} GB of weights) rotated per step"),
         "e2e_call": e2e_call, "cpu_rate": cpu_rate, "launches": 4, "dtype": "bf16",
@@ -386,8 +397,7 @@ def setup_linear(args, qs, torch, device, stream, rank):
         "dense_args": (lambda l: c_args(l, None, w.d_in)),
         "phases": ["topk", "projection"], "dominant": "projection", "kernel": kernel,
         "bound": bound, "dom_work": work, "layer_work": work, "extra": extra,
-        "desc": (f"{args.workload}: sparse linear, T={T}, {w.d_in}->{w.d_out}, K={w.k}, "
-                 f"{w.dtype}"),
+        "desc": workload_desc(args, T),
         "l2": f"inputs larger than L2: {n_layers} weight copies ({n_layers * wbytes / 1e9:.2f} GB) rotated",
         "e2e_call": e2e_call, "cpu_rate": cpu_rate, "launches": 2, "dtype": w.dtype,
         "profile": f"{'prefill_gemm' if prefill else 'gemv'}_{args.workload}_T{T}",
@@ -451,8 +461,7 @@ def setup_quant(args, qs, torch, device, stream, rank):
         "phases": ["quant_topk", "projection"], "dominant": "projection",
         "kernel": "qgemv_kernel (int8 x ternary gather)", "bound": "hbm", "dom_work": work,
         "layer_work": work, "extra": {"rows_streamed": rows},
-        "desc": (f"{args.workload}: int8 x ternary sparse projection, T={T}, {w.d_in}->{w.d_out}, "
-                 f"K={w.k}, packed 2-bit weights"),
+        "desc": workload_desc(args, T),
         "l2": f"inputs larger than L2: {n_layers} packed weight copies ({n_layers * wbytes / 1e9:.2f} GB) rotated",
         "e2e_call": e2e_call, "cpu_rate": cpu_rate, "launches": 2, "dtype": "int8",
         "profile": f"qgemv_{args.workload}_T{T}",
@@ -716,8 +725,8 @@ def run_reference(args, rank, world, local):
         "vs_baseline": None,
         "dtype": "f64",
         "data": "synthetic: x ~ N(0,1), W ~ N(0,1/fan_in) (seeded)",
-        "config": {"workload": f"{args.workload} (same workload as --impl ours), CPU oracle",
-                   "batch_per_gpu": T, "global_batch": T, "parallelism": "host cores"},
+        "config": {"workload": workload_desc(args, T), "batch_per_gpu": T, "global_batch": T,
+                   "parallelism": "host cores (the fp64 oracle, rank 0)"},
         "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": _threads_in_use(),
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0,

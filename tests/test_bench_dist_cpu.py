@@ -96,3 +96,23 @@ def test_committed_profiles_match_the_kernels():
     for name in ("gemv_upgate_ffn_relu2_llama7b_T1", "prefill_gemm_prefill_bf16_2048_T2048",
                  "qgemv_quant_up_4096x11008_T32"):
         assert bench.profiled_traffic(name) is not None, name
+
+
+def test_reference_arm_runs_the_oracle_on_the_same_workload():
+    """`bench.py --impl reference` times the oracle on the host and prints the
+    contract's line, with the same workload description as our arm."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference",
+                        "--workload", "linear_f32_512", "--steps", "5", "--warmup", "3",
+                        "--ref-seconds", "1"], capture_output=True, text=True, timeout=300, cwd=root)
+    assert r.returncode == 0, r.stderr
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["value"] > 0 and line["unit"] == "tokens/s"
+    assert line["metric"] == bench.METRIC and line["higher_is_better"] is True
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
+    args = bench.parse_args(["--workload", "linear_f32_512"])
+    assert line["config"]["workload"] == bench.workload_desc(args, args.batch)
