@@ -39,7 +39,13 @@
  *             mask always has exactly K ones per row, even when fewer than K
  *             entries are nonzero.  Inputs must be finite (NaN ranks above inf).
  *   Numerics. Products accumulate in fp32 (int32 for the int8 x ternary path);
- *             a bf16 output is rounded once, to nearest-even, at the end.
+ *             a bf16 output is rounded once, to nearest-even, at the end.  With
+ *             bf16 weights and 3 to 64 tokens the projections run on the tensor
+ *             cores and the token values enter them rounded to bf16 (the
+ *             inputs are bf16 already; the FFN's f32 h is rounded for the
+ *             down projection).  Split-K partial sums are added in an order
+ *             that is not fixed, so float results may differ in their last
+ *             bits between runs; integer results never do.
  */
 #ifndef QS_H
 #define QS_H
