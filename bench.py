@@ -59,6 +59,9 @@ def parse_args(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--layers", type=int, default=0,
                     help="independent layers to rotate over (0: enough to exceed 4x L2)")
+    ap.add_argument("--gate-first", action="store_true",
+                    help="dReLU FFN workloads: gate projection first, then W_up (output-major) "
+                         "read only for open gates (qs_sparse_ffn_gate_first)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-seconds", type=float, default=120.0)
@@ -68,6 +71,8 @@ def parse_args(argv=None):
         a.batch = 1 if w.kind in ("ffn", "quant") else w.batches[0]
     if a.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if a.gate_first and workloads.WORKLOADS[a.workload].act != "drelu":
+        ap.error("--gate-first needs a dReLU FFN workload")
     if a.steps < 1:
         ap.error("--steps must be >= 1")
     return a
@@ -262,8 +267,10 @@ def workload_desc(args, T: int) -> str:
     """The workload's description, identical in both arms' `config`."""
     w = workloads.WORKLOADS[args.workload]
     if w.kind == "ffn":
+        gf = (", gate first (W_up output-major, rows of open gates only)"
+              if getattr(args, "gate_first", False) else "")
         return (f"{args.workload}: sparse FFN decode layer, d_model={w.d_in}, d_ff={w.d_out}, "
-                f"act={w.act}, K_x={w.k}, K_h={w.k_h}, bf16")
+                f"act={w.act}, K_x={w.k}, K_h={w.k_h}, bf16{gf}")
     if w.kind == "quant":
         return (f"{args.workload}: int8 x ternary sparse projection, T={T}, {w.d_in}->{w.d_out}, "
                 f"K={w.k}, packed 2-bit weights")
@@ -279,18 +286,26 @@ def setup_ffn(args, qs, torch, device, stream, rank):
     layer_bytes = 3 * d_model * d_ff * 2
     n_layers = args.layers or max(2, math.ceil(4 * L2_BYTES / layer_bytes))
     layers = [workloads.ffn_weights_device(w, l, device) for l in range(n_layers)]
+    gate_first = bool(getattr(args, "gate_first", False))
+    if gate_first:                    # W_up output-major: [d_ff, d_model]
+        layers = [(up.t().contiguous(), gate, down) for up, gate, down in layers]
+    op = qs.QS_OP_SPARSE_FFN_GATE_FIRST if gate_first else qs.QS_OP_SPARSE_FFN
     bias = None
     if w.bias is not None:
         bias = torch.full((d_ff,), float(w.bias), dtype=torch.float32, device=device)
     x = workloads.activations_device(w, T, device, salt=rank)
     y = torch.empty(T, d_model, dtype=torch.bfloat16, device=device)
-    ws = qs.new_workspace(qs.QS_OP_SPARSE_FFN, T, d_model, d_ff, k_h, device)
+    ws = qs.new_workspace(op, T, d_model, d_ff, k_h, device)
     sp = stream.cuda_stream
     bptr = bias.data_ptr() if bias is not None else None
-    fn = qs.lib().qs_sparse_ffn
+    fn = qs.lib().qs_sparse_ffn_gate_first if gate_first else qs.lib().qs_sparse_ffn
 
     def c_args(l, ev, kx=k_in, kh=k_h):
         up, gate, down = layers[l]
+        if gate_first:                # x is dense on this path (kx = d_model)
+            return (x.data_ptr(), qs.QS_BF16, T, d_model, d_ff, kh, gate.data_ptr(),
+                    up.data_ptr(), bptr, bptr, down.data_ptr(), y.data_ptr(), None, None, ev,
+                    ws.data_ptr(), ws.numel(), sp)
         return (x.data_ptr(), qs.QS_BF16, T, d_model, d_ff, act, kx, kh, up.data_ptr(),
                 gate.data_ptr(), bptr, bptr, down.data_ptr(), y.data_ptr(), None, None, ev,
                 ws.data_ptr(), ws.numel(), sp)
@@ -299,24 +314,40 @@ def setup_ffn(args, qs, torch, device, stream, rank):
     for l in range(n_layers):
         st = fn(*c_args(l, None))
         assert st == 0, qs.qs_status_string(st)
-        rows.append(qs.qs_workspace_stats(ws, qs.QS_OP_SPARSE_FFN, T, d_model, d_ff, k_h))
+        rows.append(qs.qs_workspace_stats(ws, op, T, d_model, d_ff, k_h))
     assert qs.qs_device_status(ws) == qs.QS_OK
     rows_x = float(np.mean([r[0] for r in rows]))
     rows_h = float(np.mean([r[1] for r in rows]))
-    # algorithmic bytes of the up/gate kernel per launch: the kept rows of
-    # W_up^T and W_gate^T, the staged (index, T values) entries, h written (f32)
-    upgate_bytes = rows_x * d_ff * 2 * 2 + rows_x * (4 + 4 * T) + T * d_ff * 4
+    if gate_first:
+        # the gate kernel streams the kept rows of W_gate^T (one matrix) and
+        # writes ReLU(g + b) (f32); the up kernel streams the open rows of W_up
+        # and reads and rewrites those h entries
+        rows_up = float(np.mean([r[2] for r in rows]))
+        upgate_bytes = (rows_x * d_ff * 2 + rows_x * (4 + 4 * T) + T * d_ff * 4
+                        + rows_up * d_model * 2 + T * d_model * 2 + rows_up * T * 8)
+        extra_rows = {"x": rows_x, "h": rows_h, "up_open_gates": rows_up}
+    else:
+        # algorithmic bytes of the up/gate kernel per launch: the kept rows of
+        # W_up^T and W_gate^T, the staged (index, T values) entries, h written (f32)
+        upgate_bytes = rows_x * d_ff * 2 * 2 + rows_x * (4 + 4 * T) + T * d_ff * 4
+        extra_rows = {"x": rows_x, "h": rows_h}
     down_bytes = rows_h * d_model * 2 + rows_h * (4 + 4 * T) + T * d_model * 2
     topk_bytes = T * d_model * 2 + T * d_ff * 4
     lw = layers
 
     def e2e_call(i, x_dev, y_dev):
         up, gate, down = lw[i % n_layers]
-        qs.qs_sparse_ffn(x_dev, up, gate, down, w.act, k_in, k_h, b_up=bias, b_gate=bias, y=y_dev,
-                         ws=ws)
+        if gate_first:
+            qs.qs_sparse_ffn_gate_first(x_dev, gate, up, down, k_h, b_up=bias, b_gate=bias,
+                                        y=y_dev, ws=ws)
+        else:
+            qs.qs_sparse_ffn(x_dev, up, gate, down, w.act, k_in, k_h, b_up=bias, b_gate=bias,
+                             y=y_dev, ws=ws)
 
     def cpu_rate():
         up, gate, down = (t.float().cpu().numpy() for t in layers[0])
+        if gate_first:
+            up = np.ascontiguousarray(up.T)
         return cpu_oracle_ffn(w, x.float().cpu().numpy(), up, gate, down, args.cpu_seconds)
 
     phases = ["topk_x", "upgate", "topk_h", "down"]
@@ -325,14 +356,16 @@ def setup_ffn(args, qs, torch, device, stream, rank):
         "args": lambda l, ev: c_args(l, ev), "n_events": qs.QS_FFN_PHASE_EVENTS,
         "dense_args": (lambda l: c_args(l, None, d_model, d_ff)),
         "phases": phases, "dominant": "upgate",
-        "kernel": "gemv_kernel (up/gate gather-GEMV with the gating epilogue)",
+        "kernel": ("gemv_kernel (gate gather-GEMV) + up_rows_kernel (open gates' rows of W_up)"
+                   if gate_first else "gemv_kernel (up/gate gather-GEMV with the gating epilogue)"),
         "bound": "hbm", "dom_work": upgate_bytes, "layer_work": upgate_bytes + down_bytes + topk_bytes,
-        "extra": {"rows_streamed": {"x": rows_x, "h": rows_h}},
+        "extra": {"rows_streamed": extra_rows},
         "desc": workload_desc(args, T),
         "l2": (f"inputs larger than L2: {n_layers} independent layers "
                f"({n_layers * layer_bytes / 1e9:.2f} GB of weights) rotated per step"),
-        "e2e_call": e2e_call, "cpu_rate": cpu_rate, "launches": 4, "dtype": "bf16",
-        "profile": f"gemv_upgate_{args.workload}_T{T}",
+        "e2e_call": e2e_call, "cpu_rate": cpu_rate, "launches": 5 if gate_first else 4,
+        "dtype": "bf16",
+        "profile": f"gemv_{'gatefirst' if gate_first else 'upgate'}_{args.workload}_T{T}",
     }
 
 

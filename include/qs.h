@@ -83,7 +83,8 @@ typedef enum qs_op {
   QS_OP_SPARSE_LINEAR = 1,
   QS_OP_SPARSE_FFN = 2,
   QS_OP_QUANT_SPARSE_LINEAR = 3,
-  QS_OP_TERNARY_PACK = 4
+  QS_OP_TERNARY_PACK = 4,
+  QS_OP_SPARSE_FFN_GATE_FIRST = 5
 } qs_op;
 
 /* Largest row length (d, d_in, d_ff) a top-K row may have: one CTA holds a
@@ -173,6 +174,39 @@ qs_status qs_sparse_ffn(const void* x, int dtype, int T, int d_model, int d_ff, 
                         void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * qs_sparse_ffn_gate_first -- the dReLU layer of qs_sparse_ffn (QS_ACT_DRELU,
+ *   dense x, k_in = d_model), with the up projection restricted to open gates.
+ *   Source: Turbo Sparse summary (blog.csdn.net), Eq. 2: h = ReLU(g + b_gate)
+ *   * ReLU(u + b_up) is 0 wherever g + b_gate <= 0, whatever u is.  So the
+ *   gate projection runs first (all of W_gate), and row j of W_up is read only
+ *   if some token's gate j is open.  Same result as qs_sparse_ffn with
+ *   QS_ACT_DRELU and k_in = d_model, up to float32 summation order: an exact
+ *   reordering, not an approximation.
+ *
+ *   x         [T, d_model] `dtype` (bf16 or f32), used dense.
+ *   k_h       0..d_ff: top-K on |h| before the down projection.
+ *   wt_gate   [d_model, d_ff] `dtype` (= W_gate^T, input-major as in qs_sparse_ffn).
+ *   w_up      [d_ff, d_model] `dtype` (= W_up, OUTPUT-major: the nn.Linear layout),
+ *             so that the weights of one output column are one contiguous row.
+ *   wt_down   [d_ff, d_model] `dtype` (= W_down^T).
+ *   b_up, b_gate, y, h_out, idx_h_out, phase_events: as qs_sparse_ffn (the
+ *             "up/gate" phase event follows both the gate and the up kernel).
+ *   ws        qs_workspace_size(QS_OP_SPARSE_FFN_GATE_FIRST, T, d_model, d_ff, k_h)
+ *             bytes.  qs_workspace_stats also reports rows[2] = rows of w_up read.
+ *   The first call on a device fills a constant array (a vector of 1.0 used by
+ *   the gate's epilogue) and synchronises `stream`: make it before any stream
+ *   capture.
+ *   d_model and d_ff must be multiples of 8 (bf16) or 4 (f32).
+ *   Errors: INVALID_ARG, ALIGNMENT, WORKSPACE, UNSUPPORTED, CUDA.
+ */
+qs_status qs_sparse_ffn_gate_first(const void* x, int dtype, int T, int d_model, int d_ff,
+                                   int k_h, const void* wt_gate, const void* w_up,
+                                   const float* b_up, const float* b_gate, const void* wt_down,
+                                   void* y, float* h_out, int32_t* idx_h_out,
+                                   void* const* phase_events,
+                                   void* ws, size_t ws_bytes, void* stream);
+
+/*
  * qs_quant_sparse_linear -- BitNet b1.58 + Q-Sparse projection.
  *   Source: Q-Sparse news article, Top-K section, quantized-model paragraphs
  *   (inputs are quantized before top-K, with an epsilon guarding a division;
@@ -220,8 +254,9 @@ qs_status qs_ternary_pack(const float* w, int d_out, int d_in, float eps,
 
 /* Bytes of workspace `op` needs for these sizes (0 if the sizes are invalid).
  * Arguments: QS_OP_TOPK_MASK (T, d, 0, k); QS_OP_SPARSE_LINEAR (T, d_in, d_out,
- * k); QS_OP_SPARSE_FFN (T, d_model, d_ff, k_h); QS_OP_QUANT_SPARSE_LINEAR
- * (T, d_in, d_out, k); QS_OP_TERNARY_PACK (0, d_in, d_out, 0).  The dtype does
+ * k); QS_OP_SPARSE_FFN and QS_OP_SPARSE_FFN_GATE_FIRST (T, d_model, d_ff, k_h);
+ * QS_OP_QUANT_SPARSE_LINEAR (T, d_in, d_out, k); QS_OP_TERNARY_PACK (0, d_in,
+ * d_out, 0).  The dtype does
  * not change the size, and a workspace of this size also serves calls with the
  * same sizes and any other k. */
 size_t qs_workspace_size(int op, int T, int d_in, int d_out, int k);
@@ -237,8 +272,10 @@ qs_status qs_device_status(void* ws, void* stream);
  * workspace and these sizes, how many weight rows its projections streamed:
  * rows[0] = distinct inputs with a kept nonzero value across the T tokens (the
  * rows of wt / wt_up / wt_gate read), rows[1] = the same for h (rows of
- * wt_down read; QS_OP_SPARSE_FFN only, else 0).  These counts are the
- * algorithmic weight traffic: rows * d_out * sizeof(weight). */
+ * wt_down read; the two FFN ops only, else 0), and for
+ * QS_OP_SPARSE_FFN_GATE_FIRST only (then `rows` holds 3) rows[2] = open gates
+ * across the T tokens (the rows of w_up read).  These counts are the
+ * algorithmic weight traffic: rows * row length * sizeof(weight). */
 qs_status qs_workspace_stats(const void* ws, int op, int T, int d_in, int d_out, int k,
                              int32_t* rows, void* stream);
 

@@ -21,7 +21,8 @@ def L():
 
 def test_header_declares_the_boundary():
     names = qs.header_functions()
-    for n in ("qs_topk_mask", "qs_sparse_linear", "qs_sparse_ffn", "qs_quant_sparse_linear",
+    for n in ("qs_topk_mask", "qs_sparse_linear", "qs_sparse_ffn", "qs_sparse_ffn_gate_first",
+              "qs_quant_sparse_linear",
               "qs_ternary_pack", "qs_workspace_size", "qs_workspace_init", "qs_device_status",
               "qs_workspace_stats", "qs_status_string"):
         assert n in names
@@ -53,6 +54,10 @@ def test_workspace_size_is_host_only_and_sane(L):
     assert f(qs.QS_OP_QUANT_SPARSE_LINEAR, 1, 4096, 48, 1597) == 0
     assert f(qs.QS_OP_TERNARY_PACK, 0, 4096, 11008, 0) > 0
     assert f(99, 1, 1, 1, 1) == 0
+    # the gate-first layer needs the FFN's buffers, with partial sums sized for
+    # the gate alone
+    assert f(qs.QS_OP_SPARSE_FFN_GATE_FIRST, 1, 4096, 14336, 1433) > 0
+    assert f(qs.QS_OP_SPARSE_FFN_GATE_FIRST, 1, 4096, 14336, 14337) == 0
     # more than the decode chunk of tokens does not grow the decode buffers
     c = f(qs.QS_OP_SPARSE_FFN, 64, 4096, 11008, 7705)
     assert f(qs.QS_OP_SPARSE_FFN, 640, 4096, 11008, 7705) == c
@@ -93,6 +98,17 @@ def test_invalid_arguments_are_rejected_on_the_host(L):
     assert L.qs_sparse_ffn(*bad) == qs.QS_ERR_INVALID_ARG
     bad = list(args); bad[4] = 100            # d_ff % 8 != 0
     assert L.qs_sparse_ffn(*bad) == qs.QS_ERR_ALIGNMENT
+    # qs_sparse_ffn_gate_first: k_h > d_ff, NULL w_up, d_model % 8, tiny workspace
+    gf = [_p(FAKE), 1, 1, 64, 128, 32, _p(FAKE), _p(FAKE), None, None, _p(FAKE), _p(FAKE),
+          None, None, None, ws, wsb, s]
+    bad = list(gf); bad[5] = 129
+    assert L.qs_sparse_ffn_gate_first(*bad) == qs.QS_ERR_INVALID_ARG
+    bad = list(gf); bad[7] = None
+    assert L.qs_sparse_ffn_gate_first(*bad) == qs.QS_ERR_INVALID_ARG
+    bad = list(gf); bad[3] = 60
+    assert L.qs_sparse_ffn_gate_first(*bad) == qs.QS_ERR_ALIGNMENT
+    bad = list(gf); bad[16] = 64
+    assert L.qs_sparse_ffn_gate_first(*bad) == qs.QS_ERR_WORKSPACE
     # qs_quant_sparse_linear: d_out % 16, negative eps
     assert L.qs_quant_sparse_linear(_p(FAKE), 1, 1, 64, 40, 8, _p(FAKE), ctypes.c_float(1.0),
                                     ctypes.c_float(1e-5), _p(FAKE), None, None, None, None, ws, wsb, s) == qs.QS_ERR_ALIGNMENT

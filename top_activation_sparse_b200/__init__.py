@@ -40,6 +40,7 @@ QS_OP_SPARSE_LINEAR = 1
 QS_OP_SPARSE_FFN = 2
 QS_OP_QUANT_SPARSE_LINEAR = 3
 QS_OP_TERNARY_PACK = 4
+QS_OP_SPARSE_FFN_GATE_FIRST = 5
 
 QS_MAX_ROW = 49152
 QS_NOALLOC_SCRATCH_BYTES = 4 << 20
@@ -66,6 +67,8 @@ _SIGNATURES = {
     "qs_sparse_linear": (_i, [_vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _sz, _vp]),
     "qs_sparse_ffn": (_i, [_vp, _i, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                            _vp, _vp, _vp, _sz, _vp]),
+    "qs_sparse_ffn_gate_first": (_i, [_vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                      _vp, _vp, _vp, _sz, _vp]),
     "qs_quant_sparse_linear": (_i, [_vp, _i, _i, _i, _i, _i, _vp, _f, _f, _vp, _vp, _vp, _vp,
                                     _vp, _vp, _sz, _vp]),
     "qs_ternary_pack": (_i, [_vp, _i, _i, _f, _vp, _vp, _vp, _sz, _vp]),
@@ -197,10 +200,14 @@ def qs_device_status(ws: torch.Tensor, stream=None) -> int:
 
 
 def qs_workspace_stats(ws: torch.Tensor, op: int, T: int, d_in: int, d_out: int, k: int,
-                       stream=None) -> tuple[int, int]:
-    rows = (ctypes.c_int32 * 2)()
+                       stream=None) -> tuple[int, ...]:
+    """Weight rows the last call streamed: (input rows, h rows), plus the
+    rows of W_up read for QS_OP_SPARSE_FFN_GATE_FIRST."""
+    rows = (ctypes.c_int32 * 3)()
     _check("qs_workspace_stats",
            lib().qs_workspace_stats(ws.data_ptr(), op, T, d_in, d_out, k, rows, _stream_ptr(stream)))
+    if op == QS_OP_SPARSE_FFN_GATE_FIRST:
+        return int(rows[0]), int(rows[1]), int(rows[2])
     return int(rows[0]), int(rows[1])
 
 
@@ -306,6 +313,33 @@ def qs_sparse_ffn(x, wt_up, wt_gate, wt_down, act, k_in: int, k_h: int, b_up=Non
         wt_up.data_ptr(), wt_gate.data_ptr(), _ptr(b_up), _ptr(b_gate), wt_down.data_ptr(),
         y.data_ptr(), _ptr(h_out), _ptr(idx_h_out), ev, ws.data_ptr(), ws.numel(),
         _stream_ptr(stream)))
+    return FfnResult(y, h_out, idx_h_out)
+
+
+def qs_sparse_ffn_gate_first(x, wt_gate, w_up, wt_down, k_h: int, b_up=None, b_gate=None,
+                             y=None, h_out=None, idx_h_out=None, phase_events=None, ws=None,
+                             stream=None) -> FfnResult:
+    """dReLU FFN layer with dense x, the gate first and the up projection
+    only over open gates.  w_up is [d_ff, d_model] (output-major)."""
+    dev = _need_cuda(x, wt_gate, w_up, wt_down, b_up, b_gate)
+    T, d_model = x.shape
+    d_ff = wt_gate.shape[1]
+    for w, shp in ((wt_gate, (d_model, d_ff)), (w_up, (d_ff, d_model)), (wt_down, (d_ff, d_model))):
+        if tuple(w.shape) != shp or w.dtype != x.dtype:
+            raise ValueError(f"weight must be {shp} {x.dtype}")
+    for b in (b_up, b_gate):
+        if b is not None and (tuple(b.shape) != (d_ff,) or b.dtype != torch.float32):
+            raise ValueError("biases must be [d_ff] float32")
+    y = _out(y if y is not None else True, (T, d_model), x.dtype, dev)
+    h_out = _out(h_out, (T, d_ff), torch.float32, dev)
+    idx_h_out = _out(idx_h_out, (T, k_h), torch.int32, dev)
+    _need_cuda(y, h_out, idx_h_out)
+    ev = _events(phase_events, QS_FFN_PHASE_EVENTS)
+    ws = _workspace(ws, QS_OP_SPARSE_FFN_GATE_FIRST, T, d_model, d_ff, k_h, dev)
+    _check("qs_sparse_ffn_gate_first", lib().qs_sparse_ffn_gate_first(
+        x.data_ptr(), _dtype_code(x), T, d_model, d_ff, k_h, wt_gate.data_ptr(), w_up.data_ptr(),
+        _ptr(b_up), _ptr(b_gate), wt_down.data_ptr(), y.data_ptr(), _ptr(h_out), _ptr(idx_h_out),
+        ev, ws.data_ptr(), ws.numel(), _stream_ptr(stream)))
     return FfnResult(y, h_out, idx_h_out)
 
 

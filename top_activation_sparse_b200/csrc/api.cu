@@ -3,6 +3,7 @@
 // computation runs in this library's CUDA kernels; there is no host fallback.
 #include <cstring>
 
+#include "gate_first.cuh"
 #include "qs_internal.cuh"
 
 namespace qs {
@@ -14,11 +15,13 @@ constexpr int kChunkT = QS_PREFILL_MIN_T;
 constexpr size_t kTicketBytes = 64 * 1024;       // fixed ticket region
 constexpr int kTicketCap = (int)(kTicketBytes / sizeof(int32_t));
 // fixed ticket slots
-constexpr int kTkTopkX = 0, kTkTopkH = 1, kTkAlpha = 2, kTkGemv = 8;
-// union bitmasks of the several-token path (zero between calls)
+constexpr int kTkTopkX = 0, kTkTopkH = 1, kTkAlpha = 2, kTkUpRows = 3, kTkGemv = 8;
+// union bitmasks of the several-token path, and the open gates of the
+// gate-first FFN (zero between calls)
 constexpr int kTkGemvEnd = 4096;
 constexpr int kUnionX = 4096, kUnionH = 4096 + QS_MAX_ROW / 32;
-static_assert(kUnionH + QS_MAX_ROW / 32 <= (int)(64 * 1024 / 4), "ticket region too small");
+constexpr int kGateBits = kUnionH + QS_MAX_ROW / 32;
+static_assert(kGateBits + QS_MAX_ROW / 32 <= (int)(64 * 1024 / 4), "ticket region too small");
 
 size_t align_up(size_t v) { return (v + kWsAlign - 1) / kWsAlign * kWsAlign; }
 
@@ -96,14 +99,16 @@ bool ws_layout(int op, int T, int d_in, int d_out, int k, WsLayout* L) {
       if (T >= kChunkT) L->xs_bf16 = take((size_t)T * d_in * sizeof(uint16_t));
       break;
     }
-    case QS_OP_SPARSE_FFN: {
+    case QS_OP_SPARSE_FFN:
+    case QS_OP_SPARSE_FFN_GATE_FIRST: {
       if (T < 1 || d_in < 1 || d_out < 1 || d_in > QS_MAX_ROW || d_out > QS_MAX_ROW || k < 0 ||
           k > d_out)
         return false;
       L->xsf_x = take((size_t)Tc * d_in * sizeof(float));
       L->list_x = take((size_t)d_in * sizeof(int32_t));
       L->lval_x = take((size_t)d_in * Tc * sizeof(float));
-      L->parts1_elems = max_parts(d_out, d_in, d_in, 2);
+      // up and gate together, or (gate first) the gate alone
+      L->parts1_elems = max_parts(d_out, d_in, d_in, op == QS_OP_SPARSE_FFN ? 2 : 1);
       L->parts1 = take(L->parts1_elems * sizeof(float));
       L->h = take((size_t)Tc * d_out * sizeof(float));
       L->xsf_h = take((size_t)Tc * d_out * sizeof(float));
@@ -232,8 +237,10 @@ qs_status qs_workspace_stats(const void* ws, int op, int T, int d_in, int d_out,
   QS_TRY_CUDA(cudaMemcpyAsync(c, (const unsigned char*)ws + L.cnt, sizeof(c),
                               cudaMemcpyDeviceToHost, s));
   QS_TRY_CUDA(cudaStreamSynchronize(s));
+  const bool ffn = op == QS_OP_SPARSE_FFN || op == QS_OP_SPARSE_FFN_GATE_FIRST;
   rows[0] = c[0];
-  rows[1] = (op == QS_OP_SPARSE_FFN) ? c[1] : 0;
+  rows[1] = ffn ? c[1] : 0;
+  if (op == QS_OP_SPARSE_FFN_GATE_FIRST) rows[2] = c[2];
   return QS_OK;
 }
 
@@ -339,26 +346,32 @@ qs_status qs_sparse_linear(const void* x, int dtype, int T, int d_in, int d_out,
   return QS_OK;
 }
 
-qs_status qs_sparse_ffn(const void* x, int dtype, int T, int d_model, int d_ff, int act,
-                        int k_in, int k_h, const void* wt_up, const void* wt_gate,
-                        const float* b_up, const float* b_gate, const void* wt_down, void* y,
-                        float* h_out, int32_t* idx_h_out, void* const* phase_events, void* ws,
-                        size_t ws_bytes, void* stream) {
-  if (!valid_dtype(dtype) || x == nullptr || wt_up == nullptr || wt_gate == nullptr ||
+// One sparse gated FFN layer.  With w_up_rows (W_up output-major, [d_ff,
+// d_model]) instead of wt_up it is the gate-first dReLU form: the gate
+// projection runs alone, and the up projection reads only the rows of open
+// gates (exact: the dReLU product is 0 wherever the gate branch is).
+static qs_status ffn_impl(int op, const void* x, int dtype, int T, int d_model, int d_ff, int act,
+                          int k_in, int k_h, const void* wt_up, const void* w_up_rows,
+                          const void* wt_gate, const float* b_up, const float* b_gate,
+                          const void* wt_down, void* y, float* h_out, int32_t* idx_h_out,
+                          void* const* phase_events, void* ws, size_t ws_bytes, void* stream) {
+  const bool gate_first = op == QS_OP_SPARSE_FFN_GATE_FIRST;
+  const void* up = gate_first ? w_up_rows : wt_up;
+  if (!valid_dtype(dtype) || x == nullptr || up == nullptr || wt_gate == nullptr ||
       wt_down == nullptr || y == nullptr || T < 1 || d_model < 1 || d_ff < 1 || k_in < 0 ||
       k_in > d_model || k_h < 0 || k_h > d_ff ||
-      (act != QS_ACT_RELU2_GLU && act != QS_ACT_DRELU))
+      (act != QS_ACT_RELU2_GLU && act != QS_ACT_DRELU) || (gate_first && act != QS_ACT_DRELU))
     return QS_ERR_INVALID_ARG;
   if (d_model > QS_MAX_ROW || d_ff > QS_MAX_ROW) return QS_ERR_UNSUPPORTED;
   const int eb = elem_bytes(dtype);
   const int V = 16 / eb;
   if ((d_model % V) != 0 || (d_ff % V) != 0) return QS_ERR_ALIGNMENT;
-  if (!aligned16(x) || !aligned16(wt_up) || !aligned16(wt_gate) || !aligned16(wt_down) ||
+  if (!aligned16(x) || !aligned16(up) || !aligned16(wt_gate) || !aligned16(wt_down) ||
       !aligned16(y) || !aligned16(h_out) || !aligned16(idx_h_out) || !aligned16(b_up) ||
       !aligned16(b_gate))
     return QS_ERR_ALIGNMENT;
   WsLayout L;
-  qs_status st = check_ws(QS_OP_SPARSE_FFN, T, d_model, d_ff, k_h, ws, ws_bytes, &L);
+  qs_status st = check_ws(op, T, d_model, d_ff, k_h, ws, ws_bytes, &L);
   if (st != QS_OK) return st;
   WsView w{(unsigned char*)ws};
   cudaStream_t s = (cudaStream_t)stream;
@@ -366,6 +379,8 @@ qs_status qs_sparse_ffn(const void* x, int dtype, int T, int d_model, int d_ff, 
     if (phase_events == nullptr) return cudaSuccess;
     return cudaEventRecord((cudaEvent_t)phase_events[i], s);
   };
+  const float* unit = nullptr;                   // gate first: a vector of 1.0 (see step 2)
+  if (gate_first) QS_TRY_CUDA(unit_vector_on_current_device(&unit, s));
 
   for (int t0 = 0; t0 < T; t0 += kChunkT) {
     const int Tc = (T - t0) < kChunkT ? (T - t0) : kChunkT;
@@ -384,7 +399,8 @@ qs_status qs_sparse_ffn(const void* x, int dtype, int T, int d_model, int d_ff, 
     a.ticket = w.ticket(L, kTkTopkX);
     a.union_bits = reinterpret_cast<uint32_t*>(w.ticket(L, kUnionX));
     a.status = w.status();
-    const GemvPlan p_ug = plan_gemv(Tc, d_ff, (int)rows_bound(Tc, d_model, d_model), 2, eb);
+    const GemvPlan p_ug =
+        plan_gemv(Tc, d_ff, (int)rows_bound(Tc, d_model, d_model), gate_first ? 1 : 2, eb);
     const GemvPlan p_dn = plan_gemv(Tc, d_model, (int)rows_bound(Tc, d_ff, k_h), 1, eb);
     if (!plan_fits(L, p_ug, L.parts1_elems, 0) || !plan_fits(L, p_dn, L.parts2_elems, p_ug.tickets))
       return QS_ERR_UNSUPPORTED;
@@ -411,8 +427,34 @@ qs_status qs_sparse_ffn(const void* x, int dtype, int T, int d_model, int d_ff, 
     // one token, list outputs only: the epilogue marks the nonzero h, and the
     // top-K on h starts from that bitmask (it clears it again)
     const bool h_bits = Tc == 1 && idx_h_out == nullptr && topk_bitmask_supported(Tc, d_ff, TK_F32);
-    if (h_bits) g.hbits = reinterpret_cast<uint32_t*>(w.ticket(L, kUnionH));
-    QS_TRY_CUDA(launch_gemv(g, s));
+    uint32_t* hbits = h_bits ? reinterpret_cast<uint32_t*>(w.ticket(L, kUnionH)) : nullptr;
+    if (!gate_first) {
+      g.hbits = hbits;
+      QS_TRY_CUDA(launch_gemv(g, s));
+    } else {
+      // 2a. the gate alone, through the dReLU epilogue: the gate sums sit in
+      // the first slot with b_gate, the empty second slot gets a bias of 1,
+      // so the epilogue writes ReLU(1) * ReLU(g + b_gate) = ReLU(g + b_gate)
+      // to h (exactly) and marks the open gates, over all tokens, in a bitmask
+      g.w[0] = wt_gate; g.w[1] = nullptr;
+      g.mode = 2;
+      g.b_up = b_gate; g.b_gate = unit;
+      uint32_t* gate_bits = reinterpret_cast<uint32_t*>(w.ticket(L, kGateBits));
+      g.hbits = gate_bits;
+      QS_TRY_CUDA(launch_gemv(g, s));
+      // 2b. up projection over the open gates' rows of W_up; finishes h
+      UpRowsArgs u;
+      u.x = a.x; u.T = Tc; u.d_model = d_model; u.d_ff = d_ff;
+      u.bf16 = dtype == QS_BF16;
+      u.w_up = w_up_rows; u.b_up = b_up;
+      u.gate_bits = gate_bits;
+      u.ticket = w.ticket(L, kTkUpRows);
+      u.h = h;
+      u.hbits = hbits;
+      u.n_open = w.at<int32_t>(L.cnt) + 2;
+      u.status = w.status();
+      QS_TRY_CUDA(launch_up_rows(u, s));
+    }
     if (timed) QS_TRY_CUDA(mark(2));
 
     // 3. top-K on |h|
@@ -446,6 +488,27 @@ qs_status qs_sparse_ffn(const void* x, int dtype, int T, int d_model, int d_ff, 
     if (timed) QS_TRY_CUDA(mark(4));
   }
   return QS_OK;
+}
+
+qs_status qs_sparse_ffn(const void* x, int dtype, int T, int d_model, int d_ff, int act,
+                        int k_in, int k_h, const void* wt_up, const void* wt_gate,
+                        const float* b_up, const float* b_gate, const void* wt_down, void* y,
+                        float* h_out, int32_t* idx_h_out, void* const* phase_events, void* ws,
+                        size_t ws_bytes, void* stream) {
+  return ffn_impl(QS_OP_SPARSE_FFN, x, dtype, T, d_model, d_ff, act, k_in, k_h, wt_up, nullptr,
+                  wt_gate, b_up, b_gate, wt_down, y, h_out, idx_h_out, phase_events, ws, ws_bytes,
+                  stream);
+}
+
+qs_status qs_sparse_ffn_gate_first(const void* x, int dtype, int T, int d_model, int d_ff,
+                                   int k_h, const void* wt_gate, const void* w_up,
+                                   const float* b_up, const float* b_gate, const void* wt_down,
+                                   void* y, float* h_out, int32_t* idx_h_out,
+                                   void* const* phase_events, void* ws, size_t ws_bytes,
+                                   void* stream) {
+  return ffn_impl(QS_OP_SPARSE_FFN_GATE_FIRST, x, dtype, T, d_model, d_ff, QS_ACT_DRELU, d_model,
+                  k_h, nullptr, w_up, wt_gate, b_up, b_gate, wt_down, y, h_out, idx_h_out,
+                  phase_events, ws, ws_bytes, stream);
 }
 
 qs_status qs_quant_sparse_linear(const void* x, int dtype, int T, int d_in, int d_out, int k,
