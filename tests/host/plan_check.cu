@@ -119,16 +119,19 @@ static void check_layout(int op, int T, int d_in, int d_out, int k) {
       }
     }
   }
-  if (op == QS_OP_SPARSE_FFN) {
+  if (op == QS_OP_SPARSE_FFN || op == QS_OP_SPARSE_FFN_GATE_FIRST) {
+    // up and gate together (two matrices), or the gate alone (gate first)
+    const int mats = op == QS_OP_SPARSE_FFN ? 2 : 1;
     for (int t = 1; t <= Tc; ++t)
       for (int eb : {2, 4}) {
         const long tk = (long)t * k;
         const int rb_h = (int)(tk < d_out ? tk : d_out);
-        CHECK(qs::plan_gemv(t, d_out, (int)((long)t * d_in < d_in ? t * d_in : d_in), 2, eb)
-                      .parts_elems <= L.parts1_elems,
-              f, op, T, d_in, d_out, k);
-        CHECK(qs::plan_gemv(t, d_in, rb_h, 1, eb).parts_elems <= L.parts2_elems, f, op, T, d_in,
-              d_out, k);
+        const qs::GemvPlan p1 = qs::plan_gemv(t, d_out, d_in, mats, eb);
+        const qs::GemvPlan p2 = qs::plan_gemv(t, d_in, rb_h, 1, eb);
+        CHECK(p1.parts_elems <= L.parts1_elems, f, op, T, d_in, d_out, k);
+        CHECK(p2.parts_elems <= L.parts2_elems, f, op, T, d_in, d_out, k);
+        // both projections' tickets fit the GEMV ticket slots
+        CHECK(p1.tickets + p2.tickets <= kTicketSlots, f, op, T, d_in, d_out, k);
       }
   }
 }
@@ -154,6 +157,7 @@ int main() {
       check_layout(QS_OP_SPARSE_LINEAR, T, s[0], s[1], s[2]);
       if (s[1] % 64 == 0) check_layout(QS_OP_QUANT_SPARSE_LINEAR, T, s[0], s[1], s[2]);
       if (s[2] <= s[1]) check_layout(QS_OP_SPARSE_FFN, T, s[0], s[1], s[2]);
+      if (s[2] <= s[1]) check_layout(QS_OP_SPARSE_FFN_GATE_FIRST, T, s[0], s[1], s[2]);
     }
   std::printf("%ld checks, %d failed\n", g_checked, g_fails);
   return g_fails == 0 ? 0 : 1;
