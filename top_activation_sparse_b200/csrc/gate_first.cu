@@ -14,9 +14,9 @@
 // bytes row, and the kernel below streams exactly the rows of open gates.
 //
 // Mapping (B200: 148 SMs).  One warp computes one open row at a time: its
-// lanes read 16-byte vectors of the row (8 in flight per lane, not kept in
-// L1), multiply them with the same vectors of x (tiny, L1-resident, shared by
-// every warp) and reduce across the warp.  Open rows are dealt to warps by
+// lanes read 16-byte vectors of the row (8 in flight per lane for one token,
+// 4 for several; not kept in L1), multiply them with the same vectors of x
+// (tiny, L1-resident, shared by every warp) and reduce across the warp.  Open rows are dealt to warps by
 // rank: every CTA copies the open-gate bitmask and its prefix counts into
 // shared memory, and a warp finds the word of its rank by binary search.
 // The grid is 4 CTAs of 8 warps per SM, so about 4.7 K rows are in flight
