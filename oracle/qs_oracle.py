@@ -25,6 +25,12 @@ What it computes, and where each step comes from:
   by absolute value, then apply W_down).  Reading used:
   h = ReLU(x.W_gate^T + b_gate) (.) ReLU(x.W_up^T + b_up).
   -> :func:`sparse_ffn` with act="drelu".
+* Q-Sparse news article, the same Top-K section, the paragraphs on the
+  straight-through estimator (STE): top-K
+  has zero gradient almost everywhere, so the loss gradient with respect to
+  the sparsified tensor is copied unchanged to the tensor before it was
+  sparsified.  -> :func:`sparse_linear_backward_ste` (the backward of
+  :func:`sparse_linear`; no CUDA kernel implements it yet).
 * Q-Sparse news article, same section, the paragraph on quantized models: the
   input is quantized before top-K, with a small epsilon that keeps a
   denominator away from zero, and 1-bit weights use alpha = mean|W| (both
@@ -121,6 +127,32 @@ def sparse_linear(x, wt, k: int, keep: np.ndarray | None = None) -> np.ndarray:
     m = mask_from_keep(keep, T, d_in)
     xs = x.astype(np.float64) * m
     return xs @ wt
+
+
+def sparse_linear_backward_ste(x, wt, k: int, grad_y, keep: np.ndarray | None = None) -> dict:
+    """Gradients of Y = X_sparse . W^T for an upstream gradient dL/dY [T, d_out].
+
+    Q-Sparse news article, section "Top-K sparsification", STE paragraphs: the
+    gradient with respect to the sparsified tensor is used as the gradient
+    with respect to the tensor before sparsification.  With W^T input-major:
+
+        dL/dX_sparse = dL/dY . (W^T)^T          [T, d_in]
+        dL/dX       := dL/dX_sparse             (the estimator: no mask applied)
+        dL/dW^T      = X_sparse^T . dL/dY        [d_in, d_out]
+
+    A row i of dL/dW^T can be nonzero only if some token kept input i, so a
+    backward pass needs to write only the kept rows.  All fp64.
+    """
+    x = np.asarray(x)
+    wt = np.asarray(wt, dtype=np.float64)
+    g = np.asarray(grad_y, dtype=np.float64)
+    T, d_in = x.shape
+    if wt.shape[0] != d_in or g.shape != (T, wt.shape[1]):
+        raise ValueError("need x [T, d_in], W^T [d_in, d_out], dL/dY [T, d_out]")
+    if keep is None:
+        keep = topk_keep(x, k)
+    xs = x.astype(np.float64) * mask_from_keep(keep, T, d_in)
+    return {"grad_x": g @ wt.T, "grad_wt": xs.T @ g, "keep": keep}
 
 
 # --------------------------------------------------------------------------

@@ -155,6 +155,81 @@ def test_sparse_linear_unselected_rows_do_not_matter():
     assert not np.array_equal(oracle.sparse_linear(x, wt3, k), y0)
 
 
+# ---------------------------------------------------------------- STE backward
+
+
+def test_ste_backward_golden_hand():
+    g = load_golden("ste_backward_hand.json")
+    x = np.array(g["x"], dtype=np.float32)
+    wt = np.array(g["wt"], dtype=np.float32)
+    gy = np.array(g["grad_y"], dtype=np.float32)
+    for k, want in g["grad_wt"].items():
+        r = oracle.sparse_linear_backward_ste(x, wt, int(k), gy)
+        assert r["grad_x"].tolist() == g["grad_x"]
+        assert r["grad_wt"].tolist() == want
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_ste_backward_bruteforce(seed):
+    """Plain loops: dL/dX[t, i] = sum_j dL/dY[t, j] W^T[i, j] for every K (the
+    estimator copies the gradient through the mask); dL/dW^T[i, j] = sum over
+    the tokens that kept input i of x[t, i] dL/dY[t, j], zero for inputs no
+    token kept."""
+    g = np.random.default_rng(300 + seed)
+    T, d_in, d_out = int(g.integers(1, 4)), int(g.integers(1, 8)), int(g.integers(1, 6))
+    x = g.standard_normal((T, d_in)).astype(np.float32)
+    wt = g.standard_normal((d_in, d_out)).astype(np.float32)
+    gy = g.standard_normal((T, d_out)).astype(np.float32)
+    for k in range(d_in + 1):
+        r = oracle.sparse_linear_backward_ste(x, wt, k, gy)
+        kept = [set(bf_keep(x[t], k)) for t in range(T)]
+        for t in range(T):
+            for i in range(d_in):
+                ref = sum(float(gy[t, j]) * float(wt[i, j]) for j in range(d_out))
+                assert math.isclose(r["grad_x"][t, i], ref, rel_tol=1e-12, abs_tol=1e-12)
+        for i in range(d_in):
+            for j in range(d_out):
+                ref = sum(float(x[t, i]) * float(gy[t, j]) for t in range(T) if i in kept[t])
+                assert math.isclose(r["grad_wt"][i, j], ref, rel_tol=1e-12, abs_tol=1e-12)
+            if not any(i in kt for kt in kept):
+                assert np.all(r["grad_wt"][i] == 0.0)
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_ste_backward_finite_differences(seed):
+    """L = sum(dL/dY * Y) is linear in W^T, so a central difference along any
+    direction equals <dL/dW^T, direction> up to rounding; with K = d the mask
+    is all ones, the layer is dense, and the estimator's dL/dX is the true
+    gradient, checked the same way (Y by plain loops, not the oracle)."""
+    g = np.random.default_rng(400 + seed)
+    T, d_in, d_out = 3, 7, 5
+    x = g.standard_normal((T, d_in))
+    wt = g.standard_normal((d_in, d_out))
+    gy = g.standard_normal((T, d_out))
+
+    def loss(xx, ww, k):
+        total = 0.0
+        for t in range(T):
+            kept = set(bf_keep(xx[t], k))
+            xs = [xx[t, i] if i in kept else 0.0 for i in range(d_in)]
+            y = bf_matvec(xs, ww.tolist())
+            total += sum(gy[t, j] * y[j] for j in range(d_out))
+        return total
+
+    for k in (0, 2, d_in):
+        r = oracle.sparse_linear_backward_ste(x, wt, k, gy)
+        D = g.standard_normal((d_in, d_out))
+        fd = (loss(x, wt + D, k) - loss(x, wt - D, k)) / 2.0
+        assert math.isclose(fd, float(np.sum(r["grad_wt"] * D)), rel_tol=1e-9, abs_tol=1e-9)
+    r = oracle.sparse_linear_backward_ste(x, wt, d_in, gy)
+    E = g.standard_normal((T, d_in))
+    fd = (loss(x + E, wt, d_in) - loss(x - E, wt, d_in)) / 2.0
+    assert math.isclose(fd, float(np.sum(r["grad_x"] * E)), rel_tol=1e-9, abs_tol=1e-9)
+    # the estimator's dL/dX does not depend on K
+    for k in range(d_in + 1):
+        assert np.array_equal(oracle.sparse_linear_backward_ste(x, wt, k, gy)["grad_x"], r["grad_x"])
+
+
 # ---------------------------------------------------------------- FFN
 
 
