@@ -176,7 +176,7 @@ qs_status check_ws(int op, int T, int d_in, int d_out, int k, void* ws, size_t w
 bool valid_dtype(int dt) { return dt == QS_F32 || dt == QS_BF16; }
 
 // A launch plan must fit the buffers the layout reserved for it.
-bool plan_fits(const WsLayout& L, const GemvPlan& p, size_t parts_cap, int ticket_offset) {
+bool plan_fits(const GemvPlan& p, size_t parts_cap, int ticket_offset) {
   return p.parts_elems <= parts_cap && kTkGemv + ticket_offset + p.tickets <= kTkGemvEnd;
 }
 
@@ -322,7 +322,7 @@ qs_status qs_sparse_linear(const void* x, int dtype, int T, int d_in, int d_out,
     a.union_bits = reinterpret_cast<uint32_t*>(w.ticket(L, kUnionX));
     a.status = w.status();
     const GemvPlan gp = plan_gemv(Tc, d_out, (int)rows_bound(Tc, d_in, k), 1, eb);
-    if (!plan_fits(L, gp, L.parts1_elems, 0)) return QS_ERR_UNSUPPORTED;
+    if (!plan_fits(gp, L.parts1_elems, 0)) return QS_ERR_UNSUPPORTED;
     a.zero = w.at<float>(L.parts1);
     a.zero_n = gp.parts_elems;
     QS_TRY_CUDA(launch_topk(a, s));
@@ -337,7 +337,7 @@ qs_status qs_sparse_linear(const void* x, int dtype, int T, int d_in, int d_out,
     g.parts = w.at<float>(L.parts1);
     g.plan = gp;
     g.tickets = gemv_tickets(w, L, 0, g.plan);
-    if (!plan_fits(L, g.plan, L.parts1_elems, 0)) return QS_ERR_UNSUPPORTED;
+    if (!plan_fits(g.plan, L.parts1_elems, 0)) return QS_ERR_UNSUPPORTED;
     g.y = (unsigned char*)y + (size_t)t0 * d_out * eb;
     g.status = w.status();
     QS_TRY_CUDA(launch_gemv(g, s));
@@ -402,7 +402,7 @@ static qs_status ffn_impl(int op, const void* x, int dtype, int T, int d_model, 
     const GemvPlan p_ug =
         plan_gemv(Tc, d_ff, (int)rows_bound(Tc, d_model, d_model), gate_first ? 1 : 2, eb);
     const GemvPlan p_dn = plan_gemv(Tc, d_model, (int)rows_bound(Tc, d_ff, k_h), 1, eb);
-    if (!plan_fits(L, p_ug, L.parts1_elems, 0) || !plan_fits(L, p_dn, L.parts2_elems, p_ug.tickets))
+    if (!plan_fits(p_ug, L.parts1_elems, 0) || !plan_fits(p_dn, L.parts2_elems, p_ug.tickets))
       return QS_ERR_UNSUPPORTED;
     a.zero = w.at<float>(L.parts1);
     a.zero_n = p_ug.parts_elems;
@@ -553,7 +553,7 @@ qs_status qs_quant_sparse_linear(const void* x, int dtype, int T, int d_in, int 
     a.union_bits = reinterpret_cast<uint32_t*>(w.ticket(L, kUnionX));
     a.status = w.status();
     const GemvPlan qp = plan_qgemv(Tc, d_out, (int)rows_bound(Tc, d_in, k));
-    if (!plan_fits(L, qp, L.parts1_elems, 0)) return QS_ERR_UNSUPPORTED;
+    if (!plan_fits(qp, L.parts1_elems, 0)) return QS_ERR_UNSUPPORTED;
     a.zero = w.at<float>(L.parts1);
     a.zero_n = qp.parts_elems;
     QS_TRY_CUDA(launch_topk(a, s));
