@@ -65,6 +65,13 @@ def test_parse_args_defaults_and_guards():
     assert bench.parse_args(["--workload", "prefill_bf16_2048"]).batch == 2048
     with pytest.raises(SystemExit):
         bench.parse_args(["--warmup", "2"])
+    # the gate-first layer exists only for the dReLU FFN, and says so in its config
+    with pytest.raises(SystemExit):
+        bench.parse_args(["--gate-first"])
+    g = bench.parse_args(["--workload", "ffn_drelu_mistral7b", "--gate-first", "--batch", "4"])
+    assert g.gate_first and g.batch == 4
+    assert "gate first" in bench.workload_desc(g, g.batch)
+    assert "gate first" not in bench.workload_desc(bench.parse_args(["--workload", "ffn_drelu_mistral7b"]), 1)
 
 
 def test_clock_summary():
