@@ -318,6 +318,25 @@ def test_ffn_drelu_invariants():
     assert np.all(r["h"][(r["u"] - 0.8 <= 0) | (r["g"] - 0.8 <= 0)] == 0)
 
 
+def test_ffn_drelu_closed_gates_ignore_up():
+    """The fact the gate-first dReLU layer rests on: where g + b_gate <= 0, h
+    is 0 whatever u is, so replacing u there by any finite values (here huge
+    ones) leaves h, and so y, unchanged; changing u at an open gate does not."""
+    g = np.random.default_rng(8)
+    T, dff = 3, 400
+    u = g.standard_normal((T, dff))
+    gt = g.standard_normal((T, dff))
+    b = np.full(dff, -0.8)
+    h = oracle.ffn_hidden(u, gt, "drelu", b_up=b, b_gate=b)
+    closed = gt + b <= 0
+    u2 = np.where(closed, g.standard_normal((T, dff)) * 1e30, u)
+    assert np.array_equal(oracle.ffn_hidden(u2, gt, "drelu", b_up=b, b_gate=b), h)
+    t, j = map(int, np.argwhere(~closed & (u + b > 0))[0])
+    u3 = u.copy()
+    u3[t, j] += 1.0
+    assert not np.array_equal(oracle.ffn_hidden(u3, gt, "drelu", b_up=b, b_gate=b), h)
+
+
 def test_ffn_k_full_is_dense_glu():
     g = np.random.default_rng(8)
     x = g.standard_normal((1, 5)).astype(np.float32)
