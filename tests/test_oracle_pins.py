@@ -58,6 +58,35 @@ def test_topk_golden_hand():
     assert xs[0].tolist() == r0["xs_k4"]
 
 
+def test_kept_values_golden_hand():
+    """The compacted value list is x at the kept indices, in index order and in
+    the input's own dtype (hand values in the golden file; -0.0 keeps its sign)."""
+    g = load_golden("topk_hand.json")
+    r0, r2 = g["rows"][0], g["rows"][2]
+    x0 = np.array([r0["x"]], dtype=np.float32)
+    v0 = oracle.kept_values(x0, oracle.topk_keep(x0, 4))
+    assert v0.dtype == np.float32 and v0[0].tolist() == r0["vals_k4"]
+    x2 = np.array([r2["x"]], dtype=np.float32)
+    v2 = oracle.kept_values(x2, oracle.topk_keep(x2, 2))
+    assert np.array_equal(np.signbit(v2[0]), np.signbit(np.array(r2["vals_k2"], np.float32)))
+
+
+@pytest.mark.parametrize("dtype", [np.float32, np.float64, np.int64, np.int8])
+def test_kept_values_read_by_loops(dtype):
+    """kept_values[t, j] is x[t, keep[t, j]], read here element by element
+    (same row, same bits, same dtype) for random keeps of random rows."""
+    g = workloads.rng(77)
+    x = (g.standard_normal((5, 23)) * 40).astype(dtype)
+    for k in (0, 1, 9, 23):
+        keep = np.sort(np.stack([g.permutation(23)[:k] for _ in range(5)]), axis=1).astype(np.int64)
+        v = oracle.kept_values(x, keep)
+        assert v.dtype == x.dtype and v.shape == (5, k)
+        for t in range(5):
+            for j in range(k):
+                assert v[t, j].tobytes() == x[t, keep[t, j]].tobytes()
+
+
+
 @pytest.mark.parametrize("seed", range(40))
 def test_topk_bruteforce_rank_tiny(seed):
     g = np.random.default_rng(seed)
@@ -425,6 +454,78 @@ def test_quant_sparse_linear_golden_hand():
     assert r["keep"][0].tolist() == c["keep"]
     assert r["acc"][0].tolist() == c["acc"]
     assert np.allclose(r["y"][0], c["y_approx"], rtol=2e-7)
+
+
+def _rne_f32(q):
+    """An exact rational rounded to the nearest float32, ties to even (normal
+    range), by integer arithmetic: independent of numpy's float32 operations."""
+    from fractions import Fraction
+    if q == 0:
+        return 0.0
+    a = abs(q)
+    e = a.numerator.bit_length() - a.denominator.bit_length()
+    while Fraction(2) ** e > a:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= a:
+        e += 1
+    ulp = Fraction(2) ** (e - 23)
+    m = a / ulp
+    fl = m.numerator // m.denominator
+    rem = m - fl
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and fl % 2 == 1):
+        fl += 1
+    return math.copysign(float(fl * ulp), float(q))
+
+
+def _rint_even(q):
+    from fractions import Fraction
+    fl = q.numerator // q.denominator
+    rem = q - fl
+    return fl + (1 if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and fl % 2 == 1) else 0)
+
+
+def _f32_from_hex(h):
+    return np.array([int(h, 16)], dtype=np.uint32).view(np.float32)[0]
+
+
+def _hex(v):
+    return hex(int(np.array([v], dtype=np.float32).view(np.uint32)[0]))
+
+
+def test_quant_rescale_order_golden_bits():
+    """y = float32(acc) * ((alpha * gamma) / 127), each step rounded to float32
+    in that order.  The golden case is derived again here with exact rationals
+    rounded by hand (not numpy), the oracle must give the same bits, and the
+    other grouping alpha * (gamma / 127) must differ in the last bit."""
+    from fractions import Fraction as Fr
+    g = load_golden("rescale_order_hand.json")
+    x = [np.float32(v) for v in g["x"]]
+    alpha = _f32_from_hex(g["alpha_bits"])
+    eps = _rne_f32(Fr(np.float32(g["eps"]).item()))
+    # the hand derivation
+    gamma = _rne_f32(Fr(max(abs(float(v)) for v in x)) + Fr(eps))
+    s = _rne_f32(Fr(127) / Fr(gamma))
+    q = [max(-127, min(127, _rint_even(Fr(_rne_f32(Fr(float(v)) * Fr(s)))))) for v in x]
+    r = _rne_f32(Fr(_rne_f32(Fr(float(alpha)) * Fr(gamma))) / 127)
+    r_other = _rne_f32(Fr(float(alpha)) * Fr(_rne_f32(Fr(gamma) / 127)))
+    keep = sorted(sorted(range(len(q)), key=lambda i: (-abs(q[i]), i))[:g["k"]])
+    acc = [sum(q[i] * row[i] for i in keep) for row in g["t"]]
+    y = [_rne_f32(Fr(a) * Fr(r)) for a in acc]
+    y_other = [_rne_f32(Fr(a) * Fr(r_other)) for a in acc]
+    assert _hex(gamma) == g["gamma_bits"] and _hex(s) == g["s_bits"]
+    assert q == g["q"] and keep == g["keep"] and acc == g["acc"]
+    assert _hex(r) == g["r_bits"] and _hex(r_other) == g["other_order_r_bits"]
+    assert [_hex(v) for v in y] == g["y_bits"]
+    assert [_hex(v) for v in y_other] == g["other_order_y_bits"]
+    assert all(a != b for a, b in zip(g["y_bits"], g["other_order_y_bits"]))
+    # the oracle, bit for bit
+    res = oracle.quant_sparse_linear(np.array([x], np.float32), np.array(g["t"]), alpha, g["k"],
+                                     eps=g["eps"])
+    assert _hex(res["gamma"][0]) == g["gamma_bits"]
+    assert res["q"][0].tolist() == g["q"] and res["keep"][0].tolist() == g["keep"]
+    assert res["acc"][0].tolist() == g["acc"]
+    assert _hex(res["r"][0]) == g["r_bits"]
+    assert [_hex(v) for v in res["y"][0]] == g["y_bits"]
 
 
 @pytest.mark.parametrize("seed", range(8))
