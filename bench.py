@@ -277,6 +277,12 @@ def workload_desc(args, T: int) -> str:
     return f"{args.workload}: sparse linear, T={T}, {w.d_in}->{w.d_out}, K={w.k}, {w.dtype}"
 
 
+def run_config(desc: str, T: int, world: int, layers: int, l2: str, parallelism: str) -> dict:
+    """The `config` object; both arms emit the same keys."""
+    return {"workload": desc, "batch_per_gpu": T, "global_batch": T * world,
+            "layers_rotated": layers, "l2": l2, "parallelism": parallelism}
+
+
 def setup_ffn(args, qs, torch, device, stream, rank):
     """One sparse FFN layer per step, rotating over independent layers."""
     w = workloads.WORKLOADS[args.workload]
@@ -394,7 +400,9 @@ def setup_linear(args, qs, torch, device, stream, rank):
         return (x.data_ptr(), dt, T, w.d_in, w.d_out, k, wts[l].data_ptr(), y.data_ptr(), ev,
                 ws.data_ptr(), ws.numel(), sp)
 
-    assert fn(*c_args(0, None)) == 0
+    for l in range(n_layers):             # every layer once: validation, steady state
+        assert fn(*c_args(l, None)) == 0
+    assert qs.qs_device_status(ws) == qs.QS_OK
     prefill = (w.dtype == "bf16" and T >= qs.QS_PREFILL_MIN_T)
     if prefill:
         # tensor-core bound: algorithmic FLOPs (kept inputs only) per launch
@@ -465,7 +473,9 @@ def setup_quant(args, qs, torch, device, stream, rank):
                 ctypes.c_float(alphas[l]), ctypes.c_float(1e-5), y.data_ptr(), None, None, None, ev,
                 ws.data_ptr(), ws.numel(), sp)
 
-    assert fn(*c_args(0, None)) == 0
+    for l in range(n_layers):             # every layer once: validation, steady state
+        assert fn(*c_args(l, None)) == 0
+    assert qs.qs_device_status(ws) == qs.QS_OK
     rows, _ = qs.qs_workspace_stats(ws, qs.QS_OP_QUANT_SPARSE_LINEAR, T, w.d_in, w.d_out, w.k)
     work = rows * n_words * 4 + rows * (4 + T) + T * w.d_out * 4
 
@@ -528,14 +538,9 @@ def run_ours(args, rank, world, local):
         if st != 0:
             raise RuntimeError(f"{fn.__name__}: {qs.qs_status_string(st)}")
 
-    # phase events on a sample of the timed steps
-    n_phase = min(args.steps, 256)
-    phase_steps = set(np.linspace(0, args.steps - 1, n_phase).astype(int).tolist())
-    ev = {i: _mk_events(torch, stream, c["n_events"]) for i in phase_steps}
-    torch.cuda.synchronize()
     plain = [c["args"](l, None) for l in range(n_layers)]
-    timed = {i: c["args"](i % n_layers, ev[i][1]) for i in phase_steps}
-
+    # every rotated layer was called once during setup (validation, row counts),
+    # so the warm-up steps start from a steady state
     for i in range(args.warmup):
         run(plain[i % n_layers])
     torch.cuda.synchronize()
@@ -546,8 +551,8 @@ def run_ours(args, rank, world, local):
     torch.cuda.synchronize()
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
-    for i in range(args.steps):
-        run(timed[i] if i in timed else plain[i % n_layers])
+    for i in range(args.steps):           # the timed region: plain calls only
+        run(plain[i % n_layers])
     t_end.record(stream)
     torch.cuda.synchronize()
     if dist is not None:
@@ -559,9 +564,17 @@ def run_ours(args, rank, world, local):
     tokens = sum_over_ranks(float(T * args.steps), dist, device)
     value = tokens / (ms_max / 1e3)
 
+    # per-phase device time: a separate sampled pass after the timed region,
+    # with CUDA events between the kernels of each step (they cost the launch
+    # overlap, so they never run inside the timed region)
     names = c["phases"]
-    ph = np.array([[ev[i][0][p].elapsed_time(ev[i][0][p + 1]) for p in range(len(names))]
-                   for i in sorted(phase_steps)])
+    n_phase = 256
+    evs = [_mk_events(torch, stream, c["n_events"]) for _ in range(n_phase)]
+    torch.cuda.synchronize()
+    for i in range(n_phase):
+        run(c["args"](i % n_layers, evs[i][1]))
+    torch.cuda.synchronize()
+    ph = np.array([[e[0][p].elapsed_time(e[0][p + 1]) for p in range(len(names))] for e in evs])
     ph_us = {n: round(float(v), 3) for n, v in zip(names, ph.mean(axis=0) * 1e3)}
     dom_us = ph_us[c["dominant"]]
     peaks = load_peaks()
@@ -635,14 +648,8 @@ def run_ours(args, rank, world, local):
         "vs_baseline": None,
         "dtype": c["dtype"],
         "data": "synthetic: x ~ N(0,1), W ~ N(0,1/fan_in) (seeded; random-init weights)",
-        "config": {
-            "workload": c["desc"],
-            "batch_per_gpu": T,
-            "global_batch": T * world,
-            "layers_rotated": n_layers,
-            "l2": c["l2"],
-            "parallelism": f"replicas x{world} (no data-path collective)",
-        },
+        "config": run_config(c["desc"], T, world, n_layers, c["l2"],
+                             f"replicas x{world} (no data-path collective)"),
         "hbm": {
             "step_alg_gbs": round(c["layer_work"] / step_s / 1e9, 1) if c["bound"] == "hbm" else None,
             "frac_of_peak": (round(c["layer_work"] / step_s / 1e9 / peaks["hbm_gbs"], 4)
@@ -758,8 +765,9 @@ def run_reference(args, rank, world, local):
         "vs_baseline": None,
         "dtype": "f64",
         "data": "synthetic: x ~ N(0,1), W ~ N(0,1/fan_in) (seeded)",
-        "config": {"workload": workload_desc(args, T), "batch_per_gpu": T, "global_batch": T,
-                   "parallelism": "host cores (the fp64 oracle, rank 0)"},
+        "config": run_config(workload_desc(args, T), T, 1, 1,
+                             "not applicable: host memory (one layer's weights)",
+                             "host cores (the fp64 oracle, rank 0)"),
         "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": _threads_in_use(),
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0,

@@ -279,6 +279,39 @@ qs_status qs_device_status(void* ws, void* stream);
 qs_status qs_workspace_stats(const void* ws, int op, int T, int d_in, int d_out, int k,
                              int32_t* rows, void* stream);
 
+/* Synchronise `stream` and copy to HOST memory the kept-row list that the
+ * last call of `op` made with this workspace and these sizes left in it (for
+ * inspection and tests; the two FFN ops report their last chunk of at most
+ * QS_PREFILL_MIN_T tokens).
+ *   which  0: the projection input's list: the inputs with a kept nonzero
+ *             value (rows of wt, wt_up / wt_gate or wt_packed that were read),
+ *             ascending, the union over the tokens;
+ *          1: (QS_OP_SPARSE_FFN, QS_OP_SPARSE_FFN_GATE_FIRST) the same for h
+ *             (rows of wt_down read).
+ *   rows   host int32 [cap] out: the first min(count, cap) listed rows.
+ *   vals   host out or NULL: for calls with one token (T == 1) the listed
+ *          rows' values, in list order: float32 (the kept x, exactly as given;
+ *          the kept h) or, for QS_OP_QUANT_SPARSE_LINEAR, the int8 codes q.
+ *          Must be NULL when T > 1 (several tokens keep dense masked values).
+ *   count  host out: the number of listed rows.
+ * Errors: INVALID_ARG (bad op/which/sizes, NULL rows/count, vals with T > 1),
+ * CUDA. */
+qs_status qs_workspace_list(const void* ws, int op, int T, int d_in, int d_out, int k, int which,
+                            int32_t* rows, int cap, void* vals, int32_t* count, void* stream);
+
+/* Failure-detection test hook (host side; process-wide; not thread-safe).
+ * QS_FAULT_GATHER_NO_COPIES makes the gather-GEMV launches that follow (the
+ * FMA kernel that serves one or two tokens) issue no weight copies at all:
+ * their producer warp stays idle, so no copy is ever in flight, and the
+ * consumers' bounded waits run out after `wait_polls` polls (0: the normal
+ * limit).  The kernel then records QS_ERR_TIMEOUT in the workspace's status
+ * word, skips its remaining waits and still finishes its split sums and
+ * tickets, so the workspace stays usable; its results are meaningless.
+ * QS_FAULT_NONE restores normal operation.  Nothing here faults or hangs the
+ * GPU.  Errors: INVALID_ARG (unknown mode). */
+typedef enum qs_fault { QS_FAULT_NONE = 0, QS_FAULT_GATHER_NO_COPIES = 1 } qs_fault;
+qs_status qs_debug_inject(int mode, unsigned wait_polls);
+
 /* Human-readable name of a status code (static string). */
 const char* qs_status_string(int status);
 
@@ -299,18 +332,28 @@ const char* qs_status_string(int status);
  *   - The first call on a device looks the array's address up for that device
  *     (cudaGetSymbolAddress), so make that first call before any stream
  *     capture.
- *   - Each call first clears the array's status word and counters on `stream`
- *     (cudaMemsetAsync); the rest of the array is rewritten before it is read.
+ *   - Every argument check of qs_sparse_linear runs first; an invalid call
+ *     returns its code with nothing enqueued.  A valid call then clears the
+ *     array's counters on `stream` (cudaMemsetAsync); the rest of the array
+ *     is rewritten before it is read.
  *   - All calls share the array: calls whose kernels can overlap on the GPU
  *     (different streams without ordering) race and give wrong results.
+ *   - Device-side failures (a bounded wait that gave up, an internal check)
+ *     go to the array's status word, which keeps the first one until
+ *     qs_sparse_linear_noalloc_status reads it.
  *   - Errors: as qs_sparse_linear, plus QS_ERR_UNSUPPORTED when these sizes
  *     need more than QS_NOALLOC_SCRATCH_BYTES of scratch (that is,
  *     qs_workspace_size(QS_OP_SPARSE_LINEAR, T, d_in, d_out, k) is larger),
- *     returned before anything is enqueued.  qs_device_status is not
- *     available for this entry point's scratch.
+ *     returned before anything is enqueued.
  */
 qs_status qs_sparse_linear_noalloc(const void* x, int dtype, int T, int d_in, int d_out, int k,
                                    const void* wt, void* y, void* stream);
+
+/* Synchronise `stream`, then read and clear the status word of the current
+ * device's fixed scratch array (the qs_device_status of
+ * qs_sparse_linear_noalloc): QS_OK, QS_ERR_TIMEOUT or QS_ERR_DEVICE_CHECK for
+ * the calls since the last read (or QS_ERR_CUDA).  Allocates nothing. */
+qs_status qs_sparse_linear_noalloc_status(void* stream);
 
 #ifdef __cplusplus
 }

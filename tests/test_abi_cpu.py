@@ -134,3 +134,38 @@ def test_noalloc_entry_point_checks_sizes_on_the_host(L):
     assert L.qs_sparse_linear_noalloc(_p(FAKE), 0, *big, _p(FAKE), _p(FAKE), None) == qs.QS_ERR_UNSUPPORTED
     assert L.qs_sparse_linear_noalloc(None, 0, 1, 8, 8, 4, _p(FAKE), _p(FAKE), None) == qs.QS_ERR_INVALID_ARG
     assert L.qs_sparse_linear_noalloc(_p(FAKE), 0, 1, 8, 8, 9, _p(FAKE), _p(FAKE), None) == qs.QS_ERR_INVALID_ARG
+
+
+def test_noalloc_entry_point_checks_arguments_before_enqueuing(L):
+    """Every argument check of qs_sparse_linear runs before the no-allocation
+    entry point touches its scratch array: these return their codes without a
+    device, i.e. nothing was enqueued."""
+    s = None
+    assert L.qs_sparse_linear_noalloc(_p(FAKE), 7, 1, 64, 64, 8, _p(FAKE), _p(FAKE), s) == \
+        qs.QS_ERR_INVALID_ARG                                          # dtype
+    assert L.qs_sparse_linear_noalloc(_p(FAKE + 4), 0, 1, 64, 64, 8, _p(FAKE), _p(FAKE), s) == \
+        qs.QS_ERR_ALIGNMENT                                            # misaligned x
+    assert L.qs_sparse_linear_noalloc(_p(FAKE), 1, 1, 64, 60, 8, _p(FAKE), _p(FAKE), s) == \
+        qs.QS_ERR_ALIGNMENT                                            # bf16 d_out % 8
+    assert L.qs_sparse_linear_noalloc(_p(FAKE), 0, 1, 64, 64, 65, _p(FAKE), _p(FAKE), s) == \
+        qs.QS_ERR_INVALID_ARG                                          # k > d_in
+
+
+def test_workspace_list_and_fault_hook_check_arguments_on_the_host(L):
+    rows = (ctypes.c_int32 * 8)()
+    vals = (ctypes.c_float * 8)()
+    cnt = ctypes.c_int32(0)
+    ws = _p(FAKE)
+    lin = qs.QS_OP_SPARSE_LINEAR
+    assert L.qs_workspace_list(None, lin, 1, 64, 64, 8, 0, rows, 8, None, ctypes.byref(cnt), None) == \
+        qs.QS_ERR_INVALID_ARG                                          # no workspace
+    assert L.qs_workspace_list(ws, lin, 1, 64, 64, 8, 1, rows, 8, None, ctypes.byref(cnt), None) == \
+        qs.QS_ERR_INVALID_ARG                                          # no h list here
+    assert L.qs_workspace_list(ws, lin, 2, 64, 64, 8, 0, rows, 8, vals, ctypes.byref(cnt), None) == \
+        qs.QS_ERR_INVALID_ARG                                          # values: one token only
+    assert L.qs_workspace_list(ws, qs.QS_OP_TOPK_MASK, 1, 64, 0, 8, 0, rows, 8, None,
+                               ctypes.byref(cnt), None) == qs.QS_ERR_INVALID_ARG
+    assert L.qs_workspace_list(ws, lin, 1, 64, 64, 65, 0, rows, 8, None, ctypes.byref(cnt), None) == \
+        qs.QS_ERR_INVALID_ARG                                          # k > d_in
+    assert L.qs_debug_inject(9, 0) == qs.QS_ERR_INVALID_ARG
+    assert L.qs_debug_inject(qs.QS_FAULT_NONE, 0) == qs.QS_OK

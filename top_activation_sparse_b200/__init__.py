@@ -42,6 +42,9 @@ QS_OP_QUANT_SPARSE_LINEAR = 3
 QS_OP_TERNARY_PACK = 4
 QS_OP_SPARSE_FFN_GATE_FIRST = 5
 
+QS_FAULT_NONE = 0
+QS_FAULT_GATHER_NO_COPIES = 1
+
 QS_MAX_ROW = 49152
 QS_NOALLOC_SCRATCH_BYTES = 4 << 20
 QS_PREFILL_MIN_T = 64
@@ -78,6 +81,9 @@ _SIGNATURES = {
     "qs_workspace_stats": (_i, [_vp, _i, _i, _i, _i, _i, _vp, _vp]),
     "qs_status_string": (ctypes.c_char_p, [_i]),
     "qs_sparse_linear_noalloc": (_i, [_vp, _i, _i, _i, _i, _i, _vp, _vp, _vp]),
+    "qs_sparse_linear_noalloc_status": (_i, [_vp]),
+    "qs_workspace_list": (_i, [_vp, _i, _i, _i, _i, _i, _i, _vp, _i, _vp, _vp, _vp]),
+    "qs_debug_inject": (_i, [_i, ctypes.c_uint]),
 }
 
 _lib = None
@@ -209,6 +215,37 @@ def qs_workspace_stats(ws: torch.Tensor, op: int, T: int, d_in: int, d_out: int,
     if op == QS_OP_SPARSE_FFN_GATE_FIRST:
         return int(rows[0]), int(rows[1]), int(rows[2])
     return int(rows[0]), int(rows[1])
+
+
+def qs_workspace_list(ws: torch.Tensor, op: int, T: int, d_in: int, d_out: int, k: int,
+                      which: int = 0, values: bool = False, stream=None):
+    """The kept-row list the last call left in `ws` (see include/qs.h):
+    (rows int32 [n], values or None).  values (one-token calls only): float32
+    of the kept inputs, or the int8 codes for QS_OP_QUANT_SPARSE_LINEAR."""
+    import numpy as np
+    cap = d_in if which == 0 else d_out
+    rows = np.zeros(max(cap, 1), dtype=np.int32)
+    vals = None
+    if values:
+        vals = np.zeros(max(cap, 1), dtype=np.int8 if op == QS_OP_QUANT_SPARSE_LINEAR else np.float32)
+    count = ctypes.c_int32(0)
+    _check("qs_workspace_list", lib().qs_workspace_list(
+        ws.data_ptr(), op, T, d_in, d_out, k, which, rows.ctypes.data, cap,
+        None if vals is None else vals.ctypes.data, ctypes.byref(count), _stream_ptr(stream)))
+    n = int(count.value)
+    if not 0 <= n <= cap:
+        raise RuntimeError(f"qs_workspace_list: inconsistent row count {n}")
+    return rows[:n].copy(), (None if vals is None else vals[:n].copy())
+
+
+def qs_debug_inject(mode: int, wait_polls: int = 0) -> None:
+    """Failure-detection test hook (see include/qs.h)."""
+    _check("qs_debug_inject", lib().qs_debug_inject(int(mode), int(wait_polls)))
+
+
+def qs_sparse_linear_noalloc_status(stream=None) -> int:
+    """Read and clear the status word of the no-allocation entry point's scratch."""
+    return int(lib().qs_sparse_linear_noalloc_status(_stream_ptr(stream)))
 
 
 # ---- operations -------------------------------------------------------------

@@ -7,6 +7,9 @@
 #include "qs_internal.cuh"
 
 namespace qs {
+
+FaultState g_fault;
+
 namespace {
 
 // Token rows are processed in chunks of at most this many (decode kernels
@@ -142,6 +145,21 @@ bool ws_layout(int op, int T, int d_in, int d_out, int k, WsLayout* L) {
   return true;
 }
 
+qs_status check_sparse_linear(const void* x, int dtype, int T, int d_in, int d_out, int k,
+                              const void* wt, const void* y, const void* ws, size_t ws_bytes,
+                              WsLayout* L) {
+  if ((dtype != QS_F32 && dtype != QS_BF16) || x == nullptr || wt == nullptr || y == nullptr ||
+      T < 1 || d_in < 1 || d_out < 1 || k < 0 || k > d_in)
+    return QS_ERR_INVALID_ARG;
+  if (d_in > QS_MAX_ROW || d_out > QS_MAX_ROW) return QS_ERR_UNSUPPORTED;
+  const int V = 16 / elem_bytes(dtype);
+  if ((d_out % V) != 0 || !aligned16(x) || !aligned16(wt) || !aligned16(y)) return QS_ERR_ALIGNMENT;
+  if (!ws_layout(QS_OP_SPARSE_LINEAR, T, d_in, d_out, k, L)) return QS_ERR_INVALID_ARG;
+  if (ws == nullptr || ws_bytes < L->total) return QS_ERR_WORKSPACE;
+  if (!aligned16(ws)) return QS_ERR_ALIGNMENT;
+  return QS_OK;
+}
+
 }  // namespace qs
 
 using namespace qs;
@@ -244,6 +262,45 @@ qs_status qs_workspace_stats(const void* ws, int op, int T, int d_in, int d_out,
   return QS_OK;
 }
 
+qs_status qs_workspace_list(const void* ws, int op, int T, int d_in, int d_out, int k, int which,
+                            int32_t* rows, int cap, void* vals, int32_t* count, void* stream) {
+  if (ws == nullptr || rows == nullptr || count == nullptr || cap < 0) return QS_ERR_INVALID_ARG;
+  const bool ffn = op == QS_OP_SPARSE_FFN || op == QS_OP_SPARSE_FFN_GATE_FIRST;
+  if (!(op == QS_OP_SPARSE_LINEAR || op == QS_OP_QUANT_SPARSE_LINEAR || ffn)) return QS_ERR_INVALID_ARG;
+  if (which != 0 && !(which == 1 && ffn)) return QS_ERR_INVALID_ARG;
+  if (vals != nullptr && T != 1) return QS_ERR_INVALID_ARG;
+  WsLayout L;
+  if (!ws_layout(op, T, d_in, d_out, k, &L)) return QS_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  const unsigned char* base = (const unsigned char*)ws;
+  int32_t c[4] = {0, 0, 0, 0};
+  QS_TRY_CUDA(cudaMemcpyAsync(c, base + L.cnt, sizeof(c), cudaMemcpyDeviceToHost, s));
+  QS_TRY_CUDA(cudaStreamSynchronize(s));
+  const int n = c[which];
+  const int d_rows = which == 0 ? d_in : d_out;
+  *count = n;
+  if (n < 0 || n > d_rows) return QS_OK;           // reported as is; nothing to copy
+  const int m = n < cap ? n : cap;
+  if (m > 0) {
+    QS_TRY_CUDA(cudaMemcpyAsync(rows, base + (which == 0 ? L.list_x : L.list_h),
+                                (size_t)m * sizeof(int32_t), cudaMemcpyDeviceToHost, s));
+    if (vals != nullptr) {
+      const size_t vb = op == QS_OP_QUANT_SPARSE_LINEAR ? 1 : sizeof(float);
+      QS_TRY_CUDA(cudaMemcpyAsync(vals, base + (which == 0 ? L.lval_x : L.lval_h), (size_t)m * vb,
+                                  cudaMemcpyDeviceToHost, s));
+    }
+    QS_TRY_CUDA(cudaStreamSynchronize(s));
+  }
+  return QS_OK;
+}
+
+qs_status qs_debug_inject(int mode, unsigned wait_polls) {
+  if (mode != QS_FAULT_NONE && mode != QS_FAULT_GATHER_NO_COPIES) return QS_ERR_INVALID_ARG;
+  g_fault.mode = mode;
+  g_fault.wait_polls = mode == QS_FAULT_NONE ? 0u : wait_polls;
+  return QS_OK;
+}
+
 qs_status qs_topk_mask(const void* x, int dtype, int T, int d, int k, int32_t* idx, void* val,
                        uint8_t* mask, void* xs, void* ws, size_t ws_bytes, void* stream) {
   if (!valid_dtype(dtype) || x == nullptr || T < 1 || d < 1 || k < 0 || k > d)
@@ -269,14 +326,8 @@ qs_status qs_topk_mask(const void* x, int dtype, int T, int d, int k, int32_t* i
 qs_status qs_sparse_linear(const void* x, int dtype, int T, int d_in, int d_out, int k,
                            const void* wt, void* y, void* const* phase_events, void* ws,
                            size_t ws_bytes, void* stream) {
-  if (!valid_dtype(dtype) || x == nullptr || wt == nullptr || y == nullptr || T < 1 || d_in < 1 ||
-      d_out < 1 || k < 0 || k > d_in)
-    return QS_ERR_INVALID_ARG;
-  if (d_in > QS_MAX_ROW || d_out > QS_MAX_ROW) return QS_ERR_UNSUPPORTED;
-  const int V = 16 / elem_bytes(dtype);
-  if ((d_out % V) != 0 || !aligned16(x) || !aligned16(wt) || !aligned16(y)) return QS_ERR_ALIGNMENT;
   WsLayout L;
-  qs_status st = check_ws(QS_OP_SPARSE_LINEAR, T, d_in, d_out, k, ws, ws_bytes, &L);
+  const qs_status st = qs::check_sparse_linear(x, dtype, T, d_in, d_out, k, wt, y, ws, ws_bytes, &L);
   if (st != QS_OK) return st;
   WsView w{(unsigned char*)ws};
   cudaStream_t s = (cudaStream_t)stream;

@@ -197,12 +197,14 @@ __global__ void __launch_bounds__(kMaxConsumers + 32, (TT <= 4) ? 2 : 1) gemv_ke
     __syncthreads();
     const int nstage = (np + P.rps - 1) / P.rps;
     if (producer) {
-      // the producer warp's lanes issue a stage's copies side by side
-      for (int st = 0; st < nstage; ++st) {
+      // the producer warp's lanes issue a stage's copies side by side (none at
+      // all under the failure-detection test's no-copies injection)
+      for (int st = 0; st < nstage && !a.no_copies; ++st) {
         const int g = gst + st;
         const int slot = g % P.nst;
         int ok = 1;
-        if (lane == 0 && g >= P.nst && !mbar_wait(&s_empty[slot], (uint32_t)((g / P.nst) - 1) & 1u)) {
+        if (lane == 0 && g >= P.nst &&
+            !mbar_wait(&s_empty[slot], (uint32_t)((g / P.nst) - 1) & 1u, a.wait_limit)) {
           dev_fail(a.status, DEV_TIMEOUT, 10, (uint32_t)g);
           atomicExch(&s_err, 1);
           ok = 0;
@@ -220,8 +222,10 @@ __global__ void __launch_bounds__(kMaxConsumers + 32, (TT <= 4) ? 2 : 1) gemv_ke
       for (int st = 0; st < nstage; ++st) {
         const int g = gst + st;
         const int slot = g % P.nst;
-        bool ready = mbar_wait_backoff(&s_full[slot], (uint32_t)(g / P.nst) & 1u);
-        if (!ready) {
+        // once a wait of this CTA has given up, the later stages are not waited for
+        const bool ready = !*(volatile int*)&s_err &&
+                           mbar_wait_backoff(&s_full[slot], (uint32_t)(g / P.nst) & 1u, a.wait_limit);
+        if (!ready && !*(volatile int*)&s_err) {
           if (lane == 0) dev_fail(a.status, DEV_TIMEOUT, 11, (uint32_t)g);
           atomicExch(&s_err, 1);
         }
@@ -248,11 +252,12 @@ __global__ void __launch_bounds__(kMaxConsumers + 32, (TT <= 4) ? 2 : 1) gemv_ke
     gst += nstage;
     __syncthreads();                             // piece consumed before restaging
   }
-  if (s_err && tid == 0) {
+  if (s_err && tid == 0 && !a.no_copies) {
     // a wait gave up: let the copies already issued land before the CTA exits
+    // (with no copies issued at all there is nothing to wait for)
     for (int i = 0; i < P.nst && i < gst; ++i) {
       const int g_last = gst - 1 - i;            // the newest stage of each slot
-      mbar_wait(&s_full[g_last % P.nst], (uint32_t)(g_last / P.nst) & 1u);
+      mbar_wait(&s_full[g_last % P.nst], (uint32_t)(g_last / P.nst) & 1u, a.wait_limit);
     }
   }
 
@@ -615,7 +620,12 @@ cudaError_t launch2(const GemvArgs& a, cudaStream_t s) {
 }
 
 template <typename WT>
-cudaError_t launch1(const GemvArgs& a, cudaStream_t s) {
+cudaError_t launch1(const GemvArgs& a_in, cudaStream_t s) {
+  GemvArgs a = a_in;
+  if (g_fault.mode == QS_FAULT_GATHER_NO_COPIES) {   // failure-detection tests only
+    a.no_copies = 1;
+    if (g_fault.wait_polls != 0) a.wait_limit = g_fault.wait_polls;
+  }
   switch (a.plan.TT) {
     case 1: return launch2<WT, 1>(a, s);
     case 2: return launch2<WT, 2>(a, s);

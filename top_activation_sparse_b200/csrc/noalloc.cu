@@ -10,10 +10,13 @@
 //
 // The array is QS_NOALLOC_SCRATCH_BYTES on every GPU that loads the library
 // and stays there until the process exits.  All calls share it, and it keeps
-// whatever the last call left in it: the status word and the counters that
-// must start at zero are cleared at the start of every call (a memset on the
-// caller's stream), the rest is overwritten before it is read.  Two calls whose
-// kernels overlap on the GPU (different streams, no ordering) race on it.
+// whatever the last call left in it: the counters that must start at zero are
+// cleared at the start of every call (a memset on the caller's stream, after
+// every argument check has passed), the rest is overwritten before it is read.
+// The status word is not cleared by a call: like a workspace's, it keeps the
+// first device-side failure until qs_sparse_linear_noalloc_status reads it.
+// Two calls whose kernels overlap on the GPU (different streams, no ordering)
+// race on it.
 #include <mutex>
 
 #include "qs_internal.cuh"
@@ -52,12 +55,24 @@ extern "C" qs_status qs_sparse_linear_noalloc(const void* x, int dtype, int T, i
   const size_t need = qs_workspace_size(QS_OP_SPARSE_LINEAR, T, d_in, d_out, k);
   if (need == 0) return QS_ERR_INVALID_ARG;
   if (need > kScratchBytes) return QS_ERR_UNSUPPORTED;   // sizes beyond the fixed scratch
+  // every argument check of qs_sparse_linear first (with no workspace yet, so
+  // only the missing workspace may be reported): an invalid call enqueues nothing
+  qs::WsLayout L;
+  qs_status st = qs::check_sparse_linear(x, dtype, T, d_in, d_out, k, wt, y, nullptr, 0, &L);
+  if (st != QS_ERR_WORKSPACE) return st == QS_OK ? QS_ERR_CUDA : st;
+  void* ws = nullptr;
+  st = scratch_on_current_device(&ws);
+  if (st != QS_OK) return st;
+  // the counters (between the status word and the per-call buffers) start at zero
+  if (cudaMemsetAsync((unsigned char*)ws + L.tickets, 0, L.cnt - L.tickets, (cudaStream_t)stream) !=
+      cudaSuccess)
+    return QS_ERR_CUDA;
+  return qs_sparse_linear(x, dtype, T, d_in, d_out, k, wt, y, nullptr, ws, kScratchBytes, stream);
+}
+
+extern "C" qs_status qs_sparse_linear_noalloc_status(void* stream) {
   void* ws = nullptr;
   const qs_status st = scratch_on_current_device(&ws);
   if (st != QS_OK) return st;
-  // status word and counters (everything before the per-call buffers) start at zero
-  qs::WsLayout L;
-  if (!qs::ws_layout(QS_OP_SPARSE_LINEAR, T, d_in, d_out, k, &L)) return QS_ERR_INVALID_ARG;
-  if (cudaMemsetAsync(ws, 0, L.cnt, (cudaStream_t)stream) != cudaSuccess) return QS_ERR_CUDA;
-  return qs_sparse_linear(x, dtype, T, d_in, d_out, k, wt, y, nullptr, ws, kScratchBytes, stream);
+  return qs_device_status(ws, stream);
 }

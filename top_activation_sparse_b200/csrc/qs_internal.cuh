@@ -78,15 +78,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* b, uint32_t parity) {
       : "memory");
   return done != 0;
 }
-__device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity) {
-  for (uint32_t it = 0; it < kWaitLimit; ++it)
+__device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity,
+                                          uint32_t limit = kWaitLimit) {
+  for (uint32_t it = 0; it < limit; ++it)
     if (mbar_try_wait(b, parity)) return true;
   return false;
 }
 // Consumer-side wait: poll with a short sleep so that waiting warps leave the
 // issue slots to the producer and to the warps that have data.
-__device__ __forceinline__ bool mbar_wait_backoff(uint64_t* b, uint32_t parity) {
-  for (uint32_t it = 0; it < kWaitLimit; ++it) {
+__device__ __forceinline__ bool mbar_wait_backoff(uint64_t* b, uint32_t parity,
+                                                  uint32_t limit = kWaitLimit) {
+  for (uint32_t it = 0; it < limit; ++it) {
     if (mbar_try_wait(b, parity)) return true;
     __nanosleep(64);
   }
@@ -223,6 +225,11 @@ struct WsLayout {
 // Returns false if the sizes are invalid for `op`.
 bool ws_layout(int op, int T, int d_in, int d_out, int k, WsLayout* L);
 
+// Every host-side check of qs_sparse_linear's arguments (nothing is enqueued).
+qs_status check_sparse_linear(const void* x, int dtype, int T, int d_in, int d_out, int k,
+                              const void* wt, const void* y, const void* ws, size_t ws_bytes,
+                              WsLayout* L);
+
 // ---------------------------------------------------------------------------
 // kernel launchers (host functions, defined next to their kernels)
 // ---------------------------------------------------------------------------
@@ -293,10 +300,21 @@ struct GemvArgs {
   size_t zero_n = 0;
   uint32_t* hbits = nullptr;   // mode 1/2, one token: OR the bitmask of nonzero h in here
   DevStatus* status = nullptr;
+  // failure-detection testing only (qs_debug_inject): the producer issues no
+  // copies, and every wait of the launch gives up after wait_limit polls
+  int no_copies = 0;
+  uint32_t wait_limit = kWaitLimit;
   GemvPlan plan{};
 };
 
 cudaError_t launch_gemv(const GemvArgs& a, cudaStream_t s);
+
+// Host-side fault injection state set by qs_debug_inject (tests only).
+struct FaultState {
+  int mode = QS_FAULT_NONE;
+  uint32_t wait_polls = 0;
+};
+extern FaultState g_fault;
 
 struct QGemvArgs {
   const uint32_t* wp = nullptr;  // [d_in, d_out/16]
