@@ -4,7 +4,7 @@ Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py`` (cpu_baseline leg 
 ``--impl reference`` arm) may import this package.
 """
 from .qs_oracle import (  # noqa: F401
-    topk_keep, mask_from_keep, topk_mask, kept_values, sparse_linear, sparse_linear_backward_ste,
+    topk_keep, block_topk_keep, mask_from_keep, topk_mask, kept_values, sparse_linear, sparse_linear_backward_ste,
     relu, ffn_hidden,
     sparse_ffn, absmax_quantize, ternary_quantize, ternary_pack, ternary_unpack,
     quant_sparse_linear, max_rel_err,

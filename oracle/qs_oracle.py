@@ -25,6 +25,12 @@ What it computes, and where each step comes from:
   by absolute value, then apply W_down).  Reading used:
   h = ReLU(x.W_gate^T + b_gate) (.) ReLU(x.W_up^T + b_up).
   -> :func:`sparse_ffn` with act="drelu".
+* Q-Sparse paper summary (shd-paper.top), abstract and method section (key
+  design 3): Block Q-Sparse for batched training and inference, by splitting
+  the activations into blocks.  No mechanism survives on the pages; reading
+  used: blocks of consecutive tokens share one selection, the k features with
+  the largest block magnitude max_t |x_ti|.  -> :func:`block_topk_keep` (its
+  result is passed as ``keep`` / ``keep_h`` to the projection and FFN oracles).
 * Q-Sparse news article, the same Top-K section, the paragraphs on the
   straight-through estimator (STE): top-K
   has zero gradient almost everywhere, so the loss gradient with respect to
@@ -80,6 +86,32 @@ def topk_keep(x, k: int) -> np.ndarray:
     # lower-index-first tie rule.
     order = np.argsort(-mag, axis=1, kind="stable")
     return np.sort(order[:, :k], axis=1)
+
+
+def block_topk_keep(x, k: int, block: int) -> np.ndarray:
+    """Block Q-Sparse selection: int64 [T, k] kept indices per token.
+
+    Q-Sparse paper summary (shd-paper.top), abstract and method section (key
+    design 3): Block Q-Sparse splits the activations into blocks so that
+    batched training and inference use the hardware well.  The pages give no
+    mechanism; this library's reading: the T token rows are cut into blocks of
+    `block` consecutive rows (the last one may be shorter); a block ranks its
+    features by the block magnitude s_i = max over the block's rows of |x_ti|
+    and keeps the k largest (ties -> lower index, as for one token); every row
+    of the block keeps those same k features.  block = 1 is per-token top-K.
+    """
+    x = np.asarray(x)
+    if x.ndim != 2:
+        raise ValueError("x must be [T, d]")
+    if block < 1:
+        raise ValueError("block must be >= 1")
+    T, d = x.shape
+    keep = np.zeros((T, k), dtype=np.int64)
+    for b0 in range(0, T, block):
+        rows = slice(b0, min(T, b0 + block))
+        s = np.max(np.abs(x[rows].astype(np.float64)), axis=0)   # block magnitude per feature
+        keep[rows] = topk_keep(s[None, :], k)[0]
+    return keep
 
 
 def mask_from_keep(keep: np.ndarray, T: int, d: int) -> np.ndarray:
@@ -178,7 +210,8 @@ def ffn_hidden(u, g, act: str, b_up=None, b_gate=None):
 
 
 def sparse_ffn(x, wt_up, wt_gate, wt_down, act: str, k_in: int, k_h: int,
-               b_up=None, b_gate=None, keep_h: np.ndarray | None = None) -> dict:
+               b_up=None, b_gate=None, keep_h: np.ndarray | None = None,
+               block: int = 1) -> dict:
     """One sparse FFN layer.
 
     x_s = topK(x, k_in);  u = x_s.W_up^T;  g = x_s.W_gate^T;  h = act(u, g);
@@ -186,7 +219,8 @@ def sparse_ffn(x, wt_up, wt_gate, wt_down, act: str, k_in: int, k_h: int,
 
     ``keep_h`` overrides the top-K on |h| (the CUDA path computes h in fp32, so
     near the threshold its selection may legitimately differ; the projection is
-    then re-run here on that selection).
+    then re-run here on that selection).  ``block`` > 1 selects with Block
+    Q-Sparse (:func:`block_topk_keep`) on x and on h.
     """
     x = np.asarray(x)
     T, d_model = x.shape
@@ -194,12 +228,12 @@ def sparse_ffn(x, wt_up, wt_gate, wt_down, act: str, k_in: int, k_h: int,
     wt_gate = np.asarray(wt_gate, dtype=np.float64)
     wt_down = np.asarray(wt_down, dtype=np.float64)
     d_ff = wt_up.shape[1]
-    keep_x = topk_keep(x, k_in)
+    keep_x = block_topk_keep(x, k_in, block)
     xs = x.astype(np.float64) * mask_from_keep(keep_x, T, d_model)
     u = xs @ wt_up
     g = xs @ wt_gate
     h = ffn_hidden(u, g, act, b_up, b_gate)
-    keep_h_own = topk_keep(h, k_h)
+    keep_h_own = block_topk_keep(h, k_h, block)
     kh = keep_h_own if keep_h is None else np.asarray(keep_h)
     hs = h * mask_from_keep(kh, T, d_ff)
     y = hs @ wt_down

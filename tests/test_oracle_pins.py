@@ -561,3 +561,92 @@ def test_max_rel_err_definition():
     # row 0: 0.1 / 4 ; row 1 (all-zero reference): 0.5 / 1
     assert oracle.max_rel_err(y, ref) == pytest.approx(0.5)
     assert oracle.max_rel_err(y[:1], ref[:1]) == pytest.approx(0.025)
+
+
+# ---------------------------------------------------------------- Block Q-Sparse pins
+
+
+def test_block_topk_golden_hand():
+    g = load_golden("block_topk_hand.json")
+    x = np.array(g["x"], dtype=np.float32)
+    for k, want in g["keep"].items():
+        assert oracle.block_topk_keep(x, int(k), g["block"]).tolist() == want, k
+    keep3 = oracle.block_topk_keep(x, 3, g["block"])
+    xs = x.astype(np.float64) * oracle.mask_from_keep(keep3, *x.shape)
+    assert xs[1].tolist() == g["xs_row1_k3"]
+    assert oracle.topk_keep(x, 3)[1].tolist() == g["per_row_keep_row1_k3"]
+    rows_read = sorted({int(i) for t in (0, 1) for i in keep3[t] if x[t, i] != 0})
+    assert rows_read == g["block0_rows_read_k3"]
+    assert np.unique(oracle.topk_keep(x[:2], 3)).tolist() == g["per_row_union_block0_k3"]
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_block_of_one_token_is_per_token_topk(seed):
+    g = workloads.rng(600 + seed)
+    x = workloads.adversarial_rows(seed, 5, 37) if seed % 2 else \
+        workloads.normal_f32(g, (7, 41))
+    for k in (0, 1, 5, x.shape[1] // 2, x.shape[1]):
+        assert np.array_equal(oracle.block_topk_keep(x, k, 1), oracle.topk_keep(x, k))
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_block_topk_bruteforce(seed):
+    """Block magnitude by loops (max of |x| over the block's rows), kept set by
+    the O(d^2) rank count, rows of one block sharing it."""
+    g = np.random.default_rng(700 + seed)
+    T, d = int(g.integers(1, 9)), int(g.integers(1, 13))
+    block = int(g.integers(1, T + 2))
+    x = g.integers(-4, 5, size=(T, d)).astype(np.float32) * np.float32(0.5)
+    for k in range(d + 1):
+        got = oracle.block_topk_keep(x, k, block)
+        for b0 in range(0, T, block):
+            rows = range(b0, min(T, b0 + block))
+            s = [max(abs(float(x[t, i])) for t in rows) for i in range(d)]
+            want = bf_keep(s, k)
+            for t in rows:
+                assert got[t].tolist() == want, (seed, k, block)
+
+
+def test_block_topk_invariants_at_decode_sizes():
+    w = workloads.WORKLOADS["ffn_relu2_llama7b"]
+    x = workloads.activations(w, 8)
+    for block in (2, 4, 8, 16):
+        keep = oracle.block_topk_keep(x, w.k, block)
+        for b0 in range(0, 8, block):
+            rows = list(range(b0, min(8, b0 + block)))
+            assert all(np.array_equal(keep[t], keep[rows[0]]) for t in rows)
+            s = np.max(np.abs(x[rows].astype(np.float64)), axis=0)
+            kept = np.zeros(x.shape[1], bool)
+            kept[keep[rows[0]]] = True
+            assert s[kept].min() >= s[~kept].max()
+            # the block reads at most k weight rows, fewer than the per-row union
+            union = np.unique(oracle.topk_keep(x[rows], w.k))
+            assert np.unique(keep[rows]).size == w.k <= union.size
+
+
+@pytest.mark.parametrize("act", ["relu2_glu", "drelu"])
+@pytest.mark.parametrize("seed", range(4))
+def test_block_ffn_bruteforce_tiny(act, seed):
+    """sparse_ffn with a block selection on x and on h, by plain loops."""
+    g = np.random.default_rng(800 + seed)
+    T, dm, dff, block = 5, 6, 7, 2
+    x = g.standard_normal((T, dm))
+    up, gate = g.standard_normal((dm, dff)), g.standard_normal((dm, dff))
+    down = g.standard_normal((dff, dm))
+    bu = bg = -0.2 if act == "drelu" else None
+    r = oracle.sparse_ffn(x, up, gate, down, act, 4, 3, b_up=bu, b_gate=bg, block=block)
+    kx = oracle.block_topk_keep(x, 4, block)
+    for t in range(T):
+        xs = [x[t, i] if i in kx[t] else 0.0 for i in range(dm)]
+        u = bf_matvec(xs, up.tolist())
+        gg = bf_matvec(xs, gate.tolist())
+        if act == "relu2_glu":
+            h = [max(u[j], 0.0) ** 2 * gg[j] for j in range(dff)]
+        else:
+            h = [max(gg[j] - 0.2, 0.0) * max(u[j] - 0.2, 0.0) for j in range(dff)]
+        assert np.allclose(r["h"][t], h, rtol=1e-10, atol=1e-12)
+    kh = oracle.block_topk_keep(r["h"], 3, block)
+    assert np.array_equal(r["keep_h"], kh)
+    for t in range(T):
+        hs = [r["h"][t, j] if j in kh[t] else 0.0 for j in range(dff)]
+        assert np.allclose(r["y"][t], bf_matvec(hs, down.tolist()), rtol=1e-10, atol=1e-12)
