@@ -62,6 +62,8 @@ def parse_args(argv=None):
     ap.add_argument("--gate-first", action="store_true",
                     help="dReLU FFN workloads: gate projection first, then W_up (output-major) "
                          "read only for open gates (qs_sparse_ffn_gate_first)")
+    ap.add_argument("--block", type=int, default=1,
+                    help="Block Q-Sparse: tokens sharing one top-K selection (1: per token)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-seconds", type=float, default=120.0)
@@ -73,6 +75,8 @@ def parse_args(argv=None):
         ap.error("--warmup must be >= 3")
     if a.gate_first and workloads.WORKLOADS[a.workload].act != "drelu":
         ap.error("--gate-first needs a dReLU FFN workload")
+    if not 1 <= a.block <= 64 or (a.block > 1 and a.gate_first):
+        ap.error("--block must be 1..64 (and is not available with --gate-first)")
     if a.steps < 1:
         ap.error("--steps must be >= 1")
     return a
@@ -265,6 +269,13 @@ def _mk_events(torch, stream, n):
 
 def workload_desc(args, T: int) -> str:
     """The workload's description, identical in both arms' `config`."""
+    blk = getattr(args, "block", 1)
+    if blk > 1:
+        return _workload_desc(args, T) + f", Block Q-Sparse blocks of {blk} tokens"
+    return _workload_desc(args, T)
+
+
+def _workload_desc(args, T: int) -> str:
     w = workloads.WORKLOADS[args.workload]
     if w.kind == "ffn":
         gf = (", gate first (W_up output-major, rows of open gates only)"
@@ -296,6 +307,7 @@ def setup_ffn(args, qs, torch, device, stream, rank):
     if gate_first:                    # W_up output-major: [d_ff, d_model]
         layers = [(up.t().contiguous(), gate, down) for up, gate, down in layers]
     op = qs.QS_OP_SPARSE_FFN_GATE_FIRST if gate_first else qs.QS_OP_SPARSE_FFN
+    blk = args.block
     bias = None
     if w.bias is not None:
         bias = torch.full((d_ff,), float(w.bias), dtype=torch.float32, device=device)
@@ -304,13 +316,18 @@ def setup_ffn(args, qs, torch, device, stream, rank):
     ws = qs.new_workspace(op, T, d_model, d_ff, k_h, device)
     sp = stream.cuda_stream
     bptr = bias.data_ptr() if bias is not None else None
-    fn = qs.lib().qs_sparse_ffn_gate_first if gate_first else qs.lib().qs_sparse_ffn
+    fn = (qs.lib().qs_sparse_ffn_gate_first if gate_first else
+          qs.lib().qs_block_sparse_ffn if blk > 1 else qs.lib().qs_sparse_ffn)
 
     def c_args(l, ev, kx=k_in, kh=k_h):
         up, gate, down = layers[l]
         if gate_first:                # x is dense on this path (kx = d_model)
             return (x.data_ptr(), qs.QS_BF16, T, d_model, d_ff, kh, gate.data_ptr(),
                     up.data_ptr(), bptr, bptr, down.data_ptr(), y.data_ptr(), None, None, ev,
+                    ws.data_ptr(), ws.numel(), sp)
+        if blk > 1:
+            return (x.data_ptr(), qs.QS_BF16, T, d_model, d_ff, act, kx, kh, blk, up.data_ptr(),
+                    gate.data_ptr(), bptr, bptr, down.data_ptr(), y.data_ptr(), None, None, ev,
                     ws.data_ptr(), ws.numel(), sp)
         return (x.data_ptr(), qs.QS_BF16, T, d_model, d_ff, act, kx, kh, up.data_ptr(),
                 gate.data_ptr(), bptr, bptr, down.data_ptr(), y.data_ptr(), None, None, ev,
@@ -348,13 +365,13 @@ def setup_ffn(args, qs, torch, device, stream, rank):
                                         y=y_dev, ws=ws)
         else:
             qs.qs_sparse_ffn(x_dev, up, gate, down, w.act, k_in, k_h, b_up=bias, b_gate=bias,
-                             y=y_dev, ws=ws)
+                             y=y_dev, ws=ws, block=blk)
 
     def cpu_rate():
         up, gate, down = (t.float().cpu().numpy() for t in layers[0])
         if gate_first:
             up = np.ascontiguousarray(up.T)
-        return cpu_oracle_ffn(w, x.float().cpu().numpy(), up, gate, down, args.cpu_seconds)
+        return cpu_oracle_ffn(w, x.float().cpu().numpy(), up, gate, down, args.cpu_seconds, blk)
 
     phases = ["topk_x", "upgate", "topk_h", "down"]
     return {
@@ -393,10 +410,14 @@ def setup_linear(args, qs, torch, device, stream, rank):
     y = torch.empty(T, w.d_out, dtype=tdt, device=device)
     ws = qs.new_workspace(qs.QS_OP_SPARSE_LINEAR, T, w.d_in, w.d_out, w.k, device)
     sp = stream.cuda_stream
-    fn = qs.lib().qs_sparse_linear
+    blk = args.block
+    fn = qs.lib().qs_block_sparse_linear if blk > 1 else qs.lib().qs_sparse_linear
     dt = qs.QS_BF16 if w.dtype == "bf16" else qs.QS_F32
 
     def c_args(l, ev, k=w.k):
+        if blk > 1:
+            return (x.data_ptr(), dt, T, w.d_in, w.d_out, k, blk, wts[l].data_ptr(), y.data_ptr(),
+                    ev, ws.data_ptr(), ws.numel(), sp)
         return (x.data_ptr(), dt, T, w.d_in, w.d_out, k, wts[l].data_ptr(), y.data_ptr(), ev,
                 ws.data_ptr(), ws.numel(), sp)
 
@@ -416,7 +437,7 @@ def setup_linear(args, qs, torch, device, stream, rank):
         bound, kernel = "hbm", "gemv_kernel (gather-GEMV)"
 
     def e2e_call(i, x_dev, y_dev):
-        qs.qs_sparse_linear(x_dev, wts[i % n_layers], w.k, y=y_dev, ws=ws)
+        qs.qs_sparse_linear(x_dev, wts[i % n_layers], w.k, y=y_dev, ws=ws, block=blk)
 
     def cpu_rate():
         import oracle
@@ -426,7 +447,8 @@ def setup_linear(args, qs, torch, device, stream, rank):
         t0 = time.perf_counter()
         n = 0
         while n < 2 or time.perf_counter() - t0 < args.cpu_seconds:
-            oracle.sparse_linear(xs[:rows_n], wt0, w.k)
+            oracle.sparse_linear(xs[:rows_n], wt0, w.k,
+                                 keep=oracle.block_topk_keep(xs[:rows_n], w.k, blk))
             n += 1
         dt_ = time.perf_counter() - t0
         return {"value": round(n * rows_n / dt_, 3), "unit": UNIT, "cores": _threads_in_use(),
@@ -466,9 +488,14 @@ def setup_quant(args, qs, torch, device, stream, rank):
     y = torch.empty(T, w.d_out, dtype=torch.float32, device=device)
     ws = qs.new_workspace(qs.QS_OP_QUANT_SPARSE_LINEAR, T, w.d_in, w.d_out, w.k, device)
     sp = stream.cuda_stream
-    fn = qs.lib().qs_quant_sparse_linear
+    blk = args.block
+    fn = qs.lib().qs_block_quant_sparse_linear if blk > 1 else qs.lib().qs_quant_sparse_linear
 
     def c_args(l, ev, k=w.k):
+        if blk > 1:
+            return (x.data_ptr(), qs.QS_BF16, T, w.d_in, w.d_out, k, blk, packs[l].data_ptr(),
+                    ctypes.c_float(alphas[l]), ctypes.c_float(1e-5), y.data_ptr(), None, None,
+                    None, ev, ws.data_ptr(), ws.numel(), sp)
         return (x.data_ptr(), qs.QS_BF16, T, w.d_in, w.d_out, k, packs[l].data_ptr(),
                 ctypes.c_float(alphas[l]), ctypes.c_float(1e-5), y.data_ptr(), None, None, None, ev,
                 ws.data_ptr(), ws.numel(), sp)
@@ -481,7 +508,7 @@ def setup_quant(args, qs, torch, device, stream, rank):
 
     def e2e_call(i, x_dev, y_dev):
         qs.qs_quant_sparse_linear(x_dev, packs[i % n_layers], alphas[i % n_layers], w.k, y=y_dev,
-                                  ws=ws)
+                                  ws=ws, block=blk)
 
     def cpu_rate():
         import oracle
@@ -491,7 +518,9 @@ def setup_quant(args, qs, torch, device, stream, rank):
         t0 = time.perf_counter()
         n = 0
         while n < 2 or time.perf_counter() - t0 < args.cpu_seconds:
-            oracle.quant_sparse_linear(xs[:rows_n], t, alphas[0], w.k)
+            q_, _ = oracle.absmax_quantize(xs[:rows_n])
+            oracle.quant_sparse_linear(xs[:rows_n], t, alphas[0], w.k,
+                                       keep=oracle.block_topk_keep(q_, w.k, blk))
             n += 1
         dt_ = time.perf_counter() - t0
         return {"value": round(n * rows_n / dt_, 3), "unit": UNIT, "cores": _threads_in_use(),
@@ -694,7 +723,7 @@ def _threads_in_use() -> int:
         return 1
 
 
-def cpu_oracle_ffn(w, x, up, gate, down, seconds: float) -> dict:
+def cpu_oracle_ffn(w, x, up, gate, down, seconds: float, block: int = 1) -> dict:
     """Time the oracle as it stands on a bounded sample: whole-layer calls
     for about `seconds` of host time (at least two)."""
     import oracle
@@ -703,7 +732,7 @@ def cpu_oracle_ffn(w, x, up, gate, down, seconds: float) -> dict:
     n = 0
     t0 = time.perf_counter()
     while n < 2 or time.perf_counter() - t0 < seconds:
-        oracle.sparse_ffn(x, up, gate, down, w.act, w.k, w.k_h, b_up=b, b_gate=b)
+        oracle.sparse_ffn(x, up, gate, down, w.act, w.k, w.k_h, b_up=b, b_gate=b, block=block)
         n += 1
     dt = time.perf_counter() - t0
     return {"value": round(n * T / dt, 3), "unit": UNIT, "cores": _threads_in_use(),
@@ -724,17 +753,20 @@ def run_reference(args, rank, world, local):
         b = None if w.bias is None else np.full(w.d_out, w.bias)
 
         def step():
-            oracle.sparse_ffn(x, up, gate, down, w.act, w.k, w.k_h, b_up=b, b_gate=b)
+            oracle.sparse_ffn(x, up, gate, down, w.act, w.k, w.k_h, b_up=b, b_gate=b,
+                              block=args.block)
     elif w.kind == "quant":
         t, alpha = oracle.ternary_quantize(workloads.weight_out_major(w.d_out, w.d_in, w.seed(0, 1)))
 
         def step():
-            oracle.quant_sparse_linear(x, t, alpha, w.k)
+            q_, _ = oracle.absmax_quantize(x)
+            oracle.quant_sparse_linear(x, t, alpha, w.k,
+                                       keep=oracle.block_topk_keep(q_, w.k, args.block))
     else:
         wt = workloads.weight_t(w.d_in, w.d_out, w.seed(0, 1), w.dtype)
 
         def step():
-            oracle.sparse_linear(x, wt, w.k)
+            oracle.sparse_linear(x, wt, w.k, keep=oracle.block_topk_keep(x, w.k, args.block))
 
     t0 = time.perf_counter()
     step()

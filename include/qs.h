@@ -93,6 +93,8 @@ typedef enum qs_op {
 /* From this many tokens on, qs_sparse_linear on bf16 runs the masked-dense
  * tensor-core GEMM instead of the gather-GEMV. */
 #define QS_PREFILL_MIN_T 64
+/* Largest Block Q-Sparse block (tokens sharing one selection). */
+#define QS_MAX_BLOCK 64
 /* Number of cudaEvent_t handles qs_sparse_ffn records when given phase events. */
 #define QS_FFN_PHASE_EVENTS 5
 /* ... and qs_sparse_linear / qs_quant_sparse_linear (before the top-K, after
@@ -251,6 +253,45 @@ qs_status qs_quant_sparse_linear(const void* x, int dtype, int T, int d_in, int 
 qs_status qs_ternary_pack(const float* w, int d_out, int d_in, float eps,
                           uint32_t* wt_packed, float* alpha_out,
                           void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Block Q-Sparse: the three projections above with one selection per block of
+ * tokens instead of one per token.
+ *   Source: Q-Sparse paper summary (shd-paper.top), abstract ("Block Q-Sparse
+ *   for batch training and inference") and method section, key design 3
+ *   (splitting the activations into blocks uses the hardware better in
+ *   batches).  The pages give no mechanism; this library reads it as:
+ *     the T token rows are cut into blocks of `block` consecutive rows (the
+ *     last may be shorter); a block ranks feature i by its block magnitude
+ *     s_i = max over the block's rows of |x_ti| (ties -> lower index, -0 == +0)
+ *     and keeps the k largest; every row of the block keeps those k features.
+ *   So a block's projection reads at most k weight rows however many tokens
+ *   it holds, where per-token selections read the union of theirs.  block = 1
+ *   is the per-token entry point exactly.
+ *
+ *   block  1..QS_MAX_BLOCK.  Rows (d_in; d_model and d_ff) of more than 16384
+ *          features with block > 1 return QS_ERR_UNSUPPORTED.
+ *   Every other argument, output and error is that of the per-token entry
+ *   point; idx / idx_h_out rows of one block are equal.  For the FFN the same
+ *   block size applies to the top-K on |x| and to the top-K on |h|.  Tokens
+ *   run in chunks of whole blocks (at most QS_PREFILL_MIN_T tokens), and
+ *   qs_sparse_linear's prefill path (bf16, T >= QS_PREFILL_MIN_T) multiplies
+ *   the block-masked X_sparse on the tensor cores.
+ *   Workspace: qs_workspace_size of the per-token op with the same sizes.
+ */
+qs_status qs_block_sparse_linear(const void* x, int dtype, int T, int d_in, int d_out, int k,
+                                 int block, const void* wt, void* y, void* const* phase_events,
+                                 void* ws, size_t ws_bytes, void* stream);
+qs_status qs_block_sparse_ffn(const void* x, int dtype, int T, int d_model, int d_ff, int act,
+                              int k_in, int k_h, int block, const void* wt_up, const void* wt_gate,
+                              const float* b_up, const float* b_gate, const void* wt_down, void* y,
+                              float* h_out, int32_t* idx_h_out, void* const* phase_events,
+                              void* ws, size_t ws_bytes, void* stream);
+qs_status qs_block_quant_sparse_linear(const void* x, int dtype, int T, int d_in, int d_out, int k,
+                                       int block, const uint32_t* wt_packed, float alpha, float eps,
+                                       float* y, int32_t* acc, int8_t* q, int32_t* idx,
+                                       void* const* phase_events, void* ws, size_t ws_bytes,
+                                       void* stream);
 
 /* Bytes of workspace `op` needs for these sizes (0 if the sizes are invalid).
  * Arguments: QS_OP_TOPK_MASK (T, d, 0, k); QS_OP_SPARSE_LINEAR (T, d_in, d_out,

@@ -46,6 +46,7 @@ QS_FAULT_NONE = 0
 QS_FAULT_GATHER_NO_COPIES = 1
 
 QS_MAX_ROW = 49152
+QS_MAX_BLOCK = 64
 QS_NOALLOC_SCRATCH_BYTES = 4 << 20
 QS_PREFILL_MIN_T = 64
 QS_FFN_PHASE_EVENTS = 5
@@ -80,6 +81,11 @@ _SIGNATURES = {
     "qs_device_status": (_i, [_vp, _vp]),
     "qs_workspace_stats": (_i, [_vp, _i, _i, _i, _i, _i, _vp, _vp]),
     "qs_status_string": (ctypes.c_char_p, [_i]),
+    "qs_block_sparse_linear": (_i, [_vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "qs_block_sparse_ffn": (_i, [_vp, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp,
+                                 _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "qs_block_quant_sparse_linear": (_i, [_vp, _i, _i, _i, _i, _i, _i, _vp, _f, _f, _vp, _vp, _vp,
+                                          _vp, _vp, _vp, _sz, _vp]),
     "qs_sparse_linear_noalloc": (_i, [_vp, _i, _i, _i, _i, _i, _vp, _vp, _vp]),
     "qs_sparse_linear_noalloc_status": (_i, [_vp]),
     "qs_workspace_list": (_i, [_vp, _i, _i, _i, _i, _i, _i, _vp, _i, _vp, _vp, _vp]),
@@ -283,8 +289,9 @@ def _events(phase_events, n):
 
 
 def qs_sparse_linear(x: torch.Tensor, wt: torch.Tensor, k: int, y=None, phase_events=None,
-                     ws=None, stream=None) -> torch.Tensor:
-    """Y = (X (.) topK-mask(|X|)) . W^T with wt = W^T [d_in, d_out]."""
+                     ws=None, stream=None, block: int = 1) -> torch.Tensor:
+    """Y = (X (.) topK-mask(|X|)) . W^T with wt = W^T [d_in, d_out].
+    block > 1: Block Q-Sparse (qs_block_sparse_linear)."""
     dev = _need_cuda(x, wt)
     T, d_in = x.shape
     d_out = wt.shape[1]
@@ -293,10 +300,15 @@ def qs_sparse_linear(x: torch.Tensor, wt: torch.Tensor, k: int, y=None, phase_ev
     y = _out(y if y is not None else True, (T, d_out), x.dtype, dev)
     _need_cuda(y)
     ws = _workspace(ws, QS_OP_SPARSE_LINEAR, T, d_in, d_out, k, dev)
-    _check("qs_sparse_linear", lib().qs_sparse_linear(
-        x.data_ptr(), _dtype_code(x), T, d_in, d_out, k, wt.data_ptr(), y.data_ptr(),
-        _events(phase_events, QS_LINEAR_PHASE_EVENTS), ws.data_ptr(), ws.numel(),
-        _stream_ptr(stream)))
+    ev = _events(phase_events, QS_LINEAR_PHASE_EVENTS)
+    if block == 1:
+        _check("qs_sparse_linear", lib().qs_sparse_linear(
+            x.data_ptr(), _dtype_code(x), T, d_in, d_out, k, wt.data_ptr(), y.data_ptr(), ev,
+            ws.data_ptr(), ws.numel(), _stream_ptr(stream)))
+    else:
+        _check("qs_block_sparse_linear", lib().qs_block_sparse_linear(
+            x.data_ptr(), _dtype_code(x), T, d_in, d_out, k, int(block), wt.data_ptr(),
+            y.data_ptr(), ev, ws.data_ptr(), ws.numel(), _stream_ptr(stream)))
     return y
 
 
@@ -327,8 +339,9 @@ class FfnResult(NamedTuple):
 
 def qs_sparse_ffn(x, wt_up, wt_gate, wt_down, act, k_in: int, k_h: int, b_up=None, b_gate=None,
                   y=None, h_out=None, idx_h_out=None, phase_events=None, ws=None,
-                  stream=None) -> FfnResult:
-    """One sparse gated FFN layer (top-K on x, up/gate, gating, top-K on |h|, down)."""
+                  stream=None, block: int = 1) -> FfnResult:
+    """One sparse gated FFN layer (top-K on x, up/gate, gating, top-K on |h|, down).
+    block > 1: Block Q-Sparse selections on x and h (qs_block_sparse_ffn)."""
     dev = _need_cuda(x, wt_up, wt_gate, wt_down, b_up, b_gate)
     T, d_model = x.shape
     d_ff = wt_up.shape[1]
@@ -345,11 +358,18 @@ def qs_sparse_ffn(x, wt_up, wt_gate, wt_down, act, k_in: int, k_h: int, b_up=Non
     _need_cuda(y, h_out, idx_h_out)
     ev = _events(phase_events, QS_FFN_PHASE_EVENTS)
     ws = _workspace(ws, QS_OP_SPARSE_FFN, T, d_model, d_ff, k_h, dev)
-    _check("qs_sparse_ffn", lib().qs_sparse_ffn(
-        x.data_ptr(), _dtype_code(x), T, d_model, d_ff, act_code, k_in, k_h,
-        wt_up.data_ptr(), wt_gate.data_ptr(), _ptr(b_up), _ptr(b_gate), wt_down.data_ptr(),
-        y.data_ptr(), _ptr(h_out), _ptr(idx_h_out), ev, ws.data_ptr(), ws.numel(),
-        _stream_ptr(stream)))
+    if block == 1:
+        _check("qs_sparse_ffn", lib().qs_sparse_ffn(
+            x.data_ptr(), _dtype_code(x), T, d_model, d_ff, act_code, k_in, k_h,
+            wt_up.data_ptr(), wt_gate.data_ptr(), _ptr(b_up), _ptr(b_gate), wt_down.data_ptr(),
+            y.data_ptr(), _ptr(h_out), _ptr(idx_h_out), ev, ws.data_ptr(), ws.numel(),
+            _stream_ptr(stream)))
+    else:
+        _check("qs_block_sparse_ffn", lib().qs_block_sparse_ffn(
+            x.data_ptr(), _dtype_code(x), T, d_model, d_ff, act_code, k_in, k_h, int(block),
+            wt_up.data_ptr(), wt_gate.data_ptr(), _ptr(b_up), _ptr(b_gate), wt_down.data_ptr(),
+            y.data_ptr(), _ptr(h_out), _ptr(idx_h_out), ev, ws.data_ptr(), ws.numel(),
+            _stream_ptr(stream)))
     return FfnResult(y, h_out, idx_h_out)
 
 
@@ -389,8 +409,9 @@ class QuantResult(NamedTuple):
 
 def qs_quant_sparse_linear(x, wt_packed, alpha: float, k: int, eps: float = 1e-5, y=None,
                            acc=None, q=None, idx=None, phase_events=None, ws=None,
-                           stream=None) -> QuantResult:
-    """int8 (per-token absmax) x ternary (packed 2-bit) projection of the top-K of |q|."""
+                           stream=None, block: int = 1) -> QuantResult:
+    """int8 (per-token absmax) x ternary (packed 2-bit) projection of the top-K of |q|.
+    block > 1: Block Q-Sparse on |q| (qs_block_quant_sparse_linear)."""
     dev = _need_cuda(x, wt_packed)
     T, d_in = x.shape
     if wt_packed.dtype != torch.int32 or wt_packed.shape[0] != d_in:
@@ -402,11 +423,17 @@ def qs_quant_sparse_linear(x, wt_packed, alpha: float, k: int, eps: float = 1e-5
     idx = _out(idx, (T, k), torch.int32, dev)
     _need_cuda(y, acc, q, idx)
     ws = _workspace(ws, QS_OP_QUANT_SPARSE_LINEAR, T, d_in, d_out, k, dev)
-    _check("qs_quant_sparse_linear", lib().qs_quant_sparse_linear(
-        x.data_ptr(), _dtype_code(x), T, d_in, d_out, k, wt_packed.data_ptr(), float(alpha),
-        float(eps), y.data_ptr(), _ptr(acc), _ptr(q), _ptr(idx),
-        _events(phase_events, QS_LINEAR_PHASE_EVENTS), ws.data_ptr(), ws.numel(),
-        _stream_ptr(stream)))
+    ev = _events(phase_events, QS_LINEAR_PHASE_EVENTS)
+    if block == 1:
+        _check("qs_quant_sparse_linear", lib().qs_quant_sparse_linear(
+            x.data_ptr(), _dtype_code(x), T, d_in, d_out, k, wt_packed.data_ptr(), float(alpha),
+            float(eps), y.data_ptr(), _ptr(acc), _ptr(q), _ptr(idx), ev, ws.data_ptr(),
+            ws.numel(), _stream_ptr(stream)))
+    else:
+        _check("qs_block_quant_sparse_linear", lib().qs_block_quant_sparse_linear(
+            x.data_ptr(), _dtype_code(x), T, d_in, d_out, k, int(block), wt_packed.data_ptr(),
+            float(alpha), float(eps), y.data_ptr(), _ptr(acc), _ptr(q), _ptr(idx), ev,
+            ws.data_ptr(), ws.numel(), _stream_ptr(stream)))
     return QuantResult(y, acc, q, idx)
 
 

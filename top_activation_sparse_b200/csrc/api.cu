@@ -37,6 +37,15 @@ long rows_bound(int T, int d, int k) {
   return tk < d ? tk : d;
 }
 
+// Tokens per chunk: at most kChunkT, a whole number of Block Q-Sparse blocks.
+int chunk_tokens(int block) { return block <= 1 ? kChunkT : (kChunkT / block) * block; }
+
+// Distinct rows a chunk of Tc tokens can keep: k per selection.
+long rows_bound_blocks(int Tc, int d, int k, int block) {
+  const int b = block < 1 ? 1 : block;
+  return rows_bound((Tc + b - 1) / b, d, k);
+}
+
 }  // namespace
 
 // Same layout for every dtype: each buffer is sized for the larger of the
@@ -323,12 +332,14 @@ qs_status qs_topk_mask(const void* x, int dtype, int T, int d, int k, int32_t* i
   return from_cuda(launch_topk(a, (cudaStream_t)stream));
 }
 
-qs_status qs_sparse_linear(const void* x, int dtype, int T, int d_in, int d_out, int k,
-                           const void* wt, void* y, void* const* phase_events, void* ws,
-                           size_t ws_bytes, void* stream) {
+static qs_status linear_impl(const void* x, int dtype, int T, int d_in, int d_out, int k, int block,
+                             const void* wt, void* y, void* const* phase_events, void* ws,
+                             size_t ws_bytes, void* stream) {
   WsLayout L;
   const qs_status st = qs::check_sparse_linear(x, dtype, T, d_in, d_out, k, wt, y, ws, ws_bytes, &L);
   if (st != QS_OK) return st;
+  if (block < 1 || block > QS_MAX_BLOCK) return QS_ERR_INVALID_ARG;
+  if (block > 1 && !topk_block_supported(d_in)) return QS_ERR_UNSUPPORTED;
   WsView w{(unsigned char*)ws};
   cudaStream_t s = (cudaStream_t)stream;
   const int eb = elem_bytes(dtype);
@@ -342,6 +353,7 @@ qs_status qs_sparse_linear(const void* x, int dtype, int T, int d_in, int d_out,
     QS_TRY_CUDA(mark(0));
     TopkArgs a;
     a.x = x; a.T = T; a.d = d_in; a.k = k; a.kind = TK_BF16;
+    a.block = block;
     a.xs = w.at<void>(L.xs_bf16);
     a.status = w.status();
     QS_TRY_CUDA(launch_topk(a, s));
@@ -357,13 +369,15 @@ qs_status qs_sparse_linear(const void* x, int dtype, int T, int d_in, int d_out,
     return QS_OK;
   }
 
-  for (int t0 = 0; t0 < T; t0 += kChunkT) {
+  const int chunk = chunk_tokens(block);
+  for (int t0 = 0; t0 < T; t0 += chunk) {
     const bool timed = (t0 == 0);
     if (timed) QS_TRY_CUDA(mark(0));
-    const int Tc = (T - t0) < kChunkT ? (T - t0) : kChunkT;
+    const int Tc = (T - t0) < chunk ? (T - t0) : chunk;
     TopkArgs a;
     a.x = (const unsigned char*)x + (size_t)t0 * d_in * eb;
     a.T = Tc; a.d = d_in; a.k = k;
+    a.block = Tc > 1 ? block : 1;
     a.kind = dtype == QS_F32 ? TK_F32 : TK_BF16;
     a.xsf = Tc > 1 ? w.at<float>(L.xsf_x) : nullptr;   // only the union pass reads it
     a.list = w.at<int32_t>(L.list_x);
@@ -372,7 +386,7 @@ qs_status qs_sparse_linear(const void* x, int dtype, int T, int d_in, int d_out,
     a.ticket = w.ticket(L, kTkTopkX);
     a.union_bits = reinterpret_cast<uint32_t*>(w.ticket(L, kUnionX));
     a.status = w.status();
-    const GemvPlan gp = plan_gemv(Tc, d_out, (int)rows_bound(Tc, d_in, k), 1, eb);
+    const GemvPlan gp = plan_gemv(Tc, d_out, (int)rows_bound_blocks(Tc, d_in, k, a.block), 1, eb);
     if (!plan_fits(gp, L.parts1_elems, 0)) return QS_ERR_UNSUPPORTED;
     a.zero = w.at<float>(L.parts1);
     a.zero_n = gp.parts_elems;
@@ -402,7 +416,7 @@ qs_status qs_sparse_linear(const void* x, int dtype, int T, int d_in, int d_out,
 // projection runs alone, and the up projection reads only the rows of open
 // gates (exact: the dReLU product is 0 wherever the gate branch is).
 static qs_status ffn_impl(int op, const void* x, int dtype, int T, int d_model, int d_ff, int act,
-                          int k_in, int k_h, const void* wt_up, const void* w_up_rows,
+                          int k_in, int k_h, int block, const void* wt_up, const void* w_up_rows,
                           const void* wt_gate, const float* b_up, const float* b_gate,
                           const void* wt_down, void* y, float* h_out, int32_t* idx_h_out,
                           void* const* phase_events, void* ws, size_t ws_bytes, void* stream) {
@@ -413,7 +427,10 @@ static qs_status ffn_impl(int op, const void* x, int dtype, int T, int d_model, 
       k_in > d_model || k_h < 0 || k_h > d_ff ||
       (act != QS_ACT_RELU2_GLU && act != QS_ACT_DRELU) || (gate_first && act != QS_ACT_DRELU))
     return QS_ERR_INVALID_ARG;
+  if (block < 1 || block > QS_MAX_BLOCK) return QS_ERR_INVALID_ARG;
   if (d_model > QS_MAX_ROW || d_ff > QS_MAX_ROW) return QS_ERR_UNSUPPORTED;
+  if (block > 1 && (!topk_block_supported(d_model) || !topk_block_supported(d_ff)))
+    return QS_ERR_UNSUPPORTED;
   const int eb = elem_bytes(dtype);
   const int V = 16 / eb;
   if ((d_model % V) != 0 || (d_ff % V) != 0) return QS_ERR_ALIGNMENT;
@@ -433,15 +450,18 @@ static qs_status ffn_impl(int op, const void* x, int dtype, int T, int d_model, 
   const float* unit = nullptr;                   // gate first: a vector of 1.0 (see step 2)
   if (gate_first) QS_TRY_CUDA(unit_vector_on_current_device(&unit, s));
 
-  for (int t0 = 0; t0 < T; t0 += kChunkT) {
-    const int Tc = (T - t0) < kChunkT ? (T - t0) : kChunkT;
+  const int chunk = chunk_tokens(block);
+  for (int t0 = 0; t0 < T; t0 += chunk) {
+    const int Tc = (T - t0) < chunk ? (T - t0) : chunk;
     const bool timed = (t0 == 0);
     if (timed) QS_TRY_CUDA(mark(0));
+    const int blk = Tc > 1 ? block : 1;
 
     // 1. top-K on |x|
     TopkArgs a;
     a.x = (const unsigned char*)x + (size_t)t0 * d_model * eb;
     a.T = Tc; a.d = d_model; a.k = k_in;
+    a.block = blk;
     a.kind = dtype == QS_F32 ? TK_F32 : TK_BF16;
     a.xsf = Tc > 1 ? w.at<float>(L.xsf_x) : nullptr;
     a.list = w.at<int32_t>(L.list_x);
@@ -452,7 +472,7 @@ static qs_status ffn_impl(int op, const void* x, int dtype, int T, int d_model, 
     a.status = w.status();
     const GemvPlan p_ug =
         plan_gemv(Tc, d_ff, (int)rows_bound(Tc, d_model, d_model), gate_first ? 1 : 2, eb);
-    const GemvPlan p_dn = plan_gemv(Tc, d_model, (int)rows_bound(Tc, d_ff, k_h), 1, eb);
+    const GemvPlan p_dn = plan_gemv(Tc, d_model, (int)rows_bound_blocks(Tc, d_ff, k_h, blk), 1, eb);
     if (!plan_fits(p_ug, L.parts1_elems, 0) || !plan_fits(p_dn, L.parts2_elems, p_ug.tickets))
       return QS_ERR_UNSUPPORTED;
     a.zero = w.at<float>(L.parts1);
@@ -511,6 +531,7 @@ static qs_status ffn_impl(int op, const void* x, int dtype, int T, int d_model, 
     // 3. top-K on |h|
     TopkArgs b;
     b.x = h; b.T = Tc; b.d = d_ff; b.k = k_h; b.kind = TK_F32;
+    b.block = blk;
     b.idx = (idx_h_out && k_h > 0) ? idx_h_out + (size_t)t0 * k_h : nullptr;
     b.xsf = Tc > 1 ? w.at<float>(L.xsf_h) : nullptr;
     b.list = w.at<int32_t>(L.list_h);
@@ -546,7 +567,7 @@ qs_status qs_sparse_ffn(const void* x, int dtype, int T, int d_model, int d_ff, 
                         const float* b_up, const float* b_gate, const void* wt_down, void* y,
                         float* h_out, int32_t* idx_h_out, void* const* phase_events, void* ws,
                         size_t ws_bytes, void* stream) {
-  return ffn_impl(QS_OP_SPARSE_FFN, x, dtype, T, d_model, d_ff, act, k_in, k_h, wt_up, nullptr,
+  return ffn_impl(QS_OP_SPARSE_FFN, x, dtype, T, d_model, d_ff, act, k_in, k_h, 1, wt_up, nullptr,
                   wt_gate, b_up, b_gate, wt_down, y, h_out, idx_h_out, phase_events, ws, ws_bytes,
                   stream);
 }
@@ -558,19 +579,20 @@ qs_status qs_sparse_ffn_gate_first(const void* x, int dtype, int T, int d_model,
                                    void* const* phase_events, void* ws, size_t ws_bytes,
                                    void* stream) {
   return ffn_impl(QS_OP_SPARSE_FFN_GATE_FIRST, x, dtype, T, d_model, d_ff, QS_ACT_DRELU, d_model,
-                  k_h, nullptr, w_up, wt_gate, b_up, b_gate, wt_down, y, h_out, idx_h_out,
+                  k_h, 1, nullptr, w_up, wt_gate, b_up, b_gate, wt_down, y, h_out, idx_h_out,
                   phase_events, ws, ws_bytes, stream);
 }
 
-qs_status qs_quant_sparse_linear(const void* x, int dtype, int T, int d_in, int d_out, int k,
-                                 const uint32_t* wt_packed, float alpha, float eps, float* y,
-                                 int32_t* acc, int8_t* q, int32_t* idx,
-                                 void* const* phase_events, void* ws, size_t ws_bytes,
-                                 void* stream) {
+static qs_status quant_impl(const void* x, int dtype, int T, int d_in, int d_out, int k, int block,
+                            const uint32_t* wt_packed, float alpha, float eps, float* y,
+                            int32_t* acc, int8_t* q, int32_t* idx, void* const* phase_events,
+                            void* ws, size_t ws_bytes, void* stream) {
   if (!valid_dtype(dtype) || x == nullptr || wt_packed == nullptr || y == nullptr || T < 1 ||
-      d_in < 1 || d_out < 1 || k < 0 || k > d_in || !(eps >= 0.0f) || !(alpha == alpha))
+      d_in < 1 || d_out < 1 || k < 0 || k > d_in || !(eps >= 0.0f) || !(alpha == alpha) ||
+      block < 1 || block > QS_MAX_BLOCK)
     return QS_ERR_INVALID_ARG;
   if (d_in > QS_MAX_ROW || d_out > QS_MAX_ROW) return QS_ERR_UNSUPPORTED;
+  if (block > 1 && !topk_block_supported(d_in)) return QS_ERR_UNSUPPORTED;
   if (!qgemv_supported(d_out) || !aligned16(x) || !aligned16(wt_packed) || !aligned16(y) ||
       !aligned16(acc) || !aligned16(q) || !aligned16(idx))
     return QS_ERR_ALIGNMENT;
@@ -584,13 +606,15 @@ qs_status qs_quant_sparse_linear(const void* x, int dtype, int T, int d_in, int 
     if (phase_events == nullptr) return cudaSuccess;
     return cudaEventRecord((cudaEvent_t)phase_events[i], s);
   };
-  for (int t0 = 0; t0 < T; t0 += kChunkT) {
-    const int Tc = (T - t0) < kChunkT ? (T - t0) : kChunkT;
+  const int chunk = chunk_tokens(block);
+  for (int t0 = 0; t0 < T; t0 += chunk) {
+    const int Tc = (T - t0) < chunk ? (T - t0) : chunk;
     const bool timed = (t0 == 0);
     if (timed) QS_TRY_CUDA(mark(0));
     TopkArgs a;
     a.x = (const unsigned char*)x + (size_t)t0 * d_in * eb;
     a.T = Tc; a.d = d_in; a.k = k;
+    a.block = Tc > 1 ? block : 1;
     a.kind = dtype == QS_F32 ? TK_QUANT_F32 : TK_QUANT_BF16;
     a.eps = eps;
     a.idx = (idx && k > 0) ? idx + (size_t)t0 * k : nullptr;
@@ -603,7 +627,7 @@ qs_status qs_quant_sparse_linear(const void* x, int dtype, int T, int d_in, int 
     a.ticket = w.ticket(L, kTkTopkX);
     a.union_bits = reinterpret_cast<uint32_t*>(w.ticket(L, kUnionX));
     a.status = w.status();
-    const GemvPlan qp = plan_qgemv(Tc, d_out, (int)rows_bound(Tc, d_in, k));
+    const GemvPlan qp = plan_qgemv(Tc, d_out, (int)rows_bound_blocks(Tc, d_in, k, a.block));
     if (!plan_fits(qp, L.parts1_elems, 0)) return QS_ERR_UNSUPPORTED;
     a.zero = w.at<float>(L.parts1);
     a.zero_n = qp.parts_elems;
@@ -624,6 +648,46 @@ qs_status qs_quant_sparse_linear(const void* x, int dtype, int T, int d_in, int 
     if (timed) QS_TRY_CUDA(mark(2));
   }
   return QS_OK;
+}
+
+qs_status qs_sparse_linear(const void* x, int dtype, int T, int d_in, int d_out, int k,
+                           const void* wt, void* y, void* const* phase_events, void* ws,
+                           size_t ws_bytes, void* stream) {
+  return linear_impl(x, dtype, T, d_in, d_out, k, 1, wt, y, phase_events, ws, ws_bytes, stream);
+}
+
+qs_status qs_block_sparse_linear(const void* x, int dtype, int T, int d_in, int d_out, int k,
+                                 int block, const void* wt, void* y, void* const* phase_events,
+                                 void* ws, size_t ws_bytes, void* stream) {
+  return linear_impl(x, dtype, T, d_in, d_out, k, block, wt, y, phase_events, ws, ws_bytes, stream);
+}
+
+qs_status qs_block_sparse_ffn(const void* x, int dtype, int T, int d_model, int d_ff, int act,
+                              int k_in, int k_h, int block, const void* wt_up, const void* wt_gate,
+                              const float* b_up, const float* b_gate, const void* wt_down, void* y,
+                              float* h_out, int32_t* idx_h_out, void* const* phase_events,
+                              void* ws, size_t ws_bytes, void* stream) {
+  return ffn_impl(QS_OP_SPARSE_FFN, x, dtype, T, d_model, d_ff, act, k_in, k_h, block, wt_up,
+                  nullptr, wt_gate, b_up, b_gate, wt_down, y, h_out, idx_h_out, phase_events, ws,
+                  ws_bytes, stream);
+}
+
+qs_status qs_quant_sparse_linear(const void* x, int dtype, int T, int d_in, int d_out, int k,
+                                 const uint32_t* wt_packed, float alpha, float eps, float* y,
+                                 int32_t* acc, int8_t* q, int32_t* idx,
+                                 void* const* phase_events, void* ws, size_t ws_bytes,
+                                 void* stream) {
+  return quant_impl(x, dtype, T, d_in, d_out, k, 1, wt_packed, alpha, eps, y, acc, q, idx,
+                    phase_events, ws, ws_bytes, stream);
+}
+
+qs_status qs_block_quant_sparse_linear(const void* x, int dtype, int T, int d_in, int d_out, int k,
+                                       int block, const uint32_t* wt_packed, float alpha, float eps,
+                                       float* y, int32_t* acc, int8_t* q, int32_t* idx,
+                                       void* const* phase_events, void* ws, size_t ws_bytes,
+                                       void* stream) {
+  return quant_impl(x, dtype, T, d_in, d_out, k, block, wt_packed, alpha, eps, y, acc, q, idx,
+                    phase_events, ws, ws_bytes, stream);
 }
 
 qs_status qs_ternary_pack(const float* wmat, int d_out, int d_in, float eps, uint32_t* wt_packed,

@@ -254,6 +254,7 @@ struct TopkArgs {
   int8_t* list_q = nullptr;  // [d][T] int8 codes of the listed rows (quant path)
   int32_t* list_count = nullptr;
   int32_t* ticket = nullptr;
+  int block = 1;             // Block Q-Sparse: rows per shared selection (1 = per row)
   uint32_t* union_bits = nullptr;  // [ceil(d/32)] zero between calls (several tokens)
   uint32_t* nz_bits = nullptr;     // one token: bitmask of the row's nonzero entries, written by
                                    // the kernel that produced the row; read, then zeroed, here
@@ -270,6 +271,8 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s);
 // True when launch_topk takes a one-token row of this size through the list
 // kernel, which can consume (and then clears) a producer's nonzero bitmask.
 bool topk_bitmask_supported(int T, int d, int kind);
+// Rows this long can take block selections (a.block > 1).
+bool topk_block_supported(int d);
 
 // Zero `n` floats (n % 4 == 0) cooperatively across the whole grid.
 __device__ __forceinline__ void grid_zero(float* p, size_t n) {

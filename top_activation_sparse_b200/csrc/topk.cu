@@ -785,7 +785,102 @@ __global__ void __launch_bounds__(NT) topk_list_kernel(TopkArgs a) {
   }
 }
 
+// ---- Block Q-Sparse helpers (a block of rows shares one selection) ------------
+constexpr int kMaxBlock = 64;
+
+// int8 code of one input value (the quantizer of the quant kinds)
+template <int KIND>
+__device__ __forceinline__ int quant_code(uint32_t raw, float scale) {
+  const int qi = __float2int_rn(__fmul_rn(raw_to_f32<KIND>(raw), scale));
+  return min(127, max(-127, qi));
+}
+
+// ent[j] = the block key of feature j*NT + tid: the largest |x| bits (f32 /
+// bf16) or the largest |q| (quant kinds, each row quantized with its own
+// gamma, which is also published) over rows [t0, t1).  s_bscale gets 127/gamma.
 template <int KIND, int NT, int EPT>
+__device__ __forceinline__ void block_keys(const TopkArgs& a, int t0, int t1, uint32_t (&ent)[EPT],
+                                           uint32_t* s_wred, float* s_bscale) {
+  constexpr bool QUANT = (KIND == TK_QUANT_F32 || KIND == TK_QUANT_BF16);
+  constexpr uint32_t MASK = KeyTraits<KIND>::kMask;
+  constexpr int NW = NT / 32;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int d = a.d;
+#pragma unroll
+  for (int j = 0; j < EPT; ++j) ent[j] = 0u;
+  for (int t = t0; t < t1; ++t) {
+    const size_t rb = (size_t)t * d;
+    if constexpr (QUANT) {
+      uint32_t raw[EPT];
+      uint32_t m = 0;
+#pragma unroll
+      for (int j = 0; j < EPT; ++j) {
+        const int e = j * NT + tid;
+        raw[j] = e < d ? load_raw<KIND>(a.x, rb + e) : 0u;
+        m = max(m, raw_abs_f32bits<KIND>(raw[j]));
+      }
+      m = __reduce_max_sync(kFull, m);
+      if (lane == 0) s_wred[warp] = m;
+      __syncthreads();
+      const uint32_t amax_bits = __reduce_max_sync(kFull, lane < NW ? s_wred[lane] : 0u);
+      const float gamma = __fadd_rn(__uint_as_float(amax_bits), a.eps);
+      const float scale = __fdiv_rn(127.0f, gamma);
+      if (tid == 0) {
+        if (a.gamma) a.gamma[t] = gamma;
+        s_bscale[t - t0] = scale;
+      }
+#pragma unroll
+      for (int j = 0; j < EPT; ++j) {
+        const int qi = quant_code<KIND>(raw[j], scale);
+        ent[j] = max(ent[j], (uint32_t)(qi < 0 ? -qi : qi));
+      }
+      __syncthreads();                               // s_wred is reused by the next row
+    } else {
+#pragma unroll
+      for (int j = 0; j < EPT; ++j) {
+        const int e = j * NT + tid;
+        if (e < d) ent[j] = max(ent[j], load_raw<KIND>(a.x, rb + e) & MASK);
+      }
+    }
+  }
+  __syncthreads();                                   // s_bscale visible to every thread
+}
+
+// Outputs of feature e for every row of the block (kept or not): idx / val at
+// list position `pos`, mask, X_sparse, the dense masked copies, the codes.
+template <int KIND>
+__device__ __forceinline__ void block_outputs(const TopkArgs& a, int t0, int t1, int e, bool sel,
+                                              int pos, const float* s_bscale) {
+  constexpr bool QUANT = (KIND == TK_QUANT_F32 || KIND == TK_QUANT_BF16);
+  const int d = a.d, k = a.k;
+  for (int t = t0; t < t1; ++t) {
+    const size_t o = (size_t)t * d + e;
+    const uint32_t raw = load_raw<KIND>(a.x, o);
+    if (sel && pos < k) {
+      const size_t oi = (size_t)t * k + pos;
+      if (a.idx) a.idx[oi] = e;
+      if (a.val) {
+        if constexpr (KIND == TK_F32) reinterpret_cast<uint32_t*>(a.val)[oi] = raw;
+        else if constexpr (KIND == TK_BF16) reinterpret_cast<uint16_t*>(a.val)[oi] = (uint16_t)raw;
+      }
+    }
+    if (a.mask) a.mask[o] = sel ? 1 : 0;
+    if constexpr (QUANT) {
+      const int qi = quant_code<KIND>(raw, s_bscale[t - t0]);
+      if (a.q_full) a.q_full[o] = (int8_t)qi;
+      if (a.xq) a.xq[o] = sel ? (int8_t)qi : (int8_t)0;
+    } else {
+      const uint32_t v = sel ? raw : 0u;
+      if (a.xsf) a.xsf[o] = raw_to_f32<KIND>(v);
+      if (a.xs) {
+        if constexpr (KIND == TK_F32) reinterpret_cast<uint32_t*>(a.xs)[o] = v;
+        else reinterpret_cast<uint16_t*>(a.xs)[o] = (uint16_t)v;
+      }
+    }
+  }
+}
+
+template <int KIND, int NT, int EPT, bool BLOCK>
 __global__ void __launch_bounds__(NT) topk_reg_kernel(TopkArgs a) {
   using RK = RegKeys<KIND>;
   constexpr int NW = NT / 32;
@@ -803,20 +898,26 @@ __global__ void __launch_bounds__(NT) topk_reg_kernel(TopkArgs a) {
   __shared__ uint32_t s_sel[3];
   __shared__ uint32_t s_scan[2 * (NW + 1)];
   __shared__ int s_last;
+  __shared__ float s_bscale[kMaxBlock];             // Block Q-Sparse, quant kinds: 127 / gamma_t
 
+  // One CTA per selection: a token row, or (Block Q-Sparse, a.block > 1) a
+  // block of a.block consecutive token rows that shares one selection.
   const int row = blockIdx.x;
   const int d = a.d;
   const int k = a.k;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const size_t rbase = (size_t)row * (size_t)d;
   const uint32_t lt = (1u << lane) - 1u;
+  const int blk = BLOCK ? a.block : 1;   // the per-row instantiation keeps no block code
+  const int nsel = (a.T + blk - 1) / blk;          // selection CTAs
+  const int t0 = row * blk, t1 = min(a.T, t0 + blk);
 
   pdl_begin();
-  if (row >= a.T) {
+  if (row >= nsel) {
     if (a.zero != nullptr) {
       const size_t nthr = (size_t)a.zero_ctas * NT;
       const float4 z = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-      for (size_t i = (size_t)(row - a.T) * NT + tid; i < a.zero_n / 4; i += nthr)
+      for (size_t i = (size_t)(row - nsel) * NT + tid; i < a.zero_n / 4; i += nthr)
         reinterpret_cast<float4*>(a.zero)[i] = z;
     }
     return;
@@ -825,12 +926,18 @@ __global__ void __launch_bounds__(NT) topk_reg_kernel(TopkArgs a) {
 
   // ---- 1. entries in registers ---------------------------------------------
   uint32_t ent[EPT];
+  if constexpr (BLOCK) {
+    // Block Q-Sparse: the key of feature e is the block magnitude, the
+    // largest |x| (or |q|) over the block's rows; values are read again below
+    block_keys<KIND, NT, EPT>(a, t0, t1, ent, s_wred, s_bscale);
+  } else {
 #pragma unroll
   for (int j = 0; j < EPT; ++j) {
     const int e = j * NT + tid;
     ent[j] = e < d ? load_raw<KIND>(a.x, rbase + e) : 0u;
   }
-  if constexpr (QUANT) {
+  }
+  if (QUANT && !BLOCK) {
     uint32_t m = 0;
 #pragma unroll
     for (int j = 0; j < EPT; ++j)
@@ -927,7 +1034,11 @@ __global__ void __launch_bounds__(NT) topk_reg_kernel(TopkArgs a) {
     const int eq_b = (int)(pre >> 16) + __popc(be & lt);
     const int eqnz_b = (int)s_cnz[j * NW + warp] + __popc(bz & lt);
     const bool sel = gt || (eq && eq_b < remaining);
-    if (sel) {
+    if constexpr (BLOCK) {
+      // Block Q-Sparse: every row of the block keeps the block's selection
+      if (sel && gt_b + min(eq_b, remaining) >= k) dev_fail(a.status, DEV_CHECK, 2, (uint32_t)row);
+      if (valid) block_outputs<KIND>(a, t0, t1, e, sel, gt_b + min(eq_b, remaining), s_bscale);
+    } else if (sel) {
       const int pos = gt_b + min(eq_b, remaining);
       if (pos < k) {
         const size_t o = (size_t)row * (size_t)k + (size_t)pos;
@@ -949,7 +1060,7 @@ __global__ void __launch_bounds__(NT) topk_reg_kernel(TopkArgs a) {
         }
       }
     }
-    if (valid) {
+    if (valid && !BLOCK) {
       const uint32_t v = sel ? ent[j] : 0u;
       if (a.mask) a.mask[rbase + e] = sel ? 1 : 0;
       if constexpr (QUANT) {
@@ -977,7 +1088,7 @@ __global__ void __launch_bounds__(NT) topk_reg_kernel(TopkArgs a) {
     __shared__ uint32_t s_upre[NT];
     __threadfence();
     __syncthreads();
-    if (tid == 0) s_last = (atomicAdd(a.ticket, 1) == a.T - 1);
+    if (tid == 0) s_last = (atomicAdd(a.ticket, 1) == nsel - 1);
     __syncthreads();
     if (!s_last) return;
     __threadfence();
@@ -1080,8 +1191,13 @@ __global__ void __launch_bounds__(NT) topk_dense_bf16_kernel(TopkArgs a) {
   }
 }
 
+int selections(const TopkArgs& a) {
+  const int b = a.block > 1 ? a.block : 1;
+  return (a.T + b - 1) / b;
+}
+
 bool dense_only_bf16(const TopkArgs& a) {
-  return a.kind == TK_BF16 && a.xs != nullptr && a.idx == nullptr && a.val == nullptr &&
+  return a.block <= 1 && a.kind == TK_BF16 && a.xs != nullptr && a.idx == nullptr && a.val == nullptr &&
          a.mask == nullptr && a.xsf == nullptr && a.xq == nullptr && a.list == nullptr &&
          a.zero == nullptr && a.d <= 256 * 16 && (a.d % 8) == 0 &&
          ((uintptr_t)a.x & 15u) == 0 && ((uintptr_t)a.xs & 15u) == 0;
@@ -1091,7 +1207,7 @@ bool dense_only_bf16(const TopkArgs& a) {
 // its values and count (and gamma): the projection path's decode step.
 bool list_only(const TopkArgs& a) {
   const bool quant = a.kind == TK_QUANT_F32 || a.kind == TK_QUANT_BF16;
-  return a.T == 1 && a.list != nullptr && a.list_count != nullptr && a.idx == nullptr &&
+  return a.T == 1 && a.block <= 1 && a.list != nullptr && a.list_count != nullptr && a.idx == nullptr &&
          a.val == nullptr && a.mask == nullptr && a.xs == nullptr && a.xsf == nullptr &&
          a.xq == nullptr && a.q_full == nullptr &&
          (quant ? a.list_q != nullptr : a.list_val != nullptr);
@@ -1113,8 +1229,12 @@ cudaError_t launch_reg(const TopkArgs& a_in, cudaStream_t s) {
     e = launch_pdl(topk_list_kernel<KIND, NT, EPT>, dim3((a.d + NT - 1) / NT), dim3(NT), (size_t)0, s, a);
   } else if (list_only(a))
     e = launch_pdl(topk_list_kernel<KIND, NT, EPT>, dim3(1 + a.zero_ctas), dim3(NT), (size_t)0, s, a);
+  else if (a.block > 1)
+    e = launch_pdl(topk_reg_kernel<KIND, NT, EPT, true>, dim3(selections(a) + a.zero_ctas),
+                   dim3(NT), (size_t)0, s, a);
   else
-    e = launch_pdl(topk_reg_kernel<KIND, NT, EPT>, dim3(a.T + a.zero_ctas), dim3(NT), (size_t)0, s, a);
+    e = launch_pdl(topk_reg_kernel<KIND, NT, EPT, false>, dim3(selections(a) + a.zero_ctas),
+                   dim3(NT), (size_t)0, s, a);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -1122,7 +1242,7 @@ cudaError_t launch_reg(const TopkArgs& a_in, cudaStream_t s) {
 // Register-resident launch when the row fits (EPT <= 16); false otherwise.
 template <int KIND>
 bool try_launch_reg(const TopkArgs& a, cudaStream_t s, cudaError_t* err) {
-  if (a.T >= 2 * kNumSMs) {                      // many rows: 256-thread CTAs
+  if (selections(a) >= 2 * kNumSMs) {            // many rows: 256-thread CTAs
     if (KIND == TK_BF16 && dense_only_bf16(a)) {
       *err = launch_pdl(topk_dense_bf16_kernel<256>, dim3(a.T), dim3(256), (size_t)0, s, a);
       if (*err == cudaSuccess) *err = cudaGetLastError();
@@ -1181,6 +1301,8 @@ cudaError_t launch_nt(const TopkArgs& a, cudaStream_t s) {
 
 }  // namespace
 
+bool topk_block_supported(int d) { return d >= 1 && d <= 1024 * 16; }
+
 bool topk_bitmask_supported(int T, int d, int kind) {
   return T == 1 && d >= 1 && d <= 1024 * 16 && (kind == TK_F32 || kind == TK_BF16);
 }
@@ -1197,6 +1319,7 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t s) {
     default: return cudaErrorInvalidValue;
   }
   if (done) return err;
+  if (a.block > 1) return cudaErrorInvalidValue;   // block selections: rows of up to 16 K only
   // longer rows: the shared-memory kernel
   // Few rows: a full 1024-thread CTA per row keeps the latency down.  Many
   // rows (prefill): 256-thread CTAs so that several rows share an SM.
