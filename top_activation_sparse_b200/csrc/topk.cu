@@ -787,6 +787,7 @@ __global__ void __launch_bounds__(NT) topk_list_kernel(TopkArgs a) {
 
 // ---- Block Q-Sparse helpers (a block of rows shares one selection) ------------
 constexpr int kMaxBlock = 64;
+constexpr int kMaxBlockRow = 1024 * 16;          // features of a block-selected row
 
 // int8 code of one input value (the quantizer of the quant kinds)
 template <int KIND>
@@ -795,75 +796,124 @@ __device__ __forceinline__ int quant_code(uint32_t raw, float scale) {
   return min(127, max(-127, qi));
 }
 
-// ent[j] = the block key of feature j*NT + tid: the largest |x| bits (f32 /
-// bf16) or the largest |q| (quant kinds, each row quantized with its own
-// gamma, which is also published) over rows [t0, t1).  s_bscale gets 127/gamma.
-template <int KIND, int NT, int EPT>
-__device__ __forceinline__ void block_keys(const TopkArgs& a, int t0, int t1, uint32_t (&ent)[EPT],
-                                           uint32_t* s_wred, float* s_bscale) {
-  constexpr bool QUANT = (KIND == TK_QUANT_F32 || KIND == TK_QUANT_BF16);
-  constexpr uint32_t MASK = KeyTraits<KIND>::kMask;
-  constexpr int NW = NT / 32;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int d = a.d;
-#pragma unroll
-  for (int j = 0; j < EPT; ++j) ent[j] = 0u;
-  for (int t = t0; t < t1; ++t) {
-    const size_t rb = (size_t)t * d;
-    if constexpr (QUANT) {
-      uint32_t raw[EPT];
-      uint32_t m = 0;
-#pragma unroll
-      for (int j = 0; j < EPT; ++j) {
-        const int e = j * NT + tid;
-        raw[j] = e < d ? load_raw<KIND>(a.x, rb + e) : 0u;
-        m = max(m, raw_abs_f32bits<KIND>(raw[j]));
-      }
-      m = __reduce_max_sync(kFull, m);
-      if (lane == 0) s_wred[warp] = m;
-      __syncthreads();
-      const uint32_t amax_bits = __reduce_max_sync(kFull, lane < NW ? s_wred[lane] : 0u);
-      const float gamma = __fadd_rn(__uint_as_float(amax_bits), a.eps);
-      const float scale = __fdiv_rn(127.0f, gamma);
-      if (tid == 0) {
-        if (a.gamma) a.gamma[t] = gamma;
-        s_bscale[t - t0] = scale;
-      }
-#pragma unroll
-      for (int j = 0; j < EPT; ++j) {
-        const int qi = quant_code<KIND>(raw[j], scale);
-        ent[j] = max(ent[j], (uint32_t)(qi < 0 ? -qi : qi));
-      }
-      __syncthreads();                               // s_wred is reused by the next row
-    } else {
-#pragma unroll
-      for (int j = 0; j < EPT; ++j) {
-        const int e = j * NT + tid;
-        if (e < d) ent[j] = max(ent[j], load_raw<KIND>(a.x, rb + e) & MASK);
-      }
-    }
-  }
-  __syncthreads();                                   // s_bscale visible to every thread
+// Raw element e of a 16-byte vector q (VW elements of the input type).
+template <int KIND, int VW>
+__device__ __forceinline__ uint32_t vec_elem(const uint4& q, int e) {
+  const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+  if constexpr (KIND == TK_F32 || KIND == TK_QUANT_F32) return w[e];
+  else return (w[e >> 1] >> (16 * (e & 1))) & 0xffffu;
 }
 
-// Outputs of feature e for every row of the block (kept or not): idx / val at
-// list position `pos`, mask, X_sparse, the dense masked copies, the codes.
+// Elements per 16-byte vector of the input type.
+template <int KIND> constexpr int vec_width() {
+  return (KIND == TK_F32 || KIND == TK_QUANT_F32) ? 4 : 8;
+}
+
+// Vectors of the row and the vector width the block kernels use: 16-byte
+// vectors when the row pitch keeps them aligned, else single elements.
 template <int KIND>
-__device__ __forceinline__ void block_outputs(const TopkArgs& a, int t0, int t1, int e, bool sel,
-                                              int pos, const float* s_bscale) {
+__device__ __forceinline__ bool block_vectorized(int d) { return (d % vec_width<KIND>()) == 0; }
+
+// Quant kinds: 127 / gamma_t of every row of the block (one warp per row, its
+// lanes reading 16-byte vectors), published to a.gamma and s_bscale.
+template <int KIND, int NT>
+__device__ void block_scales(const TopkArgs& a, int t0, int t1, float* s_bscale) {
+  constexpr int V = vec_width<KIND>();
+  constexpr int NW = NT / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int d = a.d;
+  const bool vec = block_vectorized<KIND>(d);
+  for (int t = t0 + warp; t < t1; t += NW) {
+    uint32_t m = 0;
+    if (vec) {
+      const uint4* row = reinterpret_cast<const uint4*>(
+          reinterpret_cast<const unsigned char*>(a.x) + (size_t)t * d * (V == 4 ? 4 : 2));
+#pragma unroll 4
+      for (int v = lane; v < d / V; v += 32) {
+        const uint4 q = __ldg(row + v);
+#pragma unroll
+        for (int e = 0; e < V; ++e) m = max(m, raw_abs_f32bits<KIND>(vec_elem<KIND, V>(q, e)));
+      }
+    } else {
+      for (int e = lane; e < d; e += 32)
+        m = max(m, raw_abs_f32bits<KIND>(load_raw<KIND>(a.x, (size_t)t * d + e)));
+    }
+    m = __reduce_max_sync(kFull, m);
+    if (lane == 0) {
+      const float gamma = __fadd_rn(__uint_as_float(m), a.eps);
+      if (a.gamma) a.gamma[t] = gamma;
+      s_bscale[t - t0] = __fdiv_rn(127.0f, gamma);
+    }
+  }
+}
+
+// s_key[e] = the block key of feature e: the largest |x| bits (f32 / bf16) or
+// the largest |q| (quant kinds) over rows [t0, t1).  Threads take 16-byte
+// vectors of the row; when the row has fewer vectors than threads, groups of
+// threads take different rows and combine with a shared-memory maximum.
+template <int KIND, int NT>
+__device__ void block_keys(const TopkArgs& a, int t0, int t1, uint32_t* s_key, const float* s_bscale) {
   constexpr bool QUANT = (KIND == TK_QUANT_F32 || KIND == TK_QUANT_BF16);
-  const int d = a.d, k = a.k;
-  for (int t = t0; t < t1; ++t) {
-    const size_t o = (size_t)t * d + e;
-    const uint32_t raw = load_raw<KIND>(a.x, o);
-    if (sel && pos < k) {
-      const size_t oi = (size_t)t * k + pos;
-      if (a.idx) a.idx[oi] = e;
-      if (a.val) {
-        if constexpr (KIND == TK_F32) reinterpret_cast<uint32_t*>(a.val)[oi] = raw;
-        else if constexpr (KIND == TK_BF16) reinterpret_cast<uint16_t*>(a.val)[oi] = (uint16_t)raw;
+  constexpr uint32_t MASK = KeyTraits<KIND>::kMask;
+  constexpr int V = vec_width<KIND>();
+  const int tid = threadIdx.x;
+  const int d = a.d;
+  for (int e = tid; e < d; e += NT) s_key[e] = 0u;
+  __syncthreads();
+  auto key_of = [&](uint32_t raw, int t) -> uint32_t {
+    if constexpr (QUANT) {
+      const int qi = quant_code<KIND>(raw, s_bscale[t - t0]);
+      return (uint32_t)(qi < 0 ? -qi : qi);
+    } else {
+      return raw & MASK;
+    }
+  };
+  if (block_vectorized<KIND>(d)) {
+    const int nvec = d / V;
+    const int groups = nvec >= NT ? 1 : min(NT / nvec, t1 - t0);
+    const int g = tid / (nvec >= NT ? NT : nvec);
+    const int v0 = tid - g * (nvec >= NT ? NT : nvec);
+    if (g < groups) {
+      for (int v = v0; v < nvec; v += (nvec >= NT ? NT : nvec)) {
+        uint32_t k[V];
+#pragma unroll
+        for (int e = 0; e < V; ++e) k[e] = 0u;
+#pragma unroll 4
+        for (int t = t0 + g; t < t1; t += groups) {
+          const uint4 q = __ldg(reinterpret_cast<const uint4*>(
+              reinterpret_cast<const unsigned char*>(a.x) + ((size_t)t * d + (size_t)v * V) * (V == 4 ? 4 : 2)));
+#pragma unroll
+          for (int e = 0; e < V; ++e) k[e] = max(k[e], key_of(vec_elem<KIND, V>(q, e), t));
+        }
+#pragma unroll
+        for (int e = 0; e < V; ++e)
+          if (k[e] != 0u) atomicMax(&s_key[v * V + e], k[e]);
       }
     }
+  } else {
+    for (int e = tid; e < d; e += NT) {
+      uint32_t k = 0;
+      for (int t = t0; t < t1; ++t) k = max(k, key_of(load_raw<KIND>(a.x, (size_t)t * d + e), t));
+      s_key[e] = k;
+    }
+  }
+  __syncthreads();
+}
+
+// Every row's dense outputs of the block (mask, X_sparse, the masked copies,
+// the codes) in one flattened (row, vector) loop, from the selection bitmask
+// s_sel (bit e = feature e kept); then idx / val of rows t0+1.. from row t0's.
+template <int KIND, int NT>
+__device__ void block_outputs(const TopkArgs& a, int t0, int t1, const uint32_t* s_sel,
+                              const float* s_bscale) {
+  constexpr bool QUANT = (KIND == TK_QUANT_F32 || KIND == TK_QUANT_BF16);
+  constexpr int V = vec_width<KIND>();
+  const int tid = threadIdx.x;
+  const int d = a.d, k = a.k;
+  const bool dense = a.mask || a.xs || a.xsf || a.xq || a.q_full;
+  auto one = [&](int t, int e, uint32_t raw) {
+    const size_t o = (size_t)t * d + e;
+    const bool sel = (s_sel[e >> 5] >> (e & 31)) & 1u;
     if (a.mask) a.mask[o] = sel ? 1 : 0;
     if constexpr (QUANT) {
       const int qi = quant_code<KIND>(raw, s_bscale[t - t0]);
@@ -875,6 +925,82 @@ __device__ __forceinline__ void block_outputs(const TopkArgs& a, int t0, int t1,
       if (a.xs) {
         if constexpr (KIND == TK_F32) reinterpret_cast<uint32_t*>(a.xs)[o] = v;
         else reinterpret_cast<uint16_t*>(a.xs)[o] = (uint16_t)v;
+      }
+    }
+  };
+  if (dense) {
+    if (block_vectorized<KIND>(d)) {
+      const int nvec = d / V;
+      const int total = (t1 - t0) * nvec;
+#pragma unroll 2
+      for (int i = tid; i < total; i += NT) {
+        const int t = t0 + i / nvec, v = i - (i / nvec) * nvec;
+        const size_t o = (size_t)t * d + (size_t)v * V;
+        const uint4 q = __ldg(reinterpret_cast<const uint4*>(
+            reinterpret_cast<const unsigned char*>(a.x) + o * (V == 4 ? 4 : 2)));
+        const uint32_t bits = (s_sel[(v * V) >> 5] >> ((v * V) & 31)) & ((1u << V) - 1u);
+        // V elements at once: vector stores of every output (offsets are
+        // multiples of V, so byte outputs are V-byte aligned)
+        uint32_t m[V / 4] = {};                       // mask bytes
+        uint32_t c8[V / 4] = {}, z8[V / 4] = {};      // codes, masked codes
+        uint32_t w[4] = {};                           // masked raw values (input layout)
+        float f[V];
+#pragma unroll
+        for (int e = 0; e < V; ++e) {
+          const bool sel = (bits >> e) & 1u;
+          const uint32_t raw = vec_elem<KIND, V>(q, e);
+          m[e >> 2] |= (sel ? 1u : 0u) << (8 * (e & 3));
+          if constexpr (QUANT) {
+            const uint32_t qb = (uint32_t)(uint8_t)(int8_t)quant_code<KIND>(raw, s_bscale[t - t0]);
+            c8[e >> 2] |= qb << (8 * (e & 3));
+            if (sel) z8[e >> 2] |= qb << (8 * (e & 3));
+          } else {
+            const uint32_t vm = sel ? raw : 0u;
+            f[e] = raw_to_f32<KIND>(vm);
+            if constexpr (V == 4) w[e] = vm;
+            else w[e >> 1] |= vm << (16 * (e & 1));
+          }
+        }
+        if (a.mask) {
+          if constexpr (V == 8) *reinterpret_cast<uint2*>(a.mask + o) = make_uint2(m[0], m[1]);
+          else *reinterpret_cast<uint32_t*>(a.mask + o) = m[0];
+        }
+        if constexpr (QUANT) {
+          if constexpr (V == 8) {
+            if (a.q_full) *reinterpret_cast<uint2*>(a.q_full + o) = make_uint2(c8[0], c8[1]);
+            if (a.xq) *reinterpret_cast<uint2*>(a.xq + o) = make_uint2(z8[0], z8[1]);
+          } else {
+            if (a.q_full) *reinterpret_cast<uint32_t*>(a.q_full + o) = c8[0];
+            if (a.xq) *reinterpret_cast<uint32_t*>(a.xq + o) = z8[0];
+          }
+        } else {
+          if (a.xsf) {
+#pragma unroll
+            for (int c = 0; c < V / 4; ++c)
+              reinterpret_cast<float4*>(a.xsf + o)[c] = make_float4(f[4 * c], f[4 * c + 1], f[4 * c + 2], f[4 * c + 3]);
+          }
+          if (a.xs)
+            *reinterpret_cast<uint4*>(reinterpret_cast<unsigned char*>(a.xs) + o * (V == 4 ? 4 : 2)) =
+                make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      }
+    } else {
+      const int total = (t1 - t0) * d;
+      for (int i = tid; i < total; i += NT) {
+        const int t = t0 + i / d, e = i - (i / d) * d;
+        one(t, e, load_raw<KIND>(a.x, (size_t)t * d + e));
+      }
+    }
+  }
+  if (a.idx != nullptr && k > 0) {
+    for (int i = tid; i < (t1 - t0 - 1) * k; i += NT) {
+      const int t = t0 + 1 + i / k, p = i - (i / k) * k;
+      const int e = __ldcg(a.idx + (size_t)t0 * k + p);
+      a.idx[(size_t)t * k + p] = e;
+      if (a.val) {
+        const uint32_t raw = load_raw<KIND>(a.x, (size_t)t * d + e);
+        if constexpr (KIND == TK_F32) reinterpret_cast<uint32_t*>(a.val)[(size_t)t * k + p] = raw;
+        else if constexpr (KIND == TK_BF16) reinterpret_cast<uint16_t*>(a.val)[(size_t)t * k + p] = (uint16_t)raw;
       }
     }
   }
@@ -898,7 +1024,9 @@ __global__ void __launch_bounds__(NT) topk_reg_kernel(TopkArgs a) {
   __shared__ uint32_t s_sel[3];
   __shared__ uint32_t s_scan[2 * (NW + 1)];
   __shared__ int s_last;
-  __shared__ float s_bscale[kMaxBlock];             // Block Q-Sparse, quant kinds: 127 / gamma_t
+  __shared__ float s_bscale[BLOCK ? kMaxBlock : 1];           // Block Q-Sparse (quant): 127 / gamma_t
+  __shared__ uint32_t s_bsel[BLOCK ? kMaxBlockRow / 32 : 1]; // Block Q-Sparse: kept features
+  extern __shared__ uint32_t s_bkey[];                       // Block Q-Sparse: [d] block keys
 
   // One CTA per selection: a token row, or (Block Q-Sparse, a.block > 1) a
   // block of a.block consecutive token rows that shares one selection.
@@ -929,7 +1057,16 @@ __global__ void __launch_bounds__(NT) topk_reg_kernel(TopkArgs a) {
   if constexpr (BLOCK) {
     // Block Q-Sparse: the key of feature e is the block magnitude, the
     // largest |x| (or |q|) over the block's rows; values are read again below
-    block_keys<KIND, NT, EPT>(a, t0, t1, ent, s_wred, s_bscale);
+    if constexpr (QUANT) {
+      block_scales<KIND, NT>(a, t0, t1, s_bscale);
+      __syncthreads();
+    }
+    block_keys<KIND, NT>(a, t0, t1, s_bkey, s_bscale);
+#pragma unroll
+    for (int j = 0; j < EPT; ++j) {
+      const int e = j * NT + tid;
+      ent[j] = e < d ? s_bkey[e] : 0u;
+    }
   } else {
 #pragma unroll
   for (int j = 0; j < EPT; ++j) {
@@ -1035,9 +1172,24 @@ __global__ void __launch_bounds__(NT) topk_reg_kernel(TopkArgs a) {
     const int eqnz_b = (int)s_cnz[j * NW + warp] + __popc(bz & lt);
     const bool sel = gt || (eq && eq_b < remaining);
     if constexpr (BLOCK) {
-      // Block Q-Sparse: every row of the block keeps the block's selection
-      if (sel && gt_b + min(eq_b, remaining) >= k) dev_fail(a.status, DEV_CHECK, 2, (uint32_t)row);
-      if (valid) block_outputs<KIND>(a, t0, t1, e, sel, gt_b + min(eq_b, remaining), s_bscale);
+      // Block Q-Sparse: row t0's idx / val here, every row's other outputs
+      // after the loop from the selection bitmask
+      const uint32_t bs = __ballot_sync(kFull, sel);
+      if (lane == 0 && j * NT + warp * 32 < d) s_bsel[(j * NT + warp * 32) >> 5] = bs;
+      if (sel) {
+        const int pos = gt_b + min(eq_b, remaining);
+        if (pos < k) {
+          const size_t o = (size_t)t0 * k + pos;
+          if (a.idx) a.idx[o] = e;
+          if (a.val) {
+            const uint32_t raw = load_raw<KIND>(a.x, (size_t)t0 * d + e);
+            if constexpr (KIND == TK_F32) reinterpret_cast<uint32_t*>(a.val)[o] = raw;
+            else if constexpr (KIND == TK_BF16) reinterpret_cast<uint16_t*>(a.val)[o] = (uint16_t)raw;
+          }
+        } else {
+          dev_fail(a.status, DEV_CHECK, 2, (uint32_t)row);
+        }
+      }
     } else if (sel) {
       const int pos = gt_b + min(eq_b, remaining);
       if (pos < k) {
@@ -1077,6 +1229,11 @@ __global__ void __launch_bounds__(NT) topk_reg_kernel(TopkArgs a) {
       const uint32_t b = __ballot_sync(kFull, sel && key != 0u);
       if (lane == 0 && b != 0u) atomicOr(a.union_bits + (j * NT + warp * 32) / 32, b);
     }
+  }
+
+  if constexpr (BLOCK) {
+    __syncthreads();                                 // s_bsel and row t0's idx complete
+    block_outputs<KIND, NT>(a, t0, t1, s_bsel, s_bscale);
   }
 
   // ---- 4. union of the rows' kept nonzeros (several tokens) ------------------
@@ -1229,9 +1386,14 @@ cudaError_t launch_reg(const TopkArgs& a_in, cudaStream_t s) {
     e = launch_pdl(topk_list_kernel<KIND, NT, EPT>, dim3((a.d + NT - 1) / NT), dim3(NT), (size_t)0, s, a);
   } else if (list_only(a))
     e = launch_pdl(topk_list_kernel<KIND, NT, EPT>, dim3(1 + a.zero_ctas), dim3(NT), (size_t)0, s, a);
-  else if (a.block > 1)
+  else if (a.block > 1) {
+    // block keys in dynamic shared memory: 4 bytes per feature
+    static unsigned configured = 0;
+    e = ensure_smem_attr(topk_reg_kernel<KIND, NT, EPT, true>, kMaxBlockRow * 4, &configured);
+    if (e != cudaSuccess) return e;
     e = launch_pdl(topk_reg_kernel<KIND, NT, EPT, true>, dim3(selections(a) + a.zero_ctas),
-                   dim3(NT), (size_t)0, s, a);
+                   dim3(NT), (size_t)a.d * 4, s, a);
+  }
   else
     e = launch_pdl(topk_reg_kernel<KIND, NT, EPT, false>, dim3(selections(a) + a.zero_ctas),
                    dim3(NT), (size_t)0, s, a);
@@ -1301,7 +1463,7 @@ cudaError_t launch_nt(const TopkArgs& a, cudaStream_t s) {
 
 }  // namespace
 
-bool topk_block_supported(int d) { return d >= 1 && d <= 1024 * 16; }
+bool topk_block_supported(int d) { return d >= 1 && d <= kMaxBlockRow; }
 
 bool topk_bitmask_supported(int T, int d, int kind) {
   return T == 1 && d >= 1 && d <= 1024 * 16 && (kind == TK_F32 || kind == TK_BF16);
