@@ -64,6 +64,9 @@ def parse_args(argv=None):
                          "read only for open gates (qs_sparse_ffn_gate_first)")
     ap.add_argument("--block", type=int, default=1,
                     help="Block Q-Sparse: tokens sharing one top-K selection (1: per token)")
+    ap.add_argument("--backward", action="store_true",
+                    help="linear / prefill workloads: time the straight-through-estimator "
+                         "backward (grad_x and grad_wt) instead of the forward")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-seconds", type=float, default=120.0)
@@ -75,6 +78,8 @@ def parse_args(argv=None):
         ap.error("--warmup must be >= 3")
     if a.gate_first and workloads.WORKLOADS[a.workload].act != "drelu":
         ap.error("--gate-first needs a dReLU FFN workload")
+    if a.backward and workloads.WORKLOADS[a.workload].kind not in ("linear", "prefill"):
+        ap.error("--backward needs a linear or prefill workload")
     if not 1 <= a.block <= 64 or (a.block > 1 and a.gate_first):
         ap.error("--block must be 1..64 (and is not available with --gate-first)")
     if a.steps < 1:
@@ -285,6 +290,10 @@ def _workload_desc(args, T: int) -> str:
     if w.kind == "quant":
         return (f"{args.workload}: int8 x ternary sparse projection, T={T}, {w.d_in}->{w.d_out}, "
                 f"K={w.k}, packed 2-bit weights")
+    if getattr(args, "backward", False):
+        return (f"{args.workload}: straight-through-estimator backward of the sparse linear "
+                f"(grad_x = dY.W, grad_wt += X_sparse^T.dY), T={T}, {w.d_in}->{w.d_out}, K={w.k}, "
+                f"{w.dtype}")
     return f"{args.workload}: sparse linear, T={T}, {w.d_in}->{w.d_out}, K={w.k}, {w.dtype}"
 
 
@@ -467,6 +476,91 @@ def setup_linear(args, qs, torch, device, stream, rank):
     }
 
 
+def setup_backward(args, qs, torch, device, stream, rank):
+    """One straight-through-estimator backward of a sparse projection per step:
+    grad_x = dY . W (every weight row) and grad_wt += X_sparse^T . dY."""
+    w = workloads.WORKLOADS[args.workload]
+    T = args.batch
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    eb = 2 if w.dtype == "bf16" else 4
+    per_layer = w.d_in * w.d_out * (eb + 4)          # weights and their f32 gradient
+    n_layers = args.layers or max(2, math.ceil(2 * L2_BYTES / per_layer))
+    g = torch.Generator(device=device)
+    wts, gwts = [], []
+    for l in range(n_layers):
+        g.manual_seed(w.seed(0, 1 + l))
+        wts.append((torch.randn(w.d_in, w.d_out, generator=g, device=device) * (w.d_in ** -0.5)).to(tdt))
+        gwts.append(torch.zeros(w.d_in, w.d_out, dtype=torch.float32, device=device))
+    x = workloads.activations_device(w, T, device, salt=rank)
+    g.manual_seed(w.seed(T, 7))
+    gy = (torch.randn(T, w.d_out, generator=g, device=device) * 0.01).to(tdt)
+    gx = torch.empty(T, w.d_in, dtype=torch.float32, device=device)
+    ws = qs.new_workspace(qs.QS_OP_SPARSE_LINEAR, T, w.d_in, w.d_out, w.k, device)
+    sp = stream.cuda_stream
+    blk = args.block
+    fn = qs.lib().qs_sparse_linear_backward
+    dt = qs.QS_BF16 if w.dtype == "bf16" else qs.QS_F32
+
+    def c_args(l, ev, k=w.k):
+        return (x.data_ptr(), dt, T, w.d_in, w.d_out, k, blk, wts[l].data_ptr(), gy.data_ptr(),
+                gx.data_ptr(), gwts[l].data_ptr(), ws.data_ptr(), ws.numel(), sp)
+
+    for l in range(n_layers):             # every layer once: validation, steady state
+        assert fn(*c_args(l, None)) == 0
+    assert qs.qs_device_status(ws) == qs.QS_OK
+    tensor = w.dtype == "bf16" and T >= qs.QS_PREFILL_MIN_T
+    if tensor:
+        # algorithmic FLOPs: grad_x is dense (the estimator applies no mask),
+        # grad_wt counts the T*K kept entries only
+        work = 2.0 * T * w.d_in * w.d_out + 2.0 * T * w.k * w.d_out
+        extra = {"executed_flops": 4.0 * T * w.d_in * w.d_out}
+        bound, kernel = "tensor", "umma_gemm_kernel (tcgen05 grad_x and grad_wt GEMMs)"
+    else:
+        # rows of grad_wt read and written: the inputs some token kept (the
+        # library's own count for the last chunk of tokens)
+        rows_kept, _ = qs.qs_workspace_stats(ws, qs.QS_OP_SPARSE_LINEAR, T, w.d_in, w.d_out, w.k)
+        # algorithmic bytes: every row of W^T read once per 8 tokens, the kept
+        # rows of grad_wt read and written, dY read, grad_x written
+        groups = (T + 7) // 8
+        work = (groups * w.d_in * w.d_out * eb + rows_kept * w.d_out * 8 + T * w.d_out * eb
+                + T * w.d_in * 4)
+        extra = {"rows_kept": rows_kept}
+        bound, kernel = "hbm", "rowdot_kernel (grad_x) + rowaxpy_kernel (kept rows of grad_wt)"
+
+    def e2e_call(i, x_dev, y_dev):
+        qs.qs_sparse_linear_backward(x_dev, wts[i % n_layers], gy, w.k, grad_x=y_dev,
+                                     grad_wt=gwts[i % n_layers], ws=ws, block=blk)
+
+    def cpu_rate():
+        import oracle
+        xs = x.float().cpu().numpy()
+        wt0 = wts[0].float().cpu().numpy()
+        gy0 = gy.float().cpu().numpy()
+        rows_n = min(T, 8)
+        t0 = time.perf_counter()
+        n = 0
+        while n < 2 or time.perf_counter() - t0 < args.cpu_seconds:
+            oracle.sparse_linear_backward_ste(xs[:rows_n], wt0, w.k, gy0[:rows_n],
+                                              keep=oracle.block_topk_keep(xs[:rows_n], w.k, blk))
+            n += 1
+        dt_ = time.perf_counter() - t0
+        return {"value": round(n * rows_n / dt_, 3), "unit": UNIT, "cores": _threads_in_use(),
+                "kind": "oracle", "sample": f"{n} oracle backward calls of {rows_n} token(s), {dt_:.1f} s"}
+
+    return {
+        "fn": fn, "T": T, "n_layers": n_layers, "ws": ws, "x": x, "y": gx,
+        "args": c_args, "n_events": 0, "dense_args": None,
+        "phases": [], "dominant": None, "kernel": kernel,
+        "bound": bound, "dom_work": work, "layer_work": work, "extra": extra,
+        "desc": workload_desc(args, T),
+        "l2": f"inputs larger than L2: {n_layers} weight + gradient copies "
+              f"({n_layers * per_layer / 1e9:.2f} GB) rotated",
+        "e2e_call": e2e_call, "cpu_rate": cpu_rate, "e2e_inputs": [gy],
+        "launches": (3 if tensor else (1 + 2 * ((T + 63) // 64) + 2)), "dtype": w.dtype,
+        "profile": f"backward_{args.workload}_T{T}",
+    }
+
+
 def setup_quant(args, qs, torch, device, stream, rank):
     """BitNet b1.58 + Q-Sparse projection per step (int8 x packed ternary)."""
     w = workloads.WORKLOADS[args.workload]
@@ -559,6 +653,8 @@ def run_ours(args, rank, world, local):
     kind = workloads.WORKLOADS[args.workload].kind
     setup = {"ffn": setup_ffn, "linear": setup_linear, "prefill": setup_linear,
              "quant": setup_quant}[kind]
+    if args.backward:
+        setup = setup_backward
     c = setup(args, qs, torch, device, stream, rank)
     fn, T, n_layers = c["fn"], c["T"], c["n_layers"]
 
@@ -597,15 +693,19 @@ def run_ours(args, rank, world, local):
     # with CUDA events between the kernels of each step (they cost the launch
     # overlap, so they never run inside the timed region)
     names = c["phases"]
-    n_phase = 256
-    evs = [_mk_events(torch, stream, c["n_events"]) for _ in range(n_phase)]
-    torch.cuda.synchronize()
-    for i in range(n_phase):
-        run(c["args"](i % n_layers, evs[i][1]))
-    torch.cuda.synchronize()
-    ph = np.array([[e[0][p].elapsed_time(e[0][p + 1]) for p in range(len(names))] for e in evs])
-    ph_us = {n: round(float(v), 3) for n, v in zip(names, ph.mean(axis=0) * 1e3)}
-    dom_us = ph_us[c["dominant"]]
+    if c["n_events"] > 0:
+        n_phase = 256
+        evs = [_mk_events(torch, stream, c["n_events"]) for _ in range(n_phase)]
+        torch.cuda.synchronize()
+        for i in range(n_phase):
+            run(c["args"](i % n_layers, evs[i][1]))
+        torch.cuda.synchronize()
+        ph = np.array([[e[0][p].elapsed_time(e[0][p + 1]) for p in range(len(names))] for e in evs])
+        ph_us = {n: round(float(v), 3) for n, v in zip(names, ph.mean(axis=0) * 1e3)}
+        dom_us = ph_us[c["dominant"]]
+    else:                                 # one call is the dominant unit: the whole step
+        ph_us = {}
+        dom_us = ms / args.steps * 1e3
     peaks = load_peaks()
     if c["bound"] == "hbm":
         achieved = c["dom_work"] / (dom_us * 1e-6) / 1e9
@@ -637,9 +737,13 @@ def run_ours(args, rank, world, local):
     x_host = x.cpu().pin_memory()
     y_host = torch.empty(y.shape, dtype=y.dtype).pin_memory()
     x_dev = torch.empty_like(x)
+    # other per-step inputs (the backward's dY) are copied in from host too
+    extra_in = [(t, t.cpu().pin_memory()) for t in c.get("e2e_inputs", [])]
     n_e2e = max(1, min(args.steps, 5000))
     for i in range(args.warmup):
         x_dev.copy_(x_host, non_blocking=True)
+        for t_dev, t_host in extra_in:
+            t_dev.copy_(t_host, non_blocking=True)
         c["e2e_call"](i, x_dev, y)
         y_host.copy_(y, non_blocking=True)
     torch.cuda.synchronize()
@@ -649,6 +753,8 @@ def run_ours(args, rank, world, local):
     e0.record(stream)
     for i in range(n_e2e):
         x_dev.copy_(x_host, non_blocking=True)
+        for t_dev, t_host in extra_in:
+            t_dev.copy_(t_host, non_blocking=True)
         c["e2e_call"](i, x_dev, y)
         y_host.copy_(y, non_blocking=True)
     e1.record(stream)
@@ -662,7 +768,7 @@ def run_ours(args, rank, world, local):
         cpu = c["cpu_rate"]()
 
     chunks = (T + qs.QS_PREFILL_MIN_T - 1) // qs.QS_PREFILL_MIN_T
-    if c["launches"] == 2 and T >= qs.QS_PREFILL_MIN_T:
+    if (c["launches"] == 2 and T >= qs.QS_PREFILL_MIN_T) or args.backward:
         chunks = 1
     result = {
         "metric": METRIC,
@@ -699,7 +805,9 @@ def run_ours(args, rank, world, local):
         },
         "dense_same_kernels": dense,
         "e2e": {"value": round(e2e_value, 1), "unit": UNIT, "steps": n_e2e,
-                "h2d_bytes_per_step": int(x.numel() * x.element_size()),
+                "h2d_bytes_per_step": int(x.numel() * x.element_size()
+                                          + sum(t.numel() * t.element_size()
+                                                for t, _ in extra_in)),
                 "d2h_bytes_per_step": int(y.numel() * y.element_size())},
         "gpu_launches": c["launches"] * chunks * args.steps,
         "clocks": clk,
@@ -762,6 +870,14 @@ def run_reference(args, rank, world, local):
             q_, _ = oracle.absmax_quantize(x)
             oracle.quant_sparse_linear(x, t, alpha, w.k,
                                        keep=oracle.block_topk_keep(q_, w.k, args.block))
+    elif args.backward:
+        wt = workloads.weight_t(w.d_in, w.d_out, w.seed(0, 1), w.dtype)
+        gy = workloads.round_to_dtype(
+            workloads.normal_f32(workloads.rng(w.seed(T, 7)), (T, w.d_out), 0.01), w.dtype)
+
+        def step():
+            oracle.sparse_linear_backward_ste(x, wt, w.k, gy,
+                                              keep=oracle.block_topk_keep(x, w.k, args.block))
     else:
         wt = workloads.weight_t(w.d_in, w.d_out, w.seed(0, 1), w.dtype)
 

@@ -293,6 +293,36 @@ qs_status qs_block_quant_sparse_linear(const void* x, int dtype, int T, int d_in
                                        void* const* phase_events, void* ws, size_t ws_bytes,
                                        void* stream);
 
+/*
+ * qs_sparse_linear_backward -- gradients of Y = X_sparse . W^T under the
+ *   straight-through estimator.
+ *   Source: Q-Sparse news article, section "Top-K sparsification", the
+ *   straight-through-estimator paragraphs: top-K has a zero gradient almost
+ *   everywhere, so the gradient with respect to the sparsified input is used
+ *   unchanged as the gradient with respect to the input:
+ *     grad_x  = grad_y . W               [T, d_in]   (no mask applied)
+ *     grad_wt += X_sparse^T . grad_y     [d_in, d_out]
+ *   X_sparse is the forward's: top-K on |x| per token (block = 1) or per
+ *   block of tokens (Block Q-Sparse, block > 1), k kept.
+ *
+ *   x, dtype, T, d_in, d_out, k, block, wt: as qs_block_sparse_linear.
+ *   grad_y   [T, d_out] `dtype`: dL/dY.
+ *   grad_x   [T, d_in] f32 out, or NULL: overwritten.
+ *   grad_wt  [d_in, d_out] f32, or NULL: ACCUMULATED into.  Only rows of
+ *            inputs that some token kept with a nonzero value are read and
+ *            written; within them an element whose added sum is exactly zero
+ *            is left as it was.  Rows no token kept are never touched.
+ *   At least one of grad_x, grad_wt.  With bf16, T >= QS_PREFILL_MIN_T and
+ *   d_in, d_out multiples of 8, both run as tcgen05 GEMMs (bf16 operands, f32
+ *   accumulation); otherwise grad_x streams W^T once per 8 tokens and grad_wt
+ *   adds into the kept rows only.
+ *   ws       qs_workspace_size(QS_OP_SPARSE_LINEAR, T, d_in, d_out, k) bytes.
+ *   Errors: INVALID_ARG, ALIGNMENT, WORKSPACE, UNSUPPORTED, CUDA.
+ */
+qs_status qs_sparse_linear_backward(const void* x, int dtype, int T, int d_in, int d_out, int k,
+                                    int block, const void* wt, const void* grad_y, float* grad_x,
+                                    float* grad_wt, void* ws, size_t ws_bytes, void* stream);
+
 /* Bytes of workspace `op` needs for these sizes (0 if the sizes are invalid).
  * Arguments: QS_OP_TOPK_MASK (T, d, 0, k); QS_OP_SPARSE_LINEAR (T, d_in, d_out,
  * k); QS_OP_SPARSE_FFN and QS_OP_SPARSE_FFN_GATE_FIRST (T, d_model, d_ff, k_h);

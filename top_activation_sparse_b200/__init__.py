@@ -86,6 +86,8 @@ _SIGNATURES = {
                                  _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "qs_block_quant_sparse_linear": (_i, [_vp, _i, _i, _i, _i, _i, _i, _vp, _f, _f, _vp, _vp, _vp,
                                           _vp, _vp, _vp, _sz, _vp]),
+    "qs_sparse_linear_backward": (_i, [_vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _sz,
+                                       _vp]),
     "qs_sparse_linear_noalloc": (_i, [_vp, _i, _i, _i, _i, _i, _vp, _vp, _vp]),
     "qs_sparse_linear_noalloc_status": (_i, [_vp]),
     "qs_workspace_list": (_i, [_vp, _i, _i, _i, _i, _i, _i, _vp, _i, _vp, _vp, _vp]),
@@ -331,6 +333,35 @@ def qs_sparse_linear_noalloc(x: torch.Tensor, wt: torch.Tensor, k: int, y=None,
     return y
 
 
+class BackwardResult(NamedTuple):
+    grad_x: torch.Tensor | None
+    grad_wt: torch.Tensor | None
+
+
+def qs_sparse_linear_backward(x, wt, grad_y, k: int, grad_x=True, grad_wt=True, block: int = 1,
+                              ws=None, stream=None) -> BackwardResult:
+    """Straight-through-estimator gradients of Y = X_sparse . W^T:
+    grad_x = grad_y . W (f32, overwritten) and grad_wt += X_sparse^T . grad_y
+    (f32, accumulated into the kept rows only; True allocates zeros)."""
+    dev = _need_cuda(x, wt, grad_y)
+    T, d_in = x.shape
+    d_out = wt.shape[1]
+    if wt.shape[0] != d_in or wt.dtype != x.dtype or tuple(grad_y.shape) != (T, d_out) \
+            or grad_y.dtype != x.dtype:
+        raise ValueError("need wt [d_in, d_out] and grad_y [T, d_out] with x's dtype")
+    grad_x = _out(grad_x, (T, d_in), torch.float32, dev)
+    if grad_wt is True:
+        grad_wt = torch.zeros(d_in, d_out, dtype=torch.float32, device=dev)
+    grad_wt = _out(grad_wt, (d_in, d_out), torch.float32, dev)
+    _need_cuda(grad_x, grad_wt)
+    ws = _workspace(ws, QS_OP_SPARSE_LINEAR, T, d_in, d_out, k, dev)
+    _check("qs_sparse_linear_backward", lib().qs_sparse_linear_backward(
+        x.data_ptr(), _dtype_code(x), T, d_in, d_out, k, int(block), wt.data_ptr(),
+        grad_y.data_ptr(), _ptr(grad_x), _ptr(grad_wt), ws.data_ptr(), ws.numel(),
+        _stream_ptr(stream)))
+    return BackwardResult(grad_x, grad_wt)
+
+
 class FfnResult(NamedTuple):
     y: torch.Tensor
     h: torch.Tensor | None
@@ -459,4 +490,4 @@ def qs_ternary_pack(w: torch.Tensor, eps: float = 1e-5, wt_packed=None, alpha_ou
 
 __all__ = [n for n in dir() if n.startswith(("qs_", "QS_"))] + [
     "lib", "new_workspace", "header_functions", "QSError", "TopkResult", "FfnResult",
-    "QuantResult"]
+    "QuantResult", "BackwardResult"]

@@ -690,6 +690,86 @@ qs_status qs_block_quant_sparse_linear(const void* x, int dtype, int T, int d_in
                     phase_events, ws, ws_bytes, stream);
 }
 
+qs_status qs_sparse_linear_backward(const void* x, int dtype, int T, int d_in, int d_out, int k,
+                                    int block, const void* wt, const void* grad_y, float* grad_x,
+                                    float* grad_wt, void* ws, size_t ws_bytes, void* stream) {
+  WsLayout L;
+  qs_status st = qs::check_sparse_linear(x, dtype, T, d_in, d_out, k, wt, grad_y, ws, ws_bytes, &L);
+  if (st != QS_OK) return st;
+  if (block < 1 || block > QS_MAX_BLOCK || (grad_x == nullptr && grad_wt == nullptr))
+    return QS_ERR_INVALID_ARG;
+  if (block > 1 && !topk_block_supported(d_in)) return QS_ERR_UNSUPPORTED;
+  if (!aligned16(grad_x) || !aligned16(grad_wt)) return QS_ERR_ALIGNMENT;
+  WsView w{(unsigned char*)ws};
+  cudaStream_t s = (cudaStream_t)stream;
+  const int eb = elem_bytes(dtype);
+  const bool bf16 = dtype == QS_BF16;
+
+  // Many tokens: both gradients are dense contractions on the tensor cores.
+  if (bf16 && T >= QS_PREFILL_MIN_T && backward_gemm_supported(T, d_in, d_out) &&
+      prefill_supported(T, d_out, d_in)) {
+    BackwardGemmArgs g;
+    g.grad_y = reinterpret_cast<const __nv_bfloat16*>(grad_y);
+    g.wt = reinterpret_cast<const __nv_bfloat16*>(wt);
+    g.xs = w.at<__nv_bfloat16>(L.xs_bf16);
+    g.grad_x = grad_x; g.grad_wt = grad_wt;
+    g.T = T; g.d_in = d_in; g.d_out = d_out;
+    g.status = w.status();
+    if (grad_wt != nullptr) {
+      TopkArgs a;
+      a.x = x; a.T = T; a.d = d_in; a.k = k; a.kind = TK_BF16;
+      a.block = block;
+      a.xs = w.at<void>(L.xs_bf16);
+      a.status = w.status();
+      QS_TRY_CUDA(launch_topk(a, s));
+      QS_TRY_CUDA(launch_grad_wt_gemm(g, s));
+    }
+    if (grad_x != nullptr) QS_TRY_CUDA(launch_grad_x_gemm(g, s));
+    return QS_OK;
+  }
+
+  // Decode-size batches: dL/dX by streaming every row of W^T once; dL/dW^T
+  // by adding into the rows the top-K listed, chunk by chunk.
+  if (grad_wt != nullptr) {
+    const int chunk = chunk_tokens(block);
+    for (int t0 = 0; t0 < T; t0 += chunk) {
+      const int Tc = (T - t0) < chunk ? (T - t0) : chunk;
+      TopkArgs a;
+      a.x = (const unsigned char*)x + (size_t)t0 * d_in * eb;
+      a.T = Tc; a.d = d_in; a.k = k;
+      a.block = Tc > 1 ? block : 1;
+      a.kind = bf16 ? TK_BF16 : TK_F32;
+      a.xsf = Tc > 1 ? w.at<float>(L.xsf_x) : nullptr;
+      a.list = w.at<int32_t>(L.list_x);
+      a.list_val = Tc == 1 ? w.at<float>(L.lval_x) : nullptr;
+      a.list_count = w.at<int32_t>(L.cnt) + 0;
+      a.ticket = w.ticket(L, kTkTopkX);
+      a.union_bits = reinterpret_cast<uint32_t*>(w.ticket(L, kUnionX));
+      a.status = w.status();
+      QS_TRY_CUDA(launch_topk(a, s));
+      RowAxpyArgs r;
+      r.grad_y = (const unsigned char*)grad_y + (size_t)t0 * d_out * eb;
+      r.grad_wt = grad_wt;
+      r.list = a.list; r.list_count = a.list_count;
+      r.list_val = a.list_val; r.xsf = a.xsf;
+      r.T = Tc; r.d_in = d_in; r.d_out = d_out;
+      r.bf16 = bf16;
+      r.status = w.status();
+      QS_TRY_CUDA(launch_rowaxpy(r, s));
+    }
+  }
+  if (grad_x != nullptr) {
+    RowDotArgs r;
+    r.wt = wt; r.grad_y = grad_y; r.grad_x = grad_x;
+    r.T = T; r.d_in = d_in; r.d_out = d_out;
+    r.bf16 = bf16;
+    r.status = w.status();
+    r.plan = plan_rowdot(T, d_in, d_out, eb);
+    QS_TRY_CUDA(launch_rowdot(r, s));
+  }
+  return QS_OK;
+}
+
 qs_status qs_ternary_pack(const float* wmat, int d_out, int d_in, float eps, uint32_t* wt_packed,
                           float* alpha_out, void* ws, size_t ws_bytes, void* stream) {
   if (wmat == nullptr || wt_packed == nullptr || d_out < 16 || d_in < 1 || !(eps >= 0.0f))

@@ -23,6 +23,16 @@
 //   * every mbarrier wait is bounded: on a timeout the CTA records
 //     DEV_TIMEOUT, waits (bounded) for its own copies and MMAs in flight,
 //     frees its TMEM and returns.
+//
+// The same kernel serves the backward of the projection under the
+// straight-through estimator (Q-Sparse news article, section "Top-K
+// sparsification", STE paragraphs), through two compile-time choices: the
+// major-ness of each operand (K-major: the reduction index is contiguous in
+// memory; MN-major: the output index is) and the epilogue (bf16 store, f32
+// store, or f32 accumulate into an existing matrix):
+//   dL/dX   = dL/dY . W       A = dL/dY [T, d_out] K-major, B = W^T [d_in, d_out] K-major
+//   dL/dW^T = X_sparse^T . dL/dY   A = X_sparse [T, d_in] read MN-major,
+//                                  B = dL/dY [T, d_out] MN-major, added to dL/dW^T
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -44,15 +54,21 @@ constexpr int kThreads = 192;                        // warp 0 TMA, warp 1 MMA, 
 constexpr int kEpiThreads = 128;
 constexpr uint32_t kTmemCols = 512;                  // two 256-column accumulators
 
-// tcgen05 instruction descriptor, kind::f16: D f32, A bf16 (K-major),
-// B bf16 (MN-major), N = 256, M = 128.
-constexpr uint32_t kIdesc = (1u << 4)            // accumulator format: f32
-                          | (1u << 7)            // A format: bf16
-                          | (1u << 10)           // B format: bf16
-                          | (0u << 15)           // A major-ness: K
-                          | (1u << 16)           // B major-ness: MN
-                          | ((uint32_t)(BN >> 3) << 17)
-                          | ((uint32_t)(BM >> 4) << 24);
+// tcgen05 instruction descriptor, kind::f16: D f32, A and B bf16, N = 256,
+// M = 128; bits 15 / 16 select MN-major A / B.
+template <bool A_MN, bool B_MN>
+constexpr uint32_t idesc() {
+  return (1u << 4)                               // accumulator format: f32
+         | (1u << 7)                             // A format: bf16
+         | (1u << 10)                            // B format: bf16
+         | ((A_MN ? 1u : 0u) << 15)              // A major-ness
+         | ((B_MN ? 1u : 0u) << 16)              // B major-ness
+         | ((uint32_t)(BN >> 3) << 17)
+         | ((uint32_t)(BM >> 4) << 24);
+}
+
+// Epilogue kinds.
+enum Epi { EPI_BF16 = 0, EPI_F32 = 1, EPI_F32_ADD = 2 };
 
 // Shared-memory matrix descriptor (sm_100 version bits), 128-byte swizzle.
 __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
@@ -75,11 +91,11 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
 }
 
 __device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
-                                          uint32_t accumulate) {
+                                          uint32_t idesc_bits, uint32_t accumulate) {
   asm volatile(
       "{\n .reg .pred p;\n setp.ne.u32 p, %4, 0;\n"
       " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem_d),
-      "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate)
+      "l"(adesc), "l"(bdesc), "r"(idesc_bits), "r"(accumulate)
       : "memory");
 }
 
@@ -117,10 +133,12 @@ __device__ __forceinline__ uint32_t pack_bf16x2(uint32_t lo_f32, uint32_t hi_f32
          ((uint32_t)f32_to_bf16_bits(__uint_as_float(hi_f32)) << 16);
 }
 
+// out[M, N] (row pitch ldo elements) = A[M, K] . B[K, N]  (or out += that, EPI_F32_ADD)
+template <bool A_MN, bool B_MN, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
-    prefill_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
-                        const __grid_constant__ CUtensorMap map_b, __nv_bfloat16* __restrict__ y,
-                        int M, int N, int K, DevStatus* status) {
+    umma_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
+                     const __grid_constant__ CUtensorMap map_b, void* __restrict__ out, int ldo,
+                     int M, int N, int K, DevStatus* status) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   pdl_begin();
   __shared__ __align__(8) uint64_t s_full[kStages];
@@ -183,10 +201,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t sa = base + (uint32_t)(s * kStageBytes);
         const uint32_t sb = sa + kABytes;
         mbar_arrive_expect_tx(&s_full[s], (uint32_t)kStageBytes);
-        tma_load_2d(sa, &map_a, kb * BK, m0, &s_full[s]);
+        if constexpr (A_MN) {                    // two 64-row (M) x 64 (K) boxes
 #pragma unroll
-        for (int j = 0; j < BN / 64; ++j)
-          tma_load_2d(sb + j * kBBox, &map_b, n0 + 64 * j, kb * BK, &s_full[s]);
+          for (int j = 0; j < BM / 64; ++j)
+            tma_load_2d(sa + j * kBBox, &map_a, m0 + 64 * j, kb * BK, &s_full[s]);
+        } else {                                 // one 64 (K) x 128 (M) box
+          tma_load_2d(sa, &map_a, kb * BK, m0, &s_full[s]);
+        }
+        if constexpr (B_MN) {                    // four 64-column (N) x 64 (K) boxes
+#pragma unroll
+          for (int j = 0; j < BN / 64; ++j)
+            tma_load_2d(sb + j * kBBox, &map_b, n0 + 64 * j, kb * BK, &s_full[s]);
+        } else {                                 // one 64 (K) x 256 (N) box
+          tma_load_2d(sb, &map_b, kb * BK, n0, &s_full[s]);
+        }
       }
     }
     // on an abort, let the copies already issued land before the CTA exits
@@ -222,12 +250,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t sb = sa + kABytes;
 #pragma unroll
         for (int kk = 0; kk < BK / 16; ++kk) {
-          // A: K-major, 128-byte rows, 8-row groups 1 KB apart; K step = 32 bytes
-          const uint64_t ad = smem_desc(sa + kk * 32, 16, 1024);
-          // B: N-major, 128-byte K rows, 8-row groups 1 KB apart (SBO),
-          //    64-column boxes 8 KB apart (LBO); K step = 16 rows = 2 KB
-          const uint64_t bd = smem_desc(sb + kk * 2048, kBBox, 1024);
-          umma_bf16(acc, ad, bd, (kb > 0 || kk > 0) ? 1u : 0u);
+          // K-major operand: 128-byte rows, 8-row groups 1 KB apart; K step = 32 bytes.
+          // MN-major operand: 128-byte K rows, 8-row groups 1 KB apart (SBO),
+          //   64-element M/N boxes 8 KB apart (LBO); K step = 16 rows = 2 KB.
+          const uint64_t ad = A_MN ? smem_desc(sa + kk * 2048, kBBox, 1024) : smem_desc(sa + kk * 32, 16, 1024);
+          const uint64_t bd = B_MN ? smem_desc(sb + kk * 2048, kBBox, 1024) : smem_desc(sb + kk * 32, 16, 1024);
+          umma_bf16(acc, ad, bd, idesc<A_MN, B_MN>(), (kb > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(&s_empty[s]);          // frees the stage once these MMAs have read it
         issued = true;
@@ -260,16 +288,37 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t r[32];
         tmem_ld32(acc + (uint32_t)c, r);
         if (abort || row >= M) continue;
-        __nv_bfloat16* dst = y + (size_t)row * N + n0 + c;
+        if constexpr (EPI == EPI_BF16) {
+          __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(out) + (size_t)row * ldo + n0 + c;
 #pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          if (n0 + c + 8 * v + 8 > N) break;       // N is a multiple of 8
-          uint4 o;
-          o.x = pack_bf16x2(r[8 * v + 0], r[8 * v + 1]);
-          o.y = pack_bf16x2(r[8 * v + 2], r[8 * v + 3]);
-          o.z = pack_bf16x2(r[8 * v + 4], r[8 * v + 5]);
-          o.w = pack_bf16x2(r[8 * v + 6], r[8 * v + 7]);
-          *reinterpret_cast<uint4*>(dst + 8 * v) = o;
+          for (int v = 0; v < 4; ++v) {
+            if (n0 + c + 8 * v + 8 > N) break;     // N is a multiple of 8
+            uint4 o;
+            o.x = pack_bf16x2(r[8 * v + 0], r[8 * v + 1]);
+            o.y = pack_bf16x2(r[8 * v + 2], r[8 * v + 3]);
+            o.z = pack_bf16x2(r[8 * v + 4], r[8 * v + 5]);
+            o.w = pack_bf16x2(r[8 * v + 6], r[8 * v + 7]);
+            *reinterpret_cast<uint4*>(dst + 8 * v) = o;
+          }
+        } else {
+          float* dst = reinterpret_cast<float*>(out) + (size_t)row * ldo + n0 + c;
+#pragma unroll
+          for (int v = 0; v < 8; ++v) {
+            if (n0 + c + 4 * v + 4 > N) break;     // N is a multiple of 4
+            float4 o = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                                   __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
+            if constexpr (EPI == EPI_F32_ADD) {
+              // add into the existing values; a sum of exactly zero (no kept
+              // input in this row) leaves them untouched
+              if (o.x == 0.0f && o.y == 0.0f && o.z == 0.0f && o.w == 0.0f) continue;
+              const float4 p = *reinterpret_cast<const float4*>(dst + 4 * v);
+              if (o.x != 0.0f) o.x += p.x; else o.x = p.x;
+              if (o.y != 0.0f) o.y += p.y; else o.y = p.y;
+              if (o.z != 0.0f) o.z += p.z; else o.z = p.z;
+              if (o.w != 0.0f) o.w += p.w; else o.w = p.w;
+            }
+            *reinterpret_cast<float4*>(dst + 4 * v) = o;
+          }
         }
       }
       tc_fence_before();
@@ -321,6 +370,25 @@ bool prefill_supported(int M, int N, int K) {
   return M >= 1 && N >= 8 && K >= 8 && (N % 8) == 0 && (K % 8) == 0 && encode_fn() != nullptr;
 }
 
+namespace {
+
+template <bool A_MN, bool B_MN, int EPI>
+cudaError_t launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, void* out, int ldo, int M,
+                        int N, int K, DevStatus* status, cudaStream_t s) {
+  static unsigned configured = 0;
+  cudaError_t e = ensure_smem_attr(umma_gemm_kernel<A_MN, B_MN, EPI>, kSmemBytes, &configured);
+  if (e != cudaSuccess) return e;
+  // persistent: one CTA per SM, each walking tiles blockIdx.x + i * gridDim.x
+  const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+  dim3 grid(tiles < kNumSMs ? tiles : kNumSMs);
+  e = launch_pdl(umma_gemm_kernel<A_MN, B_MN, EPI>, grid, dim3(kThreads), (size_t)kSmemBytes, s, ma,
+                 mb, out, ldo, M, N, K, status);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+}  // namespace
+
 cudaError_t launch_prefill_gemm(const PrefillArgs& a, cudaStream_t s) {
   CUtensorMap ma, mb;
   // A = X_sparse [M, K] row-major: inner K, box 64 x 128
@@ -329,16 +397,38 @@ cudaError_t launch_prefill_gemm(const PrefillArgs& a, cudaStream_t s) {
   // B = W^T [K, N] row-major: inner N, box 64 (N) x 64 (K)
   if (!make_map(&mb, a.wt, (uint64_t)a.N, (uint64_t)a.K, (uint64_t)a.N * 2, 64, BK))
     return cudaErrorInvalidValue;
-  static unsigned configured = 0;
-  cudaError_t e = ensure_smem_attr(prefill_gemm_kernel, kSmemBytes, &configured);
-  if (e != cudaSuccess) return e;
-  // persistent: one CTA per SM, each walking tiles blockIdx.x + i * gridDim.x
-  const int tiles = ((a.M + BM - 1) / BM) * ((a.N + BN - 1) / BN);
-  dim3 grid(tiles < kNumSMs ? tiles : kNumSMs);
-  e = launch_pdl(prefill_gemm_kernel, grid, dim3(kThreads), (size_t)kSmemBytes, s, ma, mb, a.y, a.M,
-                 a.N, a.K, a.status);
-  if (e != cudaSuccess) return e;
-  return cudaGetLastError();
+  return launch_gemm<false, true, EPI_BF16>(ma, mb, a.y, a.N, a.M, a.N, a.K, a.status, s);
+}
+
+bool backward_gemm_supported(int T, int d_in, int d_out) {
+  return T >= 1 && d_in >= 8 && d_out >= 8 && (d_in % 8) == 0 && (d_out % 8) == 0 &&
+         encode_fn() != nullptr;
+}
+
+cudaError_t launch_grad_x_gemm(const BackwardGemmArgs& a, cudaStream_t s) {
+  // grad_x [T, d_in] = dL/dY [T, d_out] . (W^T [d_in, d_out])^T
+  CUtensorMap ma, mb;
+  // A = dL/dY: M = T rows, K = d_out contiguous (K-major), box 64 (K) x 128 (M)
+  if (!make_map(&ma, a.grad_y, (uint64_t)a.d_out, (uint64_t)a.T, (uint64_t)a.d_out * 2, BK, BM))
+    return cudaErrorInvalidValue;
+  // B = W^T: N = d_in rows, K = d_out contiguous (K-major), box 64 (K) x 256 (N)
+  if (!make_map(&mb, a.wt, (uint64_t)a.d_out, (uint64_t)a.d_in, (uint64_t)a.d_out * 2, BK, BN))
+    return cudaErrorInvalidValue;
+  return launch_gemm<false, false, EPI_F32>(ma, mb, a.grad_x, a.d_in, a.T, a.d_in, a.d_out,
+                                            a.status, s);
+}
+
+cudaError_t launch_grad_wt_gemm(const BackwardGemmArgs& a, cudaStream_t s) {
+  // grad_wt [d_in, d_out] += X_sparse^T [d_in, T] . dL/dY [T, d_out]
+  CUtensorMap ma, mb;
+  // A = X_sparse^T: M = d_in contiguous in X_sparse [T, d_in] (MN-major), K = T; box 64 x 64
+  if (!make_map(&ma, a.xs, (uint64_t)a.d_in, (uint64_t)a.T, (uint64_t)a.d_in * 2, 64, BK))
+    return cudaErrorInvalidValue;
+  // B = dL/dY [T, d_out]: N = d_out contiguous (MN-major), K = T; box 64 x 64
+  if (!make_map(&mb, a.grad_y, (uint64_t)a.d_out, (uint64_t)a.T, (uint64_t)a.d_out * 2, 64, BK))
+    return cudaErrorInvalidValue;
+  return launch_gemm<true, true, EPI_F32_ADD>(ma, mb, a.grad_wt, a.d_out, a.d_in, a.d_out, a.T,
+                                              a.status, s);
 }
 
 }  // namespace qs

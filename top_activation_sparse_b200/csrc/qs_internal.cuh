@@ -365,4 +365,57 @@ struct PrefillArgs {
 cudaError_t launch_prefill_gemm(const PrefillArgs& a, cudaStream_t s);
 bool prefill_supported(int M, int N, int K);
 
+// Backward of the projection under the straight-through estimator, on the
+// tensor cores (bf16 operands, f32 results).
+struct BackwardGemmArgs {
+  const __nv_bfloat16* grad_y = nullptr;  // [T, d_out]
+  const __nv_bfloat16* wt = nullptr;      // [d_in, d_out] (W^T)
+  const __nv_bfloat16* xs = nullptr;      // [T, d_in] X_sparse
+  float* grad_x = nullptr;                // [T, d_in] out
+  float* grad_wt = nullptr;               // [d_in, d_out] accumulated into
+  int T = 0, d_in = 0, d_out = 0;
+  DevStatus* status = nullptr;
+};
+bool backward_gemm_supported(int T, int d_in, int d_out);
+
+// Decode-size backward kernels (backward.cu).
+struct RowDotPlan {
+  int TT;          // tokens per pass (1, 2, 4, 8)
+  int groups;      // ceil(T / TT)
+  int n_ct;        // column tiles of W^T
+  int S;           // row splits
+  int vec_tile;    // 16-byte vectors per row segment
+  int threads;     // consumers (multiple of 32) + one producer warp
+  int rps;         // rows per ring stage
+  int nst;         // ring stages
+  size_t smem;
+};
+RowDotPlan plan_rowdot(int T, int d_in, int d_out, int elem_bytes);
+
+struct RowDotArgs {            // grad_x [T, d_in] = grad_y [T, d_out] . (W^T)^T
+  const void* wt = nullptr;    // [d_in, d_out]
+  const void* grad_y = nullptr;
+  float* grad_x = nullptr;     // zeroed, then added into, by launch_rowdot
+  int T = 0, d_in = 0, d_out = 0;
+  int bf16 = 1;
+  DevStatus* status = nullptr;
+  RowDotPlan plan{};
+};
+cudaError_t launch_rowdot(const RowDotArgs& a, cudaStream_t s);
+
+struct RowAxpyArgs {           // grad_wt[i, :] += sum_t xs[t, i] grad_y[t, :] for listed rows i
+  const void* grad_y = nullptr;
+  float* grad_wt = nullptr;
+  const int32_t* list = nullptr;
+  const int32_t* list_count = nullptr;
+  const float* list_val = nullptr;   // one token: the listed rows' values
+  const float* xsf = nullptr;        // several tokens: [T, d_in] dense masked values
+  int T = 0, d_in = 0, d_out = 0;
+  int bf16 = 1;
+  DevStatus* status = nullptr;
+};
+cudaError_t launch_rowaxpy(const RowAxpyArgs& a, cudaStream_t s);
+cudaError_t launch_grad_x_gemm(const BackwardGemmArgs& a, cudaStream_t s);
+cudaError_t launch_grad_wt_gemm(const BackwardGemmArgs& a, cudaStream_t s);
+
 }  // namespace qs
