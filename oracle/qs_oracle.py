@@ -41,7 +41,9 @@ What it computes, and where each step comes from:
   input is quantized before top-K, with a small epsilon that keeps a
   denominator away from zero, and 1-bit weights use alpha = mean|W| (both
   formulas lost).  Readings used (per-token absmax int8, ternary round-clip):
-  :func:`absmax_quantize`, :func:`ternary_quantize`, :func:`quant_sparse_linear`.
+  :func:`absmax_quantize`, :func:`ternary_quantize`, :func:`quant_sparse_linear`;
+  the quantized FFN layer built from them, with the gating in float32 steps:
+  :func:`ffn_hidden_f32`, :func:`quant_sparse_ffn`.
 
 Readings of what the pages leave open:
 
@@ -329,6 +331,53 @@ def quant_sparse_linear(x, t, alpha, k: int, eps: float = 1e-5,
     y = acc.astype(np.float32) * r[:, None]
     return {"q": q, "gamma": gamma, "keep": keep, "acc": acc, "r": r,
             "y": y.astype(np.float32)}
+
+
+def ffn_hidden_f32(u, g, act: str, b_up=None, b_gate=None) -> np.ndarray:
+    """The gating epilogue in float32 steps (each operation rounded to float32,
+    nearest-even, in this order), for the quantized FFN whose projections
+    produce float32:  relu2_glu: r = max(u, 0); h = (r * r) * g.
+    drelu: h = max(g + b_gate, 0) * max(u + b_up, 0)."""
+    u = np.asarray(u, dtype=np.float32)
+    g = np.asarray(g, dtype=np.float32)
+    if act == "relu2_glu":
+        r = np.maximum(u, np.float32(0.0))
+        return ((r * r).astype(np.float32) * g).astype(np.float32)
+    if act == "drelu":
+        bu = np.float32(0.0) if b_up is None else np.asarray(b_up, dtype=np.float32)
+        bg = np.float32(0.0) if b_gate is None else np.asarray(b_gate, dtype=np.float32)
+        a = np.maximum((g + bg).astype(np.float32), np.float32(0.0))
+        b = np.maximum((u + bu).astype(np.float32), np.float32(0.0))
+        return (a * b).astype(np.float32)
+    raise ValueError(f"unknown activation {act!r}")
+
+
+def quant_sparse_ffn(x, t_up, alpha_up, t_gate, alpha_gate, t_down, alpha_down, act: str,
+                     k_in: int, k_h: int, eps: float = 1e-5, b_up=None, b_gate=None,
+                     block: int = 1) -> dict:
+    """BitNet b1.58 + Q-Sparse FFN layer: every projection input is quantized
+    (per-token absmax int8) and sparsified (top-K on |q|) before an int8 x
+    ternary projection (Q-Sparse news article, Top-K section, quantized-model
+    paragraphs, applied to each linear projection as the aibase.com summary
+    says top-K is):
+      u = quant_sparse_linear(x, t_up), g = quant_sparse_linear(x, t_gate)
+          (one quantization and one selection of x shared by both)
+      h = ffn_hidden_f32(u, g)                    float32 steps
+      y = quant_sparse_linear(h, t_down, k_h)     (h quantized per token)
+    block > 1 selects with Block Q-Sparse on |q| (:func:`block_topk_keep`).
+    Every step is exact integer arithmetic or a fixed float32 step, so y is
+    defined bit for bit."""
+    q, _ = absmax_quantize(x, eps)
+    keep_x = block_topk_keep(q, k_in, block)
+    ru = quant_sparse_linear(x, t_up, alpha_up, k_in, eps, keep=keep_x)
+    rg = quant_sparse_linear(x, t_gate, alpha_gate, k_in, eps, keep=keep_x)
+    h = ffn_hidden_f32(ru["y"], rg["y"], act, b_up, b_gate)
+    qh, _ = absmax_quantize(h, eps)
+    keep_h = block_topk_keep(qh, k_h, block)
+    rd = quant_sparse_linear(h, t_down, alpha_down, k_h, eps, keep=keep_h)
+    return {"u": ru["y"], "g": rg["y"], "h": h, "keep_x": keep_x, "keep_h": keep_h,
+            "acc_u": ru["acc"], "acc_g": rg["acc"], "acc_down": rd["acc"], "q_h": rd["q"],
+            "y": rd["y"]}
 
 
 # --------------------------------------------------------------------------

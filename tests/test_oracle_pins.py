@@ -650,3 +650,98 @@ def test_block_ffn_bruteforce_tiny(act, seed):
     for t in range(T):
         hs = [r["h"][t, j] if j in kh[t] else 0.0 for j in range(dff)]
         assert np.allclose(r["y"][t], bf_matvec(hs, down.tolist()), rtol=1e-10, atol=1e-12)
+
+
+# ---------------------------------------------------------------- quantized FFN chain pins
+
+
+def test_ffn_hidden_f32_golden_hand():
+    g = load_golden("quant_ffn_hand.json")
+    c = g["relu2"]
+    assert oracle.ffn_hidden_f32(c["u"], c["g"], "relu2_glu").tolist() == c["h"]
+    c = g["drelu"]
+    assert oracle.ffn_hidden_f32(c["u"], c["g"], "drelu", b_up=c["b"], b_gate=c["b"]).tolist() == c["h"]
+    c = g["rounding"]
+    u = _f32_from_hex(c["u_bits"])
+    h = oracle.ffn_hidden_f32([u], [c["g"]], "relu2_glu")[0]
+    assert _hex(h) == c["h_bits"]
+    # the fp64 epilogue is different in the last bits here: the f32 steps are pinned
+    assert oracle.ffn_hidden([float(u)], [c["g"]], "relu2_glu")[0] != float(h)
+
+
+def _bf_quant_ffn(x, t_up, a_up, t_gate, a_gate, t_down, a_down, act, k_in, k_h, b, eps=1e-5):
+    """The quantized FFN by loops, every float32 step rounded by hand from an
+    exact rational (independent of numpy's float32 arithmetic)."""
+    from fractions import Fraction as Fr
+    eps32 = _rne_f32(Fr(np.float32(eps).item()))
+
+    def quant(row):
+        gamma = _rne_f32(Fr(max(abs(float(v)) for v in row)) + Fr(eps32))
+        s = _rne_f32(Fr(127) / Fr(gamma))
+        q = [max(-127, min(127, _rint_even(Fr(_rne_f32(Fr(float(v)) * Fr(s)))))) for v in row]
+        return q, gamma
+
+    def proj(q, gamma, keep, t, alpha):
+        r = _rne_f32(Fr(_rne_f32(Fr(float(alpha)) * Fr(gamma))) / 127)
+        out = []
+        for j in range(len(t)):
+            acc = sum(q[i] * int(t[j][i]) for i in keep)
+            out.append(_rne_f32(Fr(acc) * Fr(r)))
+        return out
+
+    ys = []
+    for row in x:
+        q, gamma = quant(row)
+        keep = bf_keep([abs(v) for v in q], k_in)
+        u = proj(q, gamma, keep, t_up, a_up)
+        gg = proj(q, gamma, keep, t_gate, a_gate)
+        h = []
+        for uj, gj in zip(u, gg):
+            if act == "relu2_glu":
+                r = max(uj, 0.0)
+                h.append(_rne_f32(Fr(_rne_f32(Fr(r) * Fr(r))) * Fr(gj)))
+            else:
+                ga = max(_rne_f32(Fr(gj) + Fr(float(np.float32(b)))), 0.0)
+                ua = max(_rne_f32(Fr(uj) + Fr(float(np.float32(b)))), 0.0)
+                h.append(_rne_f32(Fr(ga) * Fr(ua)))
+        qh, gh = quant(h)
+        keep_h = bf_keep([abs(v) for v in qh], k_h)
+        ys.append(proj(qh, gh, keep_h, t_down, a_down))
+    return np.array(ys, dtype=np.float32)
+
+
+@pytest.mark.parametrize("act", ["relu2_glu", "drelu"])
+@pytest.mark.parametrize("seed", range(4))
+def test_quant_ffn_bruteforce_bits(act, seed):
+    g = np.random.default_rng(900 + seed)
+    T, dm, dff = 3, 7, 9
+    x = (g.standard_normal((T, dm)) * 2).astype(np.float32)
+    x[0, 2] = 0.0
+    ts = [oracle.ternary_quantize(g.standard_normal(shape).astype(np.float32))
+          for shape in ((dff, dm), (dff, dm), (dm, dff))]
+    b = -0.1 if act == "drelu" else None
+    for k_in, k_h in ((4, 5), (dm, dff), (1, 2)):
+        r = oracle.quant_sparse_ffn(x, ts[0][0], ts[0][1], ts[1][0], ts[1][1], ts[2][0], ts[2][1],
+                                    act, k_in, k_h, b_up=b, b_gate=b)
+        bf = _bf_quant_ffn(x, ts[0][0], ts[0][1], ts[1][0], ts[1][1], ts[2][0], ts[2][1], act, k_in,
+                           k_h, b)
+        assert np.array_equal(r["y"].view(np.int32), bf.view(np.int32)), (act, k_in, k_h)
+
+
+def test_quant_ffn_invariants():
+    g = np.random.default_rng(990)
+    T, dm, dff = 4, 32, 48
+    x = g.standard_normal((T, dm)).astype(np.float32)
+    ts = [oracle.ternary_quantize(g.standard_normal(shape).astype(np.float32))
+          for shape in ((dff, dm), (dff, dm), (dm, dff))]
+    r = oracle.quant_sparse_ffn(x, ts[0][0], ts[0][1], ts[1][0], ts[1][1], ts[2][0], ts[2][1],
+                                "relu2_glu", 20, 10)
+    assert np.all(r["h"][r["u"] <= 0] == 0)                 # squared ReLU zeroes u <= 0
+    assert all(np.count_nonzero(r["q_h"][t][r["keep_h"][t]]) <= 10 for t in range(T))
+    rd = oracle.quant_sparse_ffn(x, ts[0][0], ts[0][1], ts[1][0], ts[1][1], ts[2][0], ts[2][1],
+                                 "drelu", 20, 10, b_up=-0.2, b_gate=-0.2)
+    assert np.all(rd["h"] >= 0) and np.all(rd["h"][(rd["g"] - np.float32(0.2)) <= 0] == 0)
+    # block = 1 equals the per-token chain; a block of all tokens shares one selection
+    rb = oracle.quant_sparse_ffn(x, ts[0][0], ts[0][1], ts[1][0], ts[1][1], ts[2][0], ts[2][1],
+                                 "relu2_glu", 20, 10, block=T)
+    assert all(np.array_equal(rb["keep_x"][t], rb["keep_x"][0]) for t in range(T))
