@@ -84,7 +84,8 @@ typedef enum qs_op {
   QS_OP_SPARSE_FFN = 2,
   QS_OP_QUANT_SPARSE_LINEAR = 3,
   QS_OP_TERNARY_PACK = 4,
-  QS_OP_SPARSE_FFN_GATE_FIRST = 5
+  QS_OP_SPARSE_FFN_GATE_FIRST = 5,
+  QS_OP_QUANT_SPARSE_FFN = 6
 } qs_op;
 
 /* Largest row length (d, d_in, d_ff) a top-K row may have: one CTA holds a
@@ -323,9 +324,44 @@ qs_status qs_sparse_linear_backward(const void* x, int dtype, int T, int d_in, i
                                     int block, const void* wt, const void* grad_y, float* grad_x,
                                     float* grad_wt, void* ws, size_t ws_bytes, void* stream);
 
+/*
+ * qs_quant_sparse_ffn -- BitNet b1.58 + Q-Sparse FFN layer: every projection
+ *   input is quantized per token and sparsified before an int8 x ternary
+ *   projection.
+ *   Sources: Q-Sparse news article, Top-K section, quantized-model paragraphs
+ *   (quantize before top-K; ternary weights scaled by mean|W|) and
+ *   feed-forward paragraph (squared ReLU, Hadamard product); aibase.com
+ *   summary (top-K on every linear projection); Turbo Sparse summary, Eq. 2
+ *   (dReLU).  Read as, each step exact integer arithmetic or a float32 step:
+ *     q_x = quantize(x) (as qs_quant_sparse_linear);  keep = topK(|q_x|, k_in)
+ *     u = int8 x ternary(q_x, up),  g = int8 x ternary(q_x, gate)   (float32)
+ *     relu2_glu: r = max(u, 0); h = (r * r) * g
+ *     drelu:     h = max(g + b_gate, 0) * max(u + b_up, 0)
+ *     q_h = quantize(h);  keep_h = topK(|q_h|, k_h);  y = int8 x ternary(q_h, down)
+ *   so y is defined bit for bit.  block > 1: Block Q-Sparse selections on |q_x|
+ *   and |q_h| (see qs_block_sparse_linear); block = 1 is per token.
+ *
+ *   x         [T, d_model] `dtype` (bf16 or f32).
+ *   wp_up, wp_gate  [d_model, d_ff/16] packed ternary W^T (qs_ternary_pack),
+ *             alpha_up, alpha_gate their scales.   wp_down [d_ff, d_model/16], alpha_down.
+ *   b_up, b_gate    [d_ff] f32 or NULL (dReLU only).
+ *   y         [T, d_model] f32 out.    h_out  [T, d_ff] f32 out or NULL.
+ *   phase_events  NULL or QS_FFN_PHASE_EVENTS events (as qs_sparse_ffn).
+ *   ws        qs_workspace_size(QS_OP_QUANT_SPARSE_FFN, T, d_model, d_ff, k_h) bytes.
+ *   d_model and d_ff must be multiples of 64; 127 * d_model and 127 * d_ff < 2^24.
+ *   Errors: INVALID_ARG, ALIGNMENT, WORKSPACE, UNSUPPORTED, CUDA.
+ */
+qs_status qs_quant_sparse_ffn(const void* x, int dtype, int T, int d_model, int d_ff, int act,
+                              int k_in, int k_h, int block, const uint32_t* wp_up, float alpha_up,
+                              const uint32_t* wp_gate, float alpha_gate, const uint32_t* wp_down,
+                              float alpha_down, float eps, const float* b_up, const float* b_gate,
+                              float* y, float* h_out, void* const* phase_events, void* ws,
+                              size_t ws_bytes, void* stream);
+
 /* Bytes of workspace `op` needs for these sizes (0 if the sizes are invalid).
  * Arguments: QS_OP_TOPK_MASK (T, d, 0, k); QS_OP_SPARSE_LINEAR (T, d_in, d_out,
- * k); QS_OP_SPARSE_FFN and QS_OP_SPARSE_FFN_GATE_FIRST (T, d_model, d_ff, k_h);
+ * k); QS_OP_SPARSE_FFN, QS_OP_SPARSE_FFN_GATE_FIRST and QS_OP_QUANT_SPARSE_FFN (T,
+ * d_model, d_ff, k_h);
  * QS_OP_QUANT_SPARSE_LINEAR (T, d_in, d_out, k); QS_OP_TERNARY_PACK (0, d_in,
  * d_out, 0).  The dtype does
  * not change the size, and a workspace of this size also serves calls with the
@@ -343,7 +379,7 @@ qs_status qs_device_status(void* ws, void* stream);
  * workspace and these sizes, how many weight rows its projections streamed:
  * rows[0] = distinct inputs with a kept nonzero value across the T tokens (the
  * rows of wt / wt_up / wt_gate read), rows[1] = the same for h (rows of
- * wt_down read; the two FFN ops only, else 0), and for
+ * wt_down read; the FFN ops only, else 0), and for
  * QS_OP_SPARSE_FFN_GATE_FIRST only (then `rows` holds 3) rows[2] = open gates
  * across the T tokens (the rows of w_up read).  These counts are the
  * algorithmic weight traffic: rows * row length * sizeof(weight). */
@@ -357,12 +393,13 @@ qs_status qs_workspace_stats(const void* ws, int op, int T, int d_in, int d_out,
  *   which  0: the projection input's list: the inputs with a kept nonzero
  *             value (rows of wt, wt_up / wt_gate or wt_packed that were read),
  *             ascending, the union over the tokens;
- *          1: (QS_OP_SPARSE_FFN, QS_OP_SPARSE_FFN_GATE_FIRST) the same for h
- *             (rows of wt_down read).
+ *          1: (QS_OP_SPARSE_FFN, QS_OP_SPARSE_FFN_GATE_FIRST,
+ *             QS_OP_QUANT_SPARSE_FFN) the same for h (rows of wt_down read).
  *   rows   host int32 [cap] out: the first min(count, cap) listed rows.
  *   vals   host out or NULL: for calls with one token (T == 1) the listed
  *          rows' values, in list order: float32 (the kept x, exactly as given;
- *          the kept h) or, for QS_OP_QUANT_SPARSE_LINEAR, the int8 codes q.
+ *          the kept h) or, for QS_OP_QUANT_SPARSE_LINEAR and
+ *          QS_OP_QUANT_SPARSE_FFN, the int8 codes.
  *          Must be NULL when T > 1 (several tokens keep dense masked values).
  *   count  host out: the number of listed rows.
  * Errors: INVALID_ARG (bad op/which/sizes, NULL rows/count, vals with T > 1),

@@ -41,6 +41,7 @@ QS_OP_SPARSE_FFN = 2
 QS_OP_QUANT_SPARSE_LINEAR = 3
 QS_OP_TERNARY_PACK = 4
 QS_OP_SPARSE_FFN_GATE_FIRST = 5
+QS_OP_QUANT_SPARSE_FFN = 6
 
 QS_FAULT_NONE = 0
 QS_FAULT_GATHER_NO_COPIES = 1
@@ -88,6 +89,8 @@ _SIGNATURES = {
                                           _vp, _vp, _vp, _sz, _vp]),
     "qs_sparse_linear_backward": (_i, [_vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _sz,
                                        _vp]),
+    "qs_quant_sparse_ffn": (_i, [_vp, _i, _i, _i, _i, _i, _i, _i, _i, _vp, _f, _vp, _f, _vp, _f,
+                                 _f, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "qs_sparse_linear_noalloc": (_i, [_vp, _i, _i, _i, _i, _i, _vp, _vp, _vp]),
     "qs_sparse_linear_noalloc_status": (_i, [_vp]),
     "qs_workspace_list": (_i, [_vp, _i, _i, _i, _i, _i, _i, _vp, _i, _vp, _vp, _vp]),
@@ -235,7 +238,8 @@ def qs_workspace_list(ws: torch.Tensor, op: int, T: int, d_in: int, d_out: int, 
     rows = np.zeros(max(cap, 1), dtype=np.int32)
     vals = None
     if values:
-        vals = np.zeros(max(cap, 1), dtype=np.int8 if op == QS_OP_QUANT_SPARSE_LINEAR else np.float32)
+        codes = op in (QS_OP_QUANT_SPARSE_LINEAR, QS_OP_QUANT_SPARSE_FFN)
+        vals = np.zeros(max(cap, 1), dtype=np.int8 if codes else np.float32)
     count = ctypes.c_int32(0)
     _check("qs_workspace_list", lib().qs_workspace_list(
         ws.data_ptr(), op, T, d_in, d_out, k, which, rows.ctypes.data, cap,
@@ -468,6 +472,39 @@ def qs_quant_sparse_linear(x, wt_packed, alpha: float, k: int, eps: float = 1e-5
     return QuantResult(y, acc, q, idx)
 
 
+class QuantFfnResult(NamedTuple):
+    y: torch.Tensor
+    h: torch.Tensor | None
+
+
+def qs_quant_sparse_ffn(x, wp_up, alpha_up: float, wp_gate, alpha_gate: float, wp_down,
+                        alpha_down: float, act, k_in: int, k_h: int, eps: float = 1e-5,
+                        b_up=None, b_gate=None, y=None, h_out=None, block: int = 1,
+                        phase_events=None, ws=None, stream=None) -> QuantFfnResult:
+    """BitNet b1.58 + Q-Sparse FFN layer: int8 x ternary up, gate and down
+    projections, each input quantized per token and top-K'd (wp_*: packed
+    ternary W^T from qs_ternary_pack)."""
+    dev = _need_cuda(x, wp_up, wp_gate, wp_down, b_up, b_gate)
+    T, d_model = x.shape
+    d_ff = wp_up.shape[1] * 16
+    for p_, shp in ((wp_up, (d_model, d_ff // 16)), (wp_gate, (d_model, d_ff // 16)),
+                    (wp_down, (d_ff, d_model // 16))):
+        if tuple(p_.shape) != shp or p_.dtype != torch.int32:
+            raise ValueError(f"packed weight must be {shp} int32")
+    act_code = _ACTS[act] if isinstance(act, str) else int(act)
+    y = _out(y if y is not None else True, (T, d_model), torch.float32, dev)
+    h_out = _out(h_out, (T, d_ff), torch.float32, dev)
+    _need_cuda(y, h_out)
+    ws = _workspace(ws, QS_OP_QUANT_SPARSE_FFN, T, d_model, d_ff, k_h, dev)
+    _check("qs_quant_sparse_ffn", lib().qs_quant_sparse_ffn(
+        x.data_ptr(), _dtype_code(x), T, d_model, d_ff, act_code, k_in, k_h, int(block),
+        wp_up.data_ptr(), float(alpha_up), wp_gate.data_ptr(), float(alpha_gate),
+        wp_down.data_ptr(), float(alpha_down), float(eps), _ptr(b_up), _ptr(b_gate),
+        y.data_ptr(), _ptr(h_out), _events(phase_events, QS_FFN_PHASE_EVENTS), ws.data_ptr(),
+        ws.numel(), _stream_ptr(stream)))
+    return QuantFfnResult(y, h_out)
+
+
 def qs_ternary_pack(w: torch.Tensor, eps: float = 1e-5, wt_packed=None, alpha_out=None, ws=None,
                     stream=None):
     """Ternary-quantize W [d_out, d_in] f32 and pack it input-major 2-bit.
@@ -490,4 +527,4 @@ def qs_ternary_pack(w: torch.Tensor, eps: float = 1e-5, wt_packed=None, alpha_ou
 
 __all__ = [n for n in dir() if n.startswith(("qs_", "QS_"))] + [
     "lib", "new_workspace", "header_functions", "QSError", "TopkResult", "FfnResult",
-    "QuantResult", "BackwardResult"]
+    "QuantResult", "BackwardResult", "QuantFfnResult"]

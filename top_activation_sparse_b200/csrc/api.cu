@@ -142,6 +142,27 @@ bool ws_layout(int op, int T, int d_in, int d_out, int k, WsLayout* L) {
       L->parts1 = take(L->parts1_elems * sizeof(float));
       break;
     }
+    case QS_OP_QUANT_SPARSE_FFN: {
+      if (T < 1 || d_in < 64 || d_out < 64 || d_in > QS_MAX_ROW || d_out > QS_MAX_ROW || k < 0 ||
+          k > d_out || (d_in % 64) != 0 || (d_out % 64) != 0)
+        return false;
+      L->xq = take((size_t)Tc * d_in);
+      L->gamma = take((size_t)Tc * sizeof(float));
+      L->list_x = take((size_t)d_in * sizeof(int32_t));
+      L->lval_x = take((size_t)d_in * Tc);
+      L->parts1_elems = max_qparts(d_out, d_in, d_in);
+      L->parts1 = take(L->parts1_elems * sizeof(float));
+      L->parts1b = take(L->parts1_elems * sizeof(float));
+      L->u = take((size_t)Tc * d_out * sizeof(float));
+      L->h = take((size_t)Tc * d_out * sizeof(float));
+      L->xq_h = take((size_t)Tc * d_out);
+      L->gamma_h = take((size_t)Tc * sizeof(float));
+      L->list_h = take((size_t)d_out * sizeof(int32_t));
+      L->lval_h = take((size_t)d_out * Tc);
+      L->parts2_elems = max_qparts(d_in, d_out, d_out);
+      L->parts2 = take(L->parts2_elems * sizeof(float));
+      break;
+    }
     case QS_OP_TERNARY_PACK:
       if (d_in < 1 || d_out < 16 || (d_out % 16) != 0) return false;
       L->alpha_parts = take(kPackSumBlocks * sizeof(double));
@@ -264,7 +285,8 @@ qs_status qs_workspace_stats(const void* ws, int op, int T, int d_in, int d_out,
   QS_TRY_CUDA(cudaMemcpyAsync(c, (const unsigned char*)ws + L.cnt, sizeof(c),
                               cudaMemcpyDeviceToHost, s));
   QS_TRY_CUDA(cudaStreamSynchronize(s));
-  const bool ffn = op == QS_OP_SPARSE_FFN || op == QS_OP_SPARSE_FFN_GATE_FIRST;
+  const bool ffn = op == QS_OP_SPARSE_FFN || op == QS_OP_SPARSE_FFN_GATE_FIRST ||
+                   op == QS_OP_QUANT_SPARSE_FFN;
   rows[0] = c[0];
   rows[1] = ffn ? c[1] : 0;
   if (op == QS_OP_SPARSE_FFN_GATE_FIRST) rows[2] = c[2];
@@ -274,7 +296,8 @@ qs_status qs_workspace_stats(const void* ws, int op, int T, int d_in, int d_out,
 qs_status qs_workspace_list(const void* ws, int op, int T, int d_in, int d_out, int k, int which,
                             int32_t* rows, int cap, void* vals, int32_t* count, void* stream) {
   if (ws == nullptr || rows == nullptr || count == nullptr || cap < 0) return QS_ERR_INVALID_ARG;
-  const bool ffn = op == QS_OP_SPARSE_FFN || op == QS_OP_SPARSE_FFN_GATE_FIRST;
+  const bool ffn = op == QS_OP_SPARSE_FFN || op == QS_OP_SPARSE_FFN_GATE_FIRST ||
+                   op == QS_OP_QUANT_SPARSE_FFN;
   if (!(op == QS_OP_SPARSE_LINEAR || op == QS_OP_QUANT_SPARSE_LINEAR || ffn)) return QS_ERR_INVALID_ARG;
   if (which != 0 && !(which == 1 && ffn)) return QS_ERR_INVALID_ARG;
   if (vals != nullptr && T != 1) return QS_ERR_INVALID_ARG;
@@ -294,7 +317,8 @@ qs_status qs_workspace_list(const void* ws, int op, int T, int d_in, int d_out, 
     QS_TRY_CUDA(cudaMemcpyAsync(rows, base + (which == 0 ? L.list_x : L.list_h),
                                 (size_t)m * sizeof(int32_t), cudaMemcpyDeviceToHost, s));
     if (vals != nullptr) {
-      const size_t vb = op == QS_OP_QUANT_SPARSE_LINEAR ? 1 : sizeof(float);
+      const bool codes = op == QS_OP_QUANT_SPARSE_LINEAR || op == QS_OP_QUANT_SPARSE_FFN;
+      const size_t vb = codes ? 1 : sizeof(float);
       QS_TRY_CUDA(cudaMemcpyAsync(vals, base + (which == 0 ? L.lval_x : L.lval_h), (size_t)m * vb,
                                   cudaMemcpyDeviceToHost, s));
     }
@@ -766,6 +790,127 @@ qs_status qs_sparse_linear_backward(const void* x, int dtype, int T, int d_in, i
     r.status = w.status();
     r.plan = plan_rowdot(T, d_in, d_out, eb);
     QS_TRY_CUDA(launch_rowdot(r, s));
+  }
+  return QS_OK;
+}
+
+qs_status qs_quant_sparse_ffn(const void* x, int dtype, int T, int d_model, int d_ff, int act,
+                              int k_in, int k_h, int block, const uint32_t* wp_up, float alpha_up,
+                              const uint32_t* wp_gate, float alpha_gate, const uint32_t* wp_down,
+                              float alpha_down, float eps, const float* b_up, const float* b_gate,
+                              float* y, float* h_out, void* const* phase_events, void* ws,
+                              size_t ws_bytes, void* stream) {
+  if (!valid_dtype(dtype) || x == nullptr || wp_up == nullptr || wp_gate == nullptr ||
+      wp_down == nullptr || y == nullptr || T < 1 || d_model < 1 || d_ff < 1 || k_in < 0 ||
+      k_in > d_model || k_h < 0 || k_h > d_ff || !(eps >= 0.0f) || !(alpha_up == alpha_up) ||
+      !(alpha_gate == alpha_gate) || !(alpha_down == alpha_down) ||
+      (act != QS_ACT_RELU2_GLU && act != QS_ACT_DRELU) || block < 1 || block > QS_MAX_BLOCK)
+    return QS_ERR_INVALID_ARG;
+  if (d_model > QS_MAX_ROW || d_ff > QS_MAX_ROW) return QS_ERR_UNSUPPORTED;
+  if (block > 1 && (!topk_block_supported(d_model) || !topk_block_supported(d_ff)))
+    return QS_ERR_UNSUPPORTED;
+  if (!qgemv_supported(d_model) || !qgemv_supported(d_ff) || !aligned16(x) || !aligned16(wp_up) ||
+      !aligned16(wp_gate) || !aligned16(wp_down) || !aligned16(y) || !aligned16(h_out) ||
+      !aligned16(b_up) || !aligned16(b_gate))
+    return QS_ERR_ALIGNMENT;
+  WsLayout L;
+  qs_status st = check_ws(QS_OP_QUANT_SPARSE_FFN, T, d_model, d_ff, k_h, ws, ws_bytes, &L);
+  if (st != QS_OK) return st;
+  WsView w{(unsigned char*)ws};
+  cudaStream_t s = (cudaStream_t)stream;
+  const int eb = elem_bytes(dtype);
+  auto mark = [&](int i) -> cudaError_t {
+    if (phase_events == nullptr) return cudaSuccess;
+    return cudaEventRecord((cudaEvent_t)phase_events[i], s);
+  };
+  const int chunk = chunk_tokens(block);
+  for (int t0 = 0; t0 < T; t0 += chunk) {
+    const int Tc = (T - t0) < chunk ? (T - t0) : chunk;
+    const bool timed = (t0 == 0);
+    const int blk = Tc > 1 ? block : 1;
+    if (timed) QS_TRY_CUDA(mark(0));
+    const GemvPlan p_up = plan_qgemv(Tc, d_ff, (int)rows_bound_blocks(Tc, d_model, k_in, blk));
+    const GemvPlan p_dn = plan_qgemv(Tc, d_model, (int)rows_bound_blocks(Tc, d_ff, k_h, blk));
+    if (!plan_fits(p_up, L.parts1_elems, 0) || !plan_fits(p_up, L.parts1_elems, p_up.tickets) ||
+        !plan_fits(p_dn, L.parts2_elems, 2 * p_up.tickets))
+      return QS_ERR_UNSUPPORTED;
+
+    // 1. quantize x, top-K on |q|
+    TopkArgs a;
+    a.x = (const unsigned char*)x + (size_t)t0 * d_model * eb;
+    a.T = Tc; a.d = d_model; a.k = k_in;
+    a.block = blk;
+    a.kind = dtype == QS_F32 ? TK_QUANT_F32 : TK_QUANT_BF16;
+    a.eps = eps;
+    a.xq = Tc > 1 ? w.at<int8_t>(L.xq) : nullptr;
+    a.gamma = w.at<float>(L.gamma);
+    a.list = w.at<int32_t>(L.list_x);
+    a.list_q = Tc == 1 ? w.at<int8_t>(L.lval_x) : nullptr;
+    a.list_count = w.at<int32_t>(L.cnt) + 0;
+    a.ticket = w.ticket(L, kTkTopkX);
+    a.union_bits = reinterpret_cast<uint32_t*>(w.ticket(L, kUnionX));
+    a.zero = w.at<float>(L.parts1);
+    a.zero_n = p_up.parts_elems;
+    a.status = w.status();
+    QS_TRY_CUDA(launch_topk(a, s));
+    if (timed) QS_TRY_CUDA(mark(1));
+
+    // 2. up projection -> u; 3. gate projection, its epilogue forms h from u
+    float* h = h_out ? h_out + (size_t)t0 * d_ff : w.at<float>(L.h);
+    QGemvArgs g;
+    g.wp = wp_up; g.d_in = d_model; g.d_out = d_ff; g.T = Tc;
+    g.gamma = a.gamma; g.alpha = alpha_up;
+    g.list = a.list; g.list_q = a.list_q; g.xq = a.xq; g.list_count = a.list_count;
+    g.parts = w.at<float>(L.parts1);
+    g.plan = p_up;
+    g.tickets = w.ticket(L, kTkGemv);
+    g.y = w.at<float>(L.u);
+    g.zero = w.at<float>(L.parts1b);
+    g.zero_n = p_up.parts_elems;
+    g.status = w.status();
+    QS_TRY_CUDA(launch_qgemv(g, s));
+    g.wp = wp_gate; g.alpha = alpha_gate;
+    g.parts = w.at<float>(L.parts1b);
+    g.tickets = w.ticket(L, kTkGemv + p_up.tickets);
+    g.gating = act == QS_ACT_RELU2_GLU ? 1 : 2;
+    g.gate_u = w.at<float>(L.u);
+    g.b_up = b_up; g.b_gate = b_gate;
+    g.y = h;
+    g.zero = nullptr; g.zero_n = 0;
+    QS_TRY_CUDA(launch_qgemv(g, s));
+    if (timed) QS_TRY_CUDA(mark(2));
+
+    // 4. quantize h, top-K on |q_h|
+    TopkArgs b;
+    b.x = h; b.T = Tc; b.d = d_ff; b.k = k_h;
+    b.block = blk;
+    b.kind = TK_QUANT_F32;
+    b.eps = eps;
+    b.xq = Tc > 1 ? w.at<int8_t>(L.xq_h) : nullptr;
+    b.gamma = w.at<float>(L.gamma_h);
+    b.list = w.at<int32_t>(L.list_h);
+    b.list_q = Tc == 1 ? w.at<int8_t>(L.lval_h) : nullptr;
+    b.list_count = w.at<int32_t>(L.cnt) + 1;
+    b.ticket = w.ticket(L, kTkTopkH);
+    b.union_bits = reinterpret_cast<uint32_t*>(w.ticket(L, kUnionH));
+    b.zero = w.at<float>(L.parts2);
+    b.zero_n = p_dn.parts_elems;
+    b.status = w.status();
+    QS_TRY_CUDA(launch_topk(b, s));
+    if (timed) QS_TRY_CUDA(mark(3));
+
+    // 5. down projection
+    QGemvArgs dn;
+    dn.wp = wp_down; dn.d_in = d_ff; dn.d_out = d_model; dn.T = Tc;
+    dn.gamma = b.gamma; dn.alpha = alpha_down;
+    dn.list = b.list; dn.list_q = b.list_q; dn.xq = b.xq; dn.list_count = b.list_count;
+    dn.parts = w.at<float>(L.parts2);
+    dn.plan = p_dn;
+    dn.tickets = w.ticket(L, kTkGemv + 2 * p_up.tickets);
+    dn.y = y + (size_t)t0 * d_model;
+    dn.status = w.status();
+    QS_TRY_CUDA(launch_qgemv(dn, s));
+    if (timed) QS_TRY_CUDA(mark(4));
   }
   return QS_OK;
 }

@@ -214,6 +214,10 @@ struct WsLayout {
   size_t list_h = 0;          // [d_ff] int32 (ffn)
   size_t lval_h = 0;          // [d_ff][T] f32 (ffn)
   size_t parts2 = 0;          // down-projection partials (ffn)
+  size_t parts1b = 0;         // gate-projection partials (quantized ffn)
+  size_t u = 0;               // [T, d_ff] f32 up projection (quantized ffn)
+  size_t xq_h = 0;            // [T, d_ff] int8 dense masked codes of h (quantized ffn)
+  size_t gamma_h = 0;         // [T] f32 (quantized ffn)
   size_t xs_bf16 = 0;         // [T, d_in] bf16 (prefill)
   size_t alpha_parts = 0;     // f64 partial sums (ternary pack)
   size_t alpha = 0;           // f32 (ternary pack)
@@ -332,6 +336,14 @@ struct QGemvArgs {
   int32_t* tickets = nullptr;
   float* y = nullptr;
   int32_t* acc = nullptr;
+  // the quantized FFN's gate projection: y receives h = act(u, this
+  // projection) in float32 steps instead of the projection itself
+  int gating = 0;                  // 0: plain, 1: ReLU(u)^2 * g, 2: ReLU(g + b_gate) * ReLU(u + b_up)
+  const float* gate_u = nullptr;   // [T, d_out] the up projection, read by the gating epilogue
+  const float* b_up = nullptr;
+  const float* b_gate = nullptr;
+  float* zero = nullptr;           // accumulators of the next launch: set to 0 here
+  size_t zero_n = 0;
   DevStatus* status = nullptr;
   GemvPlan plan{};
 };

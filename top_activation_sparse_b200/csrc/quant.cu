@@ -54,6 +54,28 @@ __device__ __forceinline__ void red_add_v4_f32(float* dst, float a0, float a1, f
                : "memory");
 }
 
+// The quantized FFN's gating, float32 steps in a fixed order (y is the gate
+// projection g of column `col`, u the up projection):
+//   1: r = max(u, 0); h = (r * r) * g        2: h = max(g + b_gate, 0) * max(u + b_up, 0)
+__device__ __forceinline__ float4 quant_gating(const QGemvArgs& a, size_t o, int col, float4 gv) {
+  const float4 uv = __ldcg(reinterpret_cast<const float4*>(a.gate_u + o));
+  const float us[4] = {uv.x, uv.y, uv.z, uv.w};
+  const float gs[4] = {gv.x, gv.y, gv.z, gv.w};
+  float hs[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    if (a.gating == 1) {
+      const float r = fmaxf(us[e], 0.0f);
+      hs[e] = __fmul_rn(__fmul_rn(r, r), gs[e]);
+    } else {
+      const float bu = a.b_up ? a.b_up[col + e] : 0.0f;
+      const float bg = a.b_gate ? a.b_gate[col + e] : 0.0f;
+      hs[e] = __fmul_rn(fmaxf(__fadd_rn(gs[e], bg), 0.0f), fmaxf(__fadd_rn(us[e], bu), 0.0f));
+    }
+  }
+  return make_float4(hs[0], hs[1], hs[2], hs[3]);
+}
+
 // codes (00 = 0, 01 = +1, 10 = -1) -> u = t + 1 (00, 01, 10 for -1, 0, +1)
 __device__ __forceinline__ uint32_t ternary_to_u(uint32_t w) {
   const uint32_t hi = (w << 1) & 0xAAAAAAAAu;              // +1 -> bit 1 of the field
@@ -97,6 +119,7 @@ __global__ void __launch_bounds__(QTune<TT>::kMaxConsumers + 32, 2) qgemv_kernel
   const int k0 = lp0 & 7;                                // its first pair inside that word
 
   pdl_begin();
+  grid_zero(a.zero, a.zero_n);
   const int n = min(max(*a.list_count, 0), d_in);
   const int r0 = (int)(((long long)n * s) / S);
   const int r1 = (int)(((long long)n * (s + 1)) / S);
@@ -303,9 +326,10 @@ __global__ void __launch_bounds__(QTune<TT>::kMaxConsumers + 32, 2) qgemv_kernel
             const int4 iv = make_int4(__float2int_rn(f.x), __float2int_rn(f.y), __float2int_rn(f.z),
                                       __float2int_rn(f.w));
             const size_t e = o + i * 16 + h * 8 + kk;
-            reinterpret_cast<float4*>(a.y + e)[0] =
-                make_float4(__fmul_rn(__int2float_rn(iv.x), r), __fmul_rn(__int2float_rn(iv.y), r),
-                            __fmul_rn(__int2float_rn(iv.z), r), __fmul_rn(__int2float_rn(iv.w), r));
+            float4 yv = make_float4(__fmul_rn(__int2float_rn(iv.x), r), __fmul_rn(__int2float_rn(iv.y), r),
+                                    __fmul_rn(__int2float_rn(iv.z), r), __fmul_rn(__int2float_rn(iv.w), r));
+            if (a.gating) yv = quant_gating(a, e, (int)(e - (size_t)tok * d_out), yv);
+            reinterpret_cast<float4*>(a.y + e)[0] = yv;
             if (a.acc) reinterpret_cast<int4*>(a.acc + e)[0] = iv;
           }
       }
@@ -381,6 +405,7 @@ __global__ void __launch_bounds__(kQmWarps * 32 + 32, 2) qgemv_mma_kernel(QGemvA
   const unsigned char* Wb = reinterpret_cast<const unsigned char*>(a.wp) + (size_t)cword * 4;
 
   pdl_begin();
+  grid_zero(a.zero, a.zero_n);
   const int n = min(max(*a.list_count, 0), d_in);
   const int r0 = (int)(((long long)n * s) / S);
   const int r1 = (int)(((long long)n * (s + 1)) / S);
@@ -562,9 +587,10 @@ __global__ void __launch_bounds__(kQmWarps * 32 + 32, 2) qgemv_mma_kernel(QGemvA
     const int4 iv = make_int4(__float2int_rn(v[0]), __float2int_rn(v[1]), __float2int_rn(v[2]),
                               __float2int_rn(v[3]));
     const size_t o = (size_t)tok * d_out + col;
-    reinterpret_cast<float4*>(a.y + o)[0] =
-        make_float4(__fmul_rn(__int2float_rn(iv.x), r), __fmul_rn(__int2float_rn(iv.y), r),
-                    __fmul_rn(__int2float_rn(iv.z), r), __fmul_rn(__int2float_rn(iv.w), r));
+    float4 yv = make_float4(__fmul_rn(__int2float_rn(iv.x), r), __fmul_rn(__int2float_rn(iv.y), r),
+                            __fmul_rn(__int2float_rn(iv.z), r), __fmul_rn(__int2float_rn(iv.w), r));
+    if (a.gating) yv = quant_gating(a, o, col, yv);
+    reinterpret_cast<float4*>(a.y + o)[0] = yv;
     if (a.acc) reinterpret_cast<int4*>(a.acc + o)[0] = iv;
   }
 }
