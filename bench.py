@@ -73,7 +73,7 @@ def parse_args(argv=None):
     a = ap.parse_args(argv)
     if a.batch <= 0:
         w = workloads.WORKLOADS[a.workload]
-        a.batch = 1 if w.kind in ("ffn", "quant") else w.batches[0]
+        a.batch = 1 if w.kind in ("ffn", "quant", "quant_ffn") else w.batches[0]
     if a.warmup < 3:
         ap.error("--warmup must be >= 3")
     if a.gate_first and workloads.WORKLOADS[a.workload].act != "drelu":
@@ -290,6 +290,9 @@ def _workload_desc(args, T: int) -> str:
     if w.kind == "quant":
         return (f"{args.workload}: int8 x ternary sparse projection, T={T}, {w.d_in}->{w.d_out}, "
                 f"K={w.k}, packed 2-bit weights")
+    if w.kind == "quant_ffn":
+        return (f"{args.workload}: int8 x ternary sparse FFN layer, d_model={w.d_in}, d_ff={w.d_out}, "
+                f"act={w.act}, K_x={w.k}, K_h={w.k_h}, packed 2-bit weights")
     if getattr(args, "backward", False):
         return (f"{args.workload}: straight-through-estimator backward of the sparse linear "
                 f"(grad_x = dY.W, grad_wt += X_sparse^T.dY), T={T}, {w.d_in}->{w.d_out}, K={w.k}, "
@@ -561,6 +564,92 @@ def setup_backward(args, qs, torch, device, stream, rank):
     }
 
 
+def setup_quant_ffn(args, qs, torch, device, stream, rank):
+    """One BitNet b1.58 + Q-Sparse FFN layer per step (int8 x packed ternary up,
+    gate and down, each input quantized and top-K'd)."""
+    w = workloads.WORKLOADS[args.workload]
+    T = args.batch
+    dm, dff = w.d_in, w.d_out
+    layer_bytes = 3 * dm * dff // 4
+    n_layers = args.layers or max(2, math.ceil(2 * L2_BYTES / layer_bytes))
+    g = torch.Generator(device=device)
+    layers = []
+    wsp = qs.new_workspace(qs.QS_OP_TERNARY_PACK, 0, max(dm, dff), max(dm, dff), 0, device)
+    for l in range(n_layers):
+        mats = []
+        for j, (o, i) in enumerate(((dff, dm), (dff, dm), (dm, dff))):
+            g.manual_seed(w.seed(0, 1 + 3 * l + j))
+            wf = torch.randn(o, i, generator=g, device=device) * (i ** -0.5)
+            p, a = qs.qs_ternary_pack(wf, 1e-5, ws=wsp)
+            mats.append((p, float(a.item())))
+            del wf
+        layers.append(mats)
+    x = workloads.activations_device(w, T, device, salt=rank)
+    y = torch.empty(T, dm, dtype=torch.float32, device=device)
+    ws = qs.new_workspace(qs.QS_OP_QUANT_SPARSE_FFN, T, dm, dff, w.k_h, device)
+    sp = stream.cuda_stream
+    blk = args.block
+    act = qs.QS_ACT_RELU2_GLU if w.act == "relu2_glu" else qs.QS_ACT_DRELU
+    fn = qs.lib().qs_quant_sparse_ffn
+    f = ctypes.c_float
+
+    def c_args(l, ev, kx=w.k, kh=w.k_h):
+        (pu, au), (pg, ag), (pd, ad) = layers[l]
+        return (x.data_ptr(), qs.QS_BF16, T, dm, dff, act, kx, kh, blk, pu.data_ptr(), f(au),
+                pg.data_ptr(), f(ag), pd.data_ptr(), f(ad), f(1e-5), None, None, y.data_ptr(),
+                None, ev, ws.data_ptr(), ws.numel(), sp)
+
+    rows = []
+    for l in range(n_layers):
+        assert fn(*c_args(l, None)) == 0
+        rows.append(qs.qs_workspace_stats(ws, qs.QS_OP_QUANT_SPARSE_FFN, T, dm, dff, w.k_h))
+    assert qs.qs_device_status(ws) == qs.QS_OK
+    rows_x = float(np.mean([r[0] for r in rows]))
+    rows_h = float(np.mean([r[1] for r in rows]))
+    # algorithmic bytes: packed rows of up and gate (kept x), of down (kept h),
+    # the staged (index, code) entries, u and h written and read (f32)
+    upgate = 2 * rows_x * dff // 4 + rows_x * (4 + T) + 3 * T * dff * 4
+    down = rows_h * dm // 4 + rows_h * (4 + T) + T * dm * 4
+    topk = T * dm * 2 + T * dff * 4
+
+    def e2e_call(i, x_dev, y_dev):
+        (pu, au), (pg, ag), (pd, ad) = layers[i % n_layers]
+        qs.qs_quant_sparse_ffn(x_dev, pu, au, pg, ag, pd, ad, w.act, w.k, w.k_h, y=y_dev, ws=ws,
+                               block=blk)
+
+    def cpu_rate():
+        import oracle
+        (pu, au), (pg, ag), (pd, ad) = layers[0]
+        ts = [oracle.ternary_unpack(p.cpu().numpy().view(np.uint32), d)
+              for p, d in ((pu, dff), (pg, dff), (pd, dm))]
+        xs = x.float().cpu().numpy()
+        rows_n = min(T, 8)
+        t0 = time.perf_counter()
+        n = 0
+        while n < 2 or time.perf_counter() - t0 < args.cpu_seconds:
+            oracle.quant_sparse_ffn(xs[:rows_n], ts[0], au, ts[1], ag, ts[2], ad, w.act, w.k, w.k_h,
+                                    block=blk)
+            n += 1
+        dt_ = time.perf_counter() - t0
+        return {"value": round(n * rows_n / dt_, 3), "unit": UNIT, "cores": _threads_in_use(),
+                "kind": "oracle", "sample": f"{n} whole-layer oracle calls of {rows_n} token(s), {dt_:.1f} s"}
+
+    return {
+        "fn": fn, "T": T, "n_layers": n_layers, "ws": ws, "x": x, "y": y,
+        "args": lambda l, ev: c_args(l, ev), "n_events": qs.QS_FFN_PHASE_EVENTS,
+        "dense_args": (lambda l: c_args(l, None, dm, dff)),
+        "phases": ["quant_topk_x", "upgate", "quant_topk_h", "down"], "dominant": "upgate",
+        "kernel": "qgemv (int8 x ternary up, then gate with the gating epilogue)",
+        "bound": "hbm", "dom_work": upgate, "layer_work": upgate + down + topk,
+        "extra": {"rows_streamed": {"x": rows_x, "h": rows_h}},
+        "desc": workload_desc(args, T),
+        "l2": (f"inputs larger than L2: {n_layers} independent packed layers "
+               f"({n_layers * layer_bytes / 1e9:.2f} GB) rotated per step"),
+        "e2e_call": e2e_call, "cpu_rate": cpu_rate, "launches": 5, "dtype": "int8",
+        "profile": f"qgemv_{args.workload}_T{T}",
+    }
+
+
 def setup_quant(args, qs, torch, device, stream, rank):
     """BitNet b1.58 + Q-Sparse projection per step (int8 x packed ternary)."""
     w = workloads.WORKLOADS[args.workload]
@@ -652,7 +741,7 @@ def run_ours(args, rank, world, local):
     stream = torch.cuda.current_stream(device)
     kind = workloads.WORKLOADS[args.workload].kind
     setup = {"ffn": setup_ffn, "linear": setup_linear, "prefill": setup_linear,
-             "quant": setup_quant}[kind]
+             "quant": setup_quant, "quant_ffn": setup_quant_ffn}[kind]
     if args.backward:
         setup = setup_backward
     c = setup(args, qs, torch, device, stream, rank)
@@ -863,6 +952,13 @@ def run_reference(args, rank, world, local):
         def step():
             oracle.sparse_ffn(x, up, gate, down, w.act, w.k, w.k_h, b_up=b, b_gate=b,
                               block=args.block)
+    elif w.kind == "quant_ffn":
+        tq = [oracle.ternary_quantize(workloads.weight_out_major(o, i, w.seed(0, 1 + j)))
+              for j, (o, i) in enumerate(((w.d_out, w.d_in), (w.d_out, w.d_in), (w.d_in, w.d_out)))]
+
+        def step():
+            oracle.quant_sparse_ffn(x, tq[0][0], tq[0][1], tq[1][0], tq[1][1], tq[2][0], tq[2][1],
+                                    w.act, w.k, w.k_h, block=args.block)
     elif w.kind == "quant":
         t, alpha = oracle.ternary_quantize(workloads.weight_out_major(w.d_out, w.d_in, w.seed(0, 1)))
 

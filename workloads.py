@@ -90,7 +90,7 @@ def round_to_dtype(a: np.ndarray, dtype: str) -> np.ndarray:
 class Workload:
     name: str
     index: int
-    kind: str                     # "linear" | "ffn" | "quant" | "prefill"
+    kind: str                     # "linear" | "ffn" | "quant" | "quant_ffn" | "prefill"
     dtype: str                    # "f32" | "bf16"
     d_in: int
     d_out: int
@@ -123,6 +123,11 @@ WORKLOADS = {
     "ffn_drelu_mistral7b": Workload("ffn_drelu_mistral7b", 3, "ffn", "bf16", 4096, 14336,
                                     4096, (1, 4), act="drelu", k_h=keep_count(0.1, 14336),
                                     bias=-0.8),
+    # BitNet b1.58 + Q-Sparse FFN layer (int8 x ternary up, gate, down), Llama-7B
+    # shape, squared-ReLU gating, 39% kept at both projection inputs.
+    "quant_ffn_llama7b": Workload("quant_ffn_llama7b", 5, "quant_ffn", "bf16", 4096, 11008,
+                                  keep_count(0.39, 4096), (1, 8, 32), act="relu2_glu",
+                                  k_h=keep_count(0.39, 11008)),
     # Prefill: 2048 tokens, 4096 -> 11008, 1% outlier channels x20, K = 2048.
     "prefill_bf16_2048": Workload("prefill_bf16_2048", 4, "prefill", "bf16", 4096, 11008,
                                   2048, (2048,), outlier_frac=0.01, outlier_scale=20.0),
