@@ -18,7 +18,8 @@ constexpr int kChunkT = QS_PREFILL_MIN_T;
 constexpr size_t kTicketBytes = 64 * 1024;       // fixed ticket region
 constexpr int kTicketCap = (int)(kTicketBytes / sizeof(int32_t));
 // fixed ticket slots
-constexpr int kTkTopkX = 0, kTkTopkH = 1, kTkAlpha = 2, kTkUpRows = 3, kTkGemv = 8;
+constexpr int kTkTopkX = 0, kTkTopkH = 1, kTkAlpha = 2, kTkUpRows = 3, kTkHCount = 4,
+              kTkDownDone = 5, kTkGemv = 8;
 // union bitmasks of the several-token path, and the open gates of the
 // gate-first FFN (zero between calls)
 constexpr int kTkGemvEnd = 4096;
@@ -523,8 +524,14 @@ static qs_status ffn_impl(int op, const void* x, int dtype, int T, int d_model, 
     // top-K on h starts from that bitmask (it clears it again)
     const bool h_bits = Tc == 1 && idx_h_out == nullptr && topk_bitmask_supported(Tc, d_ff, TK_F32);
     uint32_t* hbits = h_bits ? reinterpret_cast<uint32_t*>(w.ticket(L, kUnionH)) : nullptr;
+    // one token: the down projection may take its rows straight from h (see
+    // GemvArgs::hcount) when a split's index range fits its row staging
+    const bool h_range = h_bits && !gate_first && !p_dn.mma && p_dn.TT == 1 &&
+                         (d_ff + p_dn.S - 1) / p_dn.S <= p_dn.rcap;
+    int32_t* hcount = h_range ? w.ticket(L, kTkHCount) : nullptr;
     if (!gate_first) {
       g.hbits = hbits;
+      g.hcount = hcount;
       QS_TRY_CUDA(launch_gemv(g, s));
     } else {
       // 2a. the gate alone, through the dReLU epilogue: the gate sums sit in
@@ -579,6 +586,13 @@ static qs_status ffn_impl(int op, const void* x, int dtype, int T, int d_model, 
     dn.plan = p_dn;
     dn.tickets = gemv_tickets(w, L, 1, g.plan);
     dn.y = (unsigned char*)y + (size_t)t0 * d_model * eb;
+    if (h_range) {
+      dn.hcount = hcount;
+      dn.hsrc = h;
+      dn.k_sel = k_h;
+      dn.done = w.ticket(L, kTkDownDone);
+      dn.rows_out = w.at<int32_t>(L.cnt) + 1;
+    }
     dn.status = w.status();
     QS_TRY_CUDA(launch_gemv(dn, s));
     if (timed) QS_TRY_CUDA(mark(4));

@@ -114,6 +114,7 @@ __device__ __forceinline__ void epilogue(const GemvArgs& a, int tok, int col,
 #pragma unroll
       for (int e = 0; e < V; ++e) m |= (hv[e] != 0.0f ? 1u : 0u) << e;
       if (m != 0u) atomicOr(a.hbits + col / 32, m << (col % 32));
+      if (a.hcount != nullptr && m != 0u) atomicAdd(a.hcount, __popc(m));
     }
   }
 }
@@ -151,11 +152,31 @@ __global__ void __launch_bounds__(kMaxConsumers + 32, (TT <= 4) ? 2 : 1) gemv_ke
   const unsigned char* Wb = reinterpret_cast<const unsigned char*>(a.w[mat]) + cbyte;
   const int col = (ct * P.vec_tile + tid) * V;                            // this thread's columns
 
-  pdl_begin();
+  // The down projection of a one-token FFN (a.hcount): the launch before this
+  // one (the top-K on h) releases it only after waiting for the launch before
+  // that (the up/gate projection), so h and its nonzero count are complete
+  // here.  With at most k_sel nonzero h the kept rows are exactly the nonzero
+  // h: this CTA lists those of its own index range and streams them without
+  // waiting for the top-K's list (it still waits for the top-K before it
+  // finishes, so stream order holds for the next call).
+  bool hrange = false;
+  if (MODE == 0 && a.hcount != nullptr) {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    hrange = __ldcg(a.hcount) <= a.k_sel;
+    if (!hrange) asm volatile("griddepcontrol.wait;" ::: "memory");
+  } else {
+    pdl_begin();
+  }
   grid_zero(a.zero, a.zero_n);
-  const int n = min(max(*a.list_count, 0), d_in);
-  const int r0 = (int)(((long long)n * s) / S);
-  const int r1 = (int)(((long long)n * (s + 1)) / S);
+  int r0, r1;
+  if (hrange) {
+    r0 = (int)(((long long)d_in * s) / S);
+    r1 = (int)(((long long)d_in * (s + 1)) / S);
+  } else {
+    const int n = min(max(*a.list_count, 0), d_in);
+    r0 = (int)(((long long)n * s) / S);
+    r1 = (int)(((long long)n * (s + 1)) / S);
+  }
 
   if (tid == 0) {
     for (int i = 0; i < P.nst; ++i) {
@@ -166,6 +187,33 @@ __global__ void __launch_bounds__(kMaxConsumers + 32, (TT <= 4) ? 2 : 1) gemv_ke
     s_err = 0;
   }
   __syncthreads();
+  if (hrange) {
+    // the nonzero h of [r0, r1) in index order (r1 - r0 <= rcap, checked on the
+    // host): one ballot per warp, the warps' counts in shared memory
+    __shared__ int s_wcnt[(kMaxConsumers + 32) / 32];
+    const int nw = P.threads / 32;
+    const int len = r1 - r0;
+    int base = 0;
+    for (int c0 = 0; c0 < len; c0 += P.threads) {
+      const int i = c0 + tid;
+      const float v = i < len ? __ldcg(a.hsrc + r0 + i) : 0.0f;
+      const bool nz = v != 0.0f;
+      const unsigned b = __ballot_sync(0xffffffffu, nz);
+      if (lane == 0) s_wcnt[tid >> 5] = __popc(b);
+      __syncthreads();
+      int pre = base;
+      for (int w = 0; w < (tid >> 5); ++w) pre += s_wcnt[w];
+      if (nz) {
+        const int pos = pre + __popc(b & lanemask_lt());
+        s_rows[pos] = r0 + i;
+        s_vals[pos] = v;
+      }
+      for (int w = 0; w < nw; ++w) base += s_wcnt[w];
+      __syncthreads();
+    }
+    if (blockIdx.x == 0 && blockIdx.y == 0 && tid == 0 && a.rows_out) *a.rows_out = __ldcg(a.hcount);
+    r1 = r0 + base;                                // rows of this split's piece
+  }
 
   float acc[TT][V];
 #pragma unroll
@@ -176,7 +224,7 @@ __global__ void __launch_bounds__(kMaxConsumers + 32, (TT <= 4) ? 2 : 1) gemv_ke
   int gst = 0;                                   // stages issued so far (slot/phase)
   for (int pb = r0; pb < r1; pb += P.rcap) {
     const int np = min(P.rcap, r1 - pb);
-    for (int j = tid; j < np; j += P.threads) {
+    for (int j = tid; j < np && !hrange; j += P.threads) {
       int r = a.list[pb + j];
       const bool ok = (unsigned)r < (unsigned)d_in;
       if (!ok) {                                 // a corrupted list is reported, never followed
@@ -277,6 +325,16 @@ __global__ void __launch_bounds__(kMaxConsumers + 32, (TT <= 4) ? 2 : 1) gemv_ke
         for (int q = 0; q < V / 4; ++q)
           red_add_v4(dst + 4 * q, acc[t][4 * q], acc[t][4 * q + 1], acc[t][4 * q + 2], acc[t][4 * q + 3]);
       }
+    }
+  }
+  if (MODE == 0 && a.hcount != nullptr) {
+    if (hrange) asm volatile("griddepcontrol.wait;" ::: "memory");
+    // every CTA has read the nonzero count: the grid's last one clears it
+    __syncthreads();
+    if (tid == 0 &&
+        atomicAdd(a.done, 1) == (int)(gridDim.x * gridDim.y * gridDim.z) - 1) {
+      *a.hcount = 0;
+      *a.done = 0;
     }
   }
   if (direct) return;

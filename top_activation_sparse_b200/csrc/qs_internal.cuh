@@ -306,6 +306,17 @@ struct GemvArgs {
   float* zero = nullptr;       // accumulators of the next kernel: set to 0 here
   size_t zero_n = 0;
   uint32_t* hbits = nullptr;   // mode 1/2, one token: OR the bitmask of nonzero h in here
+  // One-token FFN, counter of the nonzero h (zero between calls):
+  //   mode 1/2 add their nonzero h to it;
+  //   mode 0 (the down projection) reads it: with at most k_sel nonzero h the
+  //   kept rows are exactly the nonzero h, so each CTA takes them from its own
+  //   index range of hsrc instead of waiting for the top-K's list.  The grid's
+  //   last CTA (done ticket) clears the counter.
+  int32_t* hcount = nullptr;
+  const float* hsrc = nullptr;
+  int k_sel = 0;
+  int32_t* done = nullptr;
+  int32_t* rows_out = nullptr;   // mode 0 from h: the number of rows streamed (workspace stats)
   DevStatus* status = nullptr;
   // failure-detection testing only (qs_debug_inject): the producer issues no
   // copies, and every wait of the launch gives up after wait_limit polls
