@@ -117,3 +117,25 @@ def test_quant_tensor_core_token_groups(T, k):
     t, alpha = oracle.ternary_quantize(W)
     x = workloads.round_to_dtype(workloads.normal_f32(workloads.rng(22 + T), (T, d_in)), "bf16")
     _check_quant(x, "bf16", t, alpha, oracle.ternary_pack(t), k)
+
+
+@pytest.mark.parametrize("T,d_in,d_out,k", [
+    (8, 304, 320, 100),       # rows not a multiple of 32, a 64-column last tile
+    (9, 112, 64, 111),        # 16-token padding, one short tile
+    (16, 512, 1088, 200),
+    (17, 1024, 256, 400),     # 32-token padding
+    (33, 2048, 4096, 800),    # 48-token padding
+    (64, 4096, 11008, 1597),  # 64 tokens at the 7B shape
+    (24, 608, 384, 0),        # K = 0: y = 0
+    (40, 608, 384, 608),      # K = d: every input
+])
+def test_quant_tcgen05_int8_kernel(T, d_in, d_out, k):
+    """8 to 64 tokens with per-token selections (d_in % 16 == 0) run the
+    tcgen05 kind::i8 kernel (every packed row streamed, int32 in tensor
+    memory): q, kept indices, acc and y bit-exact against the oracle."""
+    need_gpu()
+    W = workloads.weight_out_major(d_out, d_in, d_out + 3 * d_in)
+    t, alpha = oracle.ternary_quantize(W)
+    x = workloads.round_to_dtype(workloads.normal_f32(workloads.rng(T + d_in), (T, d_in)), "bf16")
+    x[T // 2] = 0.0                          # a zero token
+    _check_quant(x, "bf16", t, alpha, oracle.ternary_pack(t), k)

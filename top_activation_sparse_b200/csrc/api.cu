@@ -665,7 +665,11 @@ static qs_status quant_impl(const void* x, int dtype, int T, int d_in, int d_out
     a.ticket = w.ticket(L, kTkTopkX);
     a.union_bits = reinterpret_cast<uint32_t*>(w.ticket(L, kUnionX));
     a.status = w.status();
-    const GemvPlan qp = plan_qgemv(Tc, d_out, (int)rows_bound_blocks(Tc, d_in, k, a.block));
+    // 8 or more tokens with per-token selections: their union covers about
+    // every input, so the tensor-core kernel streams every packed row
+    const GemvPlan qp = (a.block == 1 && qgemv_tc_supported(Tc, d_in, d_out))
+                            ? plan_qgemv_tc(Tc, d_in, d_out)
+                            : plan_qgemv(Tc, d_out, (int)rows_bound_blocks(Tc, d_in, k, a.block));
     if (!plan_fits(qp, L.parts1_elems, 0)) return QS_ERR_UNSUPPORTED;
     a.zero = w.at<float>(L.parts1);
     a.zero_n = qp.parts_elems;
@@ -843,8 +847,12 @@ qs_status qs_quant_sparse_ffn(const void* x, int dtype, int T, int d_model, int 
     const bool timed = (t0 == 0);
     const int blk = Tc > 1 ? block : 1;
     if (timed) QS_TRY_CUDA(mark(0));
-    const GemvPlan p_up = plan_qgemv(Tc, d_ff, (int)rows_bound_blocks(Tc, d_model, k_in, blk));
-    const GemvPlan p_dn = plan_qgemv(Tc, d_model, (int)rows_bound_blocks(Tc, d_ff, k_h, blk));
+    const bool tc_up = blk == 1 && qgemv_tc_supported(Tc, d_model, d_ff);
+    const bool tc_dn = blk == 1 && qgemv_tc_supported(Tc, d_ff, d_model);
+    const GemvPlan p_up = tc_up ? plan_qgemv_tc(Tc, d_model, d_ff)
+                                : plan_qgemv(Tc, d_ff, (int)rows_bound_blocks(Tc, d_model, k_in, blk));
+    const GemvPlan p_dn = tc_dn ? plan_qgemv_tc(Tc, d_ff, d_model)
+                                : plan_qgemv(Tc, d_model, (int)rows_bound_blocks(Tc, d_ff, k_h, blk));
     if (!plan_fits(p_up, L.parts1_elems, 0) || !plan_fits(p_up, L.parts1_elems, p_up.tickets) ||
         !plan_fits(p_dn, L.parts2_elems, 2 * p_up.tickets))
       return QS_ERR_UNSUPPORTED;

@@ -1,0 +1,422 @@
+// int8 x ternary projection for 8 to 64 tokens on the 5th-generation tensor
+// cores (tcgen05.mma kind::i8, int32 accumulators in tensor memory).
+//
+// Source: Q-Sparse news article (zxwl-tech.com), Top-K section, paragraphs on
+// quantized models (BitNet b1.58 + Q-Sparse): int8 activation codes q (the
+// kept entries of each token, zero elsewhere) times ternary weights t, summed
+// exactly in int32: acc[t, j] = sum_i q[t, i] * t[i, j]; y = f32(acc) * r_t.
+//
+// With 8 or more tokens the union of the tokens' kept inputs covers about
+// every input (1 - 0.61^8 = 98% at 39% kept), so this kernel streams every
+// packed row of W^T in order (2-D TMA, no gather) and multiplies it with the
+// dense masked codes (zero where a token dropped the input):
+//   * a CTA owns 256 output columns (two MMAs of M = 128) and a range of
+//     rows; per step of 32 rows (the MMA's K) one TMA brings the 32 x 64-byte
+//     packed segment and one TMA the tokens' 32 codes each (K-major, 32-byte
+//     swizzle), into a ring of stages;
+//   * four decode warps expand the 2-bit codes (00 = 0, 01 = +1, 10 = -1) into
+//     int8 and write the two A tiles in the MN-major 128-byte-swizzled layout
+//     (each 32-row x 128-byte tile: row k holds columns 0..127, 16-byte chunk
+//     c of row k at chunk c ^ (k mod 8)), then make them visible to the tensor
+//     core (fence.proxy.async) and arrive on the stage's barrier;
+//   * one thread issues tcgen05.mma.cta_group::1.kind::i8 (s8 x s8 -> s32,
+//     M = 128, N = tokens rounded up to 16, K = 32) into two accumulators and
+//     frees the stage with tcgen05.commit;
+//   * the decode warps then read the accumulators (tcgen05.ld, one column per
+//     lane), add them exactly into the split sums (integers < 2^24 in f32),
+//     and the last CTA of the column range rescales y = f32(acc) * r_t.
+// Every wait is bounded; a timeout records DEV_TIMEOUT, lets the copies and
+// MMAs in flight finish and frees the tensor memory.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "qs_internal.cuh"
+
+namespace qs {
+namespace {
+
+constexpr int kTcBlocks = 2;                       // 128-column MMA blocks per CTA
+constexpr int kTcCols = 128 * kTcBlocks;           // output columns per CTA
+constexpr int kTcWords = kTcCols / 16;             // packed words per row segment (16)
+constexpr int kTcRows = 32;                        // rows per step (the MMA's K for int8)
+constexpr int kTcStages = 6;
+constexpr int kTcATile = kTcRows * 128;            // one 128-column A tile: 4 KB
+constexpr int kTcPacked = kTcRows * kTcWords * 4;  // 2 KB
+constexpr int kTcBMax = 64 * kTcRows;              // codes of up to 64 tokens: 2 KB
+constexpr int kTcStage = kTcBlocks * kTcATile + kTcPacked + kTcBMax;   // 12 KB (multiple of 1 KB)
+constexpr int kTcSmem = kTcStages * kTcStage + 1024;
+constexpr int kTcThreads = 192;                    // warp 0 TMA, warp 1 MMA, warps 2-5 decode + epilogue
+constexpr int kTcDecoders = 128;
+
+// instruction descriptor, kind::i8: D s32, A and B signed 8-bit, A MN-major,
+// B K-major, M = 128, N = NPAD
+template <int NPAD>
+constexpr uint32_t i8_idesc() {
+  return (2u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (0u << 16) |
+         ((uint32_t)(NPAD >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+}
+
+__device__ __forceinline__ uint64_t tc_smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo,
+                                                 uint32_t layout) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;                          // sm_100 descriptor version
+  d |= (uint64_t)layout << 61;
+  return d;
+}
+
+__device__ __forceinline__ void tc_tma_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_i8(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                        uint32_t idesc_bits, uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.u32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc_bits), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// 16 consecutive 32-bit accumulator columns of this warp's 32 TMEM lanes.
+__device__ __forceinline__ void tc_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+      "%12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void red_v4(float* dst, float a0, float a1, float a2, float a3) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(a0), "f"(a1),
+               "f"(a2), "f"(a3)
+               : "memory");
+}
+
+// 4 packed 2-bit codes (one byte) -> 4 int8 in a word: 00 -> 0, 01 -> +1, 10 -> -1
+__device__ __forceinline__ uint32_t codes4(uint32_t b) {
+  const uint32_t s = (b & 3u) | ((b & 0xCu) << 6) | ((b & 0x30u) << 12) | ((b & 0xC0u) << 18);
+  return s | (((s >> 1) & 0x01010101u) * 0xFFu);
+}
+
+template <int NPAD>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    qgemv_tc_kernel(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_q,
+                    QGemvArgs a) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  __shared__ __align__(8) uint64_t s_full[kTcStages];     // TMA -> decoders
+  __shared__ __align__(8) uint64_t s_dec[kTcStages];      // decoders -> MMA
+  __shared__ __align__(8) uint64_t s_empty[kTcStages];    // MMA (commit) -> TMA
+  __shared__ __align__(8) uint64_t s_accum;               // every MMA done -> epilogue
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_abort;
+  __shared__ int s_flag;
+  constexpr uint32_t kTmemCols = (kTcBlocks * NPAD) <= 32 ? 32 : ((kTcBlocks * NPAD) <= 64 ? 64 : 128);
+  constexpr int kBBytes = NPAD * kTcRows;
+
+  pdl_begin();
+  grid_zero(a.zero, a.zero_n);
+  const GemvPlan& P = a.plan;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ct = blockIdx.x, s = blockIdx.y;
+  const int d_in = a.d_in, d_out = a.d_out;
+  const int T = a.T;
+  const int col0 = ct * kTcCols;
+  // rows [r0, r1) of this split, in whole steps of 32
+  const int steps_all = (d_in + kTcRows - 1) / kTcRows;
+  const int st0 = (int)(((long long)steps_all * s) / P.S);
+  const int st1 = (int)(((long long)steps_all * (s + 1)) / P.S);
+  const int nsteps = st1 - st0;
+  const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kTcStages; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_dec[i], kTcDecoders);
+      mbar_init(&s_empty[i], 1);
+    }
+    mbar_init(&s_accum, 1);
+    mbar_fence_init();
+    s_abort = 0;
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&s_tmem)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_before();
+  __syncthreads();
+  tc_after();
+  const uint32_t tmem = s_tmem;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---- TMA producer ----
+      int it = 0;
+      for (; it < nsteps; ++it) {
+        const int sl = it % kTcStages;
+        if (it >= kTcStages && !mbar_wait(&s_empty[sl], (uint32_t)((it / kTcStages) - 1) & 1u)) {
+          dev_fail(a.status, DEV_TIMEOUT, 50, (uint32_t)it);
+          atomicExch(&s_abort, 1);
+          break;
+        }
+        if (*(volatile int*)&s_abort) break;
+        const uint32_t sp = base + (uint32_t)(sl * kTcStage) + kTcBlocks * kTcATile;
+        const uint32_t sq = sp + kTcPacked;
+        mbar_arrive_expect_tx(&s_full[sl], (uint32_t)(kTcPacked + kBBytes));
+        const int row = (st0 + it) * kTcRows;
+        tc_tma_2d(sp, &map_w, col0 / 16, row, &s_full[sl]);
+        tc_tma_2d(sq, &map_q, row, 0, &s_full[sl]);
+      }
+      // on an abort, let the copies already issued land
+      if (*(volatile int*)&s_abort) {
+        for (int i = 0; i < kTcStages && i < it; ++i) {
+          const int g = it - 1 - i;
+          mbar_wait(&s_full[g % kTcStages], (uint32_t)(g / kTcStages) & 1u);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---- MMA issuer ----
+      bool issued = false;
+      for (int it = 0; it < nsteps && !*(volatile int*)&s_abort; ++it) {
+        const int sl = it % kTcStages;
+        if (!mbar_wait(&s_dec[sl], (uint32_t)(it / kTcStages) & 1u)) {
+          dev_fail(a.status, DEV_TIMEOUT, 51, (uint32_t)it);
+          atomicExch(&s_abort, 1);
+          break;
+        }
+        tc_after();
+        const uint32_t sa = base + (uint32_t)(sl * kTcStage);
+        const uint32_t sq = sa + kTcBlocks * kTcATile + kTcPacked;
+        // B: K-major codes, 32-byte rows (one token each), 32-byte swizzle, 8-row groups 256 B apart
+        const uint64_t bd = tc_smem_desc(sq, 16, 256, 6);
+#pragma unroll
+        for (int b = 0; b < kTcBlocks; ++b) {
+          // A: MN-major, 128-byte rows (one input row each), 128-byte swizzle, 8-row groups 1 KB apart
+          const uint64_t ad = tc_smem_desc(sa + (uint32_t)(b * kTcATile), 16, 1024, 2);
+          umma_i8(tmem + (uint32_t)(b * NPAD), ad, bd, i8_idesc<NPAD>(), it > 0 ? 1u : 0u);
+        }
+        tc_commit(&s_empty[sl]);                   // frees the stage once these MMAs have read it
+        issued = true;
+      }
+      tc_commit(&s_accum);                         // the accumulators are complete (or abandoned)
+      if (!issued) {
+        // no MMA was issued: the commit above still arrives once nothing is pending
+      }
+    }
+  } else {
+    // ---- decoders: 2-bit codes -> int8 A tiles ----
+    const int dt = threadIdx.x - 64;               // 0..127
+    const int r = dt >> 2;                         // row of the step (0..31)
+    const int w0 = (dt & 3) * 4;                   // first of this thread's 4 words (0, 4, 8, 12)
+    const int blk = w0 >> 3;                       // A tile (columns 0..127 or 128..255)
+    for (int it = 0; it < nsteps; ++it) {
+      const int sl = it % kTcStages;
+      const bool ready = !*(volatile int*)&s_abort &&
+                         mbar_wait_backoff(&s_full[sl], (uint32_t)(it / kTcStages) & 1u);
+      if (!ready && !*(volatile int*)&s_abort) {
+        if (lane == 0) dev_fail(a.status, DEV_TIMEOUT, 52, (uint32_t)it);
+        atomicExch(&s_abort, 1);
+      }
+      if (ready) {
+        unsigned char* st = smem_raw + ((base - smem_u32(smem_raw)) + (uint32_t)(sl * kTcStage));
+        const uint4 pw = *reinterpret_cast<const uint4*>(st + kTcBlocks * kTcATile + r * (kTcWords * 4) + w0 * 4);
+        const uint32_t words[4] = {pw.x, pw.y, pw.z, pw.w};
+        unsigned char* at = st + blk * kTcATile + r * 128;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint32_t wd = words[i];
+          const int c = (w0 + i) & 7;              // 16-byte chunk (16 columns) within the row
+          const uint4 v = make_uint4(codes4(wd & 0xFFu), codes4((wd >> 8) & 0xFFu),
+                                     codes4((wd >> 16) & 0xFFu), codes4(wd >> 24));
+          *reinterpret_cast<uint4*>(at + ((c ^ (r & 7)) * 16)) = v;
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      }
+      mbar_arrive(&s_dec[sl]);
+    }
+    // ---- epilogue: accumulators -> exact split sums ----
+    const bool done = mbar_wait_backoff(&s_accum, 0u);
+    if (!done && lane == 0) dev_fail(a.status, DEV_TIMEOUT, 53, 0u);
+    tc_after();
+    const int q = warp & 3;                        // this warp's TMEM lane quarter
+    const int Tp = (T + 3) & ~3;
+    const bool abort = *(volatile int*)&s_abort || !done;
+#pragma unroll
+    for (int b = 0; b < kTcBlocks; ++b) {
+      const int col = col0 + b * 128 + q * 32 + lane;
+#pragma unroll
+      for (int c0 = 0; c0 < NPAD; c0 += 16) {
+        uint32_t v[16];
+        tc_ld16(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * NPAD + c0), v);
+        if (abort || col >= d_out) continue;
+        float* dst = a.parts + (size_t)col * Tp;
+#pragma unroll
+        for (int e = 0; e < 16; e += 4) {
+          const int t = c0 + e;
+          if (t < T)                                // T is a multiple of 4 past the last group
+            red_v4(dst + t, (float)(int)v[e], (float)(int)v[e + 1], (float)(int)v[e + 2],
+                   (float)(int)v[e + 3]);
+        }
+      }
+    }
+  }
+  // ---- free the tensor memory once every read of it is done ----
+  tc_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
+                 : "memory");
+  }
+
+  // ---- the last CTA of this column range: rescale ----
+  int32_t* ticket = a.tickets + ct;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) s_flag = (atomicAdd(ticket, 1) == P.S - 1);
+  __syncthreads();
+  if (!s_flag) return;
+  __threadfence();
+  if (threadIdx.x == 0) *ticket = 0;
+  const int Tp = (T + 3) & ~3;
+  const int ncols = min(kTcCols, d_out - col0);
+  for (int i = threadIdx.x; i < ncols * T; i += kTcThreads) {
+    const int cc = i / T, t = i - cc * T;
+    const int col = col0 + cc;
+    const float v = __ldcg(a.parts + (size_t)col * Tp + t);
+    const float r = __fdiv_rn(__fmul_rn(a.alpha, a.gamma[t]), 127.0f);
+    const int iv = __float2int_rn(v);
+    const size_t o = (size_t)t * d_out + col;
+    float yv = __fmul_rn(__int2float_rn(iv), r);
+    if (a.gating) {                                // the quantized FFN's gate projection
+      const float bu = (a.gating == 2 && a.b_up) ? a.b_up[col] : 0.0f;
+      const float bg = (a.gating == 2 && a.b_gate) ? a.b_gate[col] : 0.0f;
+      yv = quant_gate_value(a.gating, __ldcg(a.gate_u + o), yv, bu, bg);
+    }
+    a.y[o] = yv;
+    if (a.acc) a.acc[o] = iv;
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tc_encode_fn() {
+  static std::once_flag once;
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &qr) ==
+            cudaSuccess &&
+        qr == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* ptr, uint64_t inner,
+                 uint64_t outer, uint64_t pitch, uint32_t bx, uint32_t by, CUtensorMapSwizzle sw) {
+  auto fn = tc_encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {pitch};
+  cuuint32_t box[2] = {bx, by};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, dt, 2, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            sw, CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int NPAD>
+cudaError_t tc_launch(const QGemvArgs& a, const CUtensorMap& mw, const CUtensorMap& mq, cudaStream_t s) {
+  static unsigned configured = 0;
+  cudaError_t e = ensure_smem_attr(qgemv_tc_kernel<NPAD>, kTcSmem, &configured);
+  if (e != cudaSuccess) return e;
+  dim3 grid(a.plan.n_ct, a.plan.S, 1);
+  e = launch_pdl(qgemv_tc_kernel<NPAD>, grid, dim3(kTcThreads), (size_t)kTcSmem, s, mw, mq, a);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool qgemv_tc_supported(int T, int d_in, int d_out) {
+  return T >= 8 && T <= 64 && d_in >= 1 && (d_in % 16) == 0 && (d_out % 64) == 0 &&
+         tc_encode_fn() != nullptr;
+}
+
+GemvPlan plan_qgemv_tc(int T, int d_in, int d_out) {
+  GemvPlan p{};
+  p.mma = 2;
+  p.TT = ((T + 15) / 16) * 16;
+  p.groups = 1;
+  p.mats = 1;
+  p.n_ct = (d_out + kTcCols - 1) / kTcCols;
+  p.vec_tile = kTcWords;
+  p.threads = kTcThreads;
+  p.rps = kTcRows;
+  p.nst = kTcStages;
+  p.rcap = 0;
+  p.smem = kTcSmem;
+  // splits: about two CTAs per SM, at most 8 (each split adds T x d_out exact
+  // partial sums), at least 4 steps of 32 rows each
+  const int steps = (d_in + kTcRows - 1) / kTcRows;
+  long S = (2L * kNumSMs) / p.n_ct;
+  if (S > 8) S = 8;
+  if (S > steps / 4) S = steps / 4;
+  if (S < 1) S = 1;
+  p.S = (int)S;
+  p.copies = 1;
+  p.parts_elems = (size_t)d_out * (size_t)((T + 3) & ~3);   // [column][T up to 4]
+  p.tickets = p.n_ct;
+  return p;
+}
+
+cudaError_t launch_qgemv_tc(const QGemvArgs& a, cudaStream_t s) {
+  if (a.T <= 0) return cudaSuccess;
+  if (a.xq == nullptr || a.plan.mma != 2) return cudaErrorInvalidValue;
+  CUtensorMap mw, mq;
+  const int row_words = a.d_out / 16;
+  // packed W^T [d_in rows][row_words] u32: box 16 words (64 B) x 32 rows, no swizzle
+  if (!make_map_2d(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT32, a.wp, (uint64_t)row_words, (uint64_t)a.d_in,
+                   (uint64_t)row_words * 4, kTcWords, kTcRows, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorInvalidValue;
+  const int npad = a.plan.TT;
+  // dense masked codes [T][d_in] int8: box 32 (rows) x npad tokens, 32-byte swizzle
+  if (!make_map_2d(&mq, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.xq, (uint64_t)a.d_in, (uint64_t)a.T,
+                   (uint64_t)a.d_in, kTcRows, (uint32_t)npad, CU_TENSOR_MAP_SWIZZLE_32B))
+    return cudaErrorInvalidValue;
+  switch (npad) {
+    case 16: return tc_launch<16>(a, mw, mq, s);
+    case 32: return tc_launch<32>(a, mw, mq, s);
+    case 48: return tc_launch<48>(a, mw, mq, s);
+    case 64: return tc_launch<64>(a, mw, mq, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace qs

@@ -361,6 +361,23 @@ struct QGemvArgs {
 
 cudaError_t launch_qgemv(const QGemvArgs& a, cudaStream_t s);
 
+// The quantized FFN's gating of one column, float32 steps in a fixed order
+// (g: this projection, u: the up projection):
+//   1: r = max(u, 0); h = (r * r) * g       2: h = max(g + b_gate, 0) * max(u + b_up, 0)
+__device__ __forceinline__ float quant_gate_value(int gating, float u, float g, float bu, float bg) {
+  if (gating == 1) {
+    const float r = fmaxf(u, 0.0f);
+    return __fmul_rn(__fmul_rn(r, r), g);
+  }
+  return __fmul_rn(fmaxf(__fadd_rn(g, bg), 0.0f), fmaxf(__fadd_rn(u, bu), 0.0f));
+}
+
+// The tensor-core (tcgen05 kind::i8) int8 x ternary kernel for 8 to 64 tokens,
+// streaming every packed row (qgemv_tc.cu); plan.mma == 2 marks its plans.
+bool qgemv_tc_supported(int T, int d_in, int d_out);
+GemvPlan plan_qgemv_tc(int T, int d_in, int d_out);
+cudaError_t launch_qgemv_tc(const QGemvArgs& a, cudaStream_t s);
+
 struct PackArgs {
   const float* w = nullptr;  // [d_out, d_in]
   int d_out = 0, d_in = 0;

@@ -54,9 +54,8 @@ __device__ __forceinline__ void red_add_v4_f32(float* dst, float a0, float a1, f
                : "memory");
 }
 
-// The quantized FFN's gating, float32 steps in a fixed order (y is the gate
-// projection g of column `col`, u the up projection):
-//   1: r = max(u, 0); h = (r * r) * g        2: h = max(g + b_gate, 0) * max(u + b_up, 0)
+// The quantized FFN's gating of 4 columns (y is the gate projection g of
+// columns col.., u the up projection), see quant_gate_value.
 __device__ __forceinline__ float4 quant_gating(const QGemvArgs& a, size_t o, int col, float4 gv) {
   const float4 uv = __ldcg(reinterpret_cast<const float4*>(a.gate_u + o));
   const float us[4] = {uv.x, uv.y, uv.z, uv.w};
@@ -64,14 +63,9 @@ __device__ __forceinline__ float4 quant_gating(const QGemvArgs& a, size_t o, int
   float hs[4];
 #pragma unroll
   for (int e = 0; e < 4; ++e) {
-    if (a.gating == 1) {
-      const float r = fmaxf(us[e], 0.0f);
-      hs[e] = __fmul_rn(__fmul_rn(r, r), gs[e]);
-    } else {
-      const float bu = a.b_up ? a.b_up[col + e] : 0.0f;
-      const float bg = a.b_gate ? a.b_gate[col + e] : 0.0f;
-      hs[e] = __fmul_rn(fmaxf(__fadd_rn(gs[e], bg), 0.0f), fmaxf(__fadd_rn(us[e], bu), 0.0f));
-    }
+    const float bu = (a.gating == 2 && a.b_up) ? a.b_up[col + e] : 0.0f;
+    const float bg = (a.gating == 2 && a.b_gate) ? a.b_gate[col + e] : 0.0f;
+    hs[e] = quant_gate_value(a.gating, us[e], gs[e], bu, bg);
   }
   return make_float4(hs[0], hs[1], hs[2], hs[3]);
 }
@@ -766,6 +760,7 @@ bool qgemv_supported(int d_out) { return d_out % 64 == 0; }   // 16-byte aligned
 
 cudaError_t launch_qgemv(const QGemvArgs& a, cudaStream_t s) {
   if (a.T <= 0) return cudaSuccess;
+  if (a.plan.mma == 2) return launch_qgemv_tc(a, s);
   if (a.plan.mma) {
     if (a.xq == nullptr) return cudaErrorInvalidValue;   // several tokens: dense codes
     switch (a.plan.TT) {
