@@ -305,23 +305,48 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (!s_flag) return;
   __threadfence();
   if (threadIdx.x == 0) *ticket = 0;
+  // per-token scales once, then (column, 4 tokens) pairs with four float4
+  // loads in flight per thread (tokens are contiguous in the split sums)
+  __shared__ float s_r[64];
+  for (int t = threadIdx.x; t < T; t += kTcThreads) s_r[t] = __fdiv_rn(__fmul_rn(a.alpha, a.gamma[t]), 127.0f);
+  __syncthreads();
   const int Tp = (T + 3) & ~3;
+  const int G = Tp / 4;
   const int ncols = min(kTcCols, d_out - col0);
-  for (int i = threadIdx.x; i < ncols * T; i += kTcThreads) {
-    const int cc = i / T, t = i - cc * T;
-    const int col = col0 + cc;
-    const float v = __ldcg(a.parts + (size_t)col * Tp + t);
-    const float r = __fdiv_rn(__fmul_rn(a.alpha, a.gamma[t]), 127.0f);
-    const int iv = __float2int_rn(v);
-    const size_t o = (size_t)t * d_out + col;
-    float yv = __fmul_rn(__int2float_rn(iv), r);
-    if (a.gating) {                                // the quantized FFN's gate projection
-      const float bu = (a.gating == 2 && a.b_up) ? a.b_up[col] : 0.0f;
-      const float bg = (a.gating == 2 && a.b_gate) ? a.b_gate[col] : 0.0f;
-      yv = quant_gate_value(a.gating, __ldcg(a.gate_u + o), yv, bu, bg);
+  const int total = ncols * G;
+  for (int i0 = threadIdx.x; i0 < total; i0 += 4 * kTcThreads) {
+    float4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = i0 + u * kTcThreads;
+      if (i < total) {
+        const int g = i / ncols, cc = i - g * ncols;
+        v[u] = __ldcg(reinterpret_cast<const float4*>(a.parts + (size_t)(col0 + cc) * Tp) + g);
+      }
     }
-    a.y[o] = yv;
-    if (a.acc) a.acc[o] = iv;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = i0 + u * kTcThreads;
+      if (i >= total) break;
+      const int g = i / ncols, cc = i - g * ncols;
+      const int col = col0 + cc;
+      const float vv[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int t = 4 * g + e;
+        if (t >= T) break;
+        const int iv = __float2int_rn(vv[e]);
+        const size_t o = (size_t)t * d_out + col;
+        float yv = __fmul_rn(__int2float_rn(iv), s_r[t]);
+        if (a.gating) {                            // the quantized FFN's gate projection
+          const float bu = (a.gating == 2 && a.b_up) ? a.b_up[col] : 0.0f;
+          const float bg = (a.gating == 2 && a.b_gate) ? a.b_gate[col] : 0.0f;
+          yv = quant_gate_value(a.gating, __ldcg(a.gate_u + o), yv, bu, bg);
+        }
+        a.y[o] = yv;
+        if (a.acc) a.acc[o] = iv;
+      }
+    }
   }
 }
 

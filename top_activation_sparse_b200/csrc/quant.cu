@@ -566,26 +566,53 @@ __global__ void __launch_bounds__(kQmWarps * 32 + 32, 2) qgemv_mma_kernel(QGemvA
   if (!s_flag) return;
   __threadfence();
   if (tid == 0) *ticket = 0;
-  const int q4 = twords * 4;                       // float4 groups of the tile
-  for (int i = tid; i < ntok * q4; i += blockDim.x) {
-    const int qi = i / ntok, t = i - qi * ntok;    // tokens fastest
-    const int tok = tok0 + t;
-    const int col = cword * 16 + qi * 4;
-    float v[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int c = 0; c < P.copies; ++c) {
-      const float* pc = a.parts + (size_t)c * d_out * Tp + (size_t)col * Tp + tok;
+  // (column, 4 tokens) pairs with four float4 loads in flight per thread:
+  // the tokens of a column are contiguous in the split sums (one copy here)
+  __shared__ float s_r[TT];
+  for (int t = tid; t < ntok; t += blockDim.x)
+    s_r[t] = __fdiv_rn(__fmul_rn(a.alpha, a.gamma[tok0 + t]), 127.0f);
+  __syncthreads();
+  const int ncols = twords * 16;
+  const int G = (ntok + 3) / 4;
+  const int total = ncols * G;
+  for (int i0 = tid; i0 < total; i0 += 4 * (int)blockDim.x) {
+    float4 v[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) v[e] += __ldcg(pc + (size_t)e * Tp);
+    for (int u = 0; u < 4; ++u) {
+      const int i = i0 + u * (int)blockDim.x;
+      v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (i < total) {
+        const int g = i / ncols, cc = i - g * ncols;
+        for (int c = 0; c < P.copies; ++c) {
+          const float4 f = __ldcg(reinterpret_cast<const float4*>(
+              a.parts + (size_t)c * d_out * Tp + (size_t)(cword * 16 + cc) * Tp + tok0) + g);
+          v[u].x += f.x; v[u].y += f.y; v[u].z += f.z; v[u].w += f.w;
+        }
+      }
     }
-    const float r = __fdiv_rn(__fmul_rn(a.alpha, a.gamma[tok]), 127.0f);
-    const int4 iv = make_int4(__float2int_rn(v[0]), __float2int_rn(v[1]), __float2int_rn(v[2]),
-                              __float2int_rn(v[3]));
-    const size_t o = (size_t)tok * d_out + col;
-    float4 yv = make_float4(__fmul_rn(__int2float_rn(iv.x), r), __fmul_rn(__int2float_rn(iv.y), r),
-                            __fmul_rn(__int2float_rn(iv.z), r), __fmul_rn(__int2float_rn(iv.w), r));
-    if (a.gating) yv = quant_gating(a, o, col, yv);
-    reinterpret_cast<float4*>(a.y + o)[0] = yv;
-    if (a.acc) reinterpret_cast<int4*>(a.acc + o)[0] = iv;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = i0 + u * (int)blockDim.x;
+      if (i >= total) break;
+      const int g = i / ncols, cc = i - g * ncols;
+      const int col = cword * 16 + cc;
+      const float vv[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int t = 4 * g + e;
+        if (t >= ntok) break;
+        const int iv = __float2int_rn(vv[e]);
+        const size_t o = (size_t)(tok0 + t) * d_out + col;
+        float yv = __fmul_rn(__int2float_rn(iv), s_r[t]);
+        if (a.gating) {                            // the quantized FFN's gate projection
+          const float bu = (a.gating == 2 && a.b_up) ? a.b_up[col] : 0.0f;
+          const float bg = (a.gating == 2 && a.b_gate) ? a.b_gate[col] : 0.0f;
+          yv = quant_gate_value(a.gating, __ldcg(a.gate_u + o), yv, bu, bg);
+        }
+        a.y[o] = yv;
+        if (a.acc) a.acc[o] = iv;
+      }
+    }
   }
 }
 
