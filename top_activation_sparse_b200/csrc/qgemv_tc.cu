@@ -238,8 +238,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int blk = w0 >> 3;                       // A tile (columns 0..127 or 128..255)
     for (int it = 0; it < nsteps; ++it) {
       const int sl = it % kTcStages;
+      // the decode warps are the stage's only consumers: poll without sleeping
+      // (a stage holds a fraction of a microsecond of work)
       const bool ready = !*(volatile int*)&s_abort &&
-                         mbar_wait_backoff(&s_full[sl], (uint32_t)(it / kTcStages) & 1u);
+                         mbar_wait(&s_full[sl], (uint32_t)(it / kTcStages) & 1u);
       if (!ready && !*(volatile int*)&s_abort) {
         if (lane == 0) dev_fail(a.status, DEV_TIMEOUT, 52, (uint32_t)it);
         atomicExch(&s_abort, 1);
