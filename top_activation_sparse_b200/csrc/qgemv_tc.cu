@@ -14,8 +14,10 @@
 //     rows; per step of 32 rows (the MMA's K) one TMA brings the 32 x 64-byte
 //     packed segment and one TMA the tokens' 32 codes each (K-major, 32-byte
 //     swizzle), into a ring of stages;
-//   * four decode warps expand the 2-bit codes (00 = 0, 01 = +1, 10 = -1) into
-//     int8 and write the two A tiles in the MN-major 128-byte-swizzled layout
+//   * eight decode warps expand the 2-bit codes (00 = 0, 01 = +1, 10 = -1) into
+//     int8 (the codes are spread into nibbles, and one byte permute per four
+//     codes selects from the bytes {0, +1, -1}) and write the two A tiles in
+//     the MN-major 128-byte-swizzled layout
 //     (each 32-row x 128-byte tile: row k holds columns 0..127, 16-byte chunk
 //     c of row k at chunk c ^ (k mod 8)), then make them visible to the tensor
 //     core (fence.proxy.async) and arrive on the stage's barrier;
@@ -47,8 +49,9 @@ constexpr int kTcPacked = kTcRows * kTcWords * 4;  // 2 KB
 constexpr int kTcBMax = 64 * kTcRows;              // codes of up to 64 tokens: 2 KB
 constexpr int kTcStage = kTcBlocks * kTcATile + kTcPacked + kTcBMax;   // 12 KB (multiple of 1 KB)
 constexpr int kTcSmem = kTcStages * kTcStage + 1024;
-constexpr int kTcThreads = 192;                    // warp 0 TMA, warp 1 MMA, warps 2-5 decode + epilogue
-constexpr int kTcDecoders = 128;
+constexpr int kTcThreads = 320;                    // warp 0 TMA, warp 1 MMA, warps 2-9 decode + epilogue
+constexpr int kTcDecoders = 256;
+static_assert(kTcBlocks * 4 == (kTcThreads - 64) / 32, "one epilogue warp per (accumulator, TMEM lane quarter)");
 
 // instruction descriptor, kind::i8: D s32, A and B signed 8-bit, A MN-major,
 // B K-major, M = 128, N = NPAD
@@ -115,10 +118,21 @@ __device__ __forceinline__ void red_v4(float* dst, float a0, float a1, float a2,
                : "memory");
 }
 
-// 4 packed 2-bit codes (one byte) -> 4 int8 in a word: 00 -> 0, 01 -> +1, 10 -> -1
-__device__ __forceinline__ uint32_t codes4(uint32_t b) {
-  const uint32_t s = (b & 3u) | ((b & 0xCu) << 6) | ((b & 0x30u) << 12) | ((b & 0xC0u) << 18);
-  return s | (((s >> 1) & 0x01010101u) * 0xFFu);
+// 8 packed 2-bit codes (16 bits) -> 8 nibbles: code k moves to bits 4k..4k+1
+__device__ __forceinline__ uint32_t spread_codes(uint32_t x) {
+  x &= 0xFFFFu;
+  x = (x | (x << 8)) & 0x00FF00FFu;
+  x = (x | (x << 4)) & 0x0F0F0F0Fu;
+  return (x | (x << 2)) & 0x33333333u;
+}
+
+// one packed word (16 codes: 00 -> 0, 01 -> +1, 10 -> -1) -> 16 int8, in
+// column order: each nibble selects a byte of {0, +1, -1} (byte permute)
+__device__ __forceinline__ uint4 decode_word(uint32_t w) {
+  constexpr uint32_t kVals = 0x00FF0100u;          // bytes 0, +1, -1
+  const uint32_t lo = spread_codes(w), hi = spread_codes(w >> 16);
+  return make_uint4(__byte_perm(kVals, 0u, lo & 0xFFFFu), __byte_perm(kVals, 0u, lo >> 16),
+                    __byte_perm(kVals, 0u, hi & 0xFFFFu), __byte_perm(kVals, 0u, hi >> 16));
 }
 
 template <int NPAD>
@@ -232,9 +246,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   } else {
     // ---- decoders: 2-bit codes -> int8 A tiles ----
-    const int dt = threadIdx.x - 64;               // 0..127
-    const int r = dt >> 2;                         // row of the step (0..31)
-    const int w0 = (dt & 3) * 4;                   // first of this thread's 4 words (0, 4, 8, 12)
+    const int dt = threadIdx.x - 64;               // 0..255
+    const int r = dt >> 3;                         // row of the step (0..31)
+    const int w0 = (dt & 7) * 2;                   // first of this thread's 2 words (0, 2, .., 14)
     const int blk = w0 >> 3;                       // A tile (columns 0..127 or 128..255)
     for (int it = 0; it < nsteps; ++it) {
       const int sl = it % kTcStages;
@@ -248,17 +262,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       if (ready) {
         unsigned char* st = smem_raw + ((base - smem_u32(smem_raw)) + (uint32_t)(sl * kTcStage));
-        const uint4 pw = *reinterpret_cast<const uint4*>(st + kTcBlocks * kTcATile + r * (kTcWords * 4) + w0 * 4);
-        const uint32_t words[4] = {pw.x, pw.y, pw.z, pw.w};
+        const uint2 pw = *reinterpret_cast<const uint2*>(st + kTcBlocks * kTcATile + r * (kTcWords * 4) + w0 * 4);
         unsigned char* at = st + blk * kTcATile + r * 128;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const uint32_t wd = words[i];
-          const int c = (w0 + i) & 7;              // 16-byte chunk (16 columns) within the row
-          const uint4 v = make_uint4(codes4(wd & 0xFFu), codes4((wd >> 8) & 0xFFu),
-                                     codes4((wd >> 16) & 0xFFu), codes4(wd >> 24));
-          *reinterpret_cast<uint4*>(at + ((c ^ (r & 7)) * 16)) = v;
-        }
+        const int c = w0 & 7;                      // 16-byte chunks c, c + 1 (16 columns each)
+        *reinterpret_cast<uint4*>(at + ((c ^ (r & 7)) * 16)) = decode_word(pw.x);
+        *reinterpret_cast<uint4*>(at + (((c + 1) ^ (r & 7)) * 16)) = decode_word(pw.y);
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       }
       mbar_arrive(&s_dec[sl]);
@@ -268,10 +276,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (!done && lane == 0) dev_fail(a.status, DEV_TIMEOUT, 53, 0u);
     tc_after();
     const int q = warp & 3;                        // this warp's TMEM lane quarter
+    const int b = (warp - 2) >> 2;                 // its accumulator (128-column block)
     const int Tp = (T + 3) & ~3;
     const bool abort = *(volatile int*)&s_abort || !done;
-#pragma unroll
-    for (int b = 0; b < kTcBlocks; ++b) {
+    {
       const int col = col0 + b * 128 + q * 32 + lane;
 #pragma unroll
       for (int c0 = 0; c0 < NPAD; c0 += 16) {
