@@ -25,8 +25,11 @@
 //     M = 128, N = tokens rounded up to 16, K = 32) into two accumulators and
 //     frees the stage with tcgen05.commit;
 //   * the decode warps then read the accumulators (tcgen05.ld, one column per
-//     lane), add them exactly into the split sums (integers < 2^24 in f32),
-//     and the last CTA of the column range rescales y = f32(acc) * r_t.
+//     lane) into the CTA's shared memory; the S CTAs that split the rows of
+//     one column range form a thread-block cluster, and after a cluster
+//     barrier each of them sums its slice of the columns over all S partial
+//     tiles through distributed shared memory (exact int32), rescales
+//     y = f32(acc) * r_t and stores it: no global atomics, no split-sum buffer.
 // Every wait is bounded; a timeout records DEV_TIMEOUT, lets the copies and
 // MMAs in flight finish and frees the tensor memory.
 #include <cuda.h>
@@ -112,12 +115,6 @@ __device__ __forceinline__ void tc_ld16(uint32_t taddr, uint32_t (&r)[16]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-__device__ __forceinline__ void red_v4(float* dst, float a0, float a1, float a2, float a3) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(a0), "f"(a1),
-               "f"(a2), "f"(a3)
-               : "memory");
-}
-
 // 8 packed 2-bit codes (16 bits) -> 8 nibbles: code k moves to bits 4k..4k+1
 __device__ __forceinline__ uint32_t spread_codes(uint32_t x) {
   x &= 0xFFFFu;
@@ -146,7 +143,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __shared__ __align__(8) uint64_t s_accum;               // every MMA done -> epilogue
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
-  __shared__ int s_flag;
   constexpr uint32_t kTmemCols = (kTcBlocks * NPAD) <= 32 ? 32 : ((kTcBlocks * NPAD) <= 64 ? 64 : 128);
   constexpr int kBBytes = NPAD * kTcRows;
 
@@ -168,7 +164,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < kTcStages; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_dec[i], kTcDecoders);
+      mbar_init(&s_dec[i], kTcDecoders / 32);        // one arrive per decode warp
       mbar_init(&s_empty[i], 1);
     }
     mbar_init(&s_accum, 1);
@@ -269,32 +265,27 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         *reinterpret_cast<uint4*>(at + (((c + 1) ^ (r & 7)) * 16)) = decode_word(pw.y);
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       }
-      mbar_arrive(&s_dec[sl]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_dec[sl]);
     }
-    // ---- epilogue: accumulators -> exact split sums ----
+    // ---- epilogue: this CTA's partial sums -> its shared memory ----
+    // (token-major [t][256 columns] int32; the ring is free: every MMA has
+    // completed, so every stage has been read)
     const bool done = mbar_wait_backoff(&s_accum, 0u);
     if (!done && lane == 0) dev_fail(a.status, DEV_TIMEOUT, 53, 0u);
     tc_after();
     const int q = warp & 3;                        // this warp's TMEM lane quarter
     const int b = (warp - 2) >> 2;                 // its accumulator (128-column block)
-    const int Tp = (T + 3) & ~3;
     const bool abort = *(volatile int*)&s_abort || !done;
-    {
-      const int col = col0 + b * 128 + q * 32 + lane;
+    int32_t* part = reinterpret_cast<int32_t*>(smem_raw + (base - smem_u32(smem_raw)));
+    const int cl = b * 128 + q * 32 + lane;        // column within the CTA's 256
 #pragma unroll
-      for (int c0 = 0; c0 < NPAD; c0 += 16) {
-        uint32_t v[16];
-        tc_ld16(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * NPAD + c0), v);
-        if (abort || col >= d_out) continue;
-        float* dst = a.parts + (size_t)col * Tp;
+    for (int c0 = 0; c0 < NPAD; c0 += 16) {
+      uint32_t v[16];
+      tc_ld16(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * NPAD + c0), v);
 #pragma unroll
-        for (int e = 0; e < 16; e += 4) {
-          const int t = c0 + e;
-          if (t < T)                                // T is a multiple of 4 past the last group
-            red_v4(dst + t, (float)(int)v[e], (float)(int)v[e + 1], (float)(int)v[e + 2],
-                   (float)(int)v[e + 3]);
-        }
-      }
+      for (int e = 0; e < 16; ++e)
+        if (c0 + e < T) part[(c0 + e) * kTcCols + cl] = abort ? 0 : (int32_t)v[e];
     }
   }
   // ---- free the tensor memory once every read of it is done ----
@@ -305,59 +296,55 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
                  : "memory");
   }
-
-  // ---- the last CTA of this column range: rescale ----
-  int32_t* ticket = a.tickets + ct;
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) s_flag = (atomicAdd(ticket, 1) == P.S - 1);
-  __syncthreads();
-  if (!s_flag) return;
-  __threadfence();
-  if (threadIdx.x == 0) *ticket = 0;
-  // per-token scales once, then (column, 4 tokens) pairs with four float4
-  // loads in flight per thread (tokens are contiguous in the split sums)
+  // per-token scales
   __shared__ float s_r[64];
   for (int t = threadIdx.x; t < T; t += kTcThreads) s_r[t] = __fdiv_rn(__fmul_rn(a.alpha, a.gamma[t]), 127.0f);
-  __syncthreads();
-  const int Tp = (T + 3) & ~3;
-  const int G = Tp / 4;
+
+  // ---- the split CTAs of this column range are one cluster: after the
+  // barrier each sums its slice of columns over every CTA's shared memory
+  // (distributed shared memory), exactly in int32, and writes y.  Every
+  // thread of every CTA reaches both cluster barriers (no early return). ----
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+  const int S = P.S;
+  const int rank = blockIdx.y;                     // the cluster spans blockIdx.y
   const int ncols = min(kTcCols, d_out - col0);
-  const int total = ncols * G;
-  for (int i0 = threadIdx.x; i0 < total; i0 += 4 * kTcThreads) {
-    float4 v[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int i = i0 + u * kTcThreads;
-      if (i < total) {
-        const int g = i / ncols, cc = i - g * ncols;
-        v[u] = __ldcg(reinterpret_cast<const float4*>(a.parts + (size_t)(col0 + cc) * Tp) + g);
-      }
+  const int slice = (((kTcCols + S - 1) / S + 3) / 4) * 4;   // ceil(256 / S), a multiple of 4
+  const int cA = min(rank * slice, ncols), cB = min(cA + slice, ncols);
+  const int ng = (cB - cA + 3) / 4;                // 4-column groups (ncols % 4 == 0)
+  const uint32_t part_addr = base;
+  for (int i = threadIdx.x; i < T * ng; i += kTcThreads) {
+    const int t = i / ng, g = i - t * ng;
+    const int c = cA + 4 * g;
+    const uint32_t local = part_addr + (uint32_t)((t * kTcCols + c) * 4);
+    int4 sum = make_int4(0, 0, 0, 0);
+    for (int rr = 0; rr < S; ++rr) {
+      uint32_t remote;
+      asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local), "r"(rr));
+      int4 v;
+      asm volatile("ld.shared::cluster.v4.s32 {%0, %1, %2, %3}, [%4];"
+                   : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                   : "r"(remote)
+                   : "memory");
+      sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
     }
+    const int iv[4] = {sum.x, sum.y, sum.z, sum.w};
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int i = i0 + u * kTcThreads;
-      if (i >= total) break;
-      const int g = i / ncols, cc = i - g * ncols;
-      const int col = col0 + cc;
-      const float vv[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int t = 4 * g + e;
-        if (t >= T) break;
-        const int iv = __float2int_rn(vv[e]);
-        const size_t o = (size_t)t * d_out + col;
-        float yv = __fmul_rn(__int2float_rn(iv), s_r[t]);
-        if (a.gating) {                            // the quantized FFN's gate projection
-          const float bu = (a.gating == 2 && a.b_up) ? a.b_up[col] : 0.0f;
-          const float bg = (a.gating == 2 && a.b_gate) ? a.b_gate[col] : 0.0f;
-          yv = quant_gate_value(a.gating, __ldcg(a.gate_u + o), yv, bu, bg);
-        }
-        a.y[o] = yv;
-        if (a.acc) a.acc[o] = iv;
+    for (int e = 0; e < 4; ++e) {
+      const int col = col0 + c + e;
+      if (c + e >= cB) break;
+      const size_t o = (size_t)t * d_out + col;
+      float yv = __fmul_rn(__int2float_rn(iv[e]), s_r[t]);
+      if (a.gating) {                              // the quantized FFN's gate projection
+        const float bu = (a.gating == 2 && a.b_up) ? a.b_up[col] : 0.0f;
+        const float bg = (a.gating == 2 && a.b_gate) ? a.b_gate[col] : 0.0f;
+        yv = quant_gate_value(a.gating, __ldcg(a.gate_u + o), yv, bu, bg);
       }
+      a.y[o] = yv;
+      if (a.acc) a.acc[o] = iv[e];
     }
   }
+  // no CTA leaves while another may still read its shared memory
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 tc_encode_fn() {
@@ -391,8 +378,22 @@ cudaError_t tc_launch(const QGemvArgs& a, const CUtensorMap& mw, const CUtensorM
   static unsigned configured = 0;
   cudaError_t e = ensure_smem_attr(qgemv_tc_kernel<NPAD>, kTcSmem, &configured);
   if (e != cudaSuccess) return e;
-  dim3 grid(a.plan.n_ct, a.plan.S, 1);
-  e = launch_pdl(qgemv_tc_kernel<NPAD>, grid, dim3(kTcThreads), (size_t)kTcSmem, s, mw, mq, a);
+  // one cluster per column range: its S split CTAs (S <= 8, portable)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.plan.n_ct, a.plan.S, 1);
+  cfg.blockDim = dim3(kTcThreads);
+  cfg.dynamicSmemBytes = (size_t)kTcSmem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = 1;
+  attr[1].val.clusterDim.y = (unsigned)a.plan.S;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  e = cudaLaunchKernelEx(&cfg, qgemv_tc_kernel<NPAD>, mw, mq, a);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -426,8 +427,8 @@ GemvPlan plan_qgemv_tc(int T, int d_in, int d_out) {
   if (S < 1) S = 1;
   p.S = (int)S;
   p.copies = 1;
-  p.parts_elems = (size_t)d_out * (size_t)((T + 3) & ~3);   // [column][T up to 4]
-  p.tickets = p.n_ct;
+  p.parts_elems = 0;                              // split sums meet in distributed shared memory
+  p.tickets = 0;
   return p;
 }
 
