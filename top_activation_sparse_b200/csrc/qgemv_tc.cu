@@ -14,7 +14,8 @@
 //     rows; per step of 32 rows (the MMA's K) one TMA brings the 32 x 64-byte
 //     packed segment and one TMA the tokens' 32 codes each (K-major, 32-byte
 //     swizzle), into a ring of stages;
-//   * eight decode warps expand the 2-bit codes (00 = 0, 01 = +1, 10 = -1) into
+//   * eight decode warps, in four groups that take every fourth step (their
+//     proxy fences overlap), expand the 2-bit codes (00 = 0, 01 = +1, 10 = -1) into
 //     int8 (the codes are spread into nibbles, and one byte permute per four
 //     codes selects from the bytes {0, +1, -1}) and write the two A tiles in
 //     the MN-major 128-byte-swizzled layout
@@ -46,7 +47,7 @@ constexpr int kTcBlocks = 2;                       // 128-column MMA blocks per 
 constexpr int kTcCols = 128 * kTcBlocks;           // output columns per CTA
 constexpr int kTcWords = kTcCols / 16;             // packed words per row segment (16)
 constexpr int kTcRows = 32;                        // rows per step (the MMA's K for int8)
-constexpr int kTcStages = 6;
+constexpr int kTcStages = 8;                       // two CTAs per SM fit (2 x 97 KB)
 constexpr int kTcATile = kTcRows * 128;            // one 128-column A tile: 4 KB
 constexpr int kTcPacked = kTcRows * kTcWords * 4;  // 2 KB
 constexpr int kTcBMax = 64 * kTcRows;              // codes of up to 64 tokens: 2 KB
@@ -54,6 +55,10 @@ constexpr int kTcStage = kTcBlocks * kTcATile + kTcPacked + kTcBMax;   // 12 KB 
 constexpr int kTcSmem = kTcStages * kTcStage + 1024;
 constexpr int kTcThreads = 320;                    // warp 0 TMA, warp 1 MMA, warps 2-9 decode + epilogue
 constexpr int kTcDecoders = 256;
+constexpr int kTcGroups = 4;                       // decode groups working on different steps
+// A slot is always decoded by the same group (step % stages fixes step % groups),
+// so a group that waits on a slot has seen that slot's previous phase itself.
+static_assert(kTcStages % kTcGroups == 0, "each ring slot must belong to one decode group");
 static_assert(kTcBlocks * 4 == (kTcThreads - 64) / 32, "one epilogue warp per (accumulator, TMEM lane quarter)");
 
 // instruction descriptor, kind::i8: D s32, A and B signed 8-bit, A MN-major,
@@ -82,6 +87,20 @@ __device__ __forceinline__ void tc_tma_2d(uint32_t dst, const CUtensorMap* map, 
       " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
       : "memory");
+}
+
+// Bounded wait on a stage barrier that gives up early once another role has
+// aborted.  The abort flag is read only after failed polls: a shared-memory
+// load costs hundreds of cycles while the ring, the decoders and the tensor
+// core keep shared memory busy, so the fast path (phase already complete)
+// touches nothing but the barrier.
+enum TcWait { TC_READY = 0, TC_ABORTED = 1, TC_TIMEOUT = 2 };
+__device__ __forceinline__ int tc_wait(uint64_t* bar, uint32_t parity, const int* abort_flag) {
+  for (uint32_t i = 0; i < kWaitLimit; ++i) {
+    if (mbar_try_wait(bar, parity)) return TC_READY;
+    if ((i & 15u) == 15u && *(volatile const int*)abort_flag) return TC_ABORTED;
+  }
+  return TC_TIMEOUT;
 }
 
 __device__ __forceinline__ void umma_i8(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
@@ -164,7 +183,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < kTcStages; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_dec[i], kTcDecoders / 32);        // one arrive per decode warp
+      mbar_init(&s_dec[i], kTcDecoders / 32 / kTcGroups);   // one arrive per warp of the step's group
       mbar_init(&s_empty[i], 1);
     }
     mbar_init(&s_accum, 1);
@@ -189,12 +208,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       int it = 0;
       for (; it < nsteps; ++it) {
         const int sl = it % kTcStages;
-        if (it >= kTcStages && !mbar_wait(&s_empty[sl], (uint32_t)((it / kTcStages) - 1) & 1u)) {
-          dev_fail(a.status, DEV_TIMEOUT, 50, (uint32_t)it);
-          atomicExch(&s_abort, 1);
-          break;
+        if (it >= kTcStages) {
+          const int w = tc_wait(&s_empty[sl], (uint32_t)((it / kTcStages) - 1) & 1u, &s_abort);
+          if (w == TC_TIMEOUT) {
+            dev_fail(a.status, DEV_TIMEOUT, 50, (uint32_t)it);
+            atomicExch(&s_abort, 1);
+          }
+          if (w != TC_READY) break;
         }
-        if (*(volatile int*)&s_abort) break;
         const uint32_t sp = base + (uint32_t)(sl * kTcStage) + kTcBlocks * kTcATile;
         const uint32_t sq = sp + kTcPacked;
         mbar_arrive_expect_tx(&s_full[sl], (uint32_t)(kTcPacked + kBBytes));
@@ -214,13 +235,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (lane == 0) {
       // ---- MMA issuer ----
       bool issued = false;
-      for (int it = 0; it < nsteps && !*(volatile int*)&s_abort; ++it) {
+      for (int it = 0; it < nsteps; ++it) {
         const int sl = it % kTcStages;
-        if (!mbar_wait(&s_dec[sl], (uint32_t)(it / kTcStages) & 1u)) {
+        const int w = tc_wait(&s_dec[sl], (uint32_t)(it / kTcStages) & 1u, &s_abort);
+        if (w == TC_TIMEOUT) {
           dev_fail(a.status, DEV_TIMEOUT, 51, (uint32_t)it);
           atomicExch(&s_abort, 1);
-          break;
         }
+        if (w != TC_READY) break;
         tc_after();
         const uint32_t sa = base + (uint32_t)(sl * kTcStage);
         const uint32_t sq = sa + kTcBlocks * kTcATile + kTcPacked;
@@ -242,27 +264,33 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   } else {
     // ---- decoders: 2-bit codes -> int8 A tiles ----
+    // Four groups of two warps take every fourth step, so that the steps'
+    // proxy fences (decoded tiles -> tensor core) overlap; a thread decodes
+    // one 128-column row segment (8 words) of its group's step.
     const int dt = threadIdx.x - 64;               // 0..255
-    const int r = dt >> 3;                         // row of the step (0..31)
-    const int w0 = (dt & 7) * 2;                   // first of this thread's 2 words (0, 2, .., 14)
-    const int blk = w0 >> 3;                       // A tile (columns 0..127 or 128..255)
-    for (int it = 0; it < nsteps; ++it) {
+    const int grp = dt >> 6;                       // decode group (0..3)
+    const int gt = dt & 63;
+    const int r = gt >> 1;                         // row of the step (0..31)
+    const int blk = gt & 1;                        // A tile (columns 0..127 or 128..255)
+    for (int it = grp; it < nsteps; it += kTcGroups) {
       const int sl = it % kTcStages;
       // the decode warps are the stage's only consumers: poll without sleeping
       // (a stage holds a fraction of a microsecond of work)
-      const bool ready = !*(volatile int*)&s_abort &&
-                         mbar_wait(&s_full[sl], (uint32_t)(it / kTcStages) & 1u);
-      if (!ready && !*(volatile int*)&s_abort) {
+      const int w = tc_wait(&s_full[sl], (uint32_t)(it / kTcStages) & 1u, &s_abort);
+      const bool ready = w == TC_READY;
+      if (w == TC_TIMEOUT) {
         if (lane == 0) dev_fail(a.status, DEV_TIMEOUT, 52, (uint32_t)it);
         atomicExch(&s_abort, 1);
       }
       if (ready) {
         unsigned char* st = smem_raw + ((base - smem_u32(smem_raw)) + (uint32_t)(sl * kTcStage));
-        const uint2 pw = *reinterpret_cast<const uint2*>(st + kTcBlocks * kTcATile + r * (kTcWords * 4) + w0 * 4);
+        const uint4* pw = reinterpret_cast<const uint4*>(st + kTcBlocks * kTcATile + r * (kTcWords * 4) + blk * 32);
+        const uint4 p0 = pw[0], p1 = pw[1];
+        const uint32_t words[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
         unsigned char* at = st + blk * kTcATile + r * 128;
-        const int c = w0 & 7;                      // 16-byte chunks c, c + 1 (16 columns each)
-        *reinterpret_cast<uint4*>(at + ((c ^ (r & 7)) * 16)) = decode_word(pw.x);
-        *reinterpret_cast<uint4*>(at + (((c + 1) ^ (r & 7)) * 16)) = decode_word(pw.y);
+#pragma unroll
+        for (int c = 0; c < 8; ++c)                // 16-byte chunk c holds columns 16c..16c+15
+          *reinterpret_cast<uint4*>(at + ((c ^ (r & 7)) * 16)) = decode_word(words[c]);
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       }
       __syncwarp();
