@@ -201,7 +201,15 @@ def load_peaks() -> dict:
     return {"hbm_gbs": 6650.0, "source": "fallback", "bf16_tflops": 1590.0}
 
 
-KERNEL_SOURCES = {"gemv": "gemv.cu", "prefill": "prefill_gemm.cu", "qgemv": "quant.cu"}
+KERNEL_SOURCES = {"gemv": "gemv.cu", "prefill": "prefill_gemm.cu", "qgemv": "quant.cu",
+                  "qgemvtc": "qgemv_tc.cu", "ffn": "ffn_fused.cu"}
+
+
+def quant_tc(T: int, d_in: int, d_out: int, blk: int) -> bool:
+    """Whether an int8 x ternary projection of T tokens runs on the tcgen05
+    kind::i8 kernel (the library's own rule: 8..64 tokens, d_in % 16 == 0,
+    d_out % 64 == 0, per-token selections)."""
+    return blk <= 1 and 8 <= T <= 64 and d_in % 16 == 0 and d_out % 64 == 0
 
 
 def _code_only(text: str) -> str:
@@ -386,21 +394,32 @@ def setup_ffn(args, qs, torch, device, stream, rank):
         return cpu_oracle_ffn(w, x.float().cpu().numpy(), up, gate, down, args.cpu_seconds, blk)
 
     phases = ["topk_x", "upgate", "topk_h", "down"]
+    dominant, dom_work, launches = "upgate", upgate_bytes, 5 if gate_first else 4
+    kernel = ("gemv_kernel (gate gather-GEMV) + up_rows_kernel (open gates' rows of W_up)"
+              if gate_first else "gemv_kernel (up/gate gather-GEMV with the gating epilogue)")
+    profile = f"gemv_{'gatefirst' if gate_first else 'upgate'}_{args.workload}_T{T}"
+    fused = (not gate_first and blk <= 1 and
+             qs.qs_sparse_ffn_fused(qs.QS_BF16, T, d_model, d_ff, False))
+    if fused:
+        # one persistent kernel per layer: it is the dominant (and only) kernel
+        phases, dominant = ["ffn_fused"], "ffn_fused"
+        dom_work, launches = upgate_bytes + down_bytes + topk_bytes, 1
+        kernel = "ffn_fused_kernel (the whole one-token layer, one cooperative launch)"
+        profile = f"ffn_fused_{args.workload}_T{T}"
     return {
         "fn": fn, "T": T, "n_layers": n_layers, "ws": ws, "x": x, "y": y,
         "args": lambda l, ev: c_args(l, ev), "n_events": qs.QS_FFN_PHASE_EVENTS,
         "dense_args": (lambda l: c_args(l, None, d_model, d_ff)),
-        "phases": phases, "dominant": "upgate",
-        "kernel": ("gemv_kernel (gate gather-GEMV) + up_rows_kernel (open gates' rows of W_up)"
-                   if gate_first else "gemv_kernel (up/gate gather-GEMV with the gating epilogue)"),
-        "bound": "hbm", "dom_work": upgate_bytes, "layer_work": upgate_bytes + down_bytes + topk_bytes,
+        "phases": phases, "dominant": dominant,
+        "kernel": kernel,
+        "bound": "hbm", "dom_work": dom_work, "layer_work": upgate_bytes + down_bytes + topk_bytes,
         "extra": {"rows_streamed": extra_rows},
         "desc": workload_desc(args, T),
         "l2": (f"inputs larger than L2: {n_layers} independent layers "
                f"({n_layers * layer_bytes / 1e9:.2f} GB of weights) rotated per step"),
-        "e2e_call": e2e_call, "cpu_rate": cpu_rate, "launches": 5 if gate_first else 4,
+        "e2e_call": e2e_call, "cpu_rate": cpu_rate, "launches": launches,
         "dtype": "bf16",
-        "profile": f"gemv_{'gatefirst' if gate_first else 'upgate'}_{args.workload}_T{T}",
+        "profile": profile,
     }
 
 
@@ -639,14 +658,17 @@ def setup_quant_ffn(args, qs, torch, device, stream, rank):
         "args": lambda l, ev: c_args(l, ev), "n_events": qs.QS_FFN_PHASE_EVENTS,
         "dense_args": (lambda l: c_args(l, None, dm, dff)),
         "phases": ["quant_topk_x", "upgate", "quant_topk_h", "down"], "dominant": "upgate",
-        "kernel": "qgemv (int8 x ternary up, then gate with the gating epilogue)",
+        "kernel": ("qgemv_tc_kernel (int8 x ternary up, then gate with the gating epilogue; "
+                   "tcgen05 kind::i8)" if quant_tc(T, dm, dff, blk) else
+                   "qgemv (int8 x ternary up, then gate with the gating epilogue)"),
         "bound": "hbm", "dom_work": upgate, "layer_work": upgate + down + topk,
         "extra": {"rows_streamed": {"x": rows_x, "h": rows_h}},
         "desc": workload_desc(args, T),
         "l2": (f"inputs larger than L2: {n_layers} independent packed layers "
                f"({n_layers * layer_bytes / 1e9:.2f} GB) rotated per step"),
         "e2e_call": e2e_call, "cpu_rate": cpu_rate, "launches": 5, "dtype": "int8",
-        "profile": f"qgemv_{args.workload}_T{T}",
+        "profile": (f"qgemvtc_{args.workload}_T{T}" if quant_tc(T, dm, dff, blk)
+                    else f"qgemv_{args.workload}_T{T}"),
     }
 
 
@@ -714,12 +736,15 @@ def setup_quant(args, qs, torch, device, stream, rank):
         "args": c_args, "n_events": qs.QS_LINEAR_PHASE_EVENTS,
         "dense_args": (lambda l: c_args(l, None, w.d_in)),
         "phases": ["quant_topk", "projection"], "dominant": "projection",
-        "kernel": "qgemv_kernel (int8 x ternary gather)", "bound": "hbm", "dom_work": work,
+        "kernel": ("qgemv_tc_kernel (int8 x ternary, tcgen05 kind::i8, TMEM accumulators)"
+                   if quant_tc(T, w.d_in, w.d_out, blk) else "qgemv_kernel (int8 x ternary gather)"),
+        "bound": "hbm", "dom_work": work,
         "layer_work": work, "extra": {"rows_streamed": rows},
         "desc": workload_desc(args, T),
         "l2": f"inputs larger than L2: {n_layers} packed weight copies ({n_layers * wbytes / 1e9:.2f} GB) rotated",
         "e2e_call": e2e_call, "cpu_rate": cpu_rate, "launches": 2, "dtype": "int8",
-        "profile": f"qgemv_{args.workload}_T{T}",
+        "profile": (f"qgemvtc_{args.workload}_T{T}" if quant_tc(T, w.d_in, w.d_out, blk)
+                    else f"qgemv_{args.workload}_T{T}"),
     }
 
 

@@ -165,8 +165,14 @@ qs_status qs_sparse_linear(const void* x, int dtype, int T, int d_in, int d_out,
  *             recorded on `stream` before the first kernel and after the input
  *             top-K, the up/gate projection, the top-K on |h| and the down
  *             projection (for per-phase timing; recording them costs a little).
+ *             A call that runs as one kernel (qs_sparse_ffn_fused) records the
+ *             first event before it and all the others after it.
  *   ws        qs_workspace_size(QS_OP_SPARSE_FFN, T, d_model, d_ff, k_h) bytes.
  *   d_model and d_ff must be multiples of 8 (bf16) or 4 (f32).
+ *   One token, bf16, idx_h_out NULL, d_model <= 8192: the whole layer runs as
+ *   ONE persistent kernel (a cooperative launch whose phases are separated by
+ *   grid barriers) instead of four; same results up to float32 summation
+ *   order, same lists and statistics.  qs_set_ffn_fused(0) turns this off.
  *   Errors: INVALID_ARG, ALIGNMENT, WORKSPACE, UNSUPPORTED, CUDA.
  */
 qs_status qs_sparse_ffn(const void* x, int dtype, int T, int d_model, int d_ff, int act,
@@ -175,6 +181,16 @@ qs_status qs_sparse_ffn(const void* x, int dtype, int T, int d_model, int d_ff, 
                         void* y, float* h_out, int32_t* idx_h_out,
                         void* const* phase_events,
                         void* ws, size_t ws_bytes, void* stream);
+
+/* 1 if a qs_sparse_ffn call with these sizes (and idx_h_out given or not)
+ * runs as one persistent kernel on the current device, else 0 (also without
+ * a device).  Host-only: nothing is enqueued. */
+int qs_sparse_ffn_fused(int dtype, int T, int d_model, int d_ff, int with_idx_h);
+
+/* Process-wide switch for the one-kernel path of qs_sparse_ffn (on by
+ * default): 0 makes every call use the separate kernels (for comparison and
+ * testing).  Always returns QS_OK. */
+qs_status qs_set_ffn_fused(int enable);
 
 /*
  * qs_sparse_ffn_gate_first -- the dReLU layer of qs_sparse_ffn (QS_ACT_DRELU,
@@ -409,7 +425,8 @@ qs_status qs_workspace_list(const void* ws, int op, int T, int d_in, int d_out, 
 
 /* Failure-detection test hook (host side; process-wide; not thread-safe).
  * QS_FAULT_GATHER_NO_COPIES makes the gather-GEMV launches that follow (the
- * FMA kernel that serves one or two tokens) issue no weight copies at all:
+ * FMA kernel that serves one or two tokens, and the one-kernel FFN layer of
+ * qs_sparse_ffn) issue no weight copies at all:
  * their producer warp stays idle, so no copy is ever in flight, and the
  * consumers' bounded waits run out after `wait_polls` polls (0: the normal
  * limit).  The kernel then records QS_ERR_TIMEOUT in the workspace's status

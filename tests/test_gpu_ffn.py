@@ -151,12 +151,24 @@ def test_ffn_one_token_list_path_llama7b():
     _check_ffn(x8, up, gate, down, "relu2_glu", w.k, w.k_h, "bf16")
 
 
+@pytest.mark.parametrize("fused", [True, False])
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("dm,dff", [(64, 96), (200, 328), (128, 1000), (96, 16384)])
-def test_ffn_one_token_list_path_small(dtype, dm, dff):
-    """Both branches of the bitmask start: K_h above and below the nonzero
-    count of h (and K_h = 0, K_h = d_ff), ragged d_ff, the largest d_ff it takes."""
+def test_ffn_one_token_list_path_small(dtype, dm, dff, fused):
+    """Both branches of the bitmask start (or, one-kernel path, of the kept-h
+    choice): K_h above and below the nonzero count of h (and K_h = 0,
+    K_h = d_ff), ragged d_ff, the largest d_ff it takes."""
     need_gpu()
+    if fused and dtype == "f32":
+        pytest.skip("the one-kernel path serves bf16 only")
+    qs.qs_set_ffn_fused(fused)
+    try:
+        _list_path_small(dtype, dm, dff)
+    finally:
+        qs.qs_set_ffn_fused(True)
+
+
+def _list_path_small(dtype, dm, dff):
     g = workloads.rng(dm * 7 + dff)
     x = workloads.round_to_dtype(workloads.normal_f32(g, (1, dm)), dtype)
     up = workloads.round_to_dtype(workloads.normal_f32(g, (dm, dff), dm ** -0.5), dtype)
@@ -168,3 +180,48 @@ def test_ffn_one_token_list_path_small(dtype, dm, dff):
     for act, bias in (("relu2_glu", None), ("drelu", -0.3)):
         for k_h in k_hs:
             _check_ffn_list_path(x, up, gate, down, act, (7 * dm) // 10, k_h, dtype, bias=bias, ws=ws)
+
+
+def test_ffn_one_token_fused_llama7b():
+    """The one-kernel path of a one-token bf16 layer (cooperative launch, grid
+    barriers) against the oracle and against the separate kernels: the input
+    list is the same bit for bit, y matches the oracle re-run on the GPU's own
+    kept h; then K_h below the nonzero count (every CTA selects the K_h-th
+    largest |h| itself); then tokens back to back on one workspace (the
+    barrier counters must be reset by each call)."""
+    need_gpu()
+    w = workloads.WORKLOADS["ffn_relu2_llama7b"]
+    assert qs.qs_sparse_ffn_fused(qs.QS_BF16, 1, w.d_in, w.d_out, False)
+    assert not qs.qs_sparse_ffn_fused(qs.QS_BF16, 1, w.d_in, w.d_out, True)
+    assert not qs.qs_sparse_ffn_fused(qs.QS_BF16, 2, w.d_in, w.d_out, False)
+    assert not qs.qs_sparse_ffn_fused(qs.QS_F32, 1, w.d_in, w.d_out, False)
+    up, gate, down = _ffn_weights(w.name)
+    x4 = workloads.activations(w, 4)
+    lists = {}
+    for fused in (True, False):
+        qs.qs_set_ffn_fused(fused)
+        try:
+            _, ws = _check_ffn_list_path(x4[:1], up, gate, down, "relu2_glu", w.k, w.k_h, "bf16")
+        finally:
+            qs.qs_set_ffn_fused(True)
+        lists[fused] = qs.qs_workspace_list(ws, qs.QS_OP_SPARSE_FFN, 1, w.d_in, w.d_out, w.k_h, 0,
+                                            values=True)
+    rows_f, vals_f = lists[True]
+    rows_g, vals_g = lists[False]
+    assert np.array_equal(rows_f, rows_g) and np.array_equal(vals_f, vals_g)
+    keep = oracle.topk_keep(x4[:1], w.k)[0]
+    xb = x4[0, keep]
+    assert np.array_equal(rows_f, keep[xb != 0])
+    assert np.array_equal(vals_f, xb[xb != 0].astype(np.float32))
+    # fewer kept h than nonzero h: the radix select over |h| in every CTA
+    _check_ffn_list_path(x4[1:2], up, gate, down, "relu2_glu", w.k, w.d_out // 10, "bf16")
+    # back to back on one workspace, without a host synchronisation in between
+    ws = qs.new_workspace(qs.QS_OP_SPARSE_FFN, 1, w.d_in, w.d_out, w.k_h, torch.device("cuda"))
+    upt, gatet, downt = to_dev(up, "bf16"), to_dev(gate, "bf16"), to_dev(down, "bf16")
+    xs = [to_dev(x4[t:t + 1], "bf16") for t in range(4)]
+    ys = [qs.qs_sparse_ffn(xs[t], upt, gatet, downt, "relu2_glu", w.k, w.k_h, ws=ws).y
+          for t in range(4)]
+    check_status(ws)
+    for t in range(4):
+        ref = oracle.sparse_ffn(x4[t:t + 1], up, gate, down, "relu2_glu", w.k, w.k_h)
+        assert oracle.max_rel_err(to_np(ys[t]), ref["y"]) <= 2 * TOL_BF16

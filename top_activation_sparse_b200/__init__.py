@@ -95,6 +95,8 @@ _SIGNATURES = {
     "qs_sparse_linear_noalloc_status": (_i, [_vp]),
     "qs_workspace_list": (_i, [_vp, _i, _i, _i, _i, _i, _i, _vp, _i, _vp, _vp, _vp]),
     "qs_debug_inject": (_i, [_i, ctypes.c_uint]),
+    "qs_sparse_ffn_fused": (_i, [_i, _i, _i, _i, _i]),
+    "qs_set_ffn_fused": (_i, [_i]),
 }
 
 _lib = None
@@ -248,6 +250,17 @@ def qs_workspace_list(ws: torch.Tensor, op: int, T: int, d_in: int, d_out: int, 
     if not 0 <= n <= cap:
         raise RuntimeError(f"qs_workspace_list: inconsistent row count {n}")
     return rows[:n].copy(), (None if vals is None else vals[:n].copy())
+
+
+def qs_sparse_ffn_fused(dtype: int, T: int, d_model: int, d_ff: int, with_idx_h: bool = False) -> bool:
+    """True if qs_sparse_ffn with these sizes runs as one persistent kernel."""
+    return bool(lib().qs_sparse_ffn_fused(int(dtype), int(T), int(d_model), int(d_ff),
+                                          1 if with_idx_h else 0))
+
+
+def qs_set_ffn_fused(enable: bool) -> None:
+    """Turn the one-kernel path of one-token bf16 FFN calls on or off (process-wide)."""
+    _check("qs_set_ffn_fused", lib().qs_set_ffn_fused(1 if enable else 0))
 
 
 def qs_debug_inject(mode: int, wait_polls: int = 0) -> None:

@@ -1,6 +1,7 @@
 // extern "C" entry points of include/qs.h: argument checks, the workspace
 // layout, and the order in which the kernels are enqueued.  Every step of the
 // computation runs in this library's CUDA kernels; there is no host fallback.
+#include <atomic>
 #include <cstring>
 
 #include "gate_first.cuh"
@@ -25,7 +26,9 @@ constexpr int kTkTopkX = 0, kTkTopkH = 1, kTkAlpha = 2, kTkUpRows = 3, kTkHCount
 constexpr int kTkGemvEnd = 4096;
 constexpr int kUnionX = 4096, kUnionH = 4096 + QS_MAX_ROW / 32;
 constexpr int kGateBits = kUnionH + QS_MAX_ROW / 32;
-static_assert(kGateBits + QS_MAX_ROW / 32 <= (int)(64 * 1024 / 4), "ticket region too small");
+// grid-barrier counters of the one-kernel FFN (zero between calls)
+constexpr int kTkFusedBar = kGateBits + QS_MAX_ROW / 32;
+static_assert(kTkFusedBar + 5 <= (int)(64 * 1024 / 4), "ticket region too small");
 
 size_t align_up(size_t v) { return (v + kWsAlign - 1) / kWsAlign * kWsAlign; }
 
@@ -129,6 +132,15 @@ bool ws_layout(int op, int T, int d_in, int d_out, int k, WsLayout* L) {
       L->lval_h = take((size_t)d_out * Tc * sizeof(float));
       L->parts2_elems = max_parts(d_in, d_out, k, 1);
       L->parts2 = take(L->parts2_elems * sizeof(float));
+      if (op == QS_OP_SPARSE_FFN) {
+        // the one-kernel path of one-token bf16 calls (ffn_fused.cu); its down
+        // accumulator is parts2 (>= d_model floats)
+        L->fpug_elems = ffn_fused_pug_elems(d_in, d_out);
+        if (L->fpug_elems != 0) {
+          L->fpug = take(L->fpug_elems * sizeof(float));
+          L->fhnz = take((size_t)2 * kNumSMs * sizeof(int32_t));
+        }
+      }
       break;
     }
     case QS_OP_QUANT_SPARSE_LINEAR: {
@@ -328,6 +340,42 @@ qs_status qs_workspace_list(const void* ws, int op, int T, int d_in, int d_out, 
   return QS_OK;
 }
 
+namespace {
+std::atomic<int> g_ffn_fused{1};
+
+// A one-token bf16 FFN call (list outputs only) runs as one persistent kernel
+// when the device can hold its grid and the sizes fit its staging.
+bool use_ffn_fused(int op, int dtype, int T, int d_model, int d_ff, const int32_t* idx_h_out,
+                   const WsLayout& L, FfnFusedPlan* fp) {
+  if (!g_ffn_fused.load() || op != QS_OP_SPARSE_FFN || dtype != QS_BF16 || T != 1 ||
+      idx_h_out != nullptr || L.fpug == 0)
+    return false;
+  const int G = ffn_fused_grid();
+  if (G <= 0 || !plan_ffn_fused(d_model, d_ff, G, fp)) return false;
+  return (size_t)fp->S_ug * 2 * (size_t)d_ff <= L.fpug_elems && fp->S_dn <= 2 * kNumSMs &&
+         (size_t)d_model <= L.parts2_elems;
+}
+}  // namespace
+
+qs_status qs_set_ffn_fused(int enable) {
+  g_ffn_fused.store(enable ? 1 : 0);
+  return QS_OK;
+}
+
+int qs_sparse_ffn_fused(int dtype, int T, int d_model, int d_ff, int with_idx_h) {
+  if (!valid_dtype(dtype) || T < 1 || d_model < 1 || d_ff < 1 || d_model > QS_MAX_ROW ||
+      d_ff > QS_MAX_ROW)
+    return 0;
+  WsLayout L;
+  if (!ws_layout(QS_OP_SPARSE_FFN, T, d_model, d_ff, 0, &L)) return 0;
+  FfnFusedPlan fp;
+  int32_t dummy = 0;
+  return use_ffn_fused(QS_OP_SPARSE_FFN, dtype, T, d_model, d_ff, with_idx_h ? &dummy : nullptr, L,
+                       &fp)
+             ? 1
+             : 0;
+}
+
 qs_status qs_debug_inject(int mode, unsigned wait_polls) {
   if (mode != QS_FAULT_NONE && mode != QS_FAULT_GATHER_NO_COPIES) return QS_ERR_INVALID_ARG;
   g_fault.mode = mode;
@@ -472,6 +520,31 @@ static qs_status ffn_impl(int op, const void* x, int dtype, int T, int d_model, 
     if (phase_events == nullptr) return cudaSuccess;
     return cudaEventRecord((cudaEvent_t)phase_events[i], s);
   };
+  FfnFusedPlan fp;
+  if (use_ffn_fused(op, dtype, T, d_model, d_ff, idx_h_out, L, &fp)) {
+    // one token, bf16: every step in one persistent kernel (ffn_fused.cu);
+    // phase events 1-4 are all recorded after it
+    FfnFusedArgs f;
+    f.x = x; f.w_up = wt_up; f.w_gate = wt_gate; f.w_down = wt_down;
+    f.d_model = d_model; f.d_ff = d_ff; f.k_in = k_in; f.k_h = k_h;
+    f.act = act == QS_ACT_RELU2_GLU ? 1 : 2;
+    f.b_up = b_up; f.b_gate = b_gate;
+    f.y = y;
+    f.h = h_out ? h_out : w.at<float>(L.h);
+    f.pug = w.at<float>(L.fpug);
+    f.pdn = w.at<float>(L.parts2);
+    f.hnz = w.at<int32_t>(L.fhnz);
+    f.bar = w.ticket(L, kTkFusedBar);
+    f.list_x = w.at<int32_t>(L.list_x); f.lval_x = w.at<float>(L.lval_x);
+    f.list_h = w.at<int32_t>(L.list_h); f.lval_h = w.at<float>(L.lval_h);
+    f.cnt = w.at<int32_t>(L.cnt);
+    f.status = w.status();
+    f.plan = fp;
+    QS_TRY_CUDA(mark(0));
+    QS_TRY_CUDA(launch_ffn_fused(f, s));
+    for (int i = 1; i < QS_FFN_PHASE_EVENTS; ++i) QS_TRY_CUDA(mark(i));
+    return QS_OK;
+  }
   const float* unit = nullptr;                   // gate first: a vector of 1.0 (see step 2)
   if (gate_first) QS_TRY_CUDA(unit_vector_on_current_device(&unit, s));
 
@@ -502,6 +575,9 @@ static qs_status ffn_impl(int op, const void* x, int dtype, int T, int d_model, 
       return QS_ERR_UNSUPPORTED;
     a.zero = w.at<float>(L.parts1);
     a.zero_n = p_ug.parts_elems;
+    // the nonzero-h counter of step 2 starts at zero (see GemvArgs::hcount)
+    const bool h_range_call = Tc == 1 && idx_h_out == nullptr && !gate_first;
+    a.zero_word = h_range_call ? w.ticket(L, kTkHCount) : nullptr;
     QS_TRY_CUDA(launch_topk(a, s));
     if (timed) QS_TRY_CUDA(mark(1));
 
@@ -571,6 +647,7 @@ static qs_status ffn_impl(int op, const void* x, int dtype, int T, int d_model, 
     b.ticket = w.ticket(L, kTkTopkH);
     b.union_bits = reinterpret_cast<uint32_t*>(w.ticket(L, kUnionH));
     if (h_bits) b.nz_bits = b.union_bits;
+    b.early_release = h_range ? 1 : 0;             // the down projection waits for this grid
     b.status = w.status();
     QS_TRY_CUDA(launch_topk(b, s));
     if (timed) QS_TRY_CUDA(mark(3));
@@ -590,7 +667,6 @@ static qs_status ffn_impl(int op, const void* x, int dtype, int T, int d_model, 
       dn.hcount = hcount;
       dn.hsrc = h;
       dn.k_sel = k_h;
-      dn.done = w.ticket(L, kTkDownDone);
       dn.rows_out = w.at<int32_t>(L.cnt) + 1;
     }
     dn.status = w.status();

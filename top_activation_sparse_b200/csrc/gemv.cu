@@ -87,12 +87,15 @@ __device__ __forceinline__ void store_y(void* y, size_t o, const float (&v)[VecT
 }
 
 // Output of one column vector: y (MODE 0) or the gated hidden h (MODE 1/2).
+// Returns how many of its h are nonzero when the launch counts them
+// (a.hcount), for the caller to add once per warp.
 template <typename WT, int MODE>
-__device__ __forceinline__ void epilogue(const GemvArgs& a, int tok, int col,
+__device__ __forceinline__ int epilogue(const GemvArgs& a, int tok, int col,
                                          const float (&u)[VecTraits<WT>::V],
                                          const float (&g)[VecTraits<WT>::V]) {
   constexpr int V = VecTraits<WT>::V;
   const size_t o = (size_t)tok * a.d_out + col;
+  int nz = 0;
   if constexpr (MODE == 0) {
     store_y<WT>(a.y, o, u);
   } else {
@@ -114,9 +117,17 @@ __device__ __forceinline__ void epilogue(const GemvArgs& a, int tok, int col,
 #pragma unroll
       for (int e = 0; e < V; ++e) m |= (hv[e] != 0.0f ? 1u : 0u) << e;
       if (m != 0u) atomicOr(a.hbits + col / 32, m << (col % 32));
-      if (a.hcount != nullptr && m != 0u) atomicAdd(a.hcount, __popc(m));
+      if (a.hcount != nullptr) nz = __popc(m);
     }
   }
+  return nz;
+}
+
+// One atomic per warp for the nonzero-h counter (every lane calls this).
+__device__ __forceinline__ void add_hcount(int32_t* hcount, int nz) {
+  if (hcount == nullptr) return;
+  nz = __reduce_add_sync(0xffffffffu, nz);
+  if ((threadIdx.x & 31) == 0 && nz != 0) atomicAdd(hcount, nz);
 }
 
 template <typename WT, int TT, int MODE>
@@ -153,17 +164,17 @@ __global__ void __launch_bounds__(kMaxConsumers + 32, (TT <= 4) ? 2 : 1) gemv_ke
   const int col = (ct * P.vec_tile + tid) * V;                            // this thread's columns
 
   // The down projection of a one-token FFN (a.hcount): the launch before this
-  // one (the top-K on h) releases it only after waiting for the launch before
-  // that (the up/gate projection), so h and its nonzero count are complete
-  // here.  With at most k_sel nonzero h the kept rows are exactly the nonzero
-  // h: this CTA lists those of its own index range and streams them without
-  // waiting for the top-K's list (it still waits for the top-K before it
-  // finishes, so stream order holds for the next call).
+  // one (the top-K on h) releases this grid as soon as it starts, and its
+  // completion, which the wait below waits for, follows that of the up/gate
+  // projection; so h and its nonzero count are complete after the wait.  With
+  // at most k_sel nonzero h the kept rows are exactly the nonzero h: this CTA
+  // lists those of its own index range and streams them (the top-K's list is
+  // used otherwise).  The counter is zeroed by the next call's first kernel.
   bool hrange = false;
   if (MODE == 0 && a.hcount != nullptr) {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     hrange = __ldcg(a.hcount) <= a.k_sel;
-    if (!hrange) asm volatile("griddepcontrol.wait;" ::: "memory");
   } else {
     pdl_begin();
   }
@@ -327,16 +338,6 @@ __global__ void __launch_bounds__(kMaxConsumers + 32, (TT <= 4) ? 2 : 1) gemv_ke
       }
     }
   }
-  if (MODE == 0 && a.hcount != nullptr) {
-    if (hrange) asm volatile("griddepcontrol.wait;" ::: "memory");
-    // every CTA has read the nonzero count: the grid's last one clears it
-    __syncthreads();
-    if (tid == 0 &&
-        atomicAdd(a.done, 1) == (int)(gridDim.x * gridDim.y * gridDim.z) - 1) {
-      *a.hcount = 0;
-      *a.done = 0;
-    }
-  }
   if (direct) return;
 
   // ---- the last CTA of this column tile: epilogue, then zero the sums -------
@@ -348,6 +349,7 @@ __global__ void __launch_bounds__(kMaxConsumers + 32, (TT <= 4) ? 2 : 1) gemv_ke
   if (!s_flag) return;
   __threadfence();
   if (tid == 0) *ticket = 0;                     // leave the counter clean
+  int nzc = 0;
   if (mine) {
     const size_t copy_stride = (size_t)P.mats * per_mat;
     for (int t = 0; t < ntok; ++t) {
@@ -370,9 +372,10 @@ __global__ void __launch_bounds__(kMaxConsumers + 32, (TT <= 4) ? 2 : 1) gemv_ke
           }
         }
       }
-      epilogue<WT, MODE>(a, tok, col, u, g);
+      nzc += epilogue<WT, MODE>(a, tok, col, u, g);
     }
   }
+  if constexpr (MODE != 0) add_hcount(a.hcount, nzc);
 }
 
 // ---- batched decode on the tensor cores ------------------------------------
@@ -631,7 +634,8 @@ __global__ void __launch_bounds__(kMmaWarps * 32 + 32, 2) gemv_mma_kernel(GemvAr
         for (int e = 0; e < V; ++e) gv[e] += __ldcg(pu + c * copy_stride + per_mat + (size_t)e * Tp);
       }
     }
-    epilogue<__nv_bfloat16, MODE>(a, tok, col, u, gv);
+    const int nz = epilogue<__nv_bfloat16, MODE>(a, tok, col, u, gv);
+    if (a.hcount != nullptr && nz != 0) atomicAdd(a.hcount, nz);
   }
 }
 

@@ -221,6 +221,9 @@ struct WsLayout {
   size_t xs_bf16 = 0;         // [T, d_in] bf16 (prefill)
   size_t alpha_parts = 0;     // f64 partial sums (ternary pack)
   size_t alpha = 0;           // f32 (ternary pack)
+  size_t fpug = 0;            // one-kernel FFN: per-split up/gate partial sums
+  size_t fpug_elems = 0;
+  size_t fhnz = 0;            // one-kernel FFN: nonzero h per index range (int32)
   size_t total = 0;
   size_t parts1_elems = 0, parts2_elems = 0;
   int ticket_topk_x = 0, ticket_topk_h = 0, ticket_g1 = 0, ticket_g2 = 0, ticket_alpha = 0;
@@ -264,6 +267,8 @@ struct TopkArgs {
                                    // the kernel that produced the row; read, then zeroed, here
   float* zero = nullptr;     // accumulators of the next kernel: set to 0 here
   size_t zero_n = 0;         // floats, multiple of 4
+  int32_t* zero_word = nullptr;    // a counter of later kernels: set to 0 here (after the wait)
+  int early_release = 0;     // release the next grid before waiting (it waits for this one)
   DevStatus* status = nullptr;
   // set by launch_topk from the sizes
   int stage = 0;             // the row's list (or idx) is staged in shared memory
@@ -310,12 +315,11 @@ struct GemvArgs {
   //   mode 1/2 add their nonzero h to it;
   //   mode 0 (the down projection) reads it: with at most k_sel nonzero h the
   //   kept rows are exactly the nonzero h, so each CTA takes them from its own
-  //   index range of hsrc instead of waiting for the top-K's list.  The grid's
-  //   last CTA (done ticket) clears the counter.
+  //   index range of hsrc instead of the top-K's list.  The first kernel of
+  //   the next FFN call (the top-K on x, TopkArgs::zero_word) clears it.
   int32_t* hcount = nullptr;
   const float* hsrc = nullptr;
   int k_sel = 0;
-  int32_t* done = nullptr;
   int32_t* rows_out = nullptr;   // mode 0 from h: the number of rows streamed (workspace stats)
   DevStatus* status = nullptr;
   // failure-detection testing only (qs_debug_inject): the producer issues no
@@ -360,6 +364,48 @@ struct QGemvArgs {
 };
 
 cudaError_t launch_qgemv(const QGemvArgs& a, cudaStream_t s);
+
+// ---- one-token FFN as one persistent kernel (ffn_fused.cu) -------------------
+struct FfnFusedPlan {
+  int G = 0;                   // CTAs (all resident: cooperative launch)
+  int n_ct_ug = 0, vt_ug = 0;  // up/gate column tiles, 16-byte vectors per tile
+  int n_ct_dn = 0, vt_dn = 0;  // down column tiles
+  int rps_ug = 0, rps_dn = 0;  // row tiles per ring stage
+  int S_ug = 0, S_dn = 0;      // index ranges (splits) of x and of h
+};
+struct FfnFusedArgs {
+  const void* x = nullptr;     // [d_model] bf16
+  const void* w_up = nullptr;  // W^T [d_model, d_ff] bf16
+  const void* w_gate = nullptr;
+  const void* w_down = nullptr;  // W^T [d_ff, d_model] bf16
+  int d_model = 0, d_ff = 0, k_in = 0, k_h = 0;
+  int act = 1;                 // 1: ReLU(u)^2 * g, 2: ReLU(g + b_gate) * ReLU(u + b_up)
+  const float* b_up = nullptr;
+  const float* b_gate = nullptr;
+  void* y = nullptr;           // [d_model] bf16
+  float* h = nullptr;          // [d_ff] f32
+  float* pug = nullptr;        // [S_ug][2][d_ff] per-split partial sums
+  float* pdn = nullptr;        // [d_model] down accumulator (cleared in the kernel)
+  int32_t* hnz = nullptr;      // [S_dn] nonzero h per index range
+  int32_t* bar = nullptr;      // [5] grid-barrier counters, zero between calls
+  int32_t* list_x = nullptr;
+  float* lval_x = nullptr;
+  int32_t* list_h = nullptr;
+  float* lval_h = nullptr;
+  int32_t* cnt = nullptr;      // [0] listed x rows, [1] listed h rows
+  DevStatus* status = nullptr;
+  // failure-detection testing only (qs_debug_inject): no weight copies, and
+  // the stage waits give up after wait_limit polls
+  int no_copies = 0;
+  uint32_t wait_limit = 0;
+  FfnFusedPlan plan{};
+};
+size_t ffn_fused_smem();
+bool plan_ffn_fused(int d_model, int d_ff, int G, FfnFusedPlan* p);
+size_t ffn_fused_pug_elems(int d_model, int d_ff);   // 0: the sizes are not supported
+int ffn_fused_grid();                                  // resident CTAs (0: unavailable)
+cudaError_t launch_ffn_fused(const FfnFusedArgs& a, cudaStream_t s);
+
 
 // The quantized FFN's gating of one column, float32 steps in a fixed order
 // (g: this projection, u: the up projection):

@@ -39,6 +39,19 @@ constexpr unsigned kFull = 0xffffffffu;
 
 // Key layout per input kind and the radix digits used to find the K-th key:
 // (shift, width) of each pass, most significant first.
+// Kernel entry: the programmatic-dependent-launch wait (with the next grid
+// released first when it waits for this one itself), then the counter that
+// this launch clears for later kernels.
+__device__ __forceinline__ void topk_begin(const TopkArgs& a) {
+  if (a.early_release) {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+  } else {
+    pdl_begin();
+  }
+  if (a.zero_word != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *a.zero_word = 0;
+}
+
 template <int KIND> struct KeyTraits;
 template <> struct KeyTraits<TK_F32> {
   static constexpr uint32_t kMask = 0x7fffffffu;  // |x| bits (31)
@@ -144,7 +157,7 @@ __global__ void __launch_bounds__(NT) topk_kernel(TopkArgs a) {
   const size_t rbase = (size_t)row * (size_t)d;
   int sbuf = 0;
 
-  pdl_begin();
+  topk_begin(a);
   if (row >= a.T) {
     // zeroing CTAs: clear the next kernel's accumulators, nothing else
     if (a.zero != nullptr) {
@@ -643,7 +656,7 @@ __global__ void __launch_bounds__(NT) topk_list_kernel(TopkArgs a) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint32_t lt = (1u << lane) - 1u;
 
-  pdl_begin();
+  topk_begin(a);
   if constexpr (!QUANT) {
     if (a.nz_bits != nullptr) {
       // The producer left a bitmask of the row's nonzero entries (d <= 32 NT,
@@ -1040,7 +1053,7 @@ __global__ void __launch_bounds__(NT) topk_reg_kernel(TopkArgs a) {
   const int nsel = (a.T + blk - 1) / blk;          // selection CTAs
   const int t0 = row * blk, t1 = min(a.T, t0 + blk);
 
-  pdl_begin();
+  topk_begin(a);
   if (row >= nsel) {
     if (a.zero != nullptr) {
       const size_t nthr = (size_t)a.zero_ctas * NT;
@@ -1290,7 +1303,7 @@ __global__ void __launch_bounds__(NT) topk_dense_bf16_kernel(TopkArgs a) {
   const uint16_t* xr = reinterpret_cast<const uint16_t*>(a.x) + (size_t)row * d;
   uint16_t* xsr = reinterpret_cast<uint16_t*>(a.xs) + (size_t)row * d;
 
-  pdl_begin();
+  topk_begin(a);
   for (int j = tid; j < NP * 256; j += NT) (&s_hist[0][0])[j] = 0;
   uint32_t ent[EPT];
   if (e0 + EPT <= d) {                               // d % 8 == 0: rows are 16-byte aligned
