@@ -376,7 +376,8 @@ __global__ void __launch_bounds__(kFThreads, 2) ffn_fused_kernel(FfnFusedArgs a)
   int n_x = 0;
   if (ug_active) {                                 // (block-uniform)
     // (an even split of the kept rows by list position measured slower: the
-    // listing costs more than the balance saves)
+    // splits' finish times spread by about 4 us even with equal row counts,
+    // from uneven bandwidth across the SMs, and the listing costs more)
     const Selection Sx = select_topk(xkey, d_model, a.k_in, 15, r0, whist, s_hist, s_pick,
                                      reinterpret_cast<int*>(s_w));
     n_x = list_range(Sx, xkey, xval, r0, r1, s_rows, s_vals, s_w);
