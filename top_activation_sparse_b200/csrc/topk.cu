@@ -828,9 +828,9 @@ template <int KIND>
 __device__ __forceinline__ bool block_vectorized(int d) { return (d % vec_width<KIND>()) == 0; }
 
 // Quant kinds: 127 / gamma_t of every row of the block (one warp per row, its
-// lanes reading 16-byte vectors), published to a.gamma and s_bscale.
+// lanes reading 16-byte vectors) into s_bscale; gamma of row `own` to a.gamma.
 template <int KIND, int NT>
-__device__ void block_scales(const TopkArgs& a, int t0, int t1, float* s_bscale) {
+__device__ void block_scales(const TopkArgs& a, int t0, int t1, int own, float* s_bscale) {
   constexpr int V = vec_width<KIND>();
   constexpr int NW = NT / 32;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -854,7 +854,7 @@ __device__ void block_scales(const TopkArgs& a, int t0, int t1, float* s_bscale)
     m = __reduce_max_sync(kFull, m);
     if (lane == 0) {
       const float gamma = __fadd_rn(__uint_as_float(m), a.eps);
-      if (a.gamma) a.gamma[t] = gamma;
+      if (a.gamma && t == own) a.gamma[t] = gamma;
       s_bscale[t - t0] = __fdiv_rn(127.0f, gamma);
     }
   }
@@ -913,16 +913,16 @@ __device__ void block_keys(const TopkArgs& a, int t0, int t1, uint32_t* s_key, c
   __syncthreads();
 }
 
-// Every row's dense outputs of the block (mask, X_sparse, the masked copies,
-// the codes) in one flattened (row, vector) loop, from the selection bitmask
-// s_sel (bit e = feature e kept); then idx / val of rows t0+1.. from row t0's.
+// The dense outputs of rows [t0, t1) (mask, X_sparse, the masked copies, the
+// codes) in one flattened (row, vector) loop, from the selection bitmask s_sel
+// (bit e = feature e kept); s_bscale[t - t0] = 127 / gamma_t (quant kinds).
 template <int KIND, int NT>
 __device__ void block_outputs(const TopkArgs& a, int t0, int t1, const uint32_t* s_sel,
                               const float* s_bscale) {
   constexpr bool QUANT = (KIND == TK_QUANT_F32 || KIND == TK_QUANT_BF16);
   constexpr int V = vec_width<KIND>();
   const int tid = threadIdx.x;
-  const int d = a.d, k = a.k;
+  const int d = a.d;
   const bool dense = a.mask || a.xs || a.xsf || a.xq || a.q_full;
   auto one = [&](int t, int e, uint32_t raw) {
     const size_t o = (size_t)t * d + e;
@@ -1005,18 +1005,6 @@ __device__ void block_outputs(const TopkArgs& a, int t0, int t1, const uint32_t*
       }
     }
   }
-  if (a.idx != nullptr && k > 0) {
-    for (int i = tid; i < (t1 - t0 - 1) * k; i += NT) {
-      const int t = t0 + 1 + i / k, p = i - (i / k) * k;
-      const int e = __ldcg(a.idx + (size_t)t0 * k + p);
-      a.idx[(size_t)t * k + p] = e;
-      if (a.val) {
-        const uint32_t raw = load_raw<KIND>(a.x, (size_t)t * d + e);
-        if constexpr (KIND == TK_F32) reinterpret_cast<uint32_t*>(a.val)[(size_t)t * k + p] = raw;
-        else if constexpr (KIND == TK_BF16) reinterpret_cast<uint16_t*>(a.val)[(size_t)t * k + p] = (uint16_t)raw;
-      }
-    }
-  }
 }
 
 template <int KIND, int NT, int EPT, bool BLOCK>
@@ -1041,8 +1029,10 @@ __global__ void __launch_bounds__(NT) topk_reg_kernel(TopkArgs a) {
   __shared__ uint32_t s_bsel[BLOCK ? kMaxBlockRow / 32 : 1]; // Block Q-Sparse: kept features
   extern __shared__ uint32_t s_bkey[];                       // Block Q-Sparse: [d] block keys
 
-  // One CTA per selection: a token row, or (Block Q-Sparse, a.block > 1) a
-  // block of a.block consecutive token rows that shares one selection.
+  // One CTA per token row.  Block Q-Sparse (a.block > 1): the rows of a block
+  // of a.block consecutive tokens share one selection, which each of the
+  // block's CTAs computes (the same result: the same inputs and order) and
+  // uses for its own row's outputs.
   const int row = blockIdx.x;
   const int d = a.d;
   const int k = a.k;
@@ -1050,8 +1040,8 @@ __global__ void __launch_bounds__(NT) topk_reg_kernel(TopkArgs a) {
   const size_t rbase = (size_t)row * (size_t)d;
   const uint32_t lt = (1u << lane) - 1u;
   const int blk = BLOCK ? a.block : 1;   // the per-row instantiation keeps no block code
-  const int nsel = (a.T + blk - 1) / blk;          // selection CTAs
-  const int t0 = row * blk, t1 = min(a.T, t0 + blk);
+  const int nsel = a.T;                            // row CTAs
+  const int t0 = (row / blk) * blk, t1 = min(a.T, t0 + blk);   // this row's block
 
   topk_begin(a);
   if (row >= nsel) {
@@ -1071,7 +1061,7 @@ __global__ void __launch_bounds__(NT) topk_reg_kernel(TopkArgs a) {
     // Block Q-Sparse: the key of feature e is the block magnitude, the
     // largest |x| (or |q|) over the block's rows; values are read again below
     if constexpr (QUANT) {
-      block_scales<KIND, NT>(a, t0, t1, s_bscale);
+      block_scales<KIND, NT>(a, t0, t1, row, s_bscale);
       __syncthreads();
     }
     block_keys<KIND, NT>(a, t0, t1, s_bkey, s_bscale);
@@ -1185,17 +1175,17 @@ __global__ void __launch_bounds__(NT) topk_reg_kernel(TopkArgs a) {
     const int eqnz_b = (int)s_cnz[j * NW + warp] + __popc(bz & lt);
     const bool sel = gt || (eq && eq_b < remaining);
     if constexpr (BLOCK) {
-      // Block Q-Sparse: row t0's idx / val here, every row's other outputs
-      // after the loop from the selection bitmask
+      // Block Q-Sparse: this row's idx / val here, its other outputs after
+      // the loop from the selection bitmask
       const uint32_t bs = __ballot_sync(kFull, sel);
       if (lane == 0 && j * NT + warp * 32 < d) s_bsel[(j * NT + warp * 32) >> 5] = bs;
       if (sel) {
         const int pos = gt_b + min(eq_b, remaining);
         if (pos < k) {
-          const size_t o = (size_t)t0 * k + pos;
+          const size_t o = (size_t)row * k + pos;
           if (a.idx) a.idx[o] = e;
           if (a.val) {
-            const uint32_t raw = load_raw<KIND>(a.x, (size_t)t0 * d + e);
+            const uint32_t raw = load_raw<KIND>(a.x, (size_t)row * d + e);
             if constexpr (KIND == TK_F32) reinterpret_cast<uint32_t*>(a.val)[o] = raw;
             else if constexpr (KIND == TK_BF16) reinterpret_cast<uint16_t*>(a.val)[o] = (uint16_t)raw;
           }
@@ -1245,8 +1235,8 @@ __global__ void __launch_bounds__(NT) topk_reg_kernel(TopkArgs a) {
   }
 
   if constexpr (BLOCK) {
-    __syncthreads();                                 // s_bsel and row t0's idx complete
-    block_outputs<KIND, NT>(a, t0, t1, s_bsel, s_bscale);
+    __syncthreads();                                 // s_bsel complete
+    block_outputs<KIND, NT>(a, row, row + 1, s_bsel, s_bscale + (row - t0));
   }
 
   // ---- 4. union of the rows' kept nonzeros (several tokens) ------------------
@@ -1361,10 +1351,8 @@ __global__ void __launch_bounds__(NT) topk_dense_bf16_kernel(TopkArgs a) {
   }
 }
 
-int selections(const TopkArgs& a) {
-  const int b = a.block > 1 ? a.block : 1;
-  return (a.T + b - 1) / b;
-}
+// Row CTAs of a launch (Block Q-Sparse included: one CTA per token row).
+int selections(const TopkArgs& a) { return a.T; }
 
 bool dense_only_bf16(const TopkArgs& a) {
   return a.block <= 1 && a.kind == TK_BF16 && a.xs != nullptr && a.idx == nullptr && a.val == nullptr &&
