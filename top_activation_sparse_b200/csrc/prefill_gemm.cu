@@ -335,6 +335,252 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+
+// ---- prefill forward with 2-SM tiles (tcgen05 cta_group::2) -----------------
+// A cluster of two CTAs (on two SMs) computes a 256 x 256 tile of Y: each CTA
+// loads its own 128 rows of X_sparse and its own 128-column half of the W^T
+// tile (so each SM reads half of B from L2: 32 KB per stage instead of 48), the
+// first CTA of the pair issues tcgen05.mma.cta_group::2 (M = 256: the
+// accumulator rows are split over the two CTAs' tensor memory, the B operand
+// is read from both CTAs' shared memory), and each CTA's epilogue stores its
+// own 128 rows.  Loads are plain (no multicast): each CTA's copies signal the
+// first CTA's stage barrier (its address through mapa); the MMA commits
+// multicast their arrivals to both CTAs' barriers.
+constexpr int k2Stages = 6;
+constexpr int k2ABytes = 128 * BK * 2;               // 16 KB: this CTA's 128 rows
+constexpr int k2BBytes = 2 * kBBox;                  // 16 KB: this CTA's 128 columns (two boxes)
+constexpr int k2StageBytes = k2ABytes + k2BBytes;    // 32 KB
+// + 16 KB of slack after the ring: no operand read can leave the allocation
+constexpr int k2SmemBytes = k2Stages * k2StageBytes + 16 * 1024 + 1024;
+constexpr int k2EpiWarps = 4;
+
+// kind::f16: D f32, A bf16 K-major, B bf16 MN-major, N = 256, M = 256 (pair)
+constexpr uint32_t idesc_2sm() {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (0u << 15) | (1u << 16) | ((uint32_t)(256 >> 3) << 17) |
+         ((uint32_t)(256 >> 4) << 24);
+}
+
+__device__ __forceinline__ uint32_t cluster_addr(uint32_t local, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
+  return r;
+}
+
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                                 uint32_t bar_cluster) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar_cluster)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_bf16_pair(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                               uint32_t idesc_bits, uint32_t accumulate) {
+  const uint32_t z = 0u;                           // no output lane is disabled
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.u32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, {%5, %5, %5, %5, %5, %5, %5, %5}, p;\n}\n" ::"r"(
+          tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc_bits), "r"(accumulate), "r"(z)
+      : "memory");
+}
+
+// arrives on the barrier at the same offset in both CTAs of the pair once the
+// MMAs issued so far have completed
+__device__ __forceinline__ void umma_commit_pair(uint64_t* bar) {
+  const uint16_t mask = 0x3;
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"(mask)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_commit_pair_local(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
+}
+
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    umma_gemm_2sm_kernel(const __grid_constant__ CUtensorMap map_a,
+                         const __grid_constant__ CUtensorMap map_b, __nv_bfloat16* __restrict__ out,
+                         int ldo, int M, int N, int K, DevStatus* status) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  pdl_begin();
+  __shared__ __align__(8) uint64_t s_full[k2Stages];   // first CTA: both CTAs' copies of a stage
+  __shared__ __align__(8) uint64_t s_empty[k2Stages];  // each CTA: the stage's MMAs are done
+  __shared__ __align__(8) uint64_t s_tfull[2];         // each CTA: accumulator b complete
+  __shared__ __align__(8) uint64_t s_tempty[2];        // first CTA: both epilogues drained b
+  __shared__ __align__(8) uint64_t s_done;             // first CTA: every MMA has completed
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_abort;
+
+  const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = blockIdx.x & 1u;             // position in the pair (cluster of 2)
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int mblocks = (M + 255) / 256;
+  const int ntiles = mblocks * ((N + BN - 1) / BN);
+  const int nk = (K + BK - 1) / BK;
+  const int my_tiles = pair < ntiles ? (ntiles - 1 - pair) / npairs + 1 : 0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < k2Stages; ++s) {
+      mbar_init(&s_full[s], 1);
+      mbar_init(&s_empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&s_tfull[b], 1);
+      mbar_init(&s_tempty[b], 2 * k2EpiWarps);
+    }
+    mbar_init(&s_done, 1);
+    mbar_fence_init();
+    s_abort = 0;
+  }
+  if (warp == 0) {   // the same warp of both CTAs: the pair's accumulators (2 x 256 columns)
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&s_tmem)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();                                // the peer's barriers exist before any signal
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+
+  if (warp == 0 && lane == 0) {
+    // ---- TMA producer (both CTAs) ----
+    int it = 0;
+    for (int lt = 0; lt < my_tiles && !*(volatile int*)&s_abort; ++lt) {
+      const int t = pair + lt * npairs;
+      const int m0 = (t % mblocks) * 256 + (int)rank * 128, n0 = (t / mblocks) * BN + (int)rank * 128;
+      for (int kb = 0; kb < nk; ++kb, ++it) {
+        const int s = it % k2Stages;
+        if (it >= k2Stages && !mbar_wait(&s_empty[s], (uint32_t)((it / k2Stages) - 1) & 1u)) {
+          dev_fail(status, DEV_TIMEOUT, 24, (uint32_t)it);
+          atomicExch(&s_abort, 1);
+          break;
+        }
+        if (*(volatile int*)&s_abort) break;
+        const uint32_t sa = base + (uint32_t)(s * k2StageBytes);
+        const uint32_t sb = sa + k2ABytes;
+        const uint32_t full0 = cluster_addr(smem_u32(&s_full[s]), 0);
+        if (leader) mbar_arrive_expect_tx(&s_full[s], (uint32_t)(2 * k2StageBytes));
+        tma_load_2d_pair(sa, &map_a, kb * BK, m0, full0);               // 64 (K) x 128 (M)
+#pragma unroll
+        for (int j = 0; j < 2; ++j)                                        // 2 x 64 (N) x 64 (K)
+          tma_load_2d_pair(sb + j * kBBox, &map_b, n0 + 64 * j, kb * BK, full0);
+      }
+    }
+    // on an abort, the first CTA lets the copies already issued (both CTAs') land
+    if (leader && *(volatile int*)&s_abort) {
+      for (int i = 0; i < k2Stages && i < it; ++i) {
+        const int g = it - 1 - i;
+        mbar_wait(&s_full[g % k2Stages], (uint32_t)(g / k2Stages) & 1u);
+      }
+    }
+  } else if (warp == 1 && lane == 0 && leader) {
+    // ---- MMA issuer (first CTA only) ----
+    int it = 0;
+    bool issued = false;
+    for (int lt = 0; lt < my_tiles && !*(volatile int*)&s_abort; ++lt) {
+      const int b = lt & 1;
+      if (lt >= 2 && !mbar_wait(&s_tempty[b], (uint32_t)((lt >> 1) - 1) & 1u)) {
+        dev_fail(status, DEV_TIMEOUT, 25, (uint32_t)lt);
+        atomicExch(&s_abort, 1);
+        break;
+      }
+      tc_fence_after();
+      const uint32_t acc = tmem + (uint32_t)(b * BN);
+      for (int kb = 0; kb < nk; ++kb, ++it) {
+        const int s = it % k2Stages;
+        if (!mbar_wait(&s_full[s], (uint32_t)(it / k2Stages) & 1u)) {
+          dev_fail(status, DEV_TIMEOUT, 26, (uint32_t)it);
+          atomicExch(&s_abort, 1);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t sa = base + (uint32_t)(s * k2StageBytes);
+        const uint32_t sb = sa + k2ABytes;
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; ++kk) {
+          const uint64_t ad = smem_desc(sa + kk * 32, 16, 1024);          // K-major A
+          const uint64_t bd = smem_desc(sb + kk * 2048, kBBox, 1024);     // MN-major B
+          umma_bf16_pair(acc, ad, bd, idesc_2sm(), (kb > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit_pair(&s_empty[s]);     // frees the stage in both CTAs
+        issued = true;
+      }
+      umma_commit_pair(&s_tfull[b]);       // accumulator b complete in both CTAs
+    }
+    if (issued) {
+      umma_commit_pair_local(&s_done);
+      mbar_wait(&s_done, 0u);
+    }
+  } else if (warp >= 2) {
+    // ---- epilogue (both CTAs): this CTA's 128 rows of the tile ----
+    const int q = warp & 3;
+    const uint32_t tempty0[2] = {cluster_addr(smem_u32(&s_tempty[0]), 0),
+                                 cluster_addr(smem_u32(&s_tempty[1]), 0)};
+    for (int lt = 0; lt < my_tiles; ++lt) {
+      const int b = lt & 1;
+      const int t = pair + lt * npairs;
+      const int m0 = (t % mblocks) * 256 + (int)rank * 128, n0 = (t / mblocks) * BN;
+      if (!mbar_wait_backoff(&s_tfull[b], (uint32_t)(lt >> 1) & 1u)) {
+        if (lane == 0) dev_fail(status, DEV_TIMEOUT, 27, (uint32_t)lt);
+        atomicExch(&s_abort, 1);
+        break;
+      }
+      tc_fence_after();
+      const bool abort = *(volatile int*)&s_abort;
+      const int row = m0 + q * 32 + lane;
+      const uint32_t acc = tmem + (uint32_t)(b * BN) + ((uint32_t)(q * 32) << 16);
+#pragma unroll 1
+      for (int c = 0; c < BN; c += 32) {
+        uint32_t r[32];
+        tmem_ld32(acc + (uint32_t)c, r);
+        if (abort || row >= M) continue;
+        __nv_bfloat16* dst = out + (size_t)row * ldo + n0 + c;
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          if (n0 + c + 8 * v + 8 > N) break;       // N is a multiple of 8
+          uint4 o;
+          o.x = pack_bf16x2(r[8 * v + 0], r[8 * v + 1]);
+          o.y = pack_bf16x2(r[8 * v + 2], r[8 * v + 3]);
+          o.z = pack_bf16x2(r[8 * v + 4], r[8 * v + 5]);
+          o.w = pack_bf16x2(r[8 * v + 6], r[8 * v + 7]);
+          *reinterpret_cast<uint4*>(dst + 8 * v) = o;
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(tempty0[b]);   // this warp's reads of accumulator b are done
+      if (abort) break;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();                                // both CTAs are done with the pair's TMEM
+  if (warp == 0) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static std::once_flag once;
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -387,6 +633,57 @@ cudaError_t launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, void* out,
   return cudaGetLastError();
 }
 
+// Pairs of CTAs resident at once for the 2-SM kernel (0: not available).
+int pair_clusters() {
+  static int n = -1;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    n = 0;
+    if (cudaFuncSetAttribute(umma_gemm_2sm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             k2SmemBytes) != cudaSuccess)
+      return;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * kNumSMs);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = (size_t)k2SmemBytes;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int c = 0;
+    if (cudaOccupancyMaxActiveClusters(&c, umma_gemm_2sm_kernel, &cfg) == cudaSuccess && c > 0) n = c;
+    (void)cudaGetLastError();
+  });
+  return n;
+}
+
+cudaError_t launch_prefill_2sm(const CUtensorMap& ma, const CUtensorMap& mb, const PrefillArgs& a,
+                               int clusters, cudaStream_t s) {
+  const int tiles = ((a.M + 255) / 256) * ((a.N + BN - 1) / BN);
+  const int pairs = tiles < clusters ? tiles : clusters;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(2 * pairs));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = (size_t)k2SmemBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, umma_gemm_2sm_kernel, ma, mb,
+                                     reinterpret_cast<__nv_bfloat16*>(a.y), a.N, a.M, a.N, a.K, a.status);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_prefill_gemm(const PrefillArgs& a, cudaStream_t s) {
@@ -397,6 +694,9 @@ cudaError_t launch_prefill_gemm(const PrefillArgs& a, cudaStream_t s) {
   // B = W^T [K, N] row-major: inner N, box 64 (N) x 64 (K)
   if (!make_map(&mb, a.wt, (uint64_t)a.N, (uint64_t)a.K, (uint64_t)a.N * 2, 64, BK))
     return cudaErrorInvalidValue;
+  // pairs of SMs on one 256 x 256 tile (each loads half of the W^T tile)
+  const int clusters = pair_clusters();
+  if (clusters > 0) return launch_prefill_2sm(ma, mb, a, clusters, s);
   return launch_gemm<false, true, EPI_BF16>(ma, mb, a.y, a.N, a.M, a.N, a.K, a.status, s);
 }
 
