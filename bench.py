@@ -410,6 +410,8 @@ def setup_ffn(args, qs, torch, device, stream, rank):
         "fn": fn, "T": T, "n_layers": n_layers, "ws": ws, "x": x, "y": y,
         "args": lambda l, ev: c_args(l, ev), "n_events": qs.QS_FFN_PHASE_EVENTS,
         "dense_args": (lambda l: c_args(l, None, d_model, d_ff)),
+        "dense_note": ("gate-first path with K_h = d_ff: W_up is still read only for open gates"
+                       if gate_first else None),
         "phases": phases, "dominant": dominant,
         "kernel": kernel,
         "bound": "hbm", "dom_work": dom_work, "layer_work": upgate_bytes + down_bytes + topk_bytes,
@@ -845,6 +847,8 @@ def run_ours(args, rank, world, local):
         torch.cuda.synchronize()
         dense_ms = d0.elapsed_time(d1) / n_dense
         dense = {"ms_per_step": round(dense_ms, 6), "value": round(T / (dense_ms / 1e3), 1)}
+        if c.get("dense_note"):
+            dense["note"] = c["dense_note"]
 
     # end to end through the public Python API, host buffers in and out
     x, y = c["x"], c["y"]

@@ -440,6 +440,12 @@ qs_status qs_debug_inject(int mode, unsigned wait_polls);
 /* Human-readable name of a status code (static string). */
 const char* qs_status_string(int status);
 
+/* Device state kept per process: the library caches, per device ordinal, the
+ * address of two static device arrays (a vector of 1.0 used by the gate-first
+ * FFN, and the scratch array of qs_sparse_linear_noalloc).  cudaDeviceReset
+ * (or any new primary context on a device) invalidates them and is not
+ * supported while the library is in use in the process. */
+
 /* Size of the fixed device scratch array behind qs_sparse_linear_noalloc. */
 #define QS_NOALLOC_SCRATCH_BYTES (4u << 20)
 
