@@ -354,10 +354,12 @@ constexpr int k2StageBytes = k2ABytes + k2BBytes;    // 32 KB
 constexpr int k2SmemBytes = k2Stages * k2StageBytes + 16 * 1024 + 1024;
 constexpr int k2EpiWarps = 4;
 
-// kind::f16: D f32, A bf16 K-major, B bf16 MN-major, N = 256, M = 256 (pair)
+// kind::f16: D f32, A and B bf16 (bits 15 / 16: MN-major A / B), N = 256,
+// M = 256 (the pair)
+template <bool A_MN, bool B_MN>
 constexpr uint32_t idesc_2sm() {
-  return (1u << 4) | (1u << 7) | (1u << 10) | (0u << 15) | (1u << 16) | ((uint32_t)(256 >> 3) << 17) |
-         ((uint32_t)(256 >> 4) << 24);
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((A_MN ? 1u : 0u) << 15) | ((B_MN ? 1u : 0u) << 16) |
+         ((uint32_t)(256 >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
 }
 
 __device__ __forceinline__ uint32_t cluster_addr(uint32_t local, uint32_t rank) {
@@ -411,9 +413,13 @@ __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
+// The operand major-ness and the epilogue as in umma_gemm_kernel: the forward
+// prefill is <K-major A, MN-major B, bf16>, the STE backward's dL/dX
+// <K-major, K-major, f32> and dL/dW^T <MN-major, MN-major, f32 add>.
+template <bool A_MN, bool B_MN, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
     umma_gemm_2sm_kernel(const __grid_constant__ CUtensorMap map_a,
-                         const __grid_constant__ CUtensorMap map_b, __nv_bfloat16* __restrict__ out,
+                         const __grid_constant__ CUtensorMap map_b, void* __restrict__ out,
                          int ldo, int M, int N, int K, DevStatus* status) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   pdl_begin();
@@ -479,10 +485,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t sb = sa + k2ABytes;
         const uint32_t full0 = cluster_addr(smem_u32(&s_full[s]), 0);
         if (leader) mbar_arrive_expect_tx(&s_full[s], (uint32_t)(2 * k2StageBytes));
-        tma_load_2d_pair(sa, &map_a, kb * BK, m0, full0);               // 64 (K) x 128 (M)
+        if constexpr (A_MN) {                      // 2 x 64 (M) x 64 (K)
 #pragma unroll
-        for (int j = 0; j < 2; ++j)                                        // 2 x 64 (N) x 64 (K)
-          tma_load_2d_pair(sb + j * kBBox, &map_b, n0 + 64 * j, kb * BK, full0);
+          for (int j = 0; j < 2; ++j) tma_load_2d_pair(sa + j * kBBox, &map_a, m0 + 64 * j, kb * BK, full0);
+        } else {                                   // 64 (K) x 128 (M)
+          tma_load_2d_pair(sa, &map_a, kb * BK, m0, full0);
+        }
+        if constexpr (B_MN) {                      // 2 x 64 (N) x 64 (K)
+#pragma unroll
+          for (int j = 0; j < 2; ++j) tma_load_2d_pair(sb + j * kBBox, &map_b, n0 + 64 * j, kb * BK, full0);
+        } else {                                   // 64 (K) x 128 (N)
+          tma_load_2d_pair(sb, &map_b, kb * BK, n0, full0);
+        }
       }
     }
     // on an abort, the first CTA lets the copies already issued (both CTAs') land
@@ -517,9 +531,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t sb = sa + k2ABytes;
 #pragma unroll
         for (int kk = 0; kk < BK / 16; ++kk) {
-          const uint64_t ad = smem_desc(sa + kk * 32, 16, 1024);          // K-major A
-          const uint64_t bd = smem_desc(sb + kk * 2048, kBBox, 1024);     // MN-major B
-          umma_bf16_pair(acc, ad, bd, idesc_2sm(), (kb > 0 || kk > 0) ? 1u : 0u);
+          const uint64_t ad = A_MN ? smem_desc(sa + kk * 2048, kBBox, 1024) : smem_desc(sa + kk * 32, 16, 1024);
+          const uint64_t bd = B_MN ? smem_desc(sb + kk * 2048, kBBox, 1024) : smem_desc(sb + kk * 32, 16, 1024);
+          umma_bf16_pair(acc, ad, bd, idesc_2sm<A_MN, B_MN>(), (kb > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit_pair(&s_empty[s]);     // frees the stage in both CTAs
         issued = true;
@@ -553,16 +567,37 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t r[32];
         tmem_ld32(acc + (uint32_t)c, r);
         if (abort || row >= M) continue;
-        __nv_bfloat16* dst = out + (size_t)row * ldo + n0 + c;
+        if constexpr (EPI == EPI_BF16) {
+          __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(out) + (size_t)row * ldo + n0 + c;
 #pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          if (n0 + c + 8 * v + 8 > N) break;       // N is a multiple of 8
-          uint4 o;
-          o.x = pack_bf16x2(r[8 * v + 0], r[8 * v + 1]);
-          o.y = pack_bf16x2(r[8 * v + 2], r[8 * v + 3]);
-          o.z = pack_bf16x2(r[8 * v + 4], r[8 * v + 5]);
-          o.w = pack_bf16x2(r[8 * v + 6], r[8 * v + 7]);
-          *reinterpret_cast<uint4*>(dst + 8 * v) = o;
+          for (int v = 0; v < 4; ++v) {
+            if (n0 + c + 8 * v + 8 > N) break;     // N is a multiple of 8
+            uint4 o;
+            o.x = pack_bf16x2(r[8 * v + 0], r[8 * v + 1]);
+            o.y = pack_bf16x2(r[8 * v + 2], r[8 * v + 3]);
+            o.z = pack_bf16x2(r[8 * v + 4], r[8 * v + 5]);
+            o.w = pack_bf16x2(r[8 * v + 6], r[8 * v + 7]);
+            *reinterpret_cast<uint4*>(dst + 8 * v) = o;
+          }
+        } else {
+          float* dst = reinterpret_cast<float*>(out) + (size_t)row * ldo + n0 + c;
+#pragma unroll
+          for (int v = 0; v < 8; ++v) {
+            if (n0 + c + 4 * v + 4 > N) break;     // N is a multiple of 4
+            float4 o = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                                   __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
+            if constexpr (EPI == EPI_F32_ADD) {
+              // add into the existing values; a sum of exactly zero (no kept
+              // input in this row) leaves them untouched
+              if (o.x == 0.0f && o.y == 0.0f && o.z == 0.0f && o.w == 0.0f) continue;
+              const float4 p = *reinterpret_cast<const float4*>(dst + 4 * v);
+              if (o.x != 0.0f) o.x += p.x; else o.x = p.x;
+              if (o.y != 0.0f) o.y += p.y; else o.y = p.y;
+              if (o.z != 0.0f) o.z += p.z; else o.z = p.z;
+              if (o.w != 0.0f) o.w += p.w; else o.w = p.w;
+            }
+            *reinterpret_cast<float4*>(dst + 4 * v) = o;
+          }
         }
       }
       tc_fence_before();
@@ -633,14 +668,15 @@ cudaError_t launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, void* out,
   return cudaGetLastError();
 }
 
-// Pairs of CTAs resident at once for the 2-SM kernel (0: not available).
+// Pairs of CTAs resident at once for one 2-SM kernel instance (0: not available).
+template <bool A_MN, bool B_MN, int EPI>
 int pair_clusters() {
   static int n = -1;
   static std::once_flag once;
   std::call_once(once, [] {
     n = 0;
-    if (cudaFuncSetAttribute(umma_gemm_2sm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             k2SmemBytes) != cudaSuccess)
+    if (cudaFuncSetAttribute(umma_gemm_2sm_kernel<A_MN, B_MN, EPI>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, k2SmemBytes) != cudaSuccess)
       return;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * kNumSMs);
@@ -654,15 +690,18 @@ int pair_clusters() {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int c = 0;
-    if (cudaOccupancyMaxActiveClusters(&c, umma_gemm_2sm_kernel, &cfg) == cudaSuccess && c > 0) n = c;
+    if (cudaOccupancyMaxActiveClusters(&c, umma_gemm_2sm_kernel<A_MN, B_MN, EPI>, &cfg) == cudaSuccess &&
+        c > 0)
+      n = c;
     (void)cudaGetLastError();
   });
   return n;
 }
 
-cudaError_t launch_prefill_2sm(const CUtensorMap& ma, const CUtensorMap& mb, const PrefillArgs& a,
-                               int clusters, cudaStream_t s) {
-  const int tiles = ((a.M + 255) / 256) * ((a.N + BN - 1) / BN);
+template <bool A_MN, bool B_MN, int EPI>
+cudaError_t launch_gemm_2sm(const CUtensorMap& ma, const CUtensorMap& mb, void* out, int ldo, int M,
+                            int N, int K, DevStatus* status, int clusters, cudaStream_t s) {
+  const int tiles = ((M + 255) / 256) * ((N + BN - 1) / BN);
   const int pairs = tiles < clusters ? tiles : clusters;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(2 * pairs));
@@ -678,8 +717,8 @@ cudaError_t launch_prefill_2sm(const CUtensorMap& ma, const CUtensorMap& mb, con
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, umma_gemm_2sm_kernel, ma, mb,
-                                     reinterpret_cast<__nv_bfloat16*>(a.y), a.N, a.M, a.N, a.K, a.status);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, umma_gemm_2sm_kernel<A_MN, B_MN, EPI>, ma, mb, out, ldo, M,
+                                     N, K, status);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -695,8 +734,9 @@ cudaError_t launch_prefill_gemm(const PrefillArgs& a, cudaStream_t s) {
   if (!make_map(&mb, a.wt, (uint64_t)a.N, (uint64_t)a.K, (uint64_t)a.N * 2, 64, BK))
     return cudaErrorInvalidValue;
   // pairs of SMs on one 256 x 256 tile (each loads half of the W^T tile)
-  const int clusters = pair_clusters();
-  if (clusters > 0) return launch_prefill_2sm(ma, mb, a, clusters, s);
+  const int clusters = pair_clusters<false, true, EPI_BF16>();
+  if (clusters > 0)
+    return launch_gemm_2sm<false, true, EPI_BF16>(ma, mb, a.y, a.N, a.M, a.N, a.K, a.status, clusters, s);
   return launch_gemm<false, true, EPI_BF16>(ma, mb, a.y, a.N, a.M, a.N, a.K, a.status, s);
 }
 
@@ -711,9 +751,15 @@ cudaError_t launch_grad_x_gemm(const BackwardGemmArgs& a, cudaStream_t s) {
   // A = dL/dY: M = T rows, K = d_out contiguous (K-major), box 64 (K) x 128 (M)
   if (!make_map(&ma, a.grad_y, (uint64_t)a.d_out, (uint64_t)a.T, (uint64_t)a.d_out * 2, BK, BM))
     return cudaErrorInvalidValue;
-  // B = W^T: N = d_in rows, K = d_out contiguous (K-major), box 64 (K) x 256 (N)
-  if (!make_map(&mb, a.wt, (uint64_t)a.d_out, (uint64_t)a.d_in, (uint64_t)a.d_out * 2, BK, BN))
+  // B = W^T: N = d_in rows, K = d_out contiguous (K-major): box 64 (K) x 128 (N) for a CTA of a
+  // pair (2-SM tiles), else 64 x 256
+  const int clusters = pair_clusters<false, false, EPI_F32>();
+  if (!make_map(&mb, a.wt, (uint64_t)a.d_out, (uint64_t)a.d_in, (uint64_t)a.d_out * 2, BK,
+                clusters > 0 ? 128 : BN))
     return cudaErrorInvalidValue;
+  if (clusters > 0)
+    return launch_gemm_2sm<false, false, EPI_F32>(ma, mb, a.grad_x, a.d_in, a.T, a.d_in, a.d_out,
+                                                  a.status, clusters, s);
   return launch_gemm<false, false, EPI_F32>(ma, mb, a.grad_x, a.d_in, a.T, a.d_in, a.d_out,
                                             a.status, s);
 }
@@ -727,6 +773,10 @@ cudaError_t launch_grad_wt_gemm(const BackwardGemmArgs& a, cudaStream_t s) {
   // B = dL/dY [T, d_out]: N = d_out contiguous (MN-major), K = T; box 64 x 64
   if (!make_map(&mb, a.grad_y, (uint64_t)a.d_out, (uint64_t)a.T, (uint64_t)a.d_out * 2, 64, BK))
     return cudaErrorInvalidValue;
+  const int clusters = pair_clusters<true, true, EPI_F32_ADD>();
+  if (clusters > 0)
+    return launch_gemm_2sm<true, true, EPI_F32_ADD>(ma, mb, a.grad_wt, a.d_out, a.d_in, a.d_out, a.T,
+                                                    a.status, clusters, s);
   return launch_gemm<true, true, EPI_F32_ADD>(ma, mb, a.grad_wt, a.d_out, a.d_in, a.d_out, a.T,
                                               a.status, s);
 }
