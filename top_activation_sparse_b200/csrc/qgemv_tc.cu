@@ -11,20 +11,22 @@
 // packed row of W^T in order (2-D TMA, no gather) and multiplies it with the
 // dense masked codes (zero where a token dropped the input):
 //   * a CTA owns 256 output columns (two MMAs of M = 128) and a range of
-//     rows; per step of 32 rows (the MMA's K) one TMA brings the 32 x 64-byte
-//     packed segment and one TMA the tokens' 32 codes each (K-major, 32-byte
-//     swizzle), into a ring of stages;
+//     rows; per step of 64 rows (two of the MMA's K = 32) one TMA brings the
+//     64 x 64-byte packed segment and two TMAs the tokens' codes (32 rows
+//     each, K-major, 32-byte swizzle), into a ring of 4 stages (fewer barrier
+//     handshakes per byte than 32-row steps: each costs shared-memory round
+//     trips in the single-thread loops);
 //   * eight decode warps, in four groups that take every fourth step (their
 //     proxy fences overlap), expand the 2-bit codes (00 = 0, 01 = +1, 10 = -1) into
 //     int8 (the codes are spread into nibbles, and one byte permute per four
 //     codes selects from the bytes {0, +1, -1}) and write the two A tiles in
 //     the MN-major 128-byte-swizzled layout
-//     (each 32-row x 128-byte tile: row k holds columns 0..127, 16-byte chunk
+//     (each 64-row x 128-byte tile: row k holds columns 0..127, 16-byte chunk
 //     c of row k at chunk c ^ (k mod 8)), then make them visible to the tensor
 //     core (fence.proxy.async) and arrive on the stage's barrier;
 //   * one thread issues tcgen05.mma.cta_group::1.kind::i8 (s8 x s8 -> s32,
-//     M = 128, N = tokens rounded up to 16, K = 32) into two accumulators and
-//     frees the stage with tcgen05.commit;
+//     M = 128, N = tokens rounded up to 16, K = 32; four per step) into two
+//     accumulators and frees the stage with tcgen05.commit;
 //   * the decode warps then read the accumulators (tcgen05.ld, one column per
 //     lane) into the CTA's shared memory; the S CTAs that split the rows of
 //     one column range form a thread-block cluster, and after a cluster
@@ -46,12 +48,15 @@ namespace {
 constexpr int kTcBlocks = 2;                       // 128-column MMA blocks per CTA
 constexpr int kTcCols = 128 * kTcBlocks;           // output columns per CTA
 constexpr int kTcWords = kTcCols / 16;             // packed words per row segment (16)
-constexpr int kTcRows = 32;                        // rows per step (the MMA's K for int8)
-constexpr int kTcStages = 8;                       // two CTAs per SM fit (2 x 97 KB)
-constexpr int kTcATile = kTcRows * 128;            // one 128-column A tile: 4 KB
-constexpr int kTcPacked = kTcRows * kTcWords * 4;  // 2 KB
-constexpr int kTcBMax = 64 * kTcRows;              // codes of up to 64 tokens: 2 KB
-constexpr int kTcStage = kTcBlocks * kTcATile + kTcPacked + kTcBMax;   // 12 KB (multiple of 1 KB)
+constexpr int kTcK = 32;                           // the MMA's K for int8 (rows per MMA)
+constexpr int kTcKc = 2;                           // K chunks (MMAs per accumulator) per step
+constexpr int kTcRows = kTcK * kTcKc;              // rows per step: fewer handshakes per byte
+constexpr int kTcStages = 4;                       // two CTAs per SM fit (2 x 97 KB)
+constexpr int kTcATile = kTcRows * 128;            // one 128-column A tile: 8 KB
+constexpr int kTcPacked = kTcRows * kTcWords * 4;  // 4 KB
+constexpr int kTcBChunk = 64 * kTcK;               // codes of up to 64 tokens for one K chunk: 2 KB
+constexpr int kTcBMax = kTcKc * kTcBChunk;         // 4 KB
+constexpr int kTcStage = kTcBlocks * kTcATile + kTcPacked + kTcBMax;   // 24 KB (multiple of 1 KB)
 constexpr int kTcSmem = kTcStages * kTcStage + 1024;
 constexpr int kTcThreads = 320;                    // warp 0 TMA, warp 1 MMA, warps 2-9 decode + epilogue
 constexpr int kTcDecoders = 256;
@@ -163,7 +168,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort;
   constexpr uint32_t kTmemCols = (kTcBlocks * NPAD) <= 32 ? 32 : ((kTcBlocks * NPAD) <= 64 ? 64 : 128);
-  constexpr int kBBytes = NPAD * kTcRows;
+  constexpr int kBBytes = NPAD * kTcK;             // codes of one K chunk
 
   pdl_begin();
   grid_zero(a.zero, a.zero_n);
@@ -218,10 +223,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         const uint32_t sp = base + (uint32_t)(sl * kTcStage) + kTcBlocks * kTcATile;
         const uint32_t sq = sp + kTcPacked;
-        mbar_arrive_expect_tx(&s_full[sl], (uint32_t)(kTcPacked + kBBytes));
+        mbar_arrive_expect_tx(&s_full[sl], (uint32_t)(kTcPacked + kTcKc * kBBytes));
         const int row = (st0 + it) * kTcRows;
         tc_tma_2d(sp, &map_w, col0 / 16, row, &s_full[sl]);
-        tc_tma_2d(sq, &map_q, row, 0, &s_full[sl]);
+#pragma unroll
+        for (int kc = 0; kc < kTcKc; ++kc)        // one 32-row codes box per K chunk
+          tc_tma_2d(sq + (uint32_t)(kc * kTcBChunk), &map_q, row + kc * kTcK, 0, &s_full[sl]);
       }
       // on an abort, let the copies already issued land
       if (*(volatile int*)&s_abort) {
@@ -246,13 +253,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tc_after();
         const uint32_t sa = base + (uint32_t)(sl * kTcStage);
         const uint32_t sq = sa + kTcBlocks * kTcATile + kTcPacked;
-        // B: K-major codes, 32-byte rows (one token each), 32-byte swizzle, 8-row groups 256 B apart
-        const uint64_t bd = tc_smem_desc(sq, 16, 256, 6);
 #pragma unroll
-        for (int b = 0; b < kTcBlocks; ++b) {
-          // A: MN-major, 128-byte rows (one input row each), 128-byte swizzle, 8-row groups 1 KB apart
-          const uint64_t ad = tc_smem_desc(sa + (uint32_t)(b * kTcATile), 16, 1024, 2);
-          umma_i8(tmem + (uint32_t)(b * NPAD), ad, bd, i8_idesc<NPAD>(), it > 0 ? 1u : 0u);
+        for (int kc = 0; kc < kTcKc; ++kc) {
+          // B: K-major codes, 32-byte rows (one token each), 32-byte swizzle, 8-row groups 256 B apart
+          const uint64_t bd = tc_smem_desc(sq + (uint32_t)(kc * kTcBChunk), 16, 256, 6);
+#pragma unroll
+          for (int b = 0; b < kTcBlocks; ++b) {
+            // A: MN-major, 128-byte rows (one input row each), 128-byte swizzle, 8-row groups
+            // 1 KB apart; K chunk kc starts kTcK rows in
+            const uint64_t ad = tc_smem_desc(sa + (uint32_t)(b * kTcATile + kc * kTcK * 128), 16, 1024, 2);
+            umma_i8(tmem + (uint32_t)(b * NPAD), ad, bd, i8_idesc<NPAD>(), (it > 0 || kc > 0) ? 1u : 0u);
+          }
         }
         tc_commit(&s_empty[sl]);                   // frees the stage once these MMAs have read it
         issued = true;
@@ -270,7 +281,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int dt = threadIdx.x - 64;               // 0..255
     const int grp = dt >> 6;                       // decode group (0..3)
     const int gt = dt & 63;
-    const int r = gt >> 1;                         // row of the step (0..31)
+    const int r0 = gt >> 1;                        // rows r0 and r0 + 32 of the step
     const int blk = gt & 1;                        // A tile (columns 0..127 or 128..255)
     for (int it = grp; it < nsteps; it += kTcGroups) {
       const int sl = it % kTcStages;
@@ -284,13 +295,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       if (ready) {
         unsigned char* st = smem_raw + ((base - smem_u32(smem_raw)) + (uint32_t)(sl * kTcStage));
-        const uint4* pw = reinterpret_cast<const uint4*>(st + kTcBlocks * kTcATile + r * (kTcWords * 4) + blk * 32);
-        const uint4 p0 = pw[0], p1 = pw[1];
-        const uint32_t words[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
-        unsigned char* at = st + blk * kTcATile + r * 128;
 #pragma unroll
-        for (int c = 0; c < 8; ++c)                // 16-byte chunk c holds columns 16c..16c+15
-          *reinterpret_cast<uint4*>(at + ((c ^ (r & 7)) * 16)) = decode_word(words[c]);
+        for (int rr = 0; rr < kTcKc; ++rr) {
+          const int r = r0 + rr * kTcK;
+          const uint4* pw = reinterpret_cast<const uint4*>(st + kTcBlocks * kTcATile + r * (kTcWords * 4) + blk * 32);
+          const uint4 p0 = pw[0], p1 = pw[1];
+          const uint32_t words[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+          unsigned char* at = st + blk * kTcATile + r * 128;
+#pragma unroll
+          for (int c = 0; c < 8; ++c)              // 16-byte chunk c holds columns 16c..16c+15
+            *reinterpret_cast<uint4*>(at + ((c ^ (r & 7)) * 16)) = decode_word(words[c]);
+        }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       }
       __syncwarp();
@@ -447,7 +462,7 @@ GemvPlan plan_qgemv_tc(int T, int d_in, int d_out) {
   p.rcap = 0;
   p.smem = kTcSmem;
   // splits: about two CTAs per SM, at most 8 (each split adds T x d_out exact
-  // partial sums), at least 4 steps of 32 rows each
+  // partial sums), at least 4 steps of 64 rows each
   const int steps = (d_in + kTcRows - 1) / kTcRows;
   long S = (2L * kNumSMs) / p.n_ct;
   if (S > 8) S = 8;
@@ -465,14 +480,14 @@ cudaError_t launch_qgemv_tc(const QGemvArgs& a, cudaStream_t s) {
   if (a.xq == nullptr || a.plan.mma != 2) return cudaErrorInvalidValue;
   CUtensorMap mw, mq;
   const int row_words = a.d_out / 16;
-  // packed W^T [d_in rows][row_words] u32: box 16 words (64 B) x 32 rows, no swizzle
+  // packed W^T [d_in rows][row_words] u32: box 16 words (64 B) x 64 rows, no swizzle
   if (!make_map_2d(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT32, a.wp, (uint64_t)row_words, (uint64_t)a.d_in,
                    (uint64_t)row_words * 4, kTcWords, kTcRows, CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
   const int npad = a.plan.TT;
-  // dense masked codes [T][d_in] int8: box 32 (rows) x npad tokens, 32-byte swizzle
+  // dense masked codes [T][d_in] int8: box 32 (rows, one K chunk) x npad tokens, 32-byte swizzle
   if (!make_map_2d(&mq, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.xq, (uint64_t)a.d_in, (uint64_t)a.T,
-                   (uint64_t)a.d_in, kTcRows, (uint32_t)npad, CU_TENSOR_MAP_SWIZZLE_32B))
+                   (uint64_t)a.d_in, kTcK, (uint32_t)npad, CU_TENSOR_MAP_SWIZZLE_32B))
     return cudaErrorInvalidValue;
   switch (npad) {
     case 16: return tc_launch<16>(a, mw, mq, s);
