@@ -343,9 +343,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 // first CTA of the pair issues tcgen05.mma.cta_group::2 (M = 256: the
 // accumulator rows are split over the two CTAs' tensor memory, the B operand
 // is read from both CTAs' shared memory), and each CTA's epilogue stores its
-// own 128 rows.  Loads are plain (no multicast): each CTA's copies signal the
-// first CTA's stage barrier (its address through mapa); the MMA commits
-// multicast their arrivals to both CTAs' barriers.
+// own 128 rows.  Each copy writes only its own CTA's shared memory and
+// signals the first CTA's stage barrier (its address through mapa); each MMA
+// commit arrives on the barriers of both CTAs (a tcgen05.commit with a CTA mask).
 constexpr int k2Stages = 6;
 constexpr int k2ABytes = 128 * BK * 2;               // 16 KB: this CTA's 128 rows
 constexpr int k2BBytes = 2 * kBBox;                  // 16 KB: this CTA's 128 columns (two boxes)
