@@ -170,9 +170,10 @@ qs_status qs_sparse_linear(const void* x, int dtype, int T, int d_in, int d_out,
  *   ws        qs_workspace_size(QS_OP_SPARSE_FFN, T, d_model, d_ff, k_h) bytes.
  *   d_model and d_ff must be multiples of 8 (bf16) or 4 (f32).
  *   One token, bf16, idx_h_out NULL, d_model <= 8192: the whole layer runs as
- *   ONE persistent kernel (a cooperative launch whose phases are separated by
- *   grid barriers) instead of four; same results up to float32 summation
- *   order, same lists and statistics.  qs_set_ffn_fused(0) turns this off.
+ *   ONE persistent kernel (every CTA resident, phases separated by grid
+ *   barriers) instead of four; same results up to float32 summation order,
+ *   same lists and statistics.  qs_set_ffn_fused selects how it is launched
+ *   or turns it off.
  *   Errors: INVALID_ARG, ALIGNMENT, WORKSPACE, UNSUPPORTED, CUDA.
  */
 qs_status qs_sparse_ffn(const void* x, int dtype, int T, int d_model, int d_ff, int act,
@@ -187,10 +188,19 @@ qs_status qs_sparse_ffn(const void* x, int dtype, int T, int d_model, int d_ff, 
  * a device).  Host-only: nothing is enqueued. */
 int qs_sparse_ffn_fused(int dtype, int T, int d_model, int d_ff, int with_idx_h);
 
-/* Process-wide switch for the one-kernel path of qs_sparse_ffn (on by
- * default): 0 makes every call use the separate kernels (for comparison and
- * testing).  Always returns QS_OK. */
-qs_status qs_set_ffn_fused(int enable);
+/* Process-wide switch for the one-kernel path of qs_sparse_ffn:
+ *   1 (default) an ordinary launch with programmatic dependent launch: the
+ *     next launch's set-up overlaps this one's exit.  Its grid barriers need
+ *     every CTA resident, which holds on a device that runs these layers alone
+ *     on their stream; another kernel running concurrently on the device can
+ *     hold SMs that its CTAs wait for, and a barrier wait that runs out ends in
+ *     QS_ERR_TIMEOUT (qs_device_status), never a hang;
+ *   2 a cooperative launch, which the driver admits only when the whole grid
+ *     can be resident (for callers that overlap other kernels; ~1.7 us more a
+ *     launch, launches do not overlap);
+ *   0 every call uses the separate kernels (for comparison and testing).
+ * Returns QS_ERR_INVALID_ARG for any other value, else QS_OK. */
+qs_status qs_set_ffn_fused(int mode);
 
 /*
  * qs_sparse_ffn_gate_first -- the dReLU layer of qs_sparse_ffn (QS_ACT_DRELU,

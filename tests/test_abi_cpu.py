@@ -169,3 +169,10 @@ def test_workspace_list_and_fault_hook_check_arguments_on_the_host(L):
         qs.QS_ERR_INVALID_ARG                                          # k > d_in
     assert L.qs_debug_inject(9, 0) == qs.QS_ERR_INVALID_ARG
     assert L.qs_debug_inject(qs.QS_FAULT_NONE, 0) == qs.QS_OK
+
+
+def test_ffn_fused_switch_takes_three_modes(L):
+    for bad in (-1, 3):
+        assert L.qs_set_ffn_fused(bad) == qs.QS_ERR_INVALID_ARG
+    for mode in (0, 2, 1):                             # ends on the default
+        assert L.qs_set_ffn_fused(mode) == qs.QS_OK

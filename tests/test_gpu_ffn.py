@@ -151,7 +151,7 @@ def test_ffn_one_token_list_path_llama7b():
     _check_ffn(x8, up, gate, down, "relu2_glu", w.k, w.k_h, "bf16")
 
 
-@pytest.mark.parametrize("fused", [True, False])
+@pytest.mark.parametrize("fused", [1, 2, 0])       # ordinary launch, cooperative launch, off
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("dm,dff", [(64, 96), (200, 328), (128, 1000), (96, 16384)])
 def test_ffn_one_token_list_path_small(dtype, dm, dff, fused):
@@ -183,12 +183,14 @@ def _list_path_small(dtype, dm, dff):
 
 
 def test_ffn_one_token_fused_llama7b():
-    """The one-kernel path of a one-token bf16 layer (cooperative launch, grid
+    """The one-kernel path of a one-token bf16 layer (every CTA resident, grid
     barriers) against the oracle and against the separate kernels: the input
     list is the same bit for bit, y matches the oracle re-run on the GPU's own
     kept h; then K_h below the nonzero count (every CTA selects the K_h-th
     largest |h| itself); then tokens back to back on one workspace (the
-    barrier counters must be reset by each call)."""
+    barrier counters must be reset by each call), launched both ways (an
+    ordinary and a cooperative launch; the down projection's partial sums are
+    float atomic additions, so y is checked against the oracle each time)."""
     need_gpu()
     w = workloads.WORKLOADS["ffn_relu2_llama7b"]
     assert qs.qs_sparse_ffn_fused(qs.QS_BF16, 1, w.d_in, w.d_out, False)
@@ -222,6 +224,14 @@ def test_ffn_one_token_fused_llama7b():
     ys = [qs.qs_sparse_ffn(xs[t], upt, gatet, downt, "relu2_glu", w.k, w.k_h, ws=ws).y
           for t in range(4)]
     check_status(ws)
+    qs.qs_set_ffn_fused(2)
+    try:
+        ys_coop = [qs.qs_sparse_ffn(xs[t], upt, gatet, downt, "relu2_glu", w.k, w.k_h, ws=ws).y
+                   for t in range(4)]
+        check_status(ws)
+    finally:
+        qs.qs_set_ffn_fused(True)
     for t in range(4):
         ref = oracle.sparse_ffn(x4[t:t + 1], up, gate, down, "relu2_glu", w.k, w.k_h)
         assert oracle.max_rel_err(to_np(ys[t]), ref["y"]) <= 2 * TOL_BF16
+        assert oracle.max_rel_err(to_np(ys_coop[t]), ref["y"]) <= 2 * TOL_BF16

@@ -258,9 +258,10 @@ def qs_sparse_ffn_fused(dtype: int, T: int, d_model: int, d_ff: int, with_idx_h:
                                           1 if with_idx_h else 0))
 
 
-def qs_set_ffn_fused(enable: bool) -> None:
-    """Turn the one-kernel path of one-token bf16 FFN calls on or off (process-wide)."""
-    _check("qs_set_ffn_fused", lib().qs_set_ffn_fused(1 if enable else 0))
+def qs_set_ffn_fused(mode) -> None:
+    """The one-kernel path of one-token bf16 FFN calls (process-wide): False/0 off,
+    True/1 on with an ordinary launch (the default), 2 on with a cooperative launch."""
+    _check("qs_set_ffn_fused", lib().qs_set_ffn_fused(int(mode)))
 
 
 def qs_debug_inject(mode: int, wait_polls: int = 0) -> None:

@@ -20,7 +20,7 @@ constexpr size_t kTicketBytes = 64 * 1024;       // fixed ticket region
 constexpr int kTicketCap = (int)(kTicketBytes / sizeof(int32_t));
 // fixed ticket slots
 constexpr int kTkTopkX = 0, kTkTopkH = 1, kTkAlpha = 2, kTkUpRows = 3, kTkHCount = 4,
-              kTkDownDone = 5, kTkGemv = 8;
+              kTkGemv = 8;                        // (slots 5-7 unused)
 // union bitmasks of the several-token path, and the open gates of the
 // gate-first FFN (zero between calls)
 constexpr int kTkGemvEnd = 4096;
@@ -357,8 +357,9 @@ bool use_ffn_fused(int op, int dtype, int T, int d_model, int d_ff, const int32_
 }
 }  // namespace
 
-qs_status qs_set_ffn_fused(int enable) {
-  g_ffn_fused.store(enable ? 1 : 0);
+qs_status qs_set_ffn_fused(int mode) {
+  if (mode < 0 || mode > 2) return QS_ERR_INVALID_ARG;
+  g_ffn_fused.store(mode);
   return QS_OK;
 }
 
@@ -541,7 +542,7 @@ static qs_status ffn_impl(int op, const void* x, int dtype, int T, int d_model, 
     f.status = w.status();
     f.plan = fp;
     QS_TRY_CUDA(mark(0));
-    QS_TRY_CUDA(launch_ffn_fused(f, s));
+    QS_TRY_CUDA(launch_ffn_fused(f, g_ffn_fused.load() == 2, s));
     for (int i = 1; i < QS_FFN_PHASE_EVENTS; ++i) QS_TRY_CUDA(mark(i));
     return QS_OK;
   }

@@ -1,4 +1,4 @@
-// One-token sparse FFN layer as ONE persistent kernel (cooperative launch).
+// One-token sparse FFN layer as ONE persistent kernel (every CTA resident).
 //
 // Q-Sparse news article (zxwl-tech.com), "Top-K sparsification": the K
 // largest |x| of the token are kept, the rest set to zero; the projections
@@ -35,7 +35,6 @@
 //      barrier counters.
 // The row lists and their counts are written as by the general path (so the
 // workspace statistics and list read-back stay valid).
-#include <atomic>
 #include <mutex>
 
 #include "qs_internal.cuh"
@@ -114,69 +113,105 @@ __device__ __forceinline__ int block_sum(int v, int* s_w) {
   return s;
 }
 
-// The k-th largest of n magnitude keys (1 <= k <= n): returns tau (that key)
-// and need (how many of the keys equal to tau are among the k largest).
-// Radix select from the top digit (8 bits a pass).  Each warp counts into its
-// own 256-bin histogram (whist: kFWarps x 256 ints of idle shared memory), so
-// the atomics of different warps never meet on the few bins that hold most
-// keys; the histograms are then summed bin by bin.
+// The k-th largest of n magnitude keys (1 <= k <= n, keys < 2^nbits, nbits >=
+// 11): returns tau (that key) and need (how many of the keys equal to tau are
+// among the k largest).  Radix select from the top: the first pass counts the
+// top 11 bits into one 2048-bin histogram (h2k: idle shared memory), which
+// spreads the keys of a warp over many bins (a narrow first digit would be the
+// exponent alone, a few bins for most data, and serialise the atomics); the
+// later passes take up to 8 bits each into s_hist.
 template <typename KeyFn>
-__device__ void block_kth_largest(KeyFn key, int n, int k, int nbits, int* whist, int* s_hist,
-                                  int* s_pick, uint32_t& tau, int& need) {
+__device__ void block_kth_largest(KeyFn key, int n, int k, int nbits, int* h2k, int* s_hist,
+                                  int* s_pick, int* s_w, uint32_t& tau, int& need) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int nd = (nbits + 7) / 8;
-  uint32_t prefix = 0, pmask = 0;
-  int rem = k;
-  int* wh = whist + warp * 256;
-  for (int p = 0; p < nd; ++p) {
-    const int shift = 8 * (nd - 1 - p);
-    for (int j = tid; j < kFWarps * 256; j += kFThreads) whist[j] = 0;
-    __syncthreads();
-    for (int e = tid; e < n; e += kFThreads) {     // (warp aggregation by match_any measured slower)
-      const uint32_t kk = key(e);
-      if ((kk & pmask) == prefix) atomicAdd(&wh[(kk >> shift) & 255u], 1);
-    }
-    __syncthreads();
-    for (int j = tid; j < 256; j += kFThreads) {
-      int v = 0;
+  const int sh1 = nbits - 11;
+  for (int j = tid; j < 2048; j += kFThreads) h2k[j] = 0;
+  for (int j = tid; j < 256; j += kFThreads) s_hist[j] = 0;
+  __syncthreads();
+  for (int e = tid; e < n; e += kFThreads) atomicAdd(&h2k[key(e) >> sh1], 1);
+  __syncthreads();
+  // threads 0..255 hold 8 bins each, in descending order from the top bin
+  int c[8], sum = 0;
+  if (tid < 256) {
 #pragma unroll
-      for (int w = 0; w < kFWarps; ++w) v += whist[w * 256 + j];
-      s_hist[j] = v;
+    for (int q = 0; q < 8; ++q) {
+      c[q] = h2k[2047 - 8 * tid - q];
+      sum += c[q];
+    }
+  }
+  int incl = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31 && warp < 8) s_w[warp] = incl;
+  __syncthreads();
+  if (tid < 256) {
+    for (int w = 0; w < warp; ++w) incl += s_w[w];
+    const int excl = incl - sum;
+    if (excl < k && k <= incl) {
+      int run = excl;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (run + c[q] >= k) {
+          s_pick[0] = 2047 - 8 * tid - q;
+          s_pick[1] = run;
+          break;
+        }
+        run += c[q];
+      }
+    }
+  }
+  __syncthreads();
+  uint32_t prefix = (uint32_t)s_pick[0] << sh1, pmask = 0x7ffu << sh1;
+  int rem = k - s_pick[1];
+  int sh = sh1;
+  while (sh > 0) {                                 // (block-uniform)
+    const int w = sh < 8 ? sh : 8;
+    sh -= w;
+    const uint32_t dmask = (1u << w) - 1u;
+    for (int e = tid; e < n; e += kFThreads) {
+      const uint32_t kk = key(e);
+      if ((kk & pmask) == prefix) atomicAdd(&s_hist[(kk >> sh) & dmask], 1);
     }
     __syncthreads();
     if (warp == 0) {
       // lane l holds digits 255 - 8l .. 248 - 8l (descending)
-      int c[8], sum = 0;
+      int d[8], dsum = 0;
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
-        c[q] = s_hist[255 - 8 * lane - q];
-        sum += c[q];
+        d[q] = s_hist[255 - 8 * lane - q];
+        dsum += d[q];
       }
-      int incl = sum;
+      int dincl = dsum;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
-        const int v = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += v;
+        const int v = __shfl_up_sync(0xffffffffu, dincl, o);
+        if (lane >= o) dincl += v;
       }
-      const int excl = incl - sum;
-      if (excl < rem && rem <= incl) {
-        int run = excl;
+      const int dexcl = dincl - dsum;
+      if (dexcl < rem && rem <= dincl) {
+        int run = dexcl;
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
-          if (run + c[q] >= rem) {
+          if (run + d[q] >= rem) {
             s_pick[0] = 255 - 8 * lane - q;
             s_pick[1] = run;
             break;
           }
-          run += c[q];
+          run += d[q];
         }
       }
     }
     __syncthreads();
-    prefix |= (uint32_t)s_pick[0] << shift;
-    pmask |= 255u << shift;
+    prefix |= (uint32_t)s_pick[0] << sh;
+    pmask |= dmask << sh;
     rem -= s_pick[1];
-    __syncthreads();
+    if (sh > 0) {                                  // the next pass counts into a cleared s_hist
+      for (int j = tid; j < 256; j += kFThreads) s_hist[j] = 0;
+      __syncthreads();
+    }
   }
   tau = prefix;
   need = rem;
@@ -230,7 +265,7 @@ __device__ Selection select_topk(KeyFn key, int n, int k, int nbits, int r0, int
   if (k >= n) {
     S.tau = 0u; S.need = n;                        // every key is > 0 or a kept tie at 0
   } else {
-    block_kth_largest(key, n, k, nbits, whist, s_hist, s_pick, S.tau, S.need);
+    block_kth_largest(key, n, k, nbits, whist, s_hist, s_pick, s_w, S.tau, S.need);
   }
   int cnt = 0;                                     // (> tau) + (== tau) << 16, each < 65536
   for (int e = (int)threadIdx.x; e < r0; e += kFThreads) {
@@ -638,7 +673,20 @@ size_t ffn_fused_pug_elems(int d_model, int d_ff) {
 
 int ffn_fused_grid() { return fused_grid(); }
 
-cudaError_t launch_ffn_fused(const FfnFusedArgs& a_in, cudaStream_t s) {
+// The grid is the occupancy-sized count of CTAs (ffn_fused_grid), all of which
+// must be resident together for the grid barriers.  An ordinary launch with
+// programmatic dependent launch is the default: a grid that follows another
+// one-kernel layer on the stream is scheduled only after every CTA of that
+// layer has started (each one triggers at entry) and takes their places as
+// they leave, so on a device that runs these layers alone every CTA becomes
+// resident, and the next layer's set-up overlaps this one's exit (about 1.7 us
+// a launch less than a cooperative launch, with which the driver does not
+// overlap launches).  `cooperative` asks for a cooperative launch instead,
+// which the driver admits only when the whole grid can be resident: for
+// callers that run other kernels concurrently on the device, where CTAs of an
+// ordinary launch could wait for SMs that another kernel holds (every grid
+// barrier wait is bounded and would end in DEV_TIMEOUT, never a hang).
+cudaError_t launch_ffn_fused(const FfnFusedArgs& a_in, bool cooperative, cudaStream_t s) {
   FfnFusedArgs a = a_in;
   a.wait_limit = kWaitLimit;
   if (g_fault.mode == QS_FAULT_GATHER_NO_COPIES) {   // failure-detection tests only
@@ -650,23 +698,17 @@ cudaError_t launch_ffn_fused(const FfnFusedArgs& a_in, cudaStream_t s) {
   cfg.blockDim = dim3(kFThreads);
   cfg.dynamicSmemBytes = ffn_fused_smem();
   cfg.stream = s;
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeCooperative;     // every CTA resident: the grid barriers
-  attr[0].val.cooperative = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  // with programmatic dependent launch where the driver takes it together with
-  // a cooperative launch, else without (the kernel's waits are no-ops then)
-  static std::atomic<int> pdl_ok{1};
-  cfg.numAttrs = pdl_ok.load() ? 2 : 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, ffn_fused_kernel, a);
-  if (e != cudaSuccess && cfg.numAttrs == 2) {
-    (void)cudaGetLastError();                      // clear the launch error, retry without
-    pdl_ok.store(0);
-    cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, ffn_fused_kernel, a);
+  cudaLaunchAttribute attr[1];
+  if (cooperative) {
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+  } else {
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
   }
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, ffn_fused_kernel, a);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

@@ -404,7 +404,7 @@ size_t ffn_fused_smem();
 bool plan_ffn_fused(int d_model, int d_ff, int G, FfnFusedPlan* p);
 size_t ffn_fused_pug_elems(int d_model, int d_ff);   // 0: the sizes are not supported
 int ffn_fused_grid();                                  // resident CTAs (0: unavailable)
-cudaError_t launch_ffn_fused(const FfnFusedArgs& a, cudaStream_t s);
+cudaError_t launch_ffn_fused(const FfnFusedArgs& a, bool cooperative, cudaStream_t s);
 
 
 // The quantized FFN's gating of one column, float32 steps in a fixed order
