@@ -414,8 +414,8 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
-template <int TT, int MODE>
-__global__ void __launch_bounds__(kMmaWarps * 32 + 32, 2) gemv_mma_kernel(GemvArgs a) {
+template <int TT, int MODE, int MINB>
+__global__ void __launch_bounds__(kMmaWarps * 32 + 32, MINB) gemv_mma_kernel(GemvArgs a) {
   constexpr int V = 8;
   constexpr int NC = kMmaWarps * 32;
   extern __shared__ __align__(128) unsigned char smem[];
@@ -639,15 +639,20 @@ __global__ void __launch_bounds__(kMmaWarps * 32 + 32, 2) gemv_mma_kernel(GemvAr
   }
 }
 
-template <int TT, int MODE>
+template <int TT, int MODE, int MINB>
 cudaError_t launch_mma(const GemvArgs& a, cudaStream_t s) {
   static unsigned configured = 0;
-  cudaError_t e = ensure_smem_attr(gemv_mma_kernel<TT, MODE>, 200 * 1024, &configured);
+  cudaError_t e = ensure_smem_attr(gemv_mma_kernel<TT, MODE, MINB>, 200 * 1024, &configured);
   if (e != cudaSuccess) return e;
   dim3 grid(a.plan.n_ct, a.plan.mats * a.plan.S, a.plan.groups);
-  e = launch_pdl(gemv_mma_kernel<TT, MODE>, grid, dim3(kMmaWarps * 32 + 32), a.plan.smem, s, a);
+  e = launch_pdl(gemv_mma_kernel<TT, MODE, MINB>, grid, dim3(kMmaWarps * 32 + 32), a.plan.smem, s, a);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
+}
+
+template <int TT, int MODE>
+cudaError_t launch_mma(const GemvArgs& a, cudaStream_t s) {
+  return a.plan.cta_sm == 1 ? launch_mma<TT, MODE, 1>(a, s) : launch_mma<TT, MODE, 2>(a, s);
 }
 
 template <int TT>
@@ -717,13 +722,20 @@ GemvPlan plan_gemv_mma(int T, int d_out, int rows_bound, int mats) {
   p.threads = kMmaWarps * 32 + 32;
   p.rps = kMmaRows;
   const long stage = (long)kMmaRows * (p.vec_tile * 16 + 16);
-  long nst = (90L * 1024) / stage;
+  // Stages of 40 KB or more (tiles of ~2.5 KB) fit only two to a CTA at two
+  // CTAs per SM, and a consumed stage leaves one in flight; one CTA per SM
+  // with four stages keeps three in flight (8 tokens of 4096 -> 2 x 11008:
+  // 51 -> 45 us).  Smaller stages stay at two CTAs per SM, which measured
+  // faster for them (4 tokens of 4096 -> 2 x 14336 with 2 KB tiles: 52 us
+  // against 62 us at one CTA per SM).
+  p.cta_sm = stage >= 40L * 1024 ? 1 : 2;
+  long nst = (p.cta_sm == 1 ? 180L * 1024 : 90L * 1024) / stage;
   if (nst < 2) nst = 2;
   if (nst > 4) nst = 4;
   p.nst = (int)nst;
   p.rcap = 512;
   p.smem = (size_t)p.nst * stage + (size_t)p.rcap * 4 * (1 + p.TT);
-  const long slots = (long)kNumSMs * 2;
+  const long slots = (long)kNumSMs * p.cta_sm;
   const long units = (long)p.n_ct * mats * p.groups;
   long S = slots / (units > 0 ? units : 1);
   if (S < 1) S = 1;

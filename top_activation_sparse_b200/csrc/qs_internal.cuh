@@ -188,6 +188,7 @@ struct GemvPlan {
   int nst;         // pipeline stages
   int copies;      // accumulator copies: split s adds into copy s % copies (fewer adds per address)
   int mma;         // bf16, 4-8 tokens: the tensor-core (mma.sync) kernel
+  int cta_sm;      // tensor-core kernel: CTAs per SM the plan is sized for (1 or 2)
   int rcap;        // rows staged in shared memory per piece
   size_t smem;     // dynamic shared memory bytes
 };
