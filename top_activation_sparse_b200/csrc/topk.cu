@@ -1116,122 +1116,144 @@ __global__ void __launch_bounds__(NT) topk_reg_kernel(TopkArgs a) {
   reg_select<KIND, NT, EPT>(ent, d, k, nnz, s_hist, s_sel, a.status, row, P, shift, remaining);
 
   // ---- 3. compaction in index order ------------------------------------------
-#pragma unroll
-  for (int j = 0; j < EPT; ++j) {
-    const bool valid = j * NT + tid < d;
-    const uint32_t key = ent[j] & MASK;
-    const uint32_t c = key >> shift;
-    const bool eq = valid && c == P;
-    const uint32_t bg = __ballot_sync(kFull, valid && c > P);
-    const uint32_t be = __ballot_sync(kFull, eq);
-    const uint32_t bz = __ballot_sync(kFull, eq && key != 0u);
-    if (lane == j) {
-      s_cnt[j * NW + warp] = (uint32_t)__popc(bg) | ((uint32_t)__popc(be) << 16);
-      s_cnz[j * NW + warp] = (uint32_t)__popc(bz);
-    }
-  }
-  __syncthreads();
-  if (warp == 0) {
-    // exclusive prefixes over the (slot, warp) table, warps fastest: index order
-    constexpr int CH = (E + 31) / 32;
-    const int b0 = min(lane * CH, E), b1 = min(b0 + CH, E);
-    uint32_t sg = 0, sz = 0;
-    for (int i = b0; i < b1; ++i) { sg += s_cnt[i]; sz += s_cnz[i]; }
-    uint32_t ig = sg, iz = sz;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t vg = __shfl_up_sync(kFull, ig, o);
-      const uint32_t vz = __shfl_up_sync(kFull, iz, o);
-      if (lane >= o) { ig += vg; iz += vz; }
-    }
-    uint32_t eg = ig - sg, ez = iz - sz;
-    for (int i = b0; i < b1; ++i) {
-      const uint32_t cg = s_cnt[i], cz = s_cnz[i];
-      s_cnt[i] = eg; s_cnz[i] = ez;
-      eg += cg; ez += cz;
-    }
-    if (lane == 31) { s_tot[0] = ig; s_tot[1] = iz; }
-  }
-  __syncthreads();
-  const int tot_gt = (int)(s_tot[0] & 0xffffu), tot_eq = (int)(s_tot[0] >> 16);
-  const int tot_eqnz = (int)s_tot[1];
   const bool list_direct = (a.list != nullptr) && (a.T == 1);
-  if (list_direct && tid == 0) *a.list_count = tot_gt + (P != 0u ? min(tot_eq, remaining) : tot_eqnz);
   const bool want_union = (a.list != nullptr) && (a.T > 1);
+  // With at most K nonzero entries every nonzero entry is kept; when the only
+  // outputs are the dense values and the union of the kept nonzeros (the
+  // several-token projection path: h has at most K_h nonzeros per token for
+  // the squared-ReLU GLU), nothing needs a position, and the ranked
+  // compaction below (ballots, prefix scans and position arithmetic for every
+  // entry, on one SM per row) is skipped.  (block-uniform)
+  const bool all_nz_kept = !BLOCK && !QUANT && nnz <= k && !list_direct && a.idx == nullptr &&
+                           a.val == nullptr && a.mask == nullptr && a.xs == nullptr;
+  if (all_nz_kept) {
 #pragma unroll
-  for (int j = 0; j < EPT; ++j) {
-    const int e = j * NT + tid;
-    const bool valid = e < d;
-    const uint32_t key = ent[j] & MASK;
-    const uint32_t c = key >> shift;
-    const bool gt = valid && c > P;
-    const bool eq = valid && c == P;
-    const uint32_t bg = __ballot_sync(kFull, gt);
-    const uint32_t be = __ballot_sync(kFull, eq);
-    const uint32_t bz = __ballot_sync(kFull, eq && key != 0u);
-    const uint32_t pre = s_cnt[j * NW + warp];
-    const int gt_b = (int)(pre & 0xffffu) + __popc(bg & lt);
-    const int eq_b = (int)(pre >> 16) + __popc(be & lt);
-    const int eqnz_b = (int)s_cnz[j * NW + warp] + __popc(bz & lt);
-    const bool sel = gt || (eq && eq_b < remaining);
-    if constexpr (BLOCK) {
-      // Block Q-Sparse: this row's idx / val here, its other outputs after
-      // the loop from the selection bitmask
-      const uint32_t bs = __ballot_sync(kFull, sel);
-      if (lane == 0 && j * NT + warp * 32 < d) s_bsel[(j * NT + warp * 32) >> 5] = bs;
-      if (sel) {
+    for (int j = 0; j < EPT; ++j) {
+      const int e = j * NT + tid;
+      const bool valid = e < d;
+      if (valid && a.xsf) a.xsf[rbase + e] = raw_to_f32<KIND>(ent[j]);
+      if (want_union) {
+        const uint32_t b = __ballot_sync(kFull, valid && (ent[j] & MASK) != 0u);
+        if (lane == 0 && b != 0u) atomicOr(a.union_bits + (j * NT + warp * 32) / 32, b);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < EPT; ++j) {
+      const bool valid = j * NT + tid < d;
+      const uint32_t key = ent[j] & MASK;
+      const uint32_t c = key >> shift;
+      const bool eq = valid && c == P;
+      const uint32_t bg = __ballot_sync(kFull, valid && c > P);
+      const uint32_t be = __ballot_sync(kFull, eq);
+      const uint32_t bz = __ballot_sync(kFull, eq && key != 0u);
+      if (lane == j) {
+        s_cnt[j * NW + warp] = (uint32_t)__popc(bg) | ((uint32_t)__popc(be) << 16);
+        s_cnz[j * NW + warp] = (uint32_t)__popc(bz);
+      }
+    }
+    __syncthreads();
+    if (warp == 0) {
+      // exclusive prefixes over the (slot, warp) table, warps fastest: index order
+      constexpr int CH = (E + 31) / 32;
+      const int b0 = min(lane * CH, E), b1 = min(b0 + CH, E);
+      uint32_t sg = 0, sz = 0;
+      for (int i = b0; i < b1; ++i) { sg += s_cnt[i]; sz += s_cnz[i]; }
+      uint32_t ig = sg, iz = sz;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t vg = __shfl_up_sync(kFull, ig, o);
+        const uint32_t vz = __shfl_up_sync(kFull, iz, o);
+        if (lane >= o) { ig += vg; iz += vz; }
+      }
+      uint32_t eg = ig - sg, ez = iz - sz;
+      for (int i = b0; i < b1; ++i) {
+        const uint32_t cg = s_cnt[i], cz = s_cnz[i];
+        s_cnt[i] = eg; s_cnz[i] = ez;
+        eg += cg; ez += cz;
+      }
+      if (lane == 31) { s_tot[0] = ig; s_tot[1] = iz; }
+    }
+    __syncthreads();
+    const int tot_gt = (int)(s_tot[0] & 0xffffu), tot_eq = (int)(s_tot[0] >> 16);
+    const int tot_eqnz = (int)s_tot[1];
+    if (list_direct && tid == 0) *a.list_count = tot_gt + (P != 0u ? min(tot_eq, remaining) : tot_eqnz);
+#pragma unroll
+    for (int j = 0; j < EPT; ++j) {
+      const int e = j * NT + tid;
+      const bool valid = e < d;
+      const uint32_t key = ent[j] & MASK;
+      const uint32_t c = key >> shift;
+      const bool gt = valid && c > P;
+      const bool eq = valid && c == P;
+      const uint32_t bg = __ballot_sync(kFull, gt);
+      const uint32_t be = __ballot_sync(kFull, eq);
+      const uint32_t bz = __ballot_sync(kFull, eq && key != 0u);
+      const uint32_t pre = s_cnt[j * NW + warp];
+      const int gt_b = (int)(pre & 0xffffu) + __popc(bg & lt);
+      const int eq_b = (int)(pre >> 16) + __popc(be & lt);
+      const int eqnz_b = (int)s_cnz[j * NW + warp] + __popc(bz & lt);
+      const bool sel = gt || (eq && eq_b < remaining);
+      if constexpr (BLOCK) {
+        // Block Q-Sparse: this row's idx / val here, its other outputs after
+        // the loop from the selection bitmask
+        const uint32_t bs = __ballot_sync(kFull, sel);
+        if (lane == 0 && j * NT + warp * 32 < d) s_bsel[(j * NT + warp * 32) >> 5] = bs;
+        if (sel) {
+          const int pos = gt_b + min(eq_b, remaining);
+          if (pos < k) {
+            const size_t o = (size_t)row * k + pos;
+            if (a.idx) a.idx[o] = e;
+            if (a.val) {
+              const uint32_t raw = load_raw<KIND>(a.x, (size_t)row * d + e);
+              if constexpr (KIND == TK_F32) reinterpret_cast<uint32_t*>(a.val)[o] = raw;
+              else if constexpr (KIND == TK_BF16) reinterpret_cast<uint16_t*>(a.val)[o] = (uint16_t)raw;
+            }
+          } else {
+            dev_fail(a.status, DEV_CHECK, 2, (uint32_t)row);
+          }
+        }
+      } else if (sel) {
         const int pos = gt_b + min(eq_b, remaining);
         if (pos < k) {
-          const size_t o = (size_t)row * k + pos;
+          const size_t o = (size_t)row * (size_t)k + (size_t)pos;
           if (a.idx) a.idx[o] = e;
           if (a.val) {
-            const uint32_t raw = load_raw<KIND>(a.x, (size_t)row * d + e);
-            if constexpr (KIND == TK_F32) reinterpret_cast<uint32_t*>(a.val)[o] = raw;
-            else if constexpr (KIND == TK_BF16) reinterpret_cast<uint16_t*>(a.val)[o] = (uint16_t)raw;
+            if constexpr (KIND == TK_F32) reinterpret_cast<uint32_t*>(a.val)[o] = ent[j];
+            else if constexpr (KIND == TK_BF16) reinterpret_cast<uint16_t*>(a.val)[o] = (uint16_t)ent[j];
           }
         } else {
           dev_fail(a.status, DEV_CHECK, 2, (uint32_t)row);
         }
-      }
-    } else if (sel) {
-      const int pos = gt_b + min(eq_b, remaining);
-      if (pos < k) {
-        const size_t o = (size_t)row * (size_t)k + (size_t)pos;
-        if (a.idx) a.idx[o] = e;
-        if (a.val) {
-          if constexpr (KIND == TK_F32) reinterpret_cast<uint32_t*>(a.val)[o] = ent[j];
-          else if constexpr (KIND == TK_BF16) reinterpret_cast<uint16_t*>(a.val)[o] = (uint16_t)ent[j];
+        if (list_direct && key != 0u) {
+          const int nzp = gt_b + (P != 0u ? min(eq_b, remaining) : eqnz_b);
+          a.list[nzp] = e;
+          if constexpr (QUANT) {
+            if (a.list_q) a.list_q[nzp] = (int8_t)(ent[j] >> 8);
+          } else {
+            if (a.list_val) a.list_val[nzp] = raw_to_f32<KIND>(ent[j]);
+          }
         }
-      } else {
-        dev_fail(a.status, DEV_CHECK, 2, (uint32_t)row);
       }
-      if (list_direct && key != 0u) {
-        const int nzp = gt_b + (P != 0u ? min(eq_b, remaining) : eqnz_b);
-        a.list[nzp] = e;
+      if (valid && !BLOCK) {
+        const uint32_t v = sel ? ent[j] : 0u;
+        if (a.mask) a.mask[rbase + e] = sel ? 1 : 0;
         if constexpr (QUANT) {
-          if (a.list_q) a.list_q[nzp] = (int8_t)(ent[j] >> 8);
+          if (a.xq) a.xq[rbase + e] = (int8_t)(v >> 8);
         } else {
-          if (a.list_val) a.list_val[nzp] = raw_to_f32<KIND>(ent[j]);
+          if (a.xsf) a.xsf[rbase + e] = raw_to_f32<KIND>(v);
+          if (a.xs) {
+            if constexpr (KIND == TK_F32) reinterpret_cast<uint32_t*>(a.xs)[rbase + e] = v;
+            else reinterpret_cast<uint16_t*>(a.xs)[rbase + e] = (uint16_t)v;
+          }
         }
       }
-    }
-    if (valid && !BLOCK) {
-      const uint32_t v = sel ? ent[j] : 0u;
-      if (a.mask) a.mask[rbase + e] = sel ? 1 : 0;
-      if constexpr (QUANT) {
-        if (a.xq) a.xq[rbase + e] = (int8_t)(v >> 8);
-      } else {
-        if (a.xsf) a.xsf[rbase + e] = raw_to_f32<KIND>(v);
-        if (a.xs) {
-          if constexpr (KIND == TK_F32) reinterpret_cast<uint32_t*>(a.xs)[rbase + e] = v;
-          else reinterpret_cast<uint16_t*>(a.xs)[rbase + e] = (uint16_t)v;
-        }
+      if (want_union) {
+        const uint32_t b = __ballot_sync(kFull, sel && key != 0u);
+        if (lane == 0 && b != 0u) atomicOr(a.union_bits + (j * NT + warp * 32) / 32, b);
       }
     }
-    if (want_union) {
-      const uint32_t b = __ballot_sync(kFull, sel && key != 0u);
-      if (lane == 0 && b != 0u) atomicOr(a.union_bits + (j * NT + warp * 32) / 32, b);
-    }
+
   }
 
   if constexpr (BLOCK) {
