@@ -51,6 +51,13 @@ static void check_gemv(int T, int d_out, int rows, int mats, int eb) {
     CHECK(p.smem == (size_t)p.nst * 16 * (p.vec_tile * 16 + 16) + (size_t)p.rcap * 4 * (1 + p.TT),
           f, T, d_out, rows, mats, eb);
     CHECK(p.parts_elems == (size_t)p.copies * mats * d_out * round4(T), f, T, d_out, rows, mats, eb);
+    // one CTA per SM exactly for stages of 40 KB or more; the shared memory of
+    // the occupancy the plan is sized for fits an SM (228 KB, 1 KB per CTA
+    // reserved, a few KB of static shared memory), and the grid is resident
+    const long stage = 16L * (p.vec_tile * 16 + 16);
+    CHECK(p.cta_sm == (stage >= 40L * 1024 ? 1 : 2), f, T, d_out, rows, mats, eb);
+    CHECK(p.cta_sm == 1 ? p.smem <= kSmemAttr : p.smem <= 108u * 1024, f, T, d_out, rows, mats, eb);
+    CHECK((long)p.n_ct * mats * p.S <= 148L * p.cta_sm || p.S == 1, f, T, d_out, rows, mats, eb);
   } else {
     const int vec_row = (int)((long)d_out * eb / 16);
     CHECK(p.TT == 1 || p.TT == 2 || p.TT == 4 || p.TT == 8, f, T, d_out, rows, mats, eb);
@@ -85,7 +92,7 @@ static void check_qgemv(int T, int d_out, int rows) {
           T, d_out, rows);
     CHECK(p.parts_elems == (size_t)d_out * round4(T), f, T, d_out, rows);
   } else {
-    const int lpt = p.TT == 1 ? 32 : (p.TT == 2 ? 16 : (p.TT == 4 ? 8 : 4));
+    const int lpt = p.TT == 1 ? 8 : (p.TT == 2 ? 16 : (p.TT == 4 ? 8 : 4));   // QTune
     CHECK(T < 8 && (p.TT == 1 || p.TT == 2 || p.TT == 4 || p.TT == 8), f, T, d_out, rows);
     CHECK(p.threads % 32 == 0 && (long)(p.threads - 32) * lpt >= (long)p.vec_tile * 8 &&
               p.threads <= 192 + 32,
@@ -159,6 +166,18 @@ int main() {
       if (s[2] <= s[1]) check_layout(QS_OP_SPARSE_FFN, T, s[0], s[1], s[2]);
       if (s[2] <= s[1]) check_layout(QS_OP_SPARSE_FFN_GATE_FIRST, T, s[0], s[1], s[2]);
     }
+  // the batched-decode up/gate plans of the two FFN shapes: 2.75 KB tiles of
+  // the Llama shape run one CTA per SM with four stages, the 2 KB tiles of the
+  // dReLU shape two CTAs per SM (both measured faster that way)
+  {
+    const qs::GemvPlan ll = qs::plan_gemv(8, 11008, 4096, 2, 2);
+    CHECK(ll.mma && ll.vec_tile == 172 && ll.cta_sm == 1 && ll.nst == 4 && ll.n_ct * 2 * ll.S == 144,
+          "llama up/gate T=8 %d", 0);
+    const qs::GemvPlan dr = qs::plan_gemv(4, 14336, 4096, 2, 2);
+    CHECK(dr.mma && dr.vec_tile == 128 && dr.cta_sm == 2 && dr.nst == 2, "drelu up/gate T=4 %d", 0);
+    const qs::GemvPlan q1 = qs::plan_qgemv(1, 11008, 1597);
+    CHECK(!q1.mma && q1.vec_tile == 172 && q1.threads == 192 + 32, "int8 4096->11008 T=1 %d", 0);
+  }
   std::printf("%ld checks, %d failed\n", g_checked, g_fails);
   return g_fails == 0 ? 0 : 1;
 }
