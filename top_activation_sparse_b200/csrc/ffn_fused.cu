@@ -57,9 +57,10 @@ __device__ __forceinline__ int ld_acquire_gpu(const int32_t* p) {
   return v;
 }
 
-// Every CTA arrives once; the waits are bounded (a grid that is not
-// co-resident cannot occur under a cooperative launch, but a wait that runs
-// out records DEV_TIMEOUT and the kernel goes on, it never hangs).
+// Every CTA arrives once; the waits are bounded (the occupancy-sized grid is
+// resident when these layers run alone on the device, and always under a
+// cooperative launch; a wait that runs out records DEV_TIMEOUT and the kernel
+// goes on, it never hangs).
 __device__ __forceinline__ void grid_barrier(int32_t* ctr, int G, DevStatus* st, int where,
                                              int* s_err) {
   __syncthreads();

@@ -368,7 +368,7 @@ cudaError_t launch_qgemv(const QGemvArgs& a, cudaStream_t s);
 
 // ---- one-token FFN as one persistent kernel (ffn_fused.cu) -------------------
 struct FfnFusedPlan {
-  int G = 0;                   // CTAs (all resident: cooperative launch)
+  int G = 0;                   // CTAs (the occupancy-sized grid: all resident)
   int n_ct_ug = 0, vt_ug = 0;  // up/gate column tiles, 16-byte vectors per tile
   int n_ct_dn = 0, vt_dn = 0;  // down column tiles
   int rps_ug = 0, rps_dn = 0;  // row tiles per ring stage
